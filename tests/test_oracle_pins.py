@@ -1,0 +1,321 @@
+"""Pins of the CPU oracle against things other than itself (CPU only).
+
+Each test ties one oracle function to a closed form, a literal fixture from
+``tests/golden/`` (with its citation), a brute-force enumeration on tiny
+inputs, or a library routine (numpy sliding-window means, torch's
+scaled_dot_product_attention in fp64)."""
+from __future__ import annotations
+
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from long_context_decode_nosa_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def _bits(t):
+    return inputs.bf16_bits(t)
+
+
+# --------------------------------------------------------------------------- geometry
+
+def test_geometry_golden(oracle_mod):
+    """Window / block / candidate counts against the literal table derived from
+    the pages' parameters (golden/geometry.txt)."""
+    for L, nc, nb, ncand, _local in (map(int, r) for r in _rows("geometry.txt")):
+        assert oracle_mod.n_windows(L) == nc, L
+        assert oracle_mod.n_blocks(L) == nb, L
+        assert oracle_mod.n_candidates(L) == ncand, L
+
+
+@pytest.mark.parametrize("L", [1, 31, 32, 47, 1024, 1025, 1088, 1089])
+def test_geometry_local_window_tokens(oracle_mod, L):
+    """With nothing selected, attention covers exactly the last local_tokens(L)
+    tokens of golden/geometry.txt (checked through attention weights: V is the
+    one-hot token index, so the output is the attention distribution)."""
+    table = {int(r[0]): int(r[4]) for r in _rows("geometry.txt")}
+    local = table[L]
+    hkv, d = 1, 128
+    b = inputs.make_batch(L, batch=1, num_q_heads=1, num_kv_heads=hkv, seed=5)
+    # zero query -> uniform weights over the attended set
+    q = torch.zeros(1, 1, d, dtype=torch.bfloat16)
+    idx = np.full((1, 1, 4), -1, np.int32)
+    cnt = np.zeros((1, 1), np.int32)
+    out, lse = oracle_mod.sparse_attention(_bits(q), _bits(b.k_cache), _bits(b.v_cache),
+                                           b.seq_start.numpy(), b.seq_len.numpy(), idx, cnt)
+    vf = b.v_cache.double()[:, 0, :].numpy()
+    np.testing.assert_allclose(out[0, 0], vf[L - local:L].mean(0), rtol=1e-12, atol=1e-12)
+    assert abs(lse[0, 0] - math.log(local)) < 1e-12
+
+
+# --------------------------------------------------------------------------- pooling
+
+def test_pool_is_window_mean(oracle_mod):
+    """Pooled key j = mean of keys [16j, 16j+32) (closed form via numpy's
+    sliding_window_view).  fp64 sums of 32 bf16 values of these magnitudes are
+    exact, so both sides round the same real number to fp32: bit-exact."""
+    b = inputs.make_batch([700, 333, 31], num_kv_heads=2, num_q_heads=4, seed=11)
+    nc_cap = oracle_mod.n_windows(700)
+    pooled = oracle_mod.pool(_bits(b.k_cache), b.seq_start.numpy(), b.seq_len.numpy(), nc_cap)
+    kf = b.k_cache.double().numpy()
+    for i in range(3):
+        L, s0 = int(b.seq_len[i]), int(b.seq_start[i])
+        nc = oracle_mod.n_windows(L)
+        if nc:
+            win = np.lib.stride_tricks.sliding_window_view(kf[s0:s0 + L], 32, axis=0)[::16]
+            ref = win.mean(-1).astype(np.float32)  # [nc, Hkv, D]
+            assert ref.shape[0] == nc
+            np.testing.assert_array_equal(pooled[i, :, :nc], ref.transpose(1, 0, 2))
+        assert not pooled[i, :, nc:].any()
+
+
+def test_pool_incremental_equals_rebuild(oracle_mod):
+    """Appending tokens one at a time gives the same pooled cache as one rebuild,
+    and windows outside [nc(len_old), nc(len_new)) are left alone."""
+    L = 300
+    b = inputs.make_batch(L, batch=2, num_kv_heads=2, num_q_heads=2, seed=3)
+    nc_cap = oracle_mod.n_windows(L)
+    full = oracle_mod.pool(_bits(b.k_cache), b.seq_start.numpy(), b.seq_len.numpy(), nc_cap)
+    inc = np.full_like(full, 7.0)
+    inc[:] = 0
+    for t in range(1, L + 1):
+        lo = np.full(2, t - 1, np.int32)
+        hi = np.full(2, t, np.int32)
+        inc = oracle_mod.pool(_bits(b.k_cache), b.seq_start.numpy(), hi, nc_cap, len_old=lo,
+                              pooled=inc)
+    np.testing.assert_array_equal(inc, full)
+    sentinel = np.full_like(full, 7.0)
+    out = oracle_mod.pool(_bits(b.k_cache), b.seq_start.numpy(), np.full(2, 100, np.int32),
+                          nc_cap, len_old=np.full(2, 50, np.int32), pooled=sentinel)
+    lo, hi = oracle_mod.n_windows(50), oracle_mod.n_windows(100)
+    np.testing.assert_array_equal(out[:, :, lo:hi], full[:, :, lo:hi])
+    assert (out[:, :, :lo] == 7.0).all() and (out[:, :, hi:] == 7.0).all()
+
+
+# --------------------------------------------------------------------------- scores
+
+def test_comp_scores_equal_mean_of_token_scores(oracle_mod):
+    """Linearity: scale * q . mean(k_t) equals the mean over the window of the
+    per-token scores scale * q . k_t (so pooling keys and pooling raw scores
+    agree).  Token scores via numpy einsum in fp64."""
+    b = inputs.make_batch([520, 97], num_q_heads=8, num_kv_heads=2, seed=21)
+    nc_cap = oracle_mod.n_windows(520)
+    pooled = oracle_mod.pool(_bits(b.k_cache), b.seq_start.numpy(), b.seq_len.numpy(), nc_cap)
+    s = oracle_mod.comp_scores(_bits(b.q), pooled, b.seq_len.numpy(), num_kv_heads=2)
+    qf, kf = b.q.double().numpy(), b.k_cache.double().numpy()
+    scale = 1 / math.sqrt(128)
+    for i in range(2):
+        L, s0 = int(b.seq_len[i]), int(b.seq_start[i])
+        nc = oracle_mod.n_windows(L)
+        tok = scale * np.einsum("hd,thd->ht", qf[i], np.repeat(kf[s0:s0 + L], 4, axis=1))
+        win = np.lib.stride_tricks.sliding_window_view(tok, 32, axis=1)[:, ::16].mean(-1)
+        np.testing.assert_allclose(s[i, :, :nc], win, rtol=2e-6, atol=2e-6)
+        assert np.isneginf(s[i, :, nc:]).all()
+
+
+def test_comp_scores_gqa_mapping(oracle_mod):
+    """Query head h reads KV head h // G: a one-hot query along dim c returns
+    scale * pooled[g][:, c] for its own group only."""
+    rng = np.random.default_rng(0)
+    B, hq, hkv, d, nc = 1, 4, 2, 128, 5
+    pooled = rng.standard_normal((B, hkv, nc, d)).astype(np.float32)
+    q = torch.zeros(B, hq, d, dtype=torch.bfloat16)
+    for h in range(hq):
+        q[0, h, 10 + h] = 1.0
+    L = np.array([32 + 16 * (nc - 1)], np.int32)
+    s = oracle_mod.comp_scores(_bits(q), pooled, L, num_kv_heads=hkv, scale=1.0)
+    for h in range(hq):
+        np.testing.assert_array_equal(s[0, h], pooled[0, h // 2, :, 10 + h])
+
+
+# --------------------------------------------------------------------------- block scores
+
+def test_block_overlap_golden(oracle_mod):
+    """A one-hot compressed score at window j lights exactly the blocks of
+    golden/block_overlap.txt."""
+    L = 64 * 40
+    nc = oracle_mod.n_windows(L)
+    nb = oracle_mod.n_blocks(L)
+    for row in _rows("block_overlap.txt"):
+        j = int(row[0])
+        want = sorted(int(x) for x in row[3].split(","))
+        s = np.zeros((1, 1, nc), np.float32)
+        s[0, 0, j] = 1.0
+        S = oracle_mod.block_scores(s, np.array([L], np.int32), nb, num_kv_heads=1)
+        lit = sorted(np.nonzero(S[0, 0, :nb - 16] == 1.0)[0].tolist())
+        assert lit == want, (j, lit, want)
+
+
+def test_block_scores_max_then_sum_over_group(oracle_mod):
+    """Literal values: max over a block's windows per head, summed over the
+    heads of the GQA group; -inf outside the candidates."""
+    L = 64 * 20  # 20 blocks, 4 candidates
+    nc = oracle_mod.n_windows(L)
+    s = np.full((1, 4, nc), -1.0, np.float32)   # heads 0,1 -> KV head 0; 2,3 -> KV head 1
+    s[0, 0, 4] = 1.0    # block 1
+    s[0, 0, 5] = 3.0    # block 1
+    s[0, 1, 7] = 2.0    # blocks 1, 2
+    s[0, 2, 0] = 5.0    # block 0
+    s[0, 3, 15] = 4.0   # blocks 3, 4 (4 is local)
+    S = oracle_mod.block_scores(s, np.array([L], np.int32), 20, num_kv_heads=2)
+    np.testing.assert_array_equal(S[0, 0, :4], np.array([-2.0, 5.0, 1.0, -2.0], np.float32))
+    np.testing.assert_array_equal(S[0, 1, :4], np.array([4.0, -2.0, -2.0, 3.0], np.float32))
+    assert np.isneginf(S[0, :, 4:]).all()
+
+
+# --------------------------------------------------------------------------- top-k
+
+def _brute_topk(scores, k):
+    """The unique size-k subset X with: for x in X, y not in X, x ranks above y
+    (higher score, or equal score and lower index); NaN ranks as -inf and
+    -0.0 equals +0.0."""
+    n = len(scores)
+    val = [(-math.inf if math.isnan(v) else (0.0 if v == 0 else v)) for v in scores]
+
+    def above(x, y):
+        return val[x] > val[y] or (val[x] == val[y] and x < y)
+
+    found = [X for X in itertools.combinations(range(n), k)
+             if all(above(x, y) for x in X for y in set(range(n)) - set(X))]
+    assert len(found) == 1
+    return list(found[0])
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_topk_brute_force(oracle_mod, seed):
+    rng = np.random.default_rng(seed)
+    ncand = int(rng.integers(0, 13))
+    L = 64 * (ncand + 16)
+    # few distinct values -> many ties; sprinkle -0.0, +0.0 and NaN
+    S = rng.integers(-3, 4, size=(1, 1, ncand + 16)).astype(np.float32)
+    if ncand and seed % 3 == 0:
+        S[0, 0, rng.integers(0, ncand)] = -0.0
+        S[0, 0, rng.integers(0, ncand)] = np.nan
+    for k in sorted({1, ncand // 2, ncand - 1, ncand, ncand + 3} - {0, -1}):
+        idx, cnt = oracle_mod.topk(S, np.array([L], np.int32), k)
+        kk = min(k, ncand)
+        assert cnt[0, 0] == kk
+        want = _brute_topk(S[0, 0, :ncand].tolist(), kk)
+        assert idx[0, 0, :kk].tolist() == want
+        assert (idx[0, 0, kk:] == -1).all()
+
+
+def test_topk_ties_go_to_lowest_index(oracle_mod):
+    S = np.zeros((1, 1, 26), np.float32)  # 10 candidates, all tied
+    idx, cnt = oracle_mod.topk(S, np.array([64 * 26], np.int32), 4)
+    assert idx[0, 0].tolist() == [0, 1, 2, 3] and cnt[0, 0] == 4
+
+
+# --------------------------------------------------------------------------- attention
+
+def _sdpa_reference(b, mask_tokens, i, scale=None):
+    """torch fp64 scaled_dot_product_attention of sequence i over a token mask."""
+    G = b.num_q_heads // b.num_kv_heads
+    L, s0 = int(b.seq_len[i]), int(b.seq_start[i])
+    q = b.q[i].double().unsqueeze(1)                           # [Hq, 1, D]
+    k = b.k_cache[s0:s0 + L].double().permute(1, 0, 2).repeat_interleave(G, 0)
+    v = b.v_cache[s0:s0 + L].double().permute(1, 0, 2).repeat_interleave(G, 0)
+    m = torch.as_tensor(mask_tokens)                           # [Hkv, L] bool
+    m = m.repeat_interleave(G, 0).unsqueeze(1)                 # [Hq, 1, L]
+    o = F.scaled_dot_product_attention(q, k, v, attn_mask=m, scale=scale)
+    logits = (q @ k.transpose(-1, -2)) * (scale if scale else 1 / math.sqrt(b.head_dim))
+    lse = torch.logsumexp(logits.masked_fill(~m, -math.inf), dim=-1)
+    return o[:, 0].numpy(), lse[:, 0].numpy()
+
+
+def test_dense_equivalence_when_budget_covers_all(oracle_mod):
+    """topk >= number of candidates: sparse attention == dense causal decode
+    attention over [0, L) (library SDPA in fp64)."""
+    lens = [1500, 2300, 700, 64 * 17 + 5]
+    b = inputs.make_batch(lens, num_q_heads=8, num_kv_heads=2, seed=7)
+    nb_max = oracle_mod.n_blocks(max(lens))
+    idx = np.full((4, 2, nb_max), -1, np.int32)
+    cnt = np.zeros((4, 2), np.int32)
+    for i, L in enumerate(lens):
+        nc = oracle_mod.n_candidates(L)
+        idx[i, :, :nc] = np.arange(nc)
+        cnt[i, :] = nc
+    out, lse = oracle_mod.sparse_attention(_bits(b.q), _bits(b.k_cache), _bits(b.v_cache),
+                                           b.seq_start.numpy(), b.seq_len.numpy(), idx, cnt)
+    for i, L in enumerate(lens):
+        o_ref, l_ref = _sdpa_reference(b, np.ones((2, L), bool), i)
+        np.testing.assert_allclose(out[i], o_ref, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(lse[i], l_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_set_matches_masked_sdpa(oracle_mod):
+    """A hand-picked selection: output equals masked SDPA over the literal token
+    set (selected blocks + block-aligned local window)."""
+    L = 64 * 30 + 17                      # nb = 31, ncand = 15, local = [960, L)
+    b = inputs.make_batch(L, batch=1, num_q_heads=4, num_kv_heads=2, seed=9)
+    sel = {0: [0, 3, 14], 1: [2, 7]}
+    idx = np.full((1, 2, 3), -1, np.int32)
+    cnt = np.zeros((1, 2), np.int32)
+    mask = np.zeros((2, L), bool)
+    for g, blocks in sel.items():
+        idx[0, g, :len(blocks)] = blocks
+        cnt[0, g] = len(blocks)
+        for blk in blocks:
+            mask[g, 64 * blk:64 * blk + 64] = True
+        mask[g, 960:] = True
+    out, lse = oracle_mod.sparse_attention(_bits(b.q), _bits(b.k_cache), _bits(b.v_cache),
+                                           b.seq_start.numpy(), b.seq_len.numpy(), idx, cnt,
+                                           scale=0.3)
+    o_ref, l_ref = _sdpa_reference(b, mask, 0, scale=0.3)
+    np.testing.assert_allclose(out[0], o_ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(lse[0], l_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_invariant_to_selection_order(oracle_mod):
+    L = 64 * 40
+    b = inputs.make_batch(L, batch=1, num_q_heads=2, num_kv_heads=1, seed=13)
+    idx = np.array([[[1, 5, 9, 20]]], np.int32)
+    cnt = np.array([[4]], np.int32)
+    a = oracle_mod.sparse_attention(_bits(b.q), _bits(b.k_cache), _bits(b.v_cache),
+                                    b.seq_start.numpy(), b.seq_len.numpy(), idx, cnt)
+    c = oracle_mod.sparse_attention(_bits(b.q), _bits(b.k_cache), _bits(b.v_cache),
+                                    b.seq_start.numpy(), b.seq_len.numpy(),
+                                    idx[:, :, ::-1].copy(), cnt)
+    np.testing.assert_allclose(a[0], c[0], rtol=1e-13, atol=1e-15)
+
+
+def test_attention_rejects_out_of_range_index(oracle_mod):
+    L = 64 * 20
+    b = inputs.make_batch(L, batch=1, num_q_heads=2, num_kv_heads=1, seed=1)
+    idx = np.array([[[4]]], np.int32)     # ncand = 4 -> index 4 is local, not a candidate
+    with pytest.raises(ValueError):
+        oracle_mod.sparse_attention(_bits(b.q), _bits(b.k_cache), _bits(b.v_cache),
+                                    b.seq_start.numpy(), b.seq_len.numpy(), idx,
+                                    np.array([[1]], np.int32))
+
+
+# --------------------------------------------------------------------------- whole step
+
+def test_planted_blocks_are_selected_with_a_clear_gap(oracle_mod):
+    """Parity workload shape (B=1, 16/2 heads, L=8192, top-k 48 of 112): every
+    planted block is selected and the top-k boundary gap is far above fp32
+    score rounding."""
+    b = inputs.make_batch(8192, batch=1, num_q_heads=16, num_kv_heads=2, seed=1)
+    planted = inputs.plant_blocks(b, seed=101)
+    nc_cap = oracle_mod.n_windows(8192)
+    pooled = oracle_mod.pool(_bits(b.k_cache), b.seq_start.numpy(), b.seq_len.numpy(), nc_cap)
+    r = oracle_mod.decode_step(_bits(b.q), _bits(b.k_cache), _bits(b.v_cache),
+                               b.seq_start.numpy(), b.seq_len.numpy(), pooled, 48)
+    for g in range(2):
+        sel = set(r["sel_idx"][0, g].tolist())
+        assert set(planted[0, g].tolist()) <= sel
+        S = np.sort(r["block_scores"][0, g, :112])[::-1]
+        gap = S[47] - S[48]
+        assert gap > 1e-3 * max(1.0, abs(S[47])), gap
