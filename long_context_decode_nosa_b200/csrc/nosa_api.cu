@@ -1,0 +1,401 @@
+// Host side of the C ABI declared in include/nosa.h: argument checks,
+// workspace layout, launch planning and the host-buffer decode step.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "nosa.h"
+#include "nosa_common.cuh"
+#include "nosa_kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local uint32_t g_last_bits = 0;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return NOSA_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(NOSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_params(const nosa_params* p) {
+  if (!p) return fail(NOSA_ERR_INVALID_ARG, "params is NULL");
+  if (p->num_kv_heads < 1 || p->num_q_heads < 1 || p->num_q_heads % p->num_kv_heads != 0)
+    return fail(NOSA_ERR_INVALID_ARG, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
+                p->num_q_heads, p->num_kv_heads);
+  const int G = p->num_q_heads / p->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
+    return fail(NOSA_ERR_UNSUPPORTED, "GQA group size %d not supported (1, 2, 4, 8 or 16)", G);
+  if (p->head_dim != nosa::kHeadDim)
+    return fail(NOSA_ERR_UNSUPPORTED, "head_dim %d not supported (128)", p->head_dim);
+  if (p->pool_kernel != nosa::kPoolKernel || p->pool_stride != nosa::kPoolStride)
+    return fail(NOSA_ERR_UNSUPPORTED, "pooling kernel/stride %d/%d not supported (32/16)",
+                p->pool_kernel, p->pool_stride);
+  if (p->block_size != nosa::kBlock)
+    return fail(NOSA_ERR_UNSUPPORTED, "block_size %d not supported (64)", p->block_size);
+  if (p->local_blocks < 0) return fail(NOSA_ERR_INVALID_ARG, "local_blocks < 0");
+  if (p->topk < 1 || p->topk > 1024) return fail(NOSA_ERR_UNSUPPORTED, "topk %d outside 1..1024", p->topk);
+  if (!(p->softmax_scale >= 0.0f) || std::isinf(p->softmax_scale))
+    return fail(NOSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  return NOSA_OK;
+}
+
+float scale_of(const nosa_params* p) {
+  return p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(p->head_dim));
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace layout (all offsets 256-byte aligned).
+struct Layout {
+  size_t status, sel_tickets, dec_tickets, bscores, part, stage_q, stage_k, stage_v, stage_out, total;
+  int nb_ws;
+};
+
+Layout layout_of(const nosa_params* p, int batch, int max_seq_len) {
+  Layout l{};
+  const size_t pairs = static_cast<size_t>(batch) * p->num_kv_heads;
+  const int G = p->num_q_heads / p->num_kv_heads;
+  l.nb_ws = static_cast<int>(nosa::n_blocks(max_seq_len));
+  size_t off = 0;
+  l.status = off;
+  off += 256;
+  l.sel_tickets = off;
+  off = round_up(off + pairs * 4, 256);
+  l.dec_tickets = off;
+  off = round_up(off + pairs * 4, 256);
+  l.bscores = off;
+  off = round_up(off + pairs * static_cast<size_t>(l.nb_ws) * 4, 256);
+  l.part = off;
+  off = round_up(off + pairs * nosa::kMaxSplits * static_cast<size_t>(G) * (nosa::kHeadDim + 2) * 4, 256);
+  const size_t qbytes = static_cast<size_t>(batch) * p->num_q_heads * nosa::kHeadDim * 2;
+  const size_t kvbytes = pairs * nosa::kHeadDim * 2;
+  l.stage_q = off;
+  off = round_up(off + qbytes, 256);
+  l.stage_k = off;
+  off = round_up(off + kvbytes, 256);
+  l.stage_v = off;
+  off = round_up(off + kvbytes, 256);
+  l.stage_out = off;
+  off = round_up(off + qbytes, 256);
+  l.total = off;
+  return l;
+}
+
+int check_ws(void* ws, size_t ws_bytes, const Layout& l) {
+  if (!ws) return fail(NOSA_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned(ws, 256)) return fail(NOSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < l.total)
+    return fail(NOSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, l.total);
+  return NOSA_OK;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, const int64_t* seq_start,
+                   const int32_t* len_old, const int32_t* len_new, int batch, float* pooled, int nc_cap,
+                   int max_new_keys, const void* k_new, const void* v_new, uint32_t* status,
+                   cudaStream_t stream) {
+  if (batch < 0 || nc_cap < 0 || max_new_keys < 0)
+    return fail(NOSA_ERR_INVALID_ARG, "batch, nc_cap and max_new_keys must be >= 0");
+  if (batch == 0) return ok();
+  if (!k_cache || !seq_start || !len_new || !pooled)
+    return fail(NOSA_ERR_INVALID_ARG, "k_cache, seq_start, len_new and pooled must not be NULL");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(NOSA_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+  if (k_new && !v_cache) return fail(NOSA_ERR_INVALID_ARG, "v_cache must not be NULL when appending");
+  if (!aligned(k_cache, 16) || !aligned(pooled, 16) || (v_cache && !aligned(v_cache, 16)) ||
+      (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16))))
+    return fail(NOSA_ERR_INVALID_ARG, "cache, pooled and new-row pointers must be 16-byte aligned");
+  if (static_cast<int64_t>(batch) * p->num_kv_heads > 65535)
+    return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 65535");
+  nosa::PoolArgs a{};
+  a.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  a.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  a.seq_start = seq_start;
+  a.len_old = len_old;
+  a.len_new = len_new;
+  a.pooled = pooled;
+  a.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  a.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  a.status = status;
+  a.batch = batch;
+  a.hkv = p->num_kv_heads;
+  a.nc_cap = nc_cap;
+  a.max_new_keys = max_new_keys;
+  cudaError_t e = nosa::launch_pool_append(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "pool_append launch");
+  return ok();
+}
+
+int do_block_select(const nosa_params* p, const void* q, const float* pooled, int nc_cap,
+                    const int32_t* seq_len, int batch, int max_seq_len, const float* bs_in, int nb_in,
+                    float* comp_out, float* bs_out, int nb_out, int32_t* sel_idx, int32_t* sel_cnt,
+                    void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (batch < 0 || max_seq_len < 1) return fail(NOSA_ERR_INVALID_ARG, "batch >= 0 and max_seq_len >= 1 required");
+  if (batch == 0) return ok();
+  const Layout l = layout_of(p, batch, max_seq_len);
+  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
+  if (!seq_len || !sel_idx || !sel_cnt) return fail(NOSA_ERR_INVALID_ARG, "seq_len, sel_idx and sel_cnt must not be NULL");
+  const int ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
+  if (bs_in) {
+    if (nb_in < ncand_max)
+      return fail(NOSA_ERR_INVALID_ARG, "nb_cap_in %d below the %d candidates of max_seq_len", nb_in, ncand_max);
+  } else {
+    if (!q || !pooled) return fail(NOSA_ERR_INVALID_ARG, "q and pooled must not be NULL when scoring");
+    if (!aligned(pooled, 16) || !aligned(q, 8)) return fail(NOSA_ERR_INVALID_ARG, "pooled must be 16-byte and q 8-byte aligned");
+    if (nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "nc_cap must be >= 1");
+    if (bs_out && nb_out < ncand_max)
+      return fail(NOSA_ERR_INVALID_ARG, "nb_cap_out %d below the %d candidates of max_seq_len", nb_out, ncand_max);
+  }
+  if (l.nb_ws * 4 > 200 * 1024) return fail(NOSA_ERR_UNSUPPORTED, "max_seq_len too long for the selector");
+  if (static_cast<int64_t>(batch) * p->num_kv_heads > 65535)
+    return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 65535");
+  nosa::SelectArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.pooled = pooled;
+  a.seq_len = seq_len;
+  a.bs_in = bs_in;
+  a.comp_out = bs_in ? nullptr : comp_out;
+  a.bs_out = bs_in ? nullptr : bs_out;
+  a.sel_idx = sel_idx;
+  a.sel_cnt = sel_cnt;
+  a.bscratch = at<float>(ws, l.bscores);
+  a.tickets = at<uint32_t>(ws, l.sel_tickets);
+  a.status = at<uint32_t>(ws, l.status);
+  a.batch = batch;
+  a.hq = p->num_q_heads;
+  a.hkv = p->num_kv_heads;
+  a.group = p->num_q_heads / p->num_kv_heads;
+  a.local_blocks = p->local_blocks;
+  a.topk = p->topk;
+  a.max_seq_len = max_seq_len;
+  a.nc_cap = nc_cap;
+  a.nb_in = nb_in;
+  a.nb_out = nb_out;
+  a.nb_ws = l.nb_ws;
+  a.scale = scale_of(p);
+  cudaError_t e = nosa::launch_block_select(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "block_select launch");
+  return ok();
+}
+
+int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                     const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
+                     const int32_t* sel_idx, const int32_t* sel_cnt, void* out, float* lse, void* ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+  if (batch < 0 || max_seq_len < 1) return fail(NOSA_ERR_INVALID_ARG, "batch >= 0 and max_seq_len >= 1 required");
+  if (batch == 0) return ok();
+  const Layout l = layout_of(p, batch, max_seq_len);
+  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
+  if (!q || !k_cache || !v_cache || !seq_start || !seq_len || !sel_idx || !sel_cnt || !out)
+    return fail(NOSA_ERR_INVALID_ARG, "q, caches, seq_start, seq_len, sel_idx, sel_cnt and out must not be NULL");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4))
+    return fail(NOSA_ERR_INVALID_ARG, "caches must be 16-byte and q 4-byte aligned");
+  if (static_cast<int64_t>(batch) * p->num_kv_heads > 65535)
+    return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 65535");
+  const int nb_max = static_cast<int>(nosa::n_blocks(max_seq_len));
+  const int ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
+  const int max_tiles = (p->topk < ncand_max ? p->topk : ncand_max) +
+                        (p->local_blocks < nb_max ? p->local_blocks : nb_max);
+  nosa::DecodeArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
+  a.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  a.seq_start = seq_start;
+  a.seq_len = seq_len;
+  a.sel_idx = sel_idx;
+  a.sel_cnt = sel_cnt;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.part = at<float>(ws, l.part);
+  a.tickets = at<uint32_t>(ws, l.dec_tickets);
+  a.status = at<uint32_t>(ws, l.status);
+  a.batch = batch;
+  a.hq = p->num_q_heads;
+  a.hkv = p->num_kv_heads;
+  a.group = p->num_q_heads / p->num_kv_heads;
+  a.local_blocks = p->local_blocks;
+  a.topk = p->topk;
+  a.max_seq_len = max_seq_len;
+  nosa::decode_split_plan(batch * p->num_kv_heads, max_tiles, sm_count(), &a.nsplit, &a.tiles_per_split);
+  a.scale_log2 = scale_of(p) * 1.4426950408889634f;
+  cudaError_t e = nosa::launch_sparse_decode(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse_decode launch");
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+void nosa_default_params(nosa_params* p) {
+  if (!p) return;
+  p->num_q_heads = 16;
+  p->num_kv_heads = 2;
+  p->head_dim = 128;
+  p->pool_kernel = 32;
+  p->pool_stride = 16;
+  p->block_size = 64;
+  p->local_blocks = 16;
+  p->topk = 64;
+  p->softmax_scale = 0.0f;
+}
+
+size_t nosa_workspace_size(const nosa_params* p, int batch, int max_seq_len) {
+  if (check_params(p) != NOSA_OK || batch < 0 || max_seq_len < 1) return 0;
+  return layout_of(p, batch, max_seq_len).total;
+}
+
+int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < 256) return fail(NOSA_ERR_WORKSPACE, "workspace NULL or smaller than 256 bytes");
+  if (!aligned(ws, 256)) return fail(NOSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "workspace memset");
+  return ok();
+}
+
+int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache, const int64_t* seq_start,
+                     const int32_t* len_old, const int32_t* len_new, int batch, float* pooled, int nc_cap,
+                     int max_new_keys, const void* k_new, const void* v_new, void* ws, size_t ws_bytes,
+                     void* stream) {
+  if (int rc = check_params(p)) return rc;
+  uint32_t* status = nullptr;
+  if (ws) {
+    if (ws_bytes < 256 || !aligned(ws, 256)) return fail(NOSA_ERR_WORKSPACE, "workspace must be 256-byte aligned and >= 256 bytes");
+    status = at<uint32_t>(ws, 0);
+  }
+  return do_pool_append(p, k_cache, v_cache, seq_start, len_old, len_new, batch, pooled, nc_cap,
+                        max_new_keys, k_new, v_new, status, static_cast<cudaStream_t>(stream));
+}
+
+int nosa_block_select(const nosa_params* p, const void* q, const float* pooled, int nc_cap,
+                      const int32_t* seq_len, int batch, int max_seq_len, const float* block_scores_in,
+                      int nb_cap_in, float* comp_scores_out, float* block_scores_out, int nb_cap_out,
+                      int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_params(p)) return rc;
+  return do_block_select(p, q, pooled, nc_cap, seq_len, batch, max_seq_len, block_scores_in, nb_cap_in,
+                         comp_scores_out, block_scores_out, nb_cap_out, sel_idx, sel_cnt, ws, ws_bytes,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int nosa_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                       const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
+                       const int32_t* sel_idx, const int32_t* sel_cnt, void* out, float* lse, void* ws,
+                       size_t ws_bytes, void* stream) {
+  if (int rc = check_params(p)) return rc;
+  return do_sparse_decode(p, q, k_cache, v_cache, seq_start, seq_len, batch, max_seq_len, sel_idx,
+                          sel_cnt, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new_host,
+                     const void* v_new_host, void* out_host, void* k_cache, void* v_cache,
+                     const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
+                     float* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* ws,
+                     size_t ws_bytes, void* stream) {
+  if (int rc = check_params(p)) return rc;
+  if (batch < 0 || max_seq_len < 1) return fail(NOSA_ERR_INVALID_ARG, "batch >= 0 and max_seq_len >= 1 required");
+  if (batch == 0) return ok();
+  if (!q_host || !k_new_host || !v_new_host || !out_host)
+    return fail(NOSA_ERR_INVALID_ARG, "host buffers must not be NULL");
+  const Layout l = layout_of(p, batch, max_seq_len);
+  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t qbytes = static_cast<size_t>(batch) * p->num_q_heads * nosa::kHeadDim * 2;
+  const size_t kvbytes = static_cast<size_t>(batch) * p->num_kv_heads * nosa::kHeadDim * 2;
+  void* dq = at<void>(ws, l.stage_q);
+  void* dk = at<void>(ws, l.stage_k);
+  void* dv = at<void>(ws, l.stage_v);
+  void* dout = at<void>(ws, l.stage_out);
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(dq, q_host, qbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy q");
+  if ((e = cudaMemcpyAsync(dk, k_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy k_new");
+  if ((e = cudaMemcpyAsync(dv, v_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy v_new");
+  int rc = do_pool_append(p, k_cache, v_cache, seq_start, nullptr, seq_len, batch, pooled, nc_cap, 1, dk, dv,
+                          at<uint32_t>(ws, l.status), s);
+  if (rc) return rc;
+  rc = do_block_select(p, dq, pooled, nc_cap, seq_len, batch, max_seq_len, nullptr, 0, nullptr, nullptr, 0,
+                       sel_idx, sel_cnt, ws, ws_bytes, s);
+  if (rc) return rc;
+  rc = do_sparse_decode(p, dq, k_cache, v_cache, seq_start, seq_len, batch, max_seq_len, sel_idx, sel_cnt,
+                        dout, nullptr, ws, ws_bytes, s);
+  if (rc) return rc;
+  if ((e = cudaMemcpyAsync(out_host, dout, qbytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess) return cuda_fail(e, "copy out");
+  return ok();
+}
+
+int nosa_read_device_status(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < 256 || !aligned(ws, 256)) return fail(NOSA_ERR_WORKSPACE, "workspace NULL, small or misaligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t bits = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&bits, ws, sizeof bits, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof bits, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "read device status");
+  g_last_bits = bits;
+  if (bits & NOSA_DEV_TIMEOUT) return fail(NOSA_ERR_TIMEOUT, "device status 0x%08x: a bounded wait gave up", bits);
+  if (bits) return fail(NOSA_ERR_DEVICE_CHECK, "device status 0x%08x", bits);
+  return ok();
+}
+
+uint32_t nosa_last_device_bits(void) { return g_last_bits; }
+
+int nosa_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t max_iters, void* stream) {
+  if (!ws || ws_bytes < 256 || !aligned(ws, 256)) return fail(NOSA_ERR_WORKSPACE, "workspace NULL, small or misaligned");
+  if (max_iters < 1 || max_iters > (1u << 20)) return fail(NOSA_ERR_INVALID_ARG, "max_iters must be 1..2^20");
+  cudaError_t e = nosa::launch_wait_selftest(at<uint32_t>(ws, 0), max_iters, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wait selftest launch");
+  return ok();
+}
+
+const char* nosa_status_string(int status) {
+  switch (status) {
+    case NOSA_OK: return "ok";
+    case NOSA_ERR_INVALID_ARG: return "invalid argument";
+    case NOSA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case NOSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case NOSA_ERR_CUDA: return "CUDA error";
+    case NOSA_ERR_DEVICE_CHECK: return "device data check failed";
+    case NOSA_ERR_TIMEOUT: return "bounded device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* nosa_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

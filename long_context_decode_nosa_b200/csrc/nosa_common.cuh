@@ -1,0 +1,117 @@
+// Shared device helpers of the NOSA sparse-decode kernels (sm_100a).
+//
+// mbarrier + bulk-copy (TMA, cp.async.bulk) wrappers written as inline PTX,
+// with every wait bounded: a wait that does not complete within
+// kWaitLimitNs of %globaltimer (or kWaitLimitIters polls) sets
+// NOSA_DEV_TIMEOUT in the device status word and returns false, so a kernel
+// never spins forever and never traps.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "nosa.h"
+
+namespace nosa {
+
+constexpr int kHeadDim = 128;
+constexpr int kPoolKernel = 32;
+constexpr int kPoolStride = 16;
+constexpr int kBlock = 64;
+constexpr int kWindowsPerBlock = kBlock / kPoolStride;  // 4
+constexpr int kMaxGroup = 16;
+constexpr int kMaxSplits = 64;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kWaitLimitIters = 1u << 30;
+
+__host__ __device__ inline int64_t n_windows(int64_t L) {
+  return L >= kPoolKernel ? (L - kPoolKernel) / kPoolStride + 1 : 0;
+}
+__host__ __device__ inline int64_t n_blocks(int64_t L) { return (L + kBlock - 1) / kBlock; }
+__host__ __device__ inline int64_t n_candidates(int64_t L, int local_blocks) {
+  int64_t c = n_blocks(L) - local_blocks;
+  return c > 0 ? c : 0;
+}
+
+__device__ inline void set_status(uint32_t* status, uint32_t bits) {
+  if (status) atomicOr(status, bits);
+}
+
+__device__ inline uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ inline uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ inline void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+// Makes barrier initialisation visible to the async (TMA) proxy.
+__device__ inline void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ inline void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ inline bool mbar_test_parity(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Waits until the phase with the given parity has completed.  Bounded by
+// `max_iters` polls and kWaitLimitNs of wall time; on giving up it sets
+// NOSA_DEV_TIMEOUT and returns false.
+__device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                 uint32_t max_iters = kWaitLimitIters) {
+  if (mbar_test_parity(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1; it < max_iters; ++it) {
+    if (mbar_test_parity(bar, parity)) return true;
+    if ((it & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) break;
+  }
+  set_status(status, NOSA_DEV_TIMEOUT);
+  return false;
+}
+
+// 1-D bulk copy global -> shared through the TMA unit, completing on `bar`.
+// dst, src and bytes must be multiples of 16.
+__device__ inline void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Order-preserving map of an fp32 score to uint32, with -0.0 == +0.0 and NaN
+// ranked as -inf (ties are then broken by index by the caller).
+__device__ inline uint32_t order_key(float f) {
+  if (f != f) f = -INFINITY;
+  if (f == 0.0f) f = 0.0f;
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+}  // namespace nosa

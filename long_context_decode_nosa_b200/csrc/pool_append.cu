@@ -1,0 +1,108 @@
+// K1 -- CIS mean pooling of the key cache, appended incrementally.
+//
+// "从论文到代码：手把手教你理解NOSA-8B的高效注意力机制实现" (nzsm.cn),
+// "NOSA-8B的核心实现模块" item 2 (keys pooled with cis_pooling(k, cu_seqlens));
+// "NOSA-1B 性能基准全解析" (wmrh.cn) §三.3 (kernel_size 32, stride 16).
+//
+// One warp per (sequence, KV head, new window).  Lane l owns dims 4l..4l+3:
+// each of the 32 rows of the window is one coalesced 256-byte warp load
+// (8 bytes per lane), summed in fp32 in ascending token order, then scaled by
+// 1/32 (exact).  A fixed order makes an incremental append bit-identical to a
+// rebuild.  With k_new/v_new given, warp 0 of chunk 0 also stores the new
+// token's K/V rows into the caches; pooling reads that token from k_new, so
+// no cross-warp ordering is needed.
+#include "nosa_common.cuh"
+#include "nosa_kernels.h"
+
+namespace nosa {
+
+namespace {
+
+constexpr int kWarpsPerCta = 4;
+
+__device__ inline float4 bf16x4_to_float4(uint2 raw) {
+  float4 f;
+  f.x = __uint_as_float(raw.x << 16);
+  f.y = __uint_as_float(raw.x & 0xFFFF0000u);
+  f.z = __uint_as_float(raw.y << 16);
+  f.w = __uint_as_float(raw.y & 0xFFFF0000u);
+  return f;
+}
+
+__global__ void __launch_bounds__(kWarpsPerCta * 32)
+    pool_append_kernel(const PoolArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.y;
+  const int i = pair / a.hkv, h = pair % a.hkv;
+  const int32_t len_new = a.len_new[i];
+  const int32_t len_old = a.len_old ? a.len_old[i] : len_new - 1;
+  if (len_old < 0 || len_new < len_old) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, NOSA_DEV_BAD_LENGTH);
+    return;
+  }
+  const int64_t base = a.seq_start[i];
+  const bool append = a.k_new != nullptr;
+  if (append && len_new != len_old + 1) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, NOSA_DEV_APPEND_ONE);
+    return;
+  }
+  const uint2* knew_row =
+      append ? reinterpret_cast<const uint2*>(a.k_new + (static_cast<int64_t>(i) * a.hkv + h) * kHeadDim)
+             : nullptr;
+  if (append && blockIdx.x == 0 && warp == 0) {
+    const int64_t row = (base + len_old) * a.hkv + h;
+    const uint2* vnew_row =
+        reinterpret_cast<const uint2*>(a.v_new + (static_cast<int64_t>(i) * a.hkv + h) * kHeadDim);
+    reinterpret_cast<uint2*>(a.k_cache + row * kHeadDim)[lane] = knew_row[lane];
+    reinterpret_cast<uint2*>(a.v_cache + row * kHeadDim)[lane] = vnew_row[lane];
+  }
+  const int64_t j_first = n_windows(len_old), j_end = n_windows(len_new);
+  if (j_end - j_first > a.max_new_keys && blockIdx.x == 0 && threadIdx.x == 0)
+    set_status(a.status, NOSA_DEV_MAX_NEW_KEYS);
+  const int64_t j = j_first + static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + warp;
+  if (j >= j_end || j - j_first >= a.max_new_keys) return;
+  if (j >= a.nc_cap) {
+    if (lane == 0) set_status(a.status, NOSA_DEV_NC_CAP);
+    return;
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int64_t t0 = j * kPoolStride;
+#pragma unroll 8
+  for (int t = 0; t < kPoolKernel; ++t) {
+    const int64_t tok = t0 + t;
+    uint2 raw;
+    if (append && tok == len_old) {
+      raw = knew_row[lane];
+    } else {
+      const uint2* src =
+          reinterpret_cast<const uint2*>(a.k_cache + ((base + tok) * a.hkv + h) * kHeadDim);
+      raw = __ldg(src + lane);
+    }
+    const float4 f = bf16x4_to_float4(raw);
+    acc.x += f.x;
+    acc.y += f.y;
+    acc.z += f.z;
+    acc.w += f.w;
+  }
+  constexpr float inv = 1.0f / kPoolKernel;
+  acc.x *= inv;
+  acc.y *= inv;
+  acc.z *= inv;
+  acc.w *= inv;
+  float4* dst = reinterpret_cast<float4*>(
+      a.pooled + ((static_cast<int64_t>(i) * a.hkv + h) * a.nc_cap + j) * kHeadDim);
+  dst[lane] = acc;
+}
+
+}  // namespace
+
+cudaError_t launch_pool_append(const PoolArgs& a, cudaStream_t stream) {
+  const int pairs = a.batch * a.hkv;
+  if (pairs == 0) return cudaSuccess;
+  const int chunks = (a.max_new_keys + kWarpsPerCta - 1) / kWarpsPerCta;
+  dim3 grid(chunks > 0 ? chunks : 1, pairs);
+  pool_append_kernel<<<grid, kWarpsPerCta * 32, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace nosa

@@ -1,0 +1,287 @@
+"""Thin Python binding of ``libnosa_b200.so`` (the C ABI in ``include/nosa.h``).
+
+Argument marshalling only: every function takes torch tensors, checks device,
+dtype and contiguity, passes raw pointers and the current CUDA stream to the
+C entry point of the same name, and raises :class:`NosaError` on a non-zero
+status.  All arithmetic runs in the library's CUDA kernels; there is no CPU
+path, and importing the library fails loudly when it has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnosa_b200.so")
+
+NOSA_OK = 0
+NOSA_ERR_INVALID_ARG = 1
+NOSA_ERR_UNSUPPORTED = 2
+NOSA_ERR_WORKSPACE = 3
+NOSA_ERR_CUDA = 4
+NOSA_ERR_DEVICE_CHECK = 5
+NOSA_ERR_TIMEOUT = 6
+
+NOSA_DEV_BAD_LENGTH = 0x1
+NOSA_DEV_NC_CAP = 0x2
+NOSA_DEV_BAD_INDEX = 0x4
+NOSA_DEV_BAD_COUNT = 0x8
+NOSA_DEV_MAX_NEW_KEYS = 0x10
+NOSA_DEV_APPEND_ONE = 0x20
+NOSA_DEV_MAX_LEN = 0x40
+NOSA_DEV_TIMEOUT = 0x80000000
+
+
+class NosaError(RuntimeError):
+    def __init__(self, code: int, func: str, detail: str):
+        self.code = code
+        super().__init__(f"{func}: {_status_string(code)} (code {code}): {detail}")
+
+
+class nosa_params(ctypes.Structure):
+    _fields_ = [("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("pool_kernel", ctypes.c_int),
+                ("pool_stride", ctypes.c_int), ("block_size", ctypes.c_int),
+                ("local_blocks", ctypes.c_int), ("topk", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float)]
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+_SIGNATURES = {
+    "nosa_default_params": (None, [_P]),
+    "nosa_workspace_size": (_SZ, [_P, _I, _I]),
+    "nosa_workspace_init": (_I, [_P, _SZ, _P]),
+    "nosa_pool_append": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
+    "nosa_block_select": (_I, [_P, _P, _P, _I, _P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _P, _SZ, _P]),
+    "nosa_sparse_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "nosa_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "nosa_read_device_status": (_I, [_P, _SZ, _P]),
+    "nosa_last_device_bits": (ctypes.c_uint32, []),
+    "nosa_selftest_wait_timeout": (_I, [_P, _SZ, ctypes.c_uint32, _P]),
+    "nosa_status_string": (ctypes.c_char_p, [_I]),
+    "nosa_last_error": (ctypes.c_char_p, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m long_context_decode_nosa_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _status_string(code: int) -> str:
+    try:
+        return lib().nosa_status_string(code).decode()
+    except Exception:  # noqa: BLE001 -- message formatting only
+        return "status"
+
+
+def _check(rc: int, func: str):
+    if rc != NOSA_OK:
+        raise NosaError(rc, func, lib().nosa_last_error().decode())
+
+
+def params(num_q_heads: int = 16, num_kv_heads: int = 2, *, topk: int = 64,
+           local_blocks: int = 16, softmax_scale: float = 0.0, head_dim: int = 128,
+           pool_kernel: int = 32, pool_stride: int = 16, block_size: int = 64) -> nosa_params:
+    return nosa_params(num_q_heads, num_kv_heads, head_dim, pool_kernel, pool_stride, block_size,
+                       local_blocks, topk, softmax_scale)
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor", cuda=True):
+    if t is None:
+        return None
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not cuda and t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def n_windows(L: int) -> int:
+    return (L - 32) // 16 + 1 if L >= 32 else 0
+
+
+def n_blocks(L: int) -> int:
+    return (L + 63) // 64
+
+
+def workspace_size(p: nosa_params, batch: int, max_seq_len: int) -> int:
+    n = lib().nosa_workspace_size(ctypes.byref(p), batch, max_seq_len)
+    if n == 0:
+        raise NosaError(NOSA_ERR_INVALID_ARG, "nosa_workspace_size", "invalid parameters")
+    return n
+
+
+def nosa_workspace_init(ws: torch.Tensor, stream=None):
+    _check(lib().nosa_workspace_init(_ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)),
+           "nosa_workspace_init")
+
+
+def workspace(p: nosa_params, batch: int, max_seq_len: int, device="cuda", stream=None) -> torch.Tensor:
+    """A zero-initialised workspace tensor (uint8) for these shapes."""
+    n = workspace_size(p, batch, max_seq_len)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    nosa_workspace_init(ws, stream)
+    return ws
+
+
+def nosa_pool_append(p: nosa_params, k_cache: torch.Tensor, v_cache: Optional[torch.Tensor],
+                     seq_start: torch.Tensor, len_new: torch.Tensor, pooled: torch.Tensor, *,
+                     len_old: Optional[torch.Tensor] = None, max_new_keys: int = 1,
+                     k_new: Optional[torch.Tensor] = None, v_new: Optional[torch.Tensor] = None,
+                     ws: Optional[torch.Tensor] = None, stream=None):
+    batch = len_new.shape[0]
+    rc = lib().nosa_pool_append(
+        ctypes.byref(p), _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
+        _ptr(seq_start, torch.int64, "seq_start"), _ptr(len_old, torch.int32, "len_old"),
+        _ptr(len_new, torch.int32, "len_new"), batch, _ptr(pooled, torch.float32, "pooled"),
+        pooled.shape[2], max_new_keys, _ptr(k_new, torch.bfloat16, "k_new"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(ws, torch.uint8, "ws"),
+        0 if ws is None else ws.numel(), _stream(stream))
+    _check(rc, "nosa_pool_append")
+
+
+def nosa_block_select(p: nosa_params, q: Optional[torch.Tensor], pooled: Optional[torch.Tensor],
+                      seq_len: torch.Tensor, max_seq_len: int, sel_idx: torch.Tensor,
+                      sel_cnt: torch.Tensor, ws: torch.Tensor, *,
+                      block_scores_in: Optional[torch.Tensor] = None,
+                      comp_scores_out: Optional[torch.Tensor] = None,
+                      block_scores_out: Optional[torch.Tensor] = None, stream=None):
+    batch = seq_len.shape[0]
+    nc_cap = pooled.shape[2] if pooled is not None else (comp_scores_out.shape[2] if comp_scores_out is not None else 0)
+    rc = lib().nosa_block_select(
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(pooled, torch.float32, "pooled"), nc_cap,
+        _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len,
+        _ptr(block_scores_in, torch.float32, "block_scores_in"),
+        0 if block_scores_in is None else block_scores_in.shape[2],
+        _ptr(comp_scores_out, torch.float32, "comp_scores_out"),
+        _ptr(block_scores_out, torch.float32, "block_scores_out"),
+        0 if block_scores_out is None else block_scores_out.shape[2],
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(rc, "nosa_block_select")
+
+
+def nosa_sparse_decode(p: nosa_params, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                       seq_start: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int,
+                       sel_idx: torch.Tensor, sel_cnt: torch.Tensor, out: torch.Tensor,
+                       ws: torch.Tensor, *, lse: Optional[torch.Tensor] = None, stream=None):
+    if sel_idx.shape[-1] != p.topk:
+        raise ValueError("sel_idx's last dimension must equal params.topk")
+    batch = seq_len.shape[0]
+    rc = lib().nosa_sparse_decode(
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), _ptr(seq_start, torch.int64, "seq_start"),
+        _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len,
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
+        _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(rc, "nosa_sparse_decode")
+
+
+def nosa_decode_step(p: nosa_params, q_host: torch.Tensor, k_new_host: torch.Tensor,
+                     v_new_host: torch.Tensor, out_host: torch.Tensor, k_cache: torch.Tensor,
+                     v_cache: torch.Tensor, seq_start: torch.Tensor, seq_len: torch.Tensor,
+                     max_seq_len: int, pooled: torch.Tensor, sel_idx: torch.Tensor,
+                     sel_cnt: torch.Tensor, ws: torch.Tensor, stream=None):
+    """Whole decode step from host buffers (pinned for asynchronous copies);
+    out_host is valid once the stream has synchronised."""
+    batch = seq_len.shape[0]
+    rc = lib().nosa_decode_step(
+        ctypes.byref(p), _ptr(q_host, torch.bfloat16, "q_host", cuda=False),
+        _ptr(k_new_host, torch.bfloat16, "k_new_host", cuda=False),
+        _ptr(v_new_host, torch.bfloat16, "v_new_host", cuda=False),
+        _ptr(out_host, torch.bfloat16, "out_host", cuda=False),
+        _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
+        _ptr(seq_start, torch.int64, "seq_start"), _ptr(seq_len, torch.int32, "seq_len"), batch,
+        max_seq_len, _ptr(pooled, torch.float32, "pooled"), pooled.shape[2],
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(rc, "nosa_decode_step")
+
+
+def nosa_read_device_status(ws: torch.Tensor, stream=None):
+    """(status code, raw device bits); synchronises the stream and clears the word."""
+    rc = lib().nosa_read_device_status(_ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    return rc, int(lib().nosa_last_device_bits())
+
+
+def nosa_selftest_wait_timeout(ws: torch.Tensor, max_iters: int = 1000, stream=None):
+    _check(lib().nosa_selftest_wait_timeout(_ptr(ws, torch.uint8, "ws"), ws.numel(), max_iters,
+                                            _stream(stream)), "nosa_selftest_wait_timeout")
+
+
+class DecodeState:
+    """Device buffers for repeated decode steps of one layer: pooled keys,
+    selection, output and workspace, sized for ``batch`` sequences of at most
+    ``max_seq_len`` tokens.  A convenience over the C entry points."""
+
+    def __init__(self, p: nosa_params, batch: int, max_seq_len: int, device="cuda"):
+        self.p = p
+        self.batch = batch
+        self.max_seq_len = max_seq_len
+        self.nc_cap = max(1, n_windows(max_seq_len))
+        self.pooled = torch.zeros(batch, p.num_kv_heads, self.nc_cap, 128, dtype=torch.float32, device=device)
+        self.sel_idx = torch.full((batch, p.num_kv_heads, p.topk), -1, dtype=torch.int32, device=device)
+        self.sel_cnt = torch.zeros(batch, p.num_kv_heads, dtype=torch.int32, device=device)
+        self.out = torch.empty(batch, p.num_q_heads, 128, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(batch, p.num_q_heads, dtype=torch.float32, device=device)
+        self.ws = workspace(p, batch, max_seq_len, device)
+
+    def rebuild_pooled(self, k_cache, seq_start, seq_len, stream=None):
+        """Pool every complete window of [0, seq_len) (the resume path)."""
+        nosa_pool_append(self.p, k_cache, None, seq_start, seq_len, self.pooled,
+                         len_old=torch.zeros_like(seq_len), max_new_keys=self.nc_cap, ws=self.ws,
+                         stream=stream)
+
+    def step(self, q, k_cache, v_cache, seq_start, seq_len, *, append=True, stream=None,
+             with_lse=False):
+        """One decode step on device-resident inputs: pool the window the newest
+        token completes (when ``append``), select, attend.  Returns ``out``."""
+        if append:
+            nosa_pool_append(self.p, k_cache, v_cache, seq_start, seq_len, self.pooled,
+                             max_new_keys=1, ws=self.ws, stream=stream)
+        nosa_block_select(self.p, q, self.pooled, seq_len, self.max_seq_len, self.sel_idx,
+                          self.sel_cnt, self.ws, stream=stream)
+        nosa_sparse_decode(self.p, q, k_cache, v_cache, seq_start, seq_len, self.max_seq_len,
+                           self.sel_idx, self.sel_cnt, self.out, self.ws,
+                           lse=self.lse if with_lse else None, stream=stream)
+        return self.out
+
+
+def default_scale(head_dim: int = 128) -> float:
+    return 1.0 / math.sqrt(head_dim)

@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports every entry point include/nosa.h declares,
+and rejects bad host-visible arguments before touching the GPU (CPU only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nosa.h")
+
+
+@pytest.fixture(scope="module")
+def nosa():
+    from long_context_decode_nosa_b200 import build
+    build.build()
+    from long_context_decode_nosa_b200 import nosa as m
+    m.lib()
+    return m
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"NOSA_API\s+[\w\s\*]*?\b(nosa_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_path():
+    names = _declared()
+    for need in ("nosa_pool_append", "nosa_block_select", "nosa_sparse_decode",
+                 "nosa_workspace_size", "nosa_read_device_status", "nosa_status_string"):
+        assert need in names
+
+
+def test_library_exports_every_declared_symbol(nosa):
+    lib_path = nosa.LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", lib_path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (nosa_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    for n in _declared():
+        getattr(nosa.lib(), n)  # resolvable through ctypes too
+
+
+def test_status_strings(nosa):
+    for code in range(7):
+        assert nosa.lib().nosa_status_string(code).decode()
+    assert nosa.lib().nosa_status_string(99).decode() == "unknown status"
+
+
+def test_workspace_size_host_only(nosa):
+    p = nosa.params(16, 2, topk=64)
+    n8 = nosa.workspace_size(p, 8, 16384)
+    n16 = nosa.workspace_size(p, 16, 16384)
+    assert n8 > 0 and n16 > n8 and n8 % 256 == 0
+    bad = nosa.params(16, 3)
+    assert nosa.lib().nosa_workspace_size(ctypes.byref(bad), 8, 16384) == 0
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 64, 2), ("pool_kernel", 16, 2), ("block_size", 128, 2), ("topk", 0, 2),
+    ("num_kv_heads", 3, 1), ("local_blocks", -1, 1), ("softmax_scale", -1.0, 1),
+])
+def test_bad_params_rejected_before_any_launch(nosa, field, value, code):
+    p = nosa.params(16, 2)
+    setattr(p, field, value)
+    rc = nosa.lib().nosa_sparse_decode(ctypes.byref(p), None, None, None, None, None, 1, 16, None,
+                                       None, None, None, None, 0, None)
+    assert rc == code
+    assert nosa.lib().nosa_last_error().decode()
+
+
+def test_null_and_workspace_checks(nosa):
+    p = nosa.params(16, 2)
+    L = nosa.lib()
+    # workspace missing
+    rc = L.nosa_block_select(ctypes.byref(p), None, None, 1, None, 4, 1024, None, 0, None, None, 0,
+                             None, None, None, 0, None)
+    assert rc == nosa.NOSA_ERR_WORKSPACE
+    # workspace too small (a host buffer stands in: the check fails before any use)
+    buf = ctypes.create_string_buffer(1024 + 256)
+    addr = (ctypes.addressof(buf) + 255) // 256 * 256
+    rc = L.nosa_sparse_decode(ctypes.byref(p), None, None, None, None, None, 4, 1024, None, None,
+                              None, None, ctypes.c_void_p(addr), 1024, None)
+    assert rc == nosa.NOSA_ERR_WORKSPACE
+    # batch 0 is a no-op
+    assert L.nosa_pool_append(ctypes.byref(p), None, None, None, None, None, 0, None, 1, 1, None,
+                              None, None, 0, None) == 0
+    # k_new without v_new
+    rc = L.nosa_pool_append(ctypes.byref(p), ctypes.c_void_p(256), None, ctypes.c_void_p(256), None,
+                            ctypes.c_void_p(256), 1, ctypes.c_void_p(256), 1, 1,
+                            ctypes.c_void_p(256), None, None, 0, None)
+    assert rc == nosa.NOSA_ERR_INVALID_ARG
