@@ -1,0 +1,509 @@
+#!/usr/bin/env python3
+"""Benchmark of NOSA sparse decode attention on B200 (one JSON line on rank 0).
+
+A *step* is one whole decode step of one layer over the batch: append the new
+token's K/V rows and pool the window it completes (nosa_pool_append), score
+the compressed keys and select the top-k blocks (nosa_block_select), attend
+over the selected blocks plus the local window (nosa_sparse_decode).  One
+*query* is one sequence's decode token through one layer's attention.
+
+Default workload (the NOSA-1B attention shape, 16 q / 2 KV heads, head_dim
+128): batch 8, context 16384, top-k 64 blocks of 64 + 16 local blocks,
+bf16 N(0,1) KV cache.  Inputs stay resident in HBM; to keep the 126 MB L2
+from serving them, steps rotate over R independent replicas of the caches
+(R x 142 MB).  The timed steps run as one CUDA graph, bracketed by events on
+the launching stream; events inside the graph give each kernel's duration.
+
+Also reported: ``e2e`` (the same metric through nosa_decode_step with pinned
+host buffers, H2D/D2H copies inside the timed region), ``roofline`` of the
+dominant kernel against the measured HBM copy bandwidth, the CPU oracle timed
+on the host cores (``cpu_baseline``), and SM clocks sampled during the run.
+
+``--impl reference`` times the CPU oracle on the same workload instead.
+Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no
+collective on the data path); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from long_context_decode_nosa_b200 import inputs  # noqa: E402
+
+METRIC = "sparse decode-attn queries/s and achieved HBM GB/s vs ~8 TB/s, 16K–64K ctx"
+UNIT = "queries/s"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOADS = {
+    # name: (description, batch, lengths spec, Hq, Hkv, topk, layers, key dist)
+    "nosa1b_b8_16k": ("NOSA-1B attention (16 q / 2 KV heads, d128), batch 8, context 16384, "
+                      "top-k 64 blocks + 16 local blocks, bf16 N(0,1) KV",
+                      8, 16384, 16, 2, 64, 1, "normal"),
+    "nosa1b_b32_ragged_28l": ("NOSA-1B attention, batch 32, ragged context U[16384, 32768], "
+                              "top-k 64 + 16 local, 28 independent layers per step",
+                              32, "ragged", 16, 2, 64, 28, "normal"),
+    "llama8b_b4_64k": ("8B-class attention (32 q / 8 KV heads, d128), batch 4, context 65536, "
+                       "top-k 64 + 16 local, Student-t(4) keys",
+                       4, 65536, 32, 8, 64, 1, "student_t"),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="nosa1b_b8_16k")
+    ap.add_argument("--context", type=int, default=0, help="override the context length")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch size")
+    ap.add_argument("--topk", type=int, default=0, help="override top-k blocks")
+    ap.add_argument("--replicas", type=int, default=0, help="cache replicas rotated (0: auto)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline time budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--settle-ms", type=float, default=300.0,
+                    help="untimed repeated steps before timing, so clocks settle")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- workload
+
+def _n_windows(L: int) -> int:
+    return (L - 32) // 16 + 1 if L >= 32 else 0
+
+
+class Workload:
+    def __init__(self, args, seed_base: int):
+        desc, batch, lens, hq, hkv, topk, layers, kdist = WORKLOADS[args.workload]
+        self.name = args.workload
+        self.batch = args.batch or batch
+        if args.context:
+            lens = args.context
+        if lens == "ragged":
+            self.lens = inputs.ragged_lengths(self.batch, 16384, 32768, seed=seed_base + 3)
+        else:
+            self.lens = [int(lens)] * self.batch
+        self.hq, self.hkv = hq, hkv
+        self.topk = args.topk or topk
+        self.layers = layers
+        self.key_dist = kdist
+        self.local_blocks = 16
+        self.desc = desc
+        if args.context or args.batch or args.topk:
+            self.desc += f" [overridden: batch {self.batch}, context {max(self.lens)}, top-k {self.topk}]"
+        self.max_len = max(self.lens)
+
+    # Algorithmic bytes per kernel for one layer-step (see the byte model in the design notes).
+    def bytes_model(self):
+        G = self.hq // self.hkv
+        pool = select = decode = 0
+        for L in self.lens:
+            nb = -(-L // 64)
+            ncand = max(0, nb - self.local_blocks)
+            nc = _n_windows(L)
+            k_eff = min(self.topk, ncand)
+            windows = min(nc, 4 * ncand)
+            attended = k_eff * 64 + (L - 64 * ncand)
+            new_window = _n_windows(L) - _n_windows(L - 1)
+            for _ in range(self.hkv):
+                pool += 2 * 256 * 2 + new_window * (31 * 256 + 512)   # new K/V row in + out, window
+                select += windows * 512 + G * 256 + self.topk * 4 + 4
+                decode += attended * 512 + 2 * G * 256 + self.topk * 4 + 4
+        return {"pool_append": pool * self.layers, "block_select": select * self.layers,
+                "sparse_decode": decode * self.layers}
+
+
+class Replica:
+    """One layer's device state: caches, pooled keys, selection, output."""
+
+    def __init__(self, nosa, wl: Workload, seed: int, device):
+        self.b = inputs.make_batch(wl.lens, num_q_heads=wl.hq, num_kv_heads=wl.hkv, seed=seed,
+                                   key_dist=wl.key_dist, device=device)
+        self.p = nosa.params(wl.hq, wl.hkv, topk=wl.topk, local_blocks=wl.local_blocks)
+        self.st = nosa.DecodeState(self.p, wl.batch, wl.max_len, device=device)
+        self.st.rebuild_pooled(self.b.k_cache, self.b.seq_start, self.b.seq_len)
+        self.k_new, self.v_new = inputs.random_kv_rows(wl.batch, wl.hkv, 128, seed=seed + 7,
+                                                       device=device)
+
+
+def step(nosa, r: Replica, events=None):
+    """One decode step on device-resident inputs.  events: 4 CUDA events
+    recorded before K1, before K2, before K3 and after K3 (or None)."""
+    b, st, p = r.b, r.st, r.p
+    if events:
+        events[0].record()
+    nosa.nosa_pool_append(p, b.k_cache, b.v_cache, b.seq_start, b.seq_len, st.pooled, max_new_keys=1,
+                          k_new=r.k_new, v_new=r.v_new, ws=st.ws)
+    if events:
+        events[1].record()
+    nosa.nosa_block_select(p, b.q, st.pooled, b.seq_len, st.max_seq_len, st.sel_idx, st.sel_cnt,
+                           st.ws)
+    if events:
+        events[2].record()
+    nosa.nosa_sparse_decode(p, b.q, b.k_cache, b.v_cache, b.seq_start, b.seq_len, st.max_seq_len,
+                            st.sel_idx, st.sel_cnt, st.out, st.ws)
+    if events:
+        events[3].record()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [ln.split(",") for ln in out.strip().splitlines() if ln.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "long_context_decode_nosa_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """Per-launch DRAM bytes of the sparse-decode kernel from the committed ncu
+    summary (profiles/), if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"sparse_decode_{workload}.md")
+    try:
+        with open(path) as f:
+            txt = f.read()
+    except OSError:
+        return None
+    src = traffic = None
+    for ln in txt.splitlines():
+        if ln.startswith("kernel_source_sha256_16:"):
+            src = ln.split(":", 1)[1].strip()
+        if ln.startswith("dram_bytes_per_launch:"):
+            try:
+                traffic = float(ln.split(":", 1)[1].strip())
+            except ValueError:
+                traffic = None
+    return traffic if src == kernel_source_hash() else None
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_steps(wl: Workload, b_host, n_steps: int, threads: int, budget_s: float):
+    """Time whole oracle decode steps (pool the new window, score, select,
+    attend) on host copies of one layer's inputs; stops after n_steps or the
+    time budget.  Returns (steps done, seconds)."""
+    import oracle
+    oracle.set_threads(threads)
+    kb = inputs.bf16_bits(b_host.k_cache)
+    vb = inputs.bf16_bits(b_host.v_cache)
+    qb = inputs.bf16_bits(b_host.q)
+    lens = b_host.seq_len.numpy()
+    starts = b_host.seq_start.numpy()
+    nc_cap = max(1, oracle.n_windows(int(lens.max())))
+    pooled = oracle.pool(kb, starts, lens - 1, nc_cap)          # state before the step (untimed)
+    done, t0 = 0, time.perf_counter()
+    while done < n_steps:
+        pooled = oracle.pool(kb, starts, lens, nc_cap, len_old=lens - 1, pooled=pooled)
+        oracle.decode_step(qb, kb, vb, starts, lens, pooled, wl.topk, local_blocks=wl.local_blocks)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    return done, time.perf_counter() - t0
+
+
+def host_batch(wl: Workload, seed: int):
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    return inputs.make_batch(wl.lens, num_q_heads=wl.hq, num_kv_heads=wl.hkv, seed=seed,
+                             key_dist=wl.key_dist, device=dev).to("cpu")
+
+
+def run_reference(args):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return 0
+    wl = Workload(args, 0)
+    b = host_batch(wl, seed=100)
+    threads = os.cpu_count() or 1
+    oracle_steps(wl, b, max(1, min(args.warmup, 1)), threads, 1e9)       # warm caches
+    per_layer_steps, secs = oracle_steps(wl, b, args.steps, threads, 1e9)
+    # one step = all layers of the workload; the oracle runs one layer and scales
+    ms = secs / per_layer_steps * wl.layers * 1e3
+    value = wl.batch * wl.layers / (ms / 1e3)
+    sample = (f"{per_layer_steps} full one-layer steps of the workload on the oracle"
+              + (f", scaled x{wl.layers} layers" if wl.layers > 1 else ""))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.desc, "batch": wl.batch, "seq_len": wl.max_len, "topk": wl.topk,
+                       "layers": wl.layers},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- ours
+
+def run_ours(args):
+    world, rank, local = dist_setup(args)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    from long_context_decode_nosa_b200 import nosa
+    nosa.lib()
+    wl = Workload(args, 0)
+    seed0 = 1000 * (rank + 1)
+
+    # Replicas so that no step finds its inputs in L2 (126 MB).
+    layer_bytes = sum(wl.lens) * wl.hkv * 128 * 2 * 2
+    if wl.layers > 1:
+        R = 1
+        layers = [Replica(nosa, wl, seed0 + 10 * l, device) for l in range(wl.layers)]
+        rotation = [layers]
+    else:
+        R = args.replicas or max(2, min(16, math.ceil(1.0e9 / max(layer_bytes, 1))))
+        rotation = [[Replica(nosa, wl, seed0 + 10 * r, device)] for r in range(R)]
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream())
+
+    def record_steps(n, with_events):
+        evs = []
+        for s in range(n):
+            for layer in rotation[s % len(rotation)]:
+                e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] if with_events else None
+                step(nosa, layer, e)
+                if e:
+                    evs.append(e)
+        return evs
+
+    with torch.cuda.stream(stream):
+        record_steps(len(rotation), False)         # eager warm-up: sets kernel attributes
+    stream.synchronize()
+
+    g_warm = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm, stream=stream):
+        record_steps(max(args.warmup, 1), False)
+    g_timed = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_timed, stream=stream):
+        inner = record_steps(args.steps, True)
+
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    with torch.cuda.stream(stream):
+        g_warm.replay()
+        t_settle = time.perf_counter()
+        while (time.perf_counter() - t_settle) * 1e3 < args.settle_ms:
+            g_warm.replay()
+            stream.synchronize()
+        barrier(world)
+        stream.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        stop = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        g_timed.replay()
+        stop.record(stream)
+    stream.synchronize()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(start.elapsed_time(stop), world)
+    ms_step = ms_total / args.steps
+    n_layers_launches = len(inner)
+    kt = {"pool_append": [], "block_select": [], "sparse_decode": []}
+    for e in inner:
+        kt["pool_append"].append(e[0].elapsed_time(e[1]))
+        kt["block_select"].append(e[1].elapsed_time(e[2]))
+        kt["sparse_decode"].append(e[2].elapsed_time(e[3]))
+    kmean_us = {k: 1e3 * statistics.fmean(v) for k, v in kt.items()}
+
+    queries_per_step = wl.batch * wl.layers
+    value = world * queries_per_step * args.steps / (ms_total / 1e3)
+    model = wl.bytes_model()
+    step_bytes = sum(model.values())
+    peak, peak_kind = peak_hbm()
+    dec_bytes_launch = model["sparse_decode"] / wl.layers
+    dec_achieved = dec_bytes_launch / (kmean_us["sparse_decode"] * 1e-6) / 1e9
+    traffic = ncu_traffic(wl.name) if wl.name == args.workload and not (args.context or args.batch or args.topk) else None
+
+    # e2e through the host-buffer entry point, one layer (replica 0), pinned buffers.
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(nosa, wl, rotation[0][0], args, stream, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        b_host = inputs.DecodeBatch(rotation[0][0].b.q.cpu(), rotation[0][0].b.k_cache.cpu(),
+                                    rotation[0][0].b.v_cache.cpu(), rotation[0][0].b.seq_start.cpu(),
+                                    rotation[0][0].b.seq_len.cpu(), rotation[0][0].b.capacity.cpu(),
+                                    wl.hq, wl.hkv, 128)
+        threads = os.cpu_count() or 1
+        n, secs = oracle_steps(wl, b_host, 10 ** 6, threads, args.cpu_seconds)
+        cpu_ms = secs / n * wl.layers * 1e3
+        cpu = {"value": queries_per_step / (cpu_ms / 1e3), "unit": UNIT, "cores": threads,
+               "kind": "oracle",
+               "sample": f"{n} one-layer decode steps of this workload (all {wl.batch} sequences) on the "
+                         f"fp64 C oracle in {secs:.1f} s" + (f", scaled x{wl.layers} layers" if wl.layers > 1 else "")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.desc, "batch": wl.batch, "seq_len": wl.max_len,
+                       "topk": wl.topk, "local_blocks": wl.local_blocks, "layers": wl.layers,
+                       "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                       "l2": (f"inputs rotate over {R} cache replicas "
+                              f"({R * layer_bytes * wl.layers / 1e9:.2f} GB) > 126 MB L2"),
+                       "clock_settle_ms": args.settle_ms, "graph": "timed steps replayed as one CUDA graph"},
+            "gpu_launches": 3 * n_layers_launches,
+            "hbm_gbs_step": step_bytes / (ms_step * 1e-3) / 1e9,
+            "algorithmic_bytes_per_step": step_bytes,
+            "kernel_us": kmean_us,
+            "roofline": {"bound": "hbm", "kernel": "sparse_decode", "achieved": dec_achieved,
+                         "peak": peak, "unit": "GB/s", "frac": dec_achieved / peak,
+                         "peak_kind": f"{peak_kind} copy bandwidth", "traffic": traffic,
+                         "algorithmic_bytes_per_launch": dec_bytes_launch},
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del g_timed, g_warm
+        dist.destroy_process_group()
+    return 0
+
+
+def measure_e2e(nosa, wl: Workload, r: Replica, args, stream, world):
+    """Same metric through nosa_decode_step with pinned host buffers: every
+    step copies q and the new K/V rows in and the output back."""
+    if wl.layers > 1:
+        return None
+    b, st, p = r.b, r.st, r.p
+    q_h = b.q.cpu().pin_memory()
+    k_h = r.k_new.cpu().pin_memory()
+    v_h = r.v_new.cpu().pin_memory()
+    o_h = torch.empty(wl.batch, wl.hq, 128, dtype=torch.bfloat16).pin_memory()
+    n = max(10, min(args.steps, 500))
+
+    def call():
+        nosa.nosa_decode_step(p, q_h, k_h, v_h, o_h, b.k_cache, b.v_cache, b.seq_start, b.seq_len,
+                              st.max_seq_len, st.pooled, st.sel_idx, st.sel_cnt, st.ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, min(args.warmup, 50))):
+            call()
+        stream.synchronize()
+        barrier(world)
+        start = torch.cuda.Event(enable_timing=True)
+        stop = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(n):
+            call()
+        stop.record(stream)
+    stream.synchronize()
+    ms = max_over_ranks(start.elapsed_time(stop), world)
+    return {"value": world * wl.batch * n / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2,
+            "d2h_bytes_per_step": o_h.numel() * 2, "steps": n, "ms_per_step": ms / n}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200); the CUDA path has no CPU fallback")
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
