@@ -41,7 +41,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from long_context_decode_nosa_b200 import inputs  # noqa: E402
+from long_context_decode_nosa_b200 import inputs, multirank  # noqa: E402
 
 METRIC = "sparse decode-attn queries/s and achieved HBM GB/s vs ~8 TB/s, 16K–64K ctx"
 UNIT = "queries/s"
@@ -247,32 +247,9 @@ def ncu_traffic(workload: str):
 
 
 def dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-
-
-def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    info = multirank.rank_info()
+    multirank.init(info, backend="nccl", timeout_s=120)
+    return info
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -335,13 +312,14 @@ def run_reference(args):
 # ----------------------------------------------------------------------------- ours
 
 def run_ours(args):
-    world, rank, local = dist_setup(args)
+    info = dist_setup(args)
+    world, rank, local = info.world, info.rank, info.local_rank
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     from long_context_decode_nosa_b200 import nosa
     nosa.lib()
     wl = Workload(args, 0)
-    seed0 = 1000 * (rank + 1)
+    seed0 = multirank.rank_seed(0, info)
 
     # Replicas so that no step finds its inputs in L2 (126 MB).
     layer_bytes = sum(wl.lens) * wl.hkv * 128 * 2 * 2
@@ -386,7 +364,7 @@ def run_ours(args):
         while (time.perf_counter() - t_settle) * 1e3 < args.settle_ms:
             g_warm.replay()
             stream.synchronize()
-        barrier(world)
+        multirank.barrier(info)
         stream.synchronize()
         start = torch.cuda.Event(enable_timing=True)
         stop = torch.cuda.Event(enable_timing=True)
@@ -395,7 +373,7 @@ def run_ours(args):
         stop.record(stream)
     stream.synchronize()
     clk = clocks.stop()
-    ms_total = max_over_ranks(start.elapsed_time(stop), world)
+    ms_total = multirank.max_over_ranks(start.elapsed_time(stop), info, device)
     ms_step = ms_total / args.steps
     n_layers_launches = len(inner)
     kt = {"pool_append": [], "block_select": [], "sparse_decode": []}
@@ -406,7 +384,7 @@ def run_ours(args):
     kmean_us = {k: 1e3 * statistics.fmean(v) for k, v in kt.items()}
 
     queries_per_step = wl.batch * wl.layers
-    value = world * queries_per_step * args.steps / (ms_total / 1e3)
+    value = multirank.aggregate_rate(queries_per_step * args.steps, info, ms_total / 1e3)
     model = wl.bytes_model()
     step_bytes = sum(model.values())
     peak, peak_kind = peak_hbm()
@@ -417,7 +395,7 @@ def run_ours(args):
     # e2e through the host-buffer entry point, one layer (replica 0), pinned buffers.
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(nosa, wl, rotation[0][0], args, stream, world)
+        e2e = measure_e2e(nosa, wl, rotation[0][0], args, stream, info, device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -455,14 +433,12 @@ def run_ours(args):
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        del g_timed, g_warm
-        dist.destroy_process_group()
+    del g_timed, g_warm
+    multirank.shutdown(info)
     return 0
 
 
-def measure_e2e(nosa, wl: Workload, r: Replica, args, stream, world):
+def measure_e2e(nosa, wl: Workload, r: Replica, args, stream, info, device):
     """Same metric through nosa_decode_step with pinned host buffers: every
     step copies q and the new K/V rows in and the output back."""
     if wl.layers > 1:
@@ -482,7 +458,7 @@ def measure_e2e(nosa, wl: Workload, r: Replica, args, stream, world):
         for _ in range(max(3, min(args.warmup, 50))):
             call()
         stream.synchronize()
-        barrier(world)
+        multirank.barrier(info)
         start = torch.cuda.Event(enable_timing=True)
         stop = torch.cuda.Event(enable_timing=True)
         start.record(stream)
@@ -490,8 +466,8 @@ def measure_e2e(nosa, wl: Workload, r: Replica, args, stream, world):
             call()
         stop.record(stream)
     stream.synchronize()
-    ms = max_over_ranks(start.elapsed_time(stop), world)
-    return {"value": world * wl.batch * n / (ms / 1e3), "unit": UNIT,
+    ms = multirank.max_over_ranks(start.elapsed_time(stop), info, device)
+    return {"value": multirank.aggregate_rate(wl.batch * n, info, ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2,
             "d2h_bytes_per_step": o_h.numel() * 2, "steps": n, "ms_per_step": ms / n}
 

@@ -31,9 +31,10 @@
  *    except nosa_read_device_status.
  *  * Layouts (row-major, innermost last):
  *      q            bf16 [batch, num_q_heads, head_dim]
- *      k_cache/v_cache bf16 [T, num_kv_heads, head_dim]; sequence i occupies
- *                   rows seq_start[i] .. seq_start[i] + len - 1 (varlen
- *                   packing as with cu_seqlens: seq_start[i] = cu_seqlens[i]).
+ *      k_cache/v_cache bf16 [cache_rows, num_kv_heads, head_dim], cache_rows
+ *                   < 2^31; sequence i occupies rows seq_start[i] ..
+ *                   seq_start[i] + len - 1 (varlen packing as with
+ *                   cu_seqlens: seq_start[i] = cu_seqlens[i]).
  *      pooled       fp32 [batch, num_kv_heads, nc_cap, head_dim]
  *      sel_idx      int32 [batch, num_kv_heads, topk] (ascending, -1 padded)
  *      sel_cnt      int32 [batch, num_kv_heads]
@@ -92,6 +93,7 @@ typedef enum {
 #define NOSA_DEV_MAX_NEW_KEYS 0x10u  /* more new windows than max_new_keys */
 #define NOSA_DEV_APPEND_ONE 0x20u    /* k_new given but len_new != len_old + 1 */
 #define NOSA_DEV_MAX_LEN 0x40u       /* seq_len above the call's max_seq_len */
+#define NOSA_DEV_CACHE_ROWS 0x80u    /* a sequence's rows reach past cache_rows */
 #define NOSA_DEV_TIMEOUT 0x80000000u /* an mbarrier wait hit its iteration limit */
 
 typedef struct {
@@ -101,7 +103,7 @@ typedef struct {
   int pool_kernel;     /* must be 32 */
   int pool_stride;     /* must be 16 */
   int block_size;      /* must be 64 */
-  int local_blocks;    /* forced local window in blocks (16 = 1024 tokens); >= 0 */
+  int local_blocks;    /* forced local window in blocks (16 = 1024 tokens); 0..256 */
   int topk;            /* selected blocks per (sequence, KV head); 1..1024 */
   float softmax_scale; /* 0 => 1/sqrt(head_dim); used for scores and attention */
 } nosa_params;
@@ -137,7 +139,7 @@ NOSA_API int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * Does not use the workspace's counters; `ws` may be NULL (then device data
  * errors are not reported). */
 NOSA_API int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache,
-                     const int64_t* seq_start, const int32_t* len_old,
+                     int64_t cache_rows, const int64_t* seq_start, const int32_t* len_old,
                      const int32_t* len_new, int batch, float* pooled,
                      int nc_cap, int max_new_keys, const void* k_new,
                      const void* v_new, void* ws, size_t ws_bytes, void* stream);
@@ -174,7 +176,7 @@ NOSA_API int nosa_block_select(const nosa_params* p, const void* q, const float*
  * reproducible run to run).  Selected indices must be distinct; the order of
  * sel_idx does not matter.  lse (fp32 [batch, Hq]) is nullable. */
 NOSA_API int nosa_sparse_decode(const nosa_params* p, const void* q, const void* k_cache,
-                       const void* v_cache, const int64_t* seq_start,
+                       const void* v_cache, int64_t cache_rows, const int64_t* seq_start,
                        const int32_t* seq_len, int batch, int max_seq_len,
                        const int32_t* sel_idx, const int32_t* sel_cnt,
                        void* out, float* lse, void* ws, size_t ws_bytes,
@@ -194,7 +196,7 @@ NOSA_API int nosa_sparse_decode(const nosa_params* p, const void* q, const void*
 NOSA_API int nosa_decode_step(const nosa_params* p, const void* q_host,
                      const void* k_new_host, const void* v_new_host,
                      void* out_host, void* k_cache, void* v_cache,
-                     const int64_t* seq_start, const int32_t* seq_len,
+                     int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len,
                      int batch, int max_seq_len, float* pooled, int nc_cap,
                      int32_t* sel_idx, int32_t* sel_cnt, void* ws,
                      size_t ws_bytes, void* stream);

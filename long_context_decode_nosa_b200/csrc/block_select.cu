@@ -200,6 +200,12 @@ __global__ void __launch_bounds__(kSelThreads) select_score_kernel(const SelectA
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int pair = blockIdx.y;
   const int i = pair / a.hkv, g = pair % a.hkv;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  grid_dependency_wait();
+  allow_dependents();
   const int L = a.seq_len[i];
   if (L < 1 || L > a.max_seq_len) {
     if (blockIdx.x == 0) {
@@ -225,11 +231,7 @@ __global__ void __launch_bounds__(kSelThreads) select_score_kernel(const SelectA
   const int nwin = jhi - jlo;
 
   if (b1 > b0 && nwin > 0) {
-    if (tid == 0) {
-      mbar_init(&bar, 1);
-      fence_barrier_init();
-    }
-    __syncthreads();
+    __syncthreads();  // barrier initialisation visible to every thread
     if (tid == 0) {
       const uint32_t bytes = static_cast<uint32_t>(nwin) * kKeyBytes;
       mbar_arrive_expect_tx(&bar, bytes);
@@ -312,6 +314,8 @@ __global__ void __launch_bounds__(kSelThreads) select_only_kernel(const SelectAr
   __shared__ TopkShared sh;
   const int pair = blockIdx.y;
   const int i = pair / a.hkv;
+  grid_dependency_wait();
+  allow_dependents();
   const int L = a.seq_len[i];
   if (L < 1 || L > a.max_seq_len) {
     if (threadIdx.x == 0) set_status(a.status, L < 1 ? NOSA_DEV_BAD_LENGTH : NOSA_DEV_MAX_LEN);
@@ -335,8 +339,7 @@ cudaError_t launch_scoring(const SelectArgs& a, cudaStream_t stream) {
   const int nbw = a.comp_out ? nb_max : static_cast<int>(n_candidates(a.max_seq_len, a.local_blocks));
   const int chunks = nbw > 0 ? (nbw + kChunkBlocks - 1) / kChunkBlocks : 1;
   dim3 grid(chunks, a.batch * a.hkv);
-  select_score_kernel<G><<<grid, kSelThreads, smem, stream>>>(a, region);
-  return cudaGetLastError();
+  return launch_overlapped(select_score_kernel<G>, grid, dim3(kSelThreads), smem, stream, a, region);
 }
 
 }  // namespace
@@ -348,8 +351,7 @@ cudaError_t launch_block_select(const SelectArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(select_only_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    select_only_kernel<<<dim3(1, a.batch * a.hkv), kSelThreads, smem, stream>>>(a);
-    return cudaGetLastError();
+    return launch_overlapped(select_only_kernel, dim3(1, a.batch * a.hkv), dim3(kSelThreads), smem, stream, a);
   }
   switch (a.group) {
     case 1: return launch_scoring<1>(a, stream);

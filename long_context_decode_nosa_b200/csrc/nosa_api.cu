@@ -6,6 +6,8 @@
 #include <cstring>
 #include <string>
 
+#include <cudaTypedefs.h>
+
 #include "nosa.h"
 #include "nosa_common.cuh"
 #include "nosa_kernels.h"
@@ -53,6 +55,8 @@ int check_params(const nosa_params* p) {
   if (p->block_size != nosa::kBlock)
     return fail(NOSA_ERR_UNSUPPORTED, "block_size %d not supported (64)", p->block_size);
   if (p->local_blocks < 0) return fail(NOSA_ERR_INVALID_ARG, "local_blocks < 0");
+  if (p->local_blocks > nosa::kMaxLocalBlocks)
+    return fail(NOSA_ERR_UNSUPPORTED, "local_blocks %d above %d", p->local_blocks, nosa::kMaxLocalBlocks);
   if (p->topk < 1 || p->topk > 1024) return fail(NOSA_ERR_UNSUPPORTED, "topk %d outside 1..1024", p->topk);
   if (!(p->softmax_scale >= 0.0f) || std::isinf(p->softmax_scale))
     return fail(NOSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
@@ -86,7 +90,7 @@ Layout layout_of(const nosa_params* p, int batch, int max_seq_len) {
   l.bscores = off;
   off = round_up(off + pairs * static_cast<size_t>(l.nb_ws) * 4, 256);
   l.part = off;
-  off = round_up(off + pairs * nosa::kMaxSplits * static_cast<size_t>(G) * (nosa::kHeadDim + 2) * 4, 256);
+  off = round_up(off + pairs * nosa::kMaxSplits * static_cast<size_t>(nosa::part_stride(G)) * 4, 256);
   const size_t qbytes = static_cast<size_t>(batch) * p->num_q_heads * nosa::kHeadDim * 2;
   const size_t kvbytes = pairs * nosa::kHeadDim * 2;
   l.stage_q = off;
@@ -121,17 +125,48 @@ int sm_count() {
   return cached[dev];
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// 3-D map over a [rows, hkv, 128] bf16 cache: boxes of {64 dims, 1 head,
+// 64 tokens}, 128-byte swizzle, zero fill past `rows`.
+int encode_kv_map(CUtensorMap* map, const void* base, int hkv, int64_t rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(NOSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(nosa::kHeadDim), static_cast<cuuint64_t>(hkv),
+                              static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(nosa::kHeadDim) * 2,
+                                 static_cast<cuuint64_t>(hkv) * nosa::kHeadDim * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(nosa::kBlock)};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                   elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NOSA_ERR_INVALID_ARG, "tensor map encode failed (code %d)", static_cast<int>(r));
+  return NOSA_OK;
+}
+
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, const int64_t* seq_start,
+int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t cache_rows, const int64_t* seq_start,
                    const int32_t* len_old, const int32_t* len_new, int batch, float* pooled, int nc_cap,
                    int max_new_keys, const void* k_new, const void* v_new, uint32_t* status,
                    cudaStream_t stream) {
-  if (batch < 0 || nc_cap < 0 || max_new_keys < 0)
-    return fail(NOSA_ERR_INVALID_ARG, "batch, nc_cap and max_new_keys must be >= 0");
+  if (batch < 0 || nc_cap < 0 || max_new_keys < 0 || cache_rows < 0)
+    return fail(NOSA_ERR_INVALID_ARG, "batch, nc_cap, max_new_keys and cache_rows must be >= 0");
   if (batch == 0) return ok();
   if (!k_cache || !seq_start || !len_new || !pooled)
     return fail(NOSA_ERR_INVALID_ARG, "k_cache, seq_start, len_new and pooled must not be NULL");
@@ -146,6 +181,7 @@ int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, const int
   nosa::PoolArgs a{};
   a.k_cache = static_cast<__nv_bfloat16*>(k_cache);
   a.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  a.cache_rows = cache_rows;
   a.seq_start = seq_start;
   a.len_old = len_old;
   a.len_new = len_new;
@@ -215,7 +251,7 @@ int do_block_select(const nosa_params* p, const void* q, const float* pooled, in
 }
 
 int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
-                     const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
+                     int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
                      const int32_t* sel_idx, const int32_t* sel_cnt, void* out, float* lse, void* ws,
                      size_t ws_bytes, cudaStream_t stream) {
   if (batch < 0 || max_seq_len < 1) return fail(NOSA_ERR_INVALID_ARG, "batch >= 0 and max_seq_len >= 1 required");
@@ -226,6 +262,8 @@ int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, c
     return fail(NOSA_ERR_INVALID_ARG, "q, caches, seq_start, seq_len, sel_idx, sel_cnt and out must not be NULL");
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4))
     return fail(NOSA_ERR_INVALID_ARG, "caches must be 16-byte and q 4-byte aligned");
+  if (cache_rows < 1 || cache_rows >= (int64_t{1} << 31))
+    return fail(NOSA_ERR_UNSUPPORTED, "cache_rows must be in [1, 2^31)");
   if (static_cast<int64_t>(batch) * p->num_kv_heads > 65535)
     return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 65535");
   const int nb_max = static_cast<int>(nosa::n_blocks(max_seq_len));
@@ -236,6 +274,7 @@ int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, c
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
   a.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
+  a.cache_rows = cache_rows;
   a.seq_start = seq_start;
   a.seq_len = seq_len;
   a.sel_idx = sel_idx;
@@ -254,7 +293,10 @@ int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, c
   a.max_seq_len = max_seq_len;
   nosa::decode_split_plan(batch * p->num_kv_heads, max_tiles, sm_count(), &a.nsplit, &a.tiles_per_split);
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
-  cudaError_t e = nosa::launch_sparse_decode(a, stream);
+  CUtensorMap tm_k, tm_v;
+  if (int rc = encode_kv_map(&tm_k, k_cache, p->num_kv_heads, cache_rows)) return rc;
+  if (int rc = encode_kv_map(&tm_v, v_cache, p->num_kv_heads, cache_rows)) return rc;
+  cudaError_t e = nosa::launch_sparse_decode(a, tm_k, tm_v, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse_decode launch");
   return ok();
 }
@@ -289,7 +331,7 @@ int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   return ok();
 }
 
-int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache, const int64_t* seq_start,
+int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t cache_rows, const int64_t* seq_start,
                      const int32_t* len_old, const int32_t* len_new, int batch, float* pooled, int nc_cap,
                      int max_new_keys, const void* k_new, const void* v_new, void* ws, size_t ws_bytes,
                      void* stream) {
@@ -299,7 +341,7 @@ int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache, const i
     if (ws_bytes < 256 || !aligned(ws, 256)) return fail(NOSA_ERR_WORKSPACE, "workspace must be 256-byte aligned and >= 256 bytes");
     status = at<uint32_t>(ws, 0);
   }
-  return do_pool_append(p, k_cache, v_cache, seq_start, len_old, len_new, batch, pooled, nc_cap,
+  return do_pool_append(p, k_cache, v_cache, cache_rows, seq_start, len_old, len_new, batch, pooled, nc_cap,
                         max_new_keys, k_new, v_new, status, static_cast<cudaStream_t>(stream));
 }
 
@@ -314,17 +356,17 @@ int nosa_block_select(const nosa_params* p, const void* q, const float* pooled, 
 }
 
 int nosa_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
-                       const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
+                       int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
                        const int32_t* sel_idx, const int32_t* sel_cnt, void* out, float* lse, void* ws,
                        size_t ws_bytes, void* stream) {
   if (int rc = check_params(p)) return rc;
-  return do_sparse_decode(p, q, k_cache, v_cache, seq_start, seq_len, batch, max_seq_len, sel_idx,
+  return do_sparse_decode(p, q, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len, sel_idx,
                           sel_cnt, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new_host,
                      const void* v_new_host, void* out_host, void* k_cache, void* v_cache,
-                     const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
+                     int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
                      float* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* ws,
                      size_t ws_bytes, void* stream) {
   if (int rc = check_params(p)) return rc;
@@ -345,13 +387,13 @@ int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new
   if ((e = cudaMemcpyAsync(dq, q_host, qbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy q");
   if ((e = cudaMemcpyAsync(dk, k_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy k_new");
   if ((e = cudaMemcpyAsync(dv, v_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy v_new");
-  int rc = do_pool_append(p, k_cache, v_cache, seq_start, nullptr, seq_len, batch, pooled, nc_cap, 1, dk, dv,
+  int rc = do_pool_append(p, k_cache, v_cache, cache_rows, seq_start, nullptr, seq_len, batch, pooled, nc_cap, 1, dk, dv,
                           at<uint32_t>(ws, l.status), s);
   if (rc) return rc;
   rc = do_block_select(p, dq, pooled, nc_cap, seq_len, batch, max_seq_len, nullptr, 0, nullptr, nullptr, 0,
                        sel_idx, sel_cnt, ws, ws_bytes, s);
   if (rc) return rc;
-  rc = do_sparse_decode(p, dq, k_cache, v_cache, seq_start, seq_len, batch, max_seq_len, sel_idx, sel_cnt,
+  rc = do_sparse_decode(p, dq, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len, sel_idx, sel_cnt,
                         dout, nullptr, ws, ws_bytes, s);
   if (rc) return rc;
   if ((e = cudaMemcpyAsync(out_host, dout, qbytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess) return cuda_fail(e, "copy out");

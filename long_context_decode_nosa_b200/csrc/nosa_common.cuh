@@ -22,8 +22,14 @@ constexpr int kBlock = 64;
 constexpr int kWindowsPerBlock = kBlock / kPoolStride;  // 4
 constexpr int kMaxGroup = 16;
 constexpr int kMaxSplits = 64;
+constexpr int kMaxTilesPerSplit = 128;
+constexpr int kMaxLocalBlocks = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint32_t kWaitLimitIters = 1u << 30;
+
+// Floats per (pair, split) partial softmax state: O[G][128], m[G], l[G],
+// padded to a multiple of 4 floats so every split's O starts 16-byte aligned.
+__host__ __device__ constexpr int part_stride(int G) { return G * kHeadDim + ((2 * G + 3) & ~3); }
 
 __host__ __device__ inline int64_t n_windows(int64_t L) {
   return L >= kPoolKernel ? (L - kPoolKernel) / kPoolStride + 1 : 0;
@@ -104,6 +110,15 @@ __device__ inline void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while its predecessor on the stream is finishing:
+// it must not touch global memory before grid_dependency_wait(), which returns
+// once the predecessor grid has completed and its writes are visible.
+// allow_dependents() lets the next kernel on the stream start its own
+// prologue early.  Both are no-ops without a programmatic predecessor.
+__device__ inline void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Order-preserving map of an fp32 score to uint32, with -0.0 == +0.0 and NaN
 // ranked as -inf (ties are then broken by index by the caller).

@@ -1,15 +1,19 @@
 // Launch interfaces of the three NOSA kernels (internal to the library).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <utility>
 
 namespace nosa {
 
 struct PoolArgs {
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
+  int64_t cache_rows;
   const int64_t* seq_start;
   const int32_t* len_old;  // nullable: len_new - 1
   const int32_t* len_new;
@@ -41,13 +45,14 @@ struct DecodeArgs {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k_cache;
   const __nv_bfloat16* v_cache;
+  int64_t cache_rows;
   const int64_t* seq_start;
   const int32_t* seq_len;
   const int32_t* sel_idx;
   const int32_t* sel_cnt;
   __nv_bfloat16* out;
   float* lse;        // nullable
-  float* part;       // [pairs, kMaxSplits, group*(128+2)] partial softmax state
+  float* part;       // [pairs, kMaxSplits, part_stride(group)] partial softmax state
   uint32_t* tickets; // [pairs]
   uint32_t* status;
   int batch, hq, hkv, group, local_blocks, topk, max_seq_len;
@@ -55,9 +60,29 @@ struct DecodeArgs {
   float scale_log2;  // softmax scale * log2(e)
 };
 
+// Launches `kernel` with programmatic stream serialization, so that it can be
+// scheduled while the previous kernel on `stream` finishes (the kernels wait
+// on the dependency themselves before touching global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_pool_append(const PoolArgs& a, cudaStream_t stream);
 cudaError_t launch_block_select(const SelectArgs& a, cudaStream_t stream);
-cudaError_t launch_sparse_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_sparse_decode(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                 cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint32_t* status, uint32_t max_iters, cudaStream_t stream);
 
 // Number of splits and tiles per split that launch_sparse_decode will use.

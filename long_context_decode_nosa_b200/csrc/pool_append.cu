@@ -34,6 +34,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.y;
   const int i = pair / a.hkv, h = pair % a.hkv;
+  grid_dependency_wait();
+  allow_dependents();
   const int32_t len_new = a.len_new[i];
   const int32_t len_old = a.len_old ? a.len_old[i] : len_new - 1;
   if (len_old < 0 || len_new < len_old) {
@@ -41,6 +43,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
     return;
   }
   const int64_t base = a.seq_start[i];
+  if (base < 0 || base + len_new > a.cache_rows) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, NOSA_DEV_CACHE_ROWS);
+    return;
+  }
   const bool append = a.k_new != nullptr;
   if (append && len_new != len_old + 1) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, NOSA_DEV_APPEND_ONE);
@@ -65,20 +71,27 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
     if (lane == 0) set_status(a.status, NOSA_DEV_NC_CAP);
     return;
   }
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // All 32 row loads are issued before any is consumed (one DRAM round trip,
+  // not 32); rows < len_new exist in the cache, so every load is in bounds.
   const int64_t t0 = j * kPoolStride;
-#pragma unroll 8
-  for (int t = 0; t < kPoolKernel; ++t) {
-    const int64_t tok = t0 + t;
-    uint2 raw;
-    if (append && tok == len_old) {
-      raw = knew_row[lane];
-    } else {
-      const uint2* src =
-          reinterpret_cast<const uint2*>(a.k_cache + ((base + tok) * a.hkv + h) * kHeadDim);
-      raw = __ldg(src + lane);
+  const uint2* src = reinterpret_cast<const uint2*>(a.k_cache + ((base + t0) * a.hkv + h) * kHeadDim) + lane;
+  const int64_t row_stride = static_cast<int64_t>(a.hkv) * kHeadDim / 4;  // in uint2
+  uint2 raw[kPoolKernel];
+#pragma unroll
+  for (int t = 0; t < kPoolKernel; ++t) raw[t] = __ldg(src + t * row_stride);
+  if (append) {
+    const int64_t r = static_cast<int64_t>(len_old) - t0;  // the new token's row inside the window
+    if (r >= 0 && r < kPoolKernel) {
+      const uint2 fresh = knew_row[lane];
+#pragma unroll
+      for (int t = 0; t < kPoolKernel; ++t)
+        if (t == r) raw[t] = fresh;
     }
-    const float4 f = bf16x4_to_float4(raw);
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int t = 0; t < kPoolKernel; ++t) {
+    const float4 f = bf16x4_to_float4(raw[t]);
     acc.x += f.x;
     acc.y += f.y;
     acc.z += f.z;
@@ -101,8 +114,7 @@ cudaError_t launch_pool_append(const PoolArgs& a, cudaStream_t stream) {
   if (pairs == 0) return cudaSuccess;
   const int chunks = (a.max_new_keys + kWarpsPerCta - 1) / kWarpsPerCta;
   dim3 grid(chunks > 0 ? chunks : 1, pairs);
-  pool_append_kernel<<<grid, kWarpsPerCta * 32, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_overlapped(pool_append_kernel, grid, dim3(kWarpsPerCta * 32), 0, stream, a);
 }
 
 }  // namespace nosa

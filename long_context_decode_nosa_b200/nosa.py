@@ -33,6 +33,7 @@ NOSA_DEV_BAD_COUNT = 0x8
 NOSA_DEV_MAX_NEW_KEYS = 0x10
 NOSA_DEV_APPEND_ONE = 0x20
 NOSA_DEV_MAX_LEN = 0x40
+NOSA_DEV_CACHE_ROWS = 0x80
 NOSA_DEV_TIMEOUT = 0x80000000
 
 
@@ -58,15 +59,16 @@ _lib = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SZ = ctypes.c_size_t
+_I64 = ctypes.c_int64
 
 _SIGNATURES = {
     "nosa_default_params": (None, [_P]),
     "nosa_workspace_size": (_SZ, [_P, _I, _I]),
     "nosa_workspace_init": (_I, [_P, _SZ, _P]),
-    "nosa_pool_append": (_I, [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
+    "nosa_pool_append": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "nosa_block_select": (_I, [_P, _P, _P, _I, _P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _P, _SZ, _P]),
-    "nosa_sparse_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
-    "nosa_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "nosa_sparse_decode": (_I, [_P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "nosa_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "nosa_read_device_status": (_I, [_P, _SZ, _P]),
     "nosa_last_device_bits": (ctypes.c_uint32, []),
     "nosa_selftest_wait_timeout": (_I, [_P, _SZ, ctypes.c_uint32, _P]),
@@ -167,7 +169,7 @@ def nosa_pool_append(p: nosa_params, k_cache: torch.Tensor, v_cache: Optional[to
     batch = len_new.shape[0]
     rc = lib().nosa_pool_append(
         ctypes.byref(p), _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
-        _ptr(seq_start, torch.int64, "seq_start"), _ptr(len_old, torch.int32, "len_old"),
+        k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"), _ptr(len_old, torch.int32, "len_old"),
         _ptr(len_new, torch.int32, "len_new"), batch, _ptr(pooled, torch.float32, "pooled"),
         pooled.shape[2], max_new_keys, _ptr(k_new, torch.bfloat16, "k_new"),
         _ptr(v_new, torch.bfloat16, "v_new"), _ptr(ws, torch.uint8, "ws"),
@@ -205,7 +207,7 @@ def nosa_sparse_decode(p: nosa_params, q: torch.Tensor, k_cache: torch.Tensor, v
     batch = seq_len.shape[0]
     rc = lib().nosa_sparse_decode(
         ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
-        _ptr(v_cache, torch.bfloat16, "v_cache"), _ptr(seq_start, torch.int64, "seq_start"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
         _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len,
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
@@ -227,8 +229,8 @@ def nosa_decode_step(p: nosa_params, q_host: torch.Tensor, k_new_host: torch.Ten
         _ptr(v_new_host, torch.bfloat16, "v_new_host", cuda=False),
         _ptr(out_host, torch.bfloat16, "out_host", cuda=False),
         _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
-        _ptr(seq_start, torch.int64, "seq_start"), _ptr(seq_len, torch.int32, "seq_len"), batch,
-        max_seq_len, _ptr(pooled, torch.float32, "pooled"), pooled.shape[2],
+        k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"), _ptr(seq_len, torch.int32, "seq_len"),
+        batch, max_seq_len, _ptr(pooled, torch.float32, "pooled"), pooled.shape[2],
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(rc, "nosa_decode_step")

@@ -63,12 +63,13 @@ def test_workspace_size_host_only(nosa):
 
 @pytest.mark.parametrize("field,value,code", [
     ("head_dim", 64, 2), ("pool_kernel", 16, 2), ("block_size", 128, 2), ("topk", 0, 2),
+    ("local_blocks", 257, 2),
     ("num_kv_heads", 3, 1), ("local_blocks", -1, 1), ("softmax_scale", -1.0, 1),
 ])
 def test_bad_params_rejected_before_any_launch(nosa, field, value, code):
     p = nosa.params(16, 2)
     setattr(p, field, value)
-    rc = nosa.lib().nosa_sparse_decode(ctypes.byref(p), None, None, None, None, None, 1, 16, None,
+    rc = nosa.lib().nosa_sparse_decode(ctypes.byref(p), None, None, None, 0, None, None, 1, 16, None,
                                        None, None, None, None, 0, None)
     assert rc == code
     assert nosa.lib().nosa_last_error().decode()
@@ -84,14 +85,14 @@ def test_null_and_workspace_checks(nosa):
     # workspace too small (a host buffer stands in: the check fails before any use)
     buf = ctypes.create_string_buffer(1024 + 256)
     addr = (ctypes.addressof(buf) + 255) // 256 * 256
-    rc = L.nosa_sparse_decode(ctypes.byref(p), None, None, None, None, None, 4, 1024, None, None,
+    rc = L.nosa_sparse_decode(ctypes.byref(p), None, None, None, 0, None, None, 4, 1024, None, None,
                               None, None, ctypes.c_void_p(addr), 1024, None)
     assert rc == nosa.NOSA_ERR_WORKSPACE
     # batch 0 is a no-op
-    assert L.nosa_pool_append(ctypes.byref(p), None, None, None, None, None, 0, None, 1, 1, None,
+    assert L.nosa_pool_append(ctypes.byref(p), None, None, 0, None, None, None, 0, None, 1, 1, None,
                               None, None, 0, None) == 0
     # k_new without v_new
-    rc = L.nosa_pool_append(ctypes.byref(p), ctypes.c_void_p(256), None, ctypes.c_void_p(256), None,
+    rc = L.nosa_pool_append(ctypes.byref(p), ctypes.c_void_p(256), None, 100, ctypes.c_void_p(256), None,
                             ctypes.c_void_p(256), 1, ctypes.c_void_p(256), 1, 1,
                             ctypes.c_void_p(256), None, None, 0, None)
     assert rc == nosa.NOSA_ERR_INVALID_ARG
