@@ -140,10 +140,17 @@ class Replica:
                                                        device=device)
 
 
-def step(nosa, r: Replica, events=None):
-    """One decode step on device-resident inputs.  events: 4 CUDA events
-    recorded before K1, before K2, before K3 and after K3 (or None)."""
+def step(nosa, r: Replica, events=None, fused=True):
+    """One decode step on device-resident inputs: append the new token's K/V
+    rows, pool the window it completes, select, attend.  ``fused``: one launch
+    (nosa_decode_step_device); otherwise the three entry points in order, with
+    ``events`` (4 CUDA events) recorded before each kernel and after the last."""
     b, st, p = r.b, r.st, r.p
+    if fused:
+        nosa.nosa_decode_step_device(p, b.q, b.k_cache, b.v_cache, b.seq_start, b.seq_len, st.max_seq_len,
+                                     st.pooled, st.sel_idx, st.sel_cnt, st.out, st.ws, k_new=r.k_new,
+                                     v_new=r.v_new)
+        return
     if events:
         events[0].record()
     nosa.nosa_pool_append(p, b.k_cache, b.v_cache, b.seq_start, b.seq_len, st.pooled, max_new_keys=1,
@@ -226,9 +233,9 @@ def kernel_source_hash():
 
 
 def ncu_traffic(workload: str):
-    """Per-launch DRAM bytes of the sparse-decode kernel from the committed ncu
+    """Per-launch DRAM bytes of the fused step kernel from the committed ncu
     summary (profiles/), if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", f"sparse_decode_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"step_kernel_{workload}.md")
     try:
         with open(path) as f:
             txt = f.read()
@@ -335,26 +342,32 @@ def run_ours(args):
     stream = torch.cuda.Stream(device)
     stream.wait_stream(torch.cuda.current_stream())
 
-    def record_steps(n, with_events):
+    def record_steps(n, fused=True, with_events=False):
         evs = []
-        for s in range(n):
-            for layer in rotation[s % len(rotation)]:
-                e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] if with_events else None
-                step(nosa, layer, e)
+        for s_ in range(n):
+            for layer in rotation[s_ % len(rotation)]:
+                e = ([torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+                     if with_events else None)
+                step(nosa, layer, e, fused=fused)
                 if e:
                     evs.append(e)
         return evs
 
     with torch.cuda.stream(stream):
-        record_steps(len(rotation), False)         # eager warm-up: sets kernel attributes
+        record_steps(len(rotation))                       # eager warm-up: kernel attributes
+        record_steps(len(rotation), fused=False)
     stream.synchronize()
 
     g_warm = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_warm, stream=stream):
-        record_steps(max(args.warmup, 1), False)
+        record_steps(max(args.warmup, 1))
     g_timed = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_timed, stream=stream):
-        inner = record_steps(args.steps, True)
+        record_steps(args.steps)
+    n_split = max(len(rotation), min(args.steps, 200))
+    g_split = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_split, stream=stream):
+        inner = record_steps(n_split, fused=False, with_events=True)
 
     clocks = ClockSampler(device.index if device.index is not None else 0)
     clocks.start()
@@ -375,22 +388,32 @@ def run_ours(args):
     clk = clocks.stop()
     ms_total = multirank.max_over_ranks(start.elapsed_time(stop), info, device)
     ms_step = ms_total / args.steps
-    n_layers_launches = len(inner)
+    # Kernel split of the unfused path (separate launches with events between
+    # them, which also stops their launches overlapping): context only.
+    with torch.cuda.stream(stream):
+        g_split.replay()
+    stream.synchronize()
     kt = {"pool_append": [], "block_select": [], "sparse_decode": []}
     for e in inner:
         kt["pool_append"].append(e[0].elapsed_time(e[1]))
         kt["block_select"].append(e[1].elapsed_time(e[2]))
         kt["sparse_decode"].append(e[2].elapsed_time(e[3]))
     kmean_us = {k: 1e3 * statistics.fmean(v) for k, v in kt.items()}
+    unfused_ms_step = sum(kmean_us.values()) * wl.layers / 1e3
 
     queries_per_step = wl.batch * wl.layers
     value = multirank.aggregate_rate(queries_per_step * args.steps, info, ms_total / 1e3)
     model = wl.bytes_model()
     step_bytes = sum(model.values())
     peak, peak_kind = peak_hbm()
-    dec_bytes_launch = model["sparse_decode"] / wl.layers
-    dec_achieved = dec_bytes_launch / (kmean_us["sparse_decode"] * 1e-6) / 1e9
-    traffic = ncu_traffic(wl.name) if wl.name == args.workload and not (args.context or args.batch or args.topk) else None
+    # The fused step kernel is the only kernel of a step: its average launch
+    # duration is the timed region over the launches (gaps included).
+    launch_s = ms_total / 1e3 / (args.steps * wl.layers)
+    fused_bytes_launch = step_bytes / wl.layers
+    achieved = fused_bytes_launch / launch_s / 1e9
+    traffic = None
+    if not (args.context or args.batch or args.topk):
+        traffic = ncu_traffic(wl.name)
 
     # e2e through the host-buffer entry point, one layer (replica 0), pinned buffers.
     e2e = None
@@ -421,19 +444,22 @@ def run_ours(args):
                        "parallelism": f"dp{world}" if world > 1 else "single GPU",
                        "l2": (f"inputs rotate over {R} cache replicas "
                               f"({R * layer_bytes * wl.layers / 1e9:.2f} GB) > 126 MB L2"),
-                       "clock_settle_ms": args.settle_ms, "graph": "timed steps replayed as one CUDA graph"},
-            "gpu_launches": 3 * n_layers_launches,
+                       "clock_settle_ms": args.settle_ms,
+                       "graph": "timed steps (one fused launch per layer-step) replayed as one CUDA graph"},
+            "gpu_launches": args.steps * wl.layers,
             "hbm_gbs_step": step_bytes / (ms_step * 1e-3) / 1e9,
             "algorithmic_bytes_per_step": step_bytes,
-            "kernel_us": kmean_us,
-            "roofline": {"bound": "hbm", "kernel": "sparse_decode", "achieved": dec_achieved,
-                         "peak": peak, "unit": "GB/s", "frac": dec_achieved / peak,
+            "kernel_us_unfused": kmean_us,
+            "ms_per_step_unfused": unfused_ms_step,
+            "roofline": {"bound": "hbm", "kernel": "step_kernel (fused pool + select + sparse decode)",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": f"{peak_kind} copy bandwidth", "traffic": traffic,
-                         "algorithmic_bytes_per_launch": dec_bytes_launch},
+                         "algorithmic_bytes_per_launch": fused_bytes_launch,
+                         "launch_us": launch_s * 1e6},
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         }
         print(json.dumps(line), flush=True)
-    del g_timed, g_warm
+    del g_timed, g_warm, g_split
     multirank.shutdown(info)
     return 0
 

@@ -182,6 +182,26 @@ NOSA_API int nosa_sparse_decode(const nosa_params* p, const void* q, const void*
                        void* out, float* lse, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* One whole decode step on DEVICE buffers, fused into a single launch of a
+ * persistent kernel (steps 1-4 above, in the pages' order): appends the new
+ * token's K/V rows (k_new / v_new, bf16 [batch, Hkv, D], nullable: then the
+ * rows must already be in the caches) at seq_start[i] + seq_len[i] - 1, pools
+ * the window it completes, scores and selects blocks (sel_idx / sel_cnt
+ * receive the selection) and attends, writing out (bf16 [batch, Hq, D]) and
+ * lse (nullable).  Results are bit-identical to nosa_pool_append +
+ * nosa_block_select + nosa_sparse_decode on the same inputs.  Work items are
+ * taken from a queue in the workspace by resident CTAs; the attention items
+ * of a sequence wait (bounded, NOSA_DEV_TIMEOUT on expiry) for that
+ * sequence's selection, published by the CTA that computed it.  With fewer
+ * than two local blocks the three separate launches run instead. */
+NOSA_API int nosa_decode_step_device(const nosa_params* p, const void* q, const void* k_new,
+                                     const void* v_new, void* k_cache, void* v_cache,
+                                     int64_t cache_rows, const int64_t* seq_start,
+                                     const int32_t* seq_len, int batch, int max_seq_len,
+                                     float* pooled, int nc_cap, int32_t* sel_idx,
+                                     int32_t* sel_cnt, void* out, float* lse, void* ws,
+                                     size_t ws_bytes, void* stream);
+
 /* One whole decode step from HOST buffers (the pages' per-token decode,
  * steps 1-4 above in order): copies q_host (bf16 [batch, Hq, D]) and the new
  * token's k_new_host / v_new_host (bf16 [batch, Hkv, D]) to the device,
@@ -191,7 +211,8 @@ NOSA_API int nosa_sparse_decode(const nosa_params* p, const void* q, const void*
  * the new token.  All copies and kernels are enqueued on `stream`; the call
  * returns without waiting, so out_host is valid after the stream synchronises.
  * Host buffers should be pinned for the copies to be asynchronous.  The
- * device staging area comes from `ws` (nosa_workspace_size covers it).
+ * device staging area comes from `ws` (nosa_workspace_size covers it).  The
+ * kernels run as in nosa_decode_step_device.
  * sel_idx / sel_cnt (device) receive the selection. */
 NOSA_API int nosa_decode_step(const nosa_params* p, const void* q_host,
                      const void* k_new_host, const void* v_new_host,

@@ -11,6 +11,8 @@
 #include "nosa.h"
 #include "nosa_common.cuh"
 #include "nosa_kernels.h"
+#include "decode_device.cuh"
+#include "select_device.cuh"
 
 namespace {
 
@@ -71,7 +73,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace layout (all offsets 256-byte aligned).
 struct Layout {
-  size_t status, sel_tickets, dec_tickets, bscores, part, stage_q, stage_k, stage_v, stage_out, total;
+  size_t status, work, sel_tickets, dec_tickets, ready, bscores, part, stage_q, stage_k, stage_v, stage_out, total;
   int nb_ws;
 };
 
@@ -81,11 +83,14 @@ Layout layout_of(const nosa_params* p, int batch, int max_seq_len) {
   const int G = p->num_q_heads / p->num_kv_heads;
   l.nb_ws = static_cast<int>(nosa::n_blocks(max_seq_len));
   size_t off = 0;
-  l.status = off;
+  l.status = off;  // uint32 device status word
+  l.work = off + 16;  // uint32[2] work queue of the step kernel
   off += 256;
   l.sel_tickets = off;
   off = round_up(off + pairs * 4, 256);
   l.dec_tickets = off;
+  off = round_up(off + pairs * 4, 256);
+  l.ready = off;
   off = round_up(off + pairs * 4, 256);
   l.bscores = off;
   off = round_up(off + pairs * static_cast<size_t>(l.nb_ws) * 4, 256);
@@ -113,17 +118,6 @@ int check_ws(void* ws, size_t ws_bytes, const Layout& l) {
   return NOSA_OK;
 }
 
-int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -198,36 +192,15 @@ int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t c
   return ok();
 }
 
-int do_block_select(const nosa_params* p, const void* q, const float* pooled, int nc_cap,
-                    const int32_t* seq_len, int batch, int max_seq_len, const float* bs_in, int nb_in,
-                    float* comp_out, float* bs_out, int nb_out, int32_t* sel_idx, int32_t* sel_cnt,
-                    void* ws, size_t ws_bytes, cudaStream_t stream) {
-  if (batch < 0 || max_seq_len < 1) return fail(NOSA_ERR_INVALID_ARG, "batch >= 0 and max_seq_len >= 1 required");
-  if (batch == 0) return ok();
-  const Layout l = layout_of(p, batch, max_seq_len);
-  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
-  if (!seq_len || !sel_idx || !sel_cnt) return fail(NOSA_ERR_INVALID_ARG, "seq_len, sel_idx and sel_cnt must not be NULL");
-  const int ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
-  if (bs_in) {
-    if (nb_in < ncand_max)
-      return fail(NOSA_ERR_INVALID_ARG, "nb_cap_in %d below the %d candidates of max_seq_len", nb_in, ncand_max);
-  } else {
-    if (!q || !pooled) return fail(NOSA_ERR_INVALID_ARG, "q and pooled must not be NULL when scoring");
-    if (!aligned(pooled, 16) || !aligned(q, 8)) return fail(NOSA_ERR_INVALID_ARG, "pooled must be 16-byte and q 8-byte aligned");
-    if (nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "nc_cap must be >= 1");
-    if (bs_out && nb_out < ncand_max)
-      return fail(NOSA_ERR_INVALID_ARG, "nb_cap_out %d below the %d candidates of max_seq_len", nb_out, ncand_max);
-  }
-  if (l.nb_ws * 4 > 200 * 1024) return fail(NOSA_ERR_UNSUPPORTED, "max_seq_len too long for the selector");
-  if (static_cast<int64_t>(batch) * p->num_kv_heads > 65535)
-    return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 65535");
-  nosa::SelectArgs a{};
+void fill_select_args(nosa::SelectArgs& a, const nosa_params* p, const void* q, const float* pooled, int nc_cap,
+                      const int32_t* seq_len, int batch, int max_seq_len, float* comp_out, float* bs_out,
+                      int nb_out, int32_t* sel_idx, int32_t* sel_cnt, void* ws, const Layout& l) {
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.pooled = pooled;
   a.seq_len = seq_len;
-  a.bs_in = bs_in;
-  a.comp_out = bs_in ? nullptr : comp_out;
-  a.bs_out = bs_in ? nullptr : bs_out;
+  a.bs_in = nullptr;
+  a.comp_out = comp_out;
+  a.bs_out = bs_out;
   a.sel_idx = sel_idx;
   a.sel_cnt = sel_cnt;
   a.bscratch = at<float>(ws, l.bscores);
@@ -241,36 +214,16 @@ int do_block_select(const nosa_params* p, const void* q, const float* pooled, in
   a.topk = p->topk;
   a.max_seq_len = max_seq_len;
   a.nc_cap = nc_cap;
-  a.nb_in = nb_in;
+  a.nb_in = 0;
   a.nb_out = nb_out;
   a.nb_ws = l.nb_ws;
   a.scale = scale_of(p);
-  cudaError_t e = nosa::launch_block_select(a, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "block_select launch");
-  return ok();
 }
 
-int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
-                     int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
-                     const int32_t* sel_idx, const int32_t* sel_cnt, void* out, float* lse, void* ws,
-                     size_t ws_bytes, cudaStream_t stream) {
-  if (batch < 0 || max_seq_len < 1) return fail(NOSA_ERR_INVALID_ARG, "batch >= 0 and max_seq_len >= 1 required");
-  if (batch == 0) return ok();
-  const Layout l = layout_of(p, batch, max_seq_len);
-  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
-  if (!q || !k_cache || !v_cache || !seq_start || !seq_len || !sel_idx || !sel_cnt || !out)
-    return fail(NOSA_ERR_INVALID_ARG, "q, caches, seq_start, seq_len, sel_idx, sel_cnt and out must not be NULL");
-  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4))
-    return fail(NOSA_ERR_INVALID_ARG, "caches must be 16-byte and q 4-byte aligned");
-  if (cache_rows < 1 || cache_rows >= (int64_t{1} << 31))
-    return fail(NOSA_ERR_UNSUPPORTED, "cache_rows must be in [1, 2^31)");
-  if (static_cast<int64_t>(batch) * p->num_kv_heads > 65535)
-    return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 65535");
-  const int nb_max = static_cast<int>(nosa::n_blocks(max_seq_len));
-  const int ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
-  const int max_tiles = (p->topk < ncand_max ? p->topk : ncand_max) +
-                        (p->local_blocks < nb_max ? p->local_blocks : nb_max);
-  nosa::DecodeArgs a{};
+void fill_decode_args(nosa::DecodeArgs& a, const nosa_params* p, const void* q, const void* k_cache,
+                      const void* v_cache, int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len,
+                      int batch, int max_seq_len, const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
+                      float* lse, void* ws, const Layout& l) {
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
   a.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
@@ -291,13 +244,171 @@ int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, c
   a.local_blocks = p->local_blocks;
   a.topk = p->topk;
   a.max_seq_len = max_seq_len;
-  nosa::decode_split_plan(batch * p->num_kv_heads, max_tiles, sm_count(), &a.nsplit, &a.tiles_per_split);
+  const int nb_max = static_cast<int>(nosa::n_blocks(max_seq_len));
+  const int ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
+  const int max_tiles = (p->topk < ncand_max ? p->topk : ncand_max) +
+                        (p->local_blocks < nb_max ? p->local_blocks : nb_max);
+  nosa::decode_split_plan(batch * p->num_kv_heads, max_tiles, nosa::step_resident_ctas(a.group), &a.nsplit);
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
+}
+
+int scoring_items(const nosa_params* p, int batch, int max_seq_len, bool full) {
+  const int nbw = static_cast<int>(full ? nosa::n_blocks(max_seq_len) : nosa::n_candidates(max_seq_len, p->local_blocks));
+  const int chunks = nbw > 0 ? (nbw + nosa::kChunkBlocks - 1) / nosa::kChunkBlocks : 1;
+  return batch * p->num_kv_heads * chunks;
+}
+
+int check_common(const nosa_params* p, int batch, int max_seq_len) {
+  if (batch < 0 || max_seq_len < 1) return fail(NOSA_ERR_INVALID_ARG, "batch >= 0 and max_seq_len >= 1 required");
+  if (static_cast<int64_t>(batch) * p->num_kv_heads > (1 << 20))
+    return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 2^20");
+  if (nosa::n_blocks(max_seq_len) * 4 > nosa::kRingBytes)
+    return fail(NOSA_ERR_UNSUPPORTED, "max_seq_len too long for the selector's shared memory");
+  return NOSA_OK;
+}
+
+int do_block_select(const nosa_params* p, const void* q, const float* pooled, int nc_cap,
+                    const int32_t* seq_len, int batch, int max_seq_len, const float* bs_in, int nb_in,
+                    float* comp_out, float* bs_out, int nb_out, int32_t* sel_idx, int32_t* sel_cnt,
+                    void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (int rc = check_common(p, batch, max_seq_len)) return rc;
+  if (batch == 0) return ok();
+  const Layout l = layout_of(p, batch, max_seq_len);
+  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
+  if (!seq_len || !sel_idx || !sel_cnt) return fail(NOSA_ERR_INVALID_ARG, "seq_len, sel_idx and sel_cnt must not be NULL");
+  const int ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
+  nosa::SelectArgs a{};
+  if (bs_in) {
+    if (nb_in < ncand_max)
+      return fail(NOSA_ERR_INVALID_ARG, "nb_cap_in %d below the %d candidates of max_seq_len", nb_in, ncand_max);
+    if (static_cast<int64_t>(batch) * p->num_kv_heads > 65535)
+      return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 65535");
+    fill_select_args(a, p, nullptr, nullptr, 0, seq_len, batch, max_seq_len, nullptr, nullptr, 0, sel_idx, sel_cnt,
+                     ws, l);
+    a.bs_in = bs_in;
+    a.nb_in = nb_in;
+    cudaError_t e = nosa::launch_select_only(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "block_select launch");
+    return ok();
+  }
+  if (!q || !pooled) return fail(NOSA_ERR_INVALID_ARG, "q and pooled must not be NULL when scoring");
+  if (!aligned(pooled, 16) || !aligned(q, 8)) return fail(NOSA_ERR_INVALID_ARG, "pooled must be 16-byte and q 8-byte aligned");
+  if (nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "nc_cap must be >= 1");
+  if (bs_out && nb_out < ncand_max)
+    return fail(NOSA_ERR_INVALID_ARG, "nb_cap_out %d below the %d candidates of max_seq_len", nb_out, ncand_max);
+  nosa::StepArgs s{};
+  fill_select_args(s.sel, p, q, pooled, nc_cap, seq_len, batch, max_seq_len, comp_out, bs_out, nb_out, sel_idx,
+                   sel_cnt, ws, l);
+  s.dec.group = s.sel.group;
+  s.work = at<uint32_t>(ws, l.work);
+  s.ready = at<uint32_t>(ws, l.ready);
+  s.mode = nosa::kStepScore;
+  s.pairs = batch * p->num_kv_heads;
+  s.n_score_items = scoring_items(p, batch, max_seq_len, comp_out != nullptr);
+  s.n_items = s.n_score_items;
+  CUtensorMap none;
+  memset(&none, 0, sizeof none);
+  cudaError_t e = nosa::launch_step(s, none, none, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "block_select launch");
+  return ok();
+}
+
+int check_decode_ptrs(const void* q, const void* k_cache, const void* v_cache, int64_t cache_rows,
+                      const int64_t* seq_start, const int32_t* seq_len, const int32_t* sel_idx,
+                      const int32_t* sel_cnt, const void* out) {
+  if (!q || !k_cache || !v_cache || !seq_start || !seq_len || !sel_idx || !sel_cnt || !out)
+    return fail(NOSA_ERR_INVALID_ARG, "q, caches, seq_start, seq_len, sel_idx, sel_cnt and out must not be NULL");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 8))
+    return fail(NOSA_ERR_INVALID_ARG, "caches must be 16-byte and q 8-byte aligned");
+  if (cache_rows < 1 || cache_rows >= (int64_t{1} << 31))
+    return fail(NOSA_ERR_UNSUPPORTED, "cache_rows must be in [1, 2^31)");
+  return NOSA_OK;
+}
+
+int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                     int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
+                     const int32_t* sel_idx, const int32_t* sel_cnt, void* out, float* lse, void* ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+  if (int rc = check_common(p, batch, max_seq_len)) return rc;
+  if (batch == 0) return ok();
+  const Layout l = layout_of(p, batch, max_seq_len);
+  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
+  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, seq_start, seq_len, sel_idx, sel_cnt, out)) return rc;
+  nosa::StepArgs s{};
+  fill_decode_args(s.dec, p, q, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len, sel_idx,
+                   sel_cnt, out, lse, ws, l);
+  s.work = at<uint32_t>(ws, l.work);
+  s.ready = at<uint32_t>(ws, l.ready);
+  s.mode = nosa::kStepDecode;
+  s.pairs = batch * p->num_kv_heads;
+  s.n_score_items = 0;
+  s.n_items = s.pairs * s.dec.nsplit;
   CUtensorMap tm_k, tm_v;
   if (int rc = encode_kv_map(&tm_k, k_cache, p->num_kv_heads, cache_rows)) return rc;
   if (int rc = encode_kv_map(&tm_v, v_cache, p->num_kv_heads, cache_rows)) return rc;
-  cudaError_t e = nosa::launch_sparse_decode(a, tm_k, tm_v, stream);
+  cudaError_t e = nosa::launch_step(s, tm_k, tm_v, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse_decode launch");
+  return ok();
+}
+
+// The fused step on device buffers: one launch appends, pools, selects and
+// attends.  Needs at least two local blocks (then the window a new token
+// completes is never read by the same step's selection); otherwise the three
+// separate launches run.
+int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                          void* v_cache, int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len,
+                          int batch, int max_seq_len, float* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt,
+                          void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (int rc = check_common(p, batch, max_seq_len)) return rc;
+  if (batch == 0) return ok();
+  const Layout l = layout_of(p, batch, max_seq_len);
+  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
+  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, seq_start, seq_len, sel_idx, sel_cnt, out)) return rc;
+  if (!pooled || nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "pooled must not be NULL and nc_cap >= 1");
+  if (!aligned(pooled, 16)) return fail(NOSA_ERR_INVALID_ARG, "pooled must be 16-byte aligned");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(NOSA_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+  if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16)))
+    return fail(NOSA_ERR_INVALID_ARG, "new-row pointers must be 16-byte aligned");
+  if (p->local_blocks < 2) {
+    int rc = do_pool_append(p, k_cache, v_cache, cache_rows, seq_start, nullptr, seq_len, batch, pooled, nc_cap, 1,
+                            k_new, v_new, at<uint32_t>(ws, l.status), stream);
+    if (!rc) rc = do_block_select(p, q, pooled, nc_cap, seq_len, batch, max_seq_len, nullptr, 0, nullptr, nullptr, 0,
+                                  sel_idx, sel_cnt, ws, ws_bytes, stream);
+    if (!rc) rc = do_sparse_decode(p, q, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len,
+                                   sel_idx, sel_cnt, out, lse, ws, ws_bytes, stream);
+    return rc;
+  }
+  nosa::StepArgs s{};
+  fill_select_args(s.sel, p, q, pooled, nc_cap, seq_len, batch, max_seq_len, nullptr, nullptr, 0, sel_idx, sel_cnt,
+                   ws, l);
+  fill_decode_args(s.dec, p, q, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len, sel_idx,
+                   sel_cnt, out, lse, ws, l);
+  s.pool.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  s.pool.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  s.pool.cache_rows = cache_rows;
+  s.pool.seq_start = seq_start;
+  s.pool.len_old = nullptr;
+  s.pool.len_new = seq_len;
+  s.pool.pooled = pooled;
+  s.pool.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  s.pool.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  s.pool.status = at<uint32_t>(ws, l.status);
+  s.pool.batch = batch;
+  s.pool.hkv = p->num_kv_heads;
+  s.pool.nc_cap = nc_cap;
+  s.pool.max_new_keys = 1;
+  s.work = at<uint32_t>(ws, l.work);
+  s.ready = at<uint32_t>(ws, l.ready);
+  s.mode = nosa::kStepScore | nosa::kStepDecode | nosa::kStepAppend;
+  s.pairs = batch * p->num_kv_heads;
+  s.n_score_items = scoring_items(p, batch, max_seq_len, false);
+  s.n_items = s.n_score_items + s.pairs * s.dec.nsplit;
+  CUtensorMap tm_k, tm_v;
+  if (int rc = encode_kv_map(&tm_k, k_cache, p->num_kv_heads, cache_rows)) return rc;
+  if (int rc = encode_kv_map(&tm_v, v_cache, p->num_kv_heads, cache_rows)) return rc;
+  cudaError_t e = nosa::launch_step(s, tm_k, tm_v, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
   return ok();
 }
 
@@ -364,13 +475,24 @@ int nosa_sparse_decode(const nosa_params* p, const void* q, const void* k_cache,
                           sel_cnt, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+int nosa_decode_step_device(const nosa_params* p, const void* q, const void* k_new, const void* v_new,
+                            void* k_cache, void* v_cache, int64_t cache_rows, const int64_t* seq_start,
+                            const int32_t* seq_len, int batch, int max_seq_len, float* pooled, int nc_cap,
+                            int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* ws, size_t ws_bytes,
+                            void* stream) {
+  if (int rc = check_params(p)) return rc;
+  return do_decode_step_device(p, q, k_new, v_new, k_cache, v_cache, cache_rows, seq_start, seq_len, batch,
+                               max_seq_len, pooled, nc_cap, sel_idx, sel_cnt, out, lse, ws, ws_bytes,
+                               static_cast<cudaStream_t>(stream));
+}
+
 int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new_host,
                      const void* v_new_host, void* out_host, void* k_cache, void* v_cache,
                      int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
                      float* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* ws,
                      size_t ws_bytes, void* stream) {
   if (int rc = check_params(p)) return rc;
-  if (batch < 0 || max_seq_len < 1) return fail(NOSA_ERR_INVALID_ARG, "batch >= 0 and max_seq_len >= 1 required");
+  if (int rc = check_common(p, batch, max_seq_len)) return rc;
   if (batch == 0) return ok();
   if (!q_host || !k_new_host || !v_new_host || !out_host)
     return fail(NOSA_ERR_INVALID_ARG, "host buffers must not be NULL");
@@ -387,14 +509,8 @@ int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new
   if ((e = cudaMemcpyAsync(dq, q_host, qbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy q");
   if ((e = cudaMemcpyAsync(dk, k_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy k_new");
   if ((e = cudaMemcpyAsync(dv, v_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy v_new");
-  int rc = do_pool_append(p, k_cache, v_cache, cache_rows, seq_start, nullptr, seq_len, batch, pooled, nc_cap, 1, dk, dv,
-                          at<uint32_t>(ws, l.status), s);
-  if (rc) return rc;
-  rc = do_block_select(p, dq, pooled, nc_cap, seq_len, batch, max_seq_len, nullptr, 0, nullptr, nullptr, 0,
-                       sel_idx, sel_cnt, ws, ws_bytes, s);
-  if (rc) return rc;
-  rc = do_sparse_decode(p, dq, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len, sel_idx, sel_cnt,
-                        dout, nullptr, ws, ws_bytes, s);
+  int rc = do_decode_step_device(p, dq, dk, dv, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len,
+                                 pooled, nc_cap, sel_idx, sel_cnt, dout, nullptr, ws, ws_bytes, s);
   if (rc) return rc;
   if ((e = cudaMemcpyAsync(out_host, dout, qbytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess) return cuda_fail(e, "copy out");
   return ok();

@@ -22,7 +22,6 @@ constexpr int kBlock = 64;
 constexpr int kWindowsPerBlock = kBlock / kPoolStride;  // 4
 constexpr int kMaxGroup = 16;
 constexpr int kMaxSplits = 64;
-constexpr int kMaxTilesPerSplit = 128;
 constexpr int kMaxLocalBlocks = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint32_t kWaitLimitIters = 1u << 30;

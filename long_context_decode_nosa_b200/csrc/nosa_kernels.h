@@ -56,8 +56,22 @@ struct DecodeArgs {
   uint32_t* tickets; // [pairs]
   uint32_t* status;
   int batch, hq, hkv, group, local_blocks, topk, max_seq_len;
-  int nsplit, tiles_per_split;
+  int nsplit;
   float scale_log2;  // softmax scale * log2(e)
+};
+
+// Work mix of one launch of the persistent step kernel.
+constexpr int kStepScore = 1;   // scoring items (+ top-k of each pair)
+constexpr int kStepDecode = 2;  // decode items
+constexpr int kStepAppend = 4;  // the first scoring item of a pair appends the new token and pools
+
+struct StepArgs {
+  SelectArgs sel;
+  DecodeArgs dec;
+  PoolArgs pool;
+  uint32_t* work;   // [2]: queue position, CTAs finished (zero between launches)
+  uint32_t* ready;  // [pairs]: selection published (zero between launches)
+  int mode, pairs, n_score_items, n_items;
 };
 
 // Launches `kernel` with programmatic stream serialization, so that it can be
@@ -80,12 +94,15 @@ cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 cudaError_t launch_pool_append(const PoolArgs& a, cudaStream_t stream);
-cudaError_t launch_block_select(const SelectArgs& a, cudaStream_t stream);
-cudaError_t launch_sparse_decode(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                 cudaStream_t stream);
+cudaError_t launch_step(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t stream);
+cudaError_t launch_select_only(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint32_t* status, uint32_t max_iters, cudaStream_t stream);
 
-// Number of splits and tiles per split that launch_sparse_decode will use.
-void decode_split_plan(int pairs, int max_tiles, int num_sms, int* nsplit, int* tiles_per_split);
+// CTAs of the step kernel that fit on the current device at once.
+int step_resident_ctas(int group);
+
+// Splits per (sequence, KV head) for the decode items: about one item per
+// resident CTA, at most one per tile and kMaxSplits.
+void decode_split_plan(int pairs, int max_tiles, int num_ctas, int* nsplit);
 
 }  // namespace nosa

@@ -13,21 +13,13 @@
 // no cross-warp ordering is needed.
 #include "nosa_common.cuh"
 #include "nosa_kernels.h"
+#include "pool_device.cuh"
 
 namespace nosa {
 
 namespace {
 
 constexpr int kWarpsPerCta = 4;
-
-__device__ inline float4 bf16x4_to_float4(uint2 raw) {
-  float4 f;
-  f.x = __uint_as_float(raw.x << 16);
-  f.y = __uint_as_float(raw.x & 0xFFFF0000u);
-  f.z = __uint_as_float(raw.y << 16);
-  f.w = __uint_as_float(raw.y & 0xFFFF0000u);
-  return f;
-}
 
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
     pool_append_kernel(const PoolArgs a) {
@@ -38,11 +30,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
   allow_dependents();
   const int32_t len_new = a.len_new[i];
   const int32_t len_old = a.len_old ? a.len_old[i] : len_new - 1;
+  const int64_t base = a.seq_start[i];
   if (len_old < 0 || len_new < len_old) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, NOSA_DEV_BAD_LENGTH);
     return;
   }
-  const int64_t base = a.seq_start[i];
   if (base < 0 || base + len_new > a.cache_rows) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, NOSA_DEV_CACHE_ROWS);
     return;
@@ -71,40 +63,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
     if (lane == 0) set_status(a.status, NOSA_DEV_NC_CAP);
     return;
   }
-  // All 32 row loads are issued before any is consumed (one DRAM round trip,
-  // not 32); rows < len_new exist in the cache, so every load is in bounds.
-  const int64_t t0 = j * kPoolStride;
-  const uint2* src = reinterpret_cast<const uint2*>(a.k_cache + ((base + t0) * a.hkv + h) * kHeadDim) + lane;
-  const int64_t row_stride = static_cast<int64_t>(a.hkv) * kHeadDim / 4;  // in uint2
-  uint2 raw[kPoolKernel];
-#pragma unroll
-  for (int t = 0; t < kPoolKernel; ++t) raw[t] = __ldg(src + t * row_stride);
-  if (append) {
-    const int64_t r = static_cast<int64_t>(len_old) - t0;  // the new token's row inside the window
-    if (r >= 0 && r < kPoolKernel) {
-      const uint2 fresh = knew_row[lane];
-#pragma unroll
-      for (int t = 0; t < kPoolKernel; ++t)
-        if (t == r) raw[t] = fresh;
-    }
-  }
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int t = 0; t < kPoolKernel; ++t) {
-    const float4 f = bf16x4_to_float4(raw[t]);
-    acc.x += f.x;
-    acc.y += f.y;
-    acc.z += f.z;
-    acc.w += f.w;
-  }
-  constexpr float inv = 1.0f / kPoolKernel;
-  acc.x *= inv;
-  acc.y *= inv;
-  acc.z *= inv;
-  acc.w *= inv;
-  float4* dst = reinterpret_cast<float4*>(
-      a.pooled + ((static_cast<int64_t>(i) * a.hkv + h) * a.nc_cap + j) * kHeadDim);
-  dst[lane] = acc;
+  pool_window_warp(a.k_cache, a.hkv, base, h, j, append ? len_old : -1, knew_row,
+                   a.pooled + ((static_cast<int64_t>(i) * a.hkv + h) * a.nc_cap + j) * kHeadDim, lane);
 }
 
 }  // namespace

@@ -1,0 +1,59 @@
+// Per-window CIS mean pooling, shared by the pool-append kernel and the fused
+// decode-step kernel.
+//
+// "从论文到代码：手把手教你理解NOSA-8B的高效注意力机制实现" (nzsm.cn),
+// "NOSA-8B的核心实现模块" item 2; "NOSA-1B 性能基准全解析" (wmrh.cn) §三.3
+// (kernel_size 32, stride 16):  pooled[j] = (1/32) * sum_{t=16j}^{16j+31} K[t].
+#pragma once
+
+#include "nosa_common.cuh"
+
+namespace nosa {
+
+__device__ inline float4 bf16x4_to_float4(uint2 raw) {
+  float4 f;
+  f.x = __uint_as_float(raw.x << 16);
+  f.y = __uint_as_float(raw.x & 0xFFFF0000u);
+  f.z = __uint_as_float(raw.y << 16);
+  f.w = __uint_as_float(raw.y & 0xFFFF0000u);
+  return f;
+}
+
+// One warp pools window j of one (sequence, KV head): lane l owns dims
+// 4l..4l+3.  All 32 rows are loaded before any is summed (one memory round
+// trip); the row of token `fresh_tok` (when >= 0) is taken from `fresh`
+// instead of the cache -- the token being appended by the same launch.  The
+// fp32 sum runs in ascending token order, then x 1/32 (exact), so appending
+// and rebuilding give identical bits.  Rows [16j, 16j+32) must lie inside
+// the cache (the caller checks the sequence against cache_rows).
+__device__ inline void pool_window_warp(const __nv_bfloat16* __restrict__ k_cache, int hkv,
+                                        int64_t seq_base, int h, int64_t j, int64_t fresh_tok,
+                                        const uint2* __restrict__ fresh, float* __restrict__ dst,
+                                        int lane) {
+  const int64_t t0 = j * kPoolStride;
+  const uint2* src = reinterpret_cast<const uint2*>(k_cache + ((seq_base + t0) * hkv + h) * kHeadDim) + lane;
+  const int64_t row_stride = static_cast<int64_t>(hkv) * kHeadDim / 4;  // in uint2
+  uint2 raw[kPoolKernel];
+#pragma unroll
+  for (int t = 0; t < kPoolKernel; ++t) raw[t] = __ldcg(src + t * row_stride);
+  const int64_t r = fresh_tok - t0;
+  if (fresh != nullptr && r >= 0 && r < kPoolKernel) {
+    const uint2 f = fresh[lane];
+#pragma unroll
+    for (int t = 0; t < kPoolKernel; ++t)
+      if (t == r) raw[t] = f;
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int t = 0; t < kPoolKernel; ++t) {
+    const float4 f = bf16x4_to_float4(raw[t]);
+    acc.x += f.x;
+    acc.y += f.y;
+    acc.z += f.z;
+    acc.w += f.w;
+  }
+  constexpr float inv = 1.0f / kPoolKernel;
+  reinterpret_cast<float4*>(dst)[lane] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+}
+
+}  // namespace nosa

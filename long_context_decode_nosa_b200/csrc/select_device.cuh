@@ -1,0 +1,286 @@
+// Compressed scores, block scores and top-k selection: device routines shared
+// by the selection-only kernel and the persistent decode-step kernel.
+//
+// "NOSA-1B 模型家族全景" (demingchina.com), 核心原理: compressed attention
+// screens the history for the TopK blocks; "NOSA-1B 性能基准全解析" (wmrh.cn)
+// §三.2 (block 64, 16 local blocks, TopK 64) and §三.3 (scores of the
+// kernel-32 / stride-16 pooled keys, then TopK).
+//
+//   s[h][j] = scale * q[h] . pooled[j]                        (j < nc)
+//   S[b]    = sum_{h in group, ascending} max_{j in J(b)} s[h][j],
+//             J(b) = {4b-1, ..., 4b+3} n [0, nc)               (b < ncand)
+//   sel     = the min(topk, ncand) largest S, ties to the lower index,
+//             ascending, -1 padded.
+#pragma once
+
+#include "nosa_common.cuh"
+
+namespace nosa {
+
+constexpr int kChunkBlocks = 16;                                     // blocks per scoring item
+constexpr int kChunkWindows = kChunkBlocks * kWindowsPerBlock + 1;   // 65 pooled rows
+constexpr int kScoreStride = 68;                                     // floats per head row
+constexpr int kKeyBytes = kHeadDim * 4;                              // one fp32 pooled key
+constexpr int kScoreKeysBytes = kChunkWindows * kKeyBytes;           // 33,280
+constexpr int kScoreSmemBytes = kScoreKeysBytes + kMaxGroup * kScoreStride * 4;
+
+// Exchange half of `v` (N values) with lane ^ off; keep the half this lane's
+// side owns, added to the partner's copy of it.
+template <int N>
+__device__ inline void xpose_step(float* v, int lane, int off) {
+  const bool upper = (lane & off) != 0;
+#pragma unroll
+  for (int k = 0; k < N / 2; ++k) {
+    const float send = upper ? v[k] : v[k + N / 2];
+    const float keep = upper ? v[k + N / 2] : v[k];
+    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+  }
+}
+
+template <int G>
+__host__ __device__ constexpr int log2_of() {
+  return G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
+}
+
+// Sum over the 32 lanes of v[h] for the head h this lane ends up owning:
+// log2(G) halving exchanges, then 5 - log2(G) plain butterfly steps.
+template <int G>
+__device__ inline float group_warp_sum(float (&v)[G], int lane, int* head) {
+  int h = 0;
+  if constexpr (G >= 2) {
+    xpose_step<G>(v, lane, 16);
+    h += (lane & 16) ? G / 2 : 0;
+  }
+  if constexpr (G >= 4) {
+    xpose_step<G / 2>(v, lane, 8);
+    h += (lane & 8) ? G / 4 : 0;
+  }
+  if constexpr (G >= 8) {
+    xpose_step<G / 4>(v, lane, 4);
+    h += (lane & 4) ? G / 8 : 0;
+  }
+  if constexpr (G >= 16) {
+    xpose_step<G / 8>(v, lane, 2);
+    h += (lane & 2) ? G / 16 : 0;
+  }
+  float s = v[0];
+#pragma unroll
+  for (int o = 16 >> log2_of<G>(); o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  *head = h;
+  return s;
+}
+
+struct TopkShared {
+  uint32_t hist[256];
+  uint32_t warp_eq[32];
+  uint32_t warp_take[32];
+  uint32_t prefix, need, run_eq, run_pos;
+};
+
+// Top-k of `ncand` scores (global; read with ld.global.cg when `coherent`) by
+// NT threads.  Exact 4 x 8-bit radix select of the k-th largest
+// order-preserving key, then an index-ordered ballot compaction: every key
+// above the threshold plus the lowest-index keys equal to it.  Writes the
+// pair's sel_idx row (ascending, -1 padded) and its count.  `ords` is
+// shared memory for ncand keys.
+template <int NT>
+__device__ void select_topk(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
+                            int32_t* sel_cnt, uint32_t* ords, TopkShared& sh) {
+  constexpr int kWarpsNT = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int k_eff = ncand < topk ? ncand : topk;
+  for (int b = tid; b < ncand; b += NT) ords[b] = order_key(coherent ? __ldcg(scores + b) : scores[b]);
+  if (tid == 0) {
+    sh.prefix = 0;
+    sh.need = 0;
+    sh.run_eq = 0;
+    sh.run_pos = 0;
+  }
+  __syncthreads();
+  uint32_t T = 0, need = 0;  // T = 0: take every key (all keys are > 0)
+  if (k_eff < ncand) {
+    uint32_t prefix = 0;
+    need = static_cast<uint32_t>(k_eff);
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
+      for (int t = tid; t < 256; t += NT) sh.hist[t] = 0;
+      __syncthreads();
+      for (int b = tid; b < ncand; b += NT) {
+        const uint32_t key = ords[b];
+        if ((key & hi_mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        uint32_t c[8], sum = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          c[k] = sh.hist[8 * lane + k];
+          sum += c[k];
+        }
+        uint32_t suf = sum;  // sum over lanes >= this lane
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t x = __shfl_down_sync(0xffffffffu, suf, o);
+          if (lane + o < 32) suf += x;
+        }
+        const uint32_t above = suf - sum;
+        if (above < need && need <= suf) {
+          uint32_t acc = above;
+#pragma unroll
+          for (int k = 7; k >= 0; --k) {
+            if (acc + c[k] >= need) {
+              sh.prefix = prefix | (static_cast<uint32_t>(8 * lane + k) << shift);
+              sh.need = need - acc;
+              break;
+            }
+            acc += c[k];
+          }
+        }
+      }
+      __syncthreads();
+      prefix = sh.prefix;
+      need = sh.need;
+    }
+    T = prefix;
+  }
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int base = 0; base < ncand; base += NT) {
+    const int b = base + tid;
+    const uint32_t key = b < ncand ? ords[b] : 0u;
+    const bool gt = b < ncand && key > T;
+    const bool eq = b < ncand && key == T && k_eff < ncand;
+    uint32_t ball = __ballot_sync(0xffffffffu, eq);
+    const uint32_t eq_in_warp = __popc(ball & lt_mask);
+    if (lane == 0) sh.warp_eq[warp] = __popc(ball);
+    __syncthreads();
+    uint32_t eq_before = sh.run_eq + eq_in_warp;
+    for (int w = 0; w < warp; ++w) eq_before += sh.warp_eq[w];
+    const bool take = gt || (eq && eq_before < need);
+    ball = __ballot_sync(0xffffffffu, take);
+    if (lane == 0) sh.warp_take[warp] = __popc(ball);
+    __syncthreads();
+    uint32_t pos = sh.run_pos + __popc(ball & lt_mask);
+    for (int w = 0; w < warp; ++w) pos += sh.warp_take[w];
+    if (take && pos < static_cast<uint32_t>(topk)) sel_row[pos] = b;
+    __syncthreads();
+    if (tid == 0) {
+      for (int w = 0; w < kWarpsNT; ++w) {
+        sh.run_eq += sh.warp_eq[w];
+        sh.run_pos += sh.warp_take[w];
+      }
+    }
+    __syncthreads();
+  }
+  for (int t = k_eff + tid; t < topk; t += NT) sel_row[t] = -1;
+  if (tid == 0) *sel_cnt = k_eff;
+}
+
+struct ScoreGeometry {
+  int L, nb, ncand, nchunks, b0, b1, jlo, jhi;
+  int64_t nc;
+};
+
+// Scores one chunk of 16 blocks of one (sequence i, KV head g) with NT
+// threads: one 1-D bulk (TMA) copy stages the chunk's pooled rows
+// [4*b0-1, 4*b1) in shared memory (`keys`), each warp scores one window at a
+// time with the group's queries in registers, and the block rule runs from
+// shared memory (`ssm`).  Writes block scores to `bscratch` (and the optional
+// outputs).  `bar` is this CTA's key barrier, `phase` its current parity.
+// Returns false when a bounded wait gave up.
+template <int G, int NT>
+__device__ bool score_chunk(const __nv_bfloat16* __restrict__ q, const float* __restrict__ pooled,
+                            int nc_cap, int hq, int hkv, int i, int g, float scale, const ScoreGeometry& geo,
+                            float* __restrict__ bscratch_row, float* __restrict__ comp_out,
+                            float* __restrict__ bs_out_row, uint8_t* smem, uint64_t* bar, uint32_t phase,
+                            uint32_t* status) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* keys = reinterpret_cast<float*>(smem);
+  float* ssm = reinterpret_cast<float*>(smem + kScoreKeysBytes);
+  const int nwin = geo.jhi - geo.jlo;
+  if (geo.b1 <= geo.b0 || nwin <= 0) return true;
+  if (tid == 0) {
+    const uint32_t bytes = static_cast<uint32_t>(nwin) * kKeyBytes;
+    mbar_arrive_expect_tx(bar, bytes);
+    const float* src = pooled + ((static_cast<int64_t>(i) * hkv + g) * nc_cap + geo.jlo) * kHeadDim;
+    bulk_copy_g2s(keys, src, bytes, bar);
+  }
+  // The group's queries, dims 4*lane .. 4*lane+3, widened to fp32.
+  float4 qv[G];
+  const __nv_bfloat16* qbase = q + (static_cast<int64_t>(i) * hq + g * G) * kHeadDim;
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qbase + hh * kHeadDim) + lane);
+    qv[hh] = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                         __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u));
+  }
+  const bool ok = mbar_wait(bar, phase, status);
+  if (ok) {
+    const int writer_mask = 32 / G - 1;
+    for (int jj = warp; jj < nwin; jj += NT / 32) {
+      const float4 kv = reinterpret_cast<const float4*>(keys + jj * kHeadDim)[lane];
+      float v[G];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        float d = qv[hh].x * kv.x;
+        d = fmaf(qv[hh].y, kv.y, d);
+        d = fmaf(qv[hh].z, kv.z, d);
+        d = fmaf(qv[hh].w, kv.w, d);
+        v[hh] = d;
+      }
+      int head;
+      const float s = group_warp_sum<G>(v, lane, &head);
+      if ((lane & writer_mask) == 0) ssm[head * kScoreStride + jj] = s * scale;
+    }
+  }
+  __syncthreads();
+  if (ok) {
+    if (comp_out) {
+      const int jo0 = kWindowsPerBlock * geo.b0, jo1 = geo.jhi;
+      const int span = jo1 - jo0;
+      for (int t = tid; t < G * span; t += NT) {
+        const int hh = t / span, j = jo0 + t % span;
+        comp_out[(static_cast<int64_t>(i) * hq + g * G + hh) * nc_cap + j] = ssm[hh * kScoreStride + (j - geo.jlo)];
+      }
+    }
+    const int bend = min(geo.b1, geo.ncand);
+    for (int t = tid; t < bend - geo.b0; t += NT) {
+      const int b = geo.b0 + t;
+      const int j0 = max(0, kWindowsPerBlock * b - 1);
+      const int j1 = static_cast<int>(geo.nc < kWindowsPerBlock * b + 4 ? geo.nc : kWindowsPerBlock * b + 4);
+      float S = 0.0f;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        float m = -INFINITY;
+        for (int j = j0; j < j1; ++j) m = fmaxf(m, ssm[hh * kScoreStride + (j - geo.jlo)]);
+        S += m;
+      }
+      bscratch_row[b] = S;
+      if (bs_out_row) bs_out_row[b] = S;
+    }
+  }
+  return ok;
+}
+
+// Geometry of scoring item `chunk` of a sequence of length L (L valid).
+// `full` = scores wanted for every window (comp_out) rather than only the
+// windows the selection reads.
+__device__ inline ScoreGeometry score_geometry(int L, int nc_cap, int local_blocks, bool full, int chunk) {
+  ScoreGeometry g;
+  g.L = L;
+  g.nc = n_windows(L);
+  if (g.nc > nc_cap) g.nc = nc_cap;
+  g.nb = static_cast<int>(n_blocks(L));
+  g.ncand = static_cast<int>(n_candidates(L, local_blocks));
+  const int nbw = full ? g.nb : g.ncand;
+  g.nchunks = nbw > 0 ? (nbw + kChunkBlocks - 1) / kChunkBlocks : 1;
+  g.b0 = chunk * kChunkBlocks;
+  g.b1 = min(g.b0 + kChunkBlocks, nbw);
+  g.jlo = max(0, kWindowsPerBlock * g.b0 - 1);
+  const int64_t jh = static_cast<int64_t>(kWindowsPerBlock) * g.b1;
+  g.jhi = static_cast<int>(g.nc < jh ? g.nc : jh);
+  return g;
+}
+
+}  // namespace nosa

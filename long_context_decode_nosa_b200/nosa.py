@@ -68,6 +68,7 @@ _SIGNATURES = {
     "nosa_pool_append": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "nosa_block_select": (_I, [_P, _P, _P, _I, _P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "nosa_sparse_decode": (_I, [_P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "nosa_decode_step_device": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "nosa_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "nosa_read_device_status": (_I, [_P, _SZ, _P]),
     "nosa_last_device_bits": (ctypes.c_uint32, []),
@@ -215,6 +216,27 @@ def nosa_sparse_decode(p: nosa_params, q: torch.Tensor, k_cache: torch.Tensor, v
     _check(rc, "nosa_sparse_decode")
 
 
+def nosa_decode_step_device(p: nosa_params, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                            seq_start: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int,
+                            pooled: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor,
+                            out: torch.Tensor, ws: torch.Tensor, *, k_new: Optional[torch.Tensor] = None,
+                            v_new: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                            stream=None):
+    """Whole decode step on device buffers in one fused launch."""
+    if sel_idx.shape[-1] != p.topk:
+        raise ValueError("sel_idx's last dimension must equal params.topk")
+    batch = seq_len.shape[0]
+    rc = lib().nosa_decode_step_device(
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
+        _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len, _ptr(pooled, torch.float32, "pooled"),
+        pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
+        _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"),
+        ws.numel(), _stream(stream))
+    _check(rc, "nosa_decode_step_device")
+
+
 def nosa_decode_step(p: nosa_params, q_host: torch.Tensor, k_new_host: torch.Tensor,
                      v_new_host: torch.Tensor, out_host: torch.Tensor, k_cache: torch.Tensor,
                      v_cache: torch.Tensor, seq_start: torch.Tensor, seq_len: torch.Tensor,
@@ -271,17 +293,26 @@ class DecodeState:
                          stream=stream)
 
     def step(self, q, k_cache, v_cache, seq_start, seq_len, *, append=True, stream=None,
-             with_lse=False):
-        """One decode step on device-resident inputs: pool the window the newest
-        token completes (when ``append``), select, attend.  Returns ``out``."""
+             with_lse=False, fused=False, k_new=None, v_new=None):
+        """One decode step on device-resident inputs: (when ``append``) write the
+        new token's K/V rows if given and pool the window the newest token
+        completes, then select and attend.  ``fused`` runs it as one launch.
+        Returns ``out``."""
+        lse = self.lse if with_lse else None
+        if fused:
+            if not append:
+                raise ValueError("the fused step always pools the newest token's window")
+            nosa_decode_step_device(self.p, q, k_cache, v_cache, seq_start, seq_len, self.max_seq_len,
+                                    self.pooled, self.sel_idx, self.sel_cnt, self.out, self.ws,
+                                    k_new=k_new, v_new=v_new, lse=lse, stream=stream)
+            return self.out
         if append:
             nosa_pool_append(self.p, k_cache, v_cache, seq_start, seq_len, self.pooled,
-                             max_new_keys=1, ws=self.ws, stream=stream)
+                             max_new_keys=1, k_new=k_new, v_new=v_new, ws=self.ws, stream=stream)
         nosa_block_select(self.p, q, self.pooled, seq_len, self.max_seq_len, self.sel_idx,
                           self.sel_cnt, self.ws, stream=stream)
         nosa_sparse_decode(self.p, q, k_cache, v_cache, seq_start, seq_len, self.max_seq_len,
-                           self.sel_idx, self.sel_cnt, self.out, self.ws,
-                           lse=self.lse if with_lse else None, stream=stream)
+                           self.sel_idx, self.sel_cnt, self.out, self.ws, lse=lse, stream=stream)
         return self.out
 
 
