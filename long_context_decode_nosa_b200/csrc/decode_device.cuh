@@ -117,6 +117,10 @@ struct DecodeShared {
   uint64_t empty_bar[kStages];
   int stage_blk[kStages];
   int last;
+#ifdef NOSA_TRACE
+  uint64_t t_flag;  // instrumented builds: when the producer saw the selection
+  uint64_t t_issue[8], t_full[8], t_done[8];  // per tile: TMA issued, landed, consumed (warp 0)
+#endif
 };
 
 // One decode item with 160 threads (4 consumer warps + 1 producer warp).
@@ -183,6 +187,9 @@ __device__ inline void decode_item(const DecodeArgs& a, const CUtensorMap* tm_k,
         if (!have_sel && t >= n_local - 1) {
           sel_ok = wait_ready(ready, a.status);
           have_sel = true;
+#ifdef NOSA_TRACE
+          sh.t_flag = global_timer_ns();
+#endif
           if (sel_ok && __ldcg(a.sel_cnt + pair) != cnt) set_status(a.status, NOSA_DEV_BAD_COUNT);
         }
         int blk;
@@ -208,6 +215,9 @@ __device__ inline void decode_item(const DecodeArgs& a, const CUtensorMap* tm_k,
         tma_load_box(st + kHalfBytes, tm_k, 64, g, row, &sh.full_bar[s]);
         tma_load_box(st + 2 * kHalfBytes, tm_v, 0, g, row, &sh.full_bar[s]);
         tma_load_box(st + 3 * kHalfBytes, tm_v, 64, g, row, &sh.full_bar[s]);
+#ifdef NOSA_TRACE
+        if (n < 8) sh.t_issue[n] = global_timer_ns();
+#endif
         issued = n + 1;
       }
       // Every copy issued has landed before shared memory is reused.
@@ -236,6 +246,9 @@ __device__ inline void decode_item(const DecodeArgs& a, const CUtensorMap* tm_k,
       const uint32_t r = ring_n + static_cast<uint32_t>(n);
       const int s = static_cast<int>(r % kStages);
       if (!mbar_wait(&sh.full_bar[s], (r / kStages) & 1u, a.status)) break;
+#ifdef NOSA_TRACE
+      if (warp == 0 && lane == 0 && n < 8) sh.t_full[n] = global_timer_ns();
+#endif
       const int blk = sh.stage_blk[s];
       uint8_t* st = smem + s * kStageBytes;
       const uint32_t k_lo = smem_addr(st);
@@ -324,6 +337,9 @@ __device__ inline void decode_item(const DecodeArgs& a, const CUtensorMap* tm_k,
       if (partial) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
+#ifdef NOSA_TRACE
+      if (warp == 0 && lane == 0 && n < 8) sh.t_done[n] = global_timer_ns();
+#endif
     }
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {

@@ -26,6 +26,19 @@
 
 namespace nosa {
 
+#ifdef NOSA_TRACE
+// Instrumented builds only (-DNOSA_TRACE): one record per work item of the
+// step kernel -- CTA, SM, item, start / selection-seen / end globaltimer.
+struct TraceRecord {
+  uint32_t cta, smid, item, pad;
+  uint64_t t_start, t_flag, t_end;
+  uint32_t issue[8], full[8], done[8];  // per tile, ns after t_start
+};
+constexpr int kTraceCapacity = 1 << 16;
+__device__ TraceRecord g_trace[kTraceCapacity];
+__device__ uint32_t g_trace_count;
+#endif
+
 namespace {
 
 constexpr int kSelOnlyThreads = 256;
@@ -142,6 +155,12 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_k) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_v) : "memory");
   }
+#ifdef NOSA_TRACE
+  if (tid == 0) {
+    dsh.t_flag = 0;
+    for (int n = 0; n < 8; ++n) dsh.t_issue[n] = dsh.t_full[n] = dsh.t_done[n] = 0;
+  }
+#endif
   grid_dependency_wait();
   allow_dependents();
   __syncthreads();
@@ -151,6 +170,9 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     __syncthreads();
     const int item = sh_item;
     if (item >= a.n_items) break;
+#ifdef NOSA_TRACE
+    const uint64_t tr_start = global_timer_ns();
+#endif
     if (item < a.n_score_items) {
       score_item<G>(a, item, smem, &key_bar, key_phase, tsh, &sh_last);
     } else {
@@ -161,6 +183,24 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     // Shared memory written by this item's threads may next be written by TMA.
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
+#ifdef NOSA_TRACE
+    if (tid == 0) {
+      const uint32_t k = atomicAdd(&g_trace_count, 1u);
+      if (k < kTraceCapacity) {
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        TraceRecord rec{blockIdx.x, smid, static_cast<uint32_t>(item), 0u, tr_start, dsh.t_flag, global_timer_ns()};
+        for (int n = 0; n < 8; ++n) {
+          rec.issue[n] = dsh.t_issue[n] ? static_cast<uint32_t>(dsh.t_issue[n] - tr_start) : 0u;
+          rec.full[n] = dsh.t_full[n] ? static_cast<uint32_t>(dsh.t_full[n] - tr_start) : 0u;
+          rec.done[n] = dsh.t_done[n] ? static_cast<uint32_t>(dsh.t_done[n] - tr_start) : 0u;
+          dsh.t_issue[n] = dsh.t_full[n] = dsh.t_done[n] = 0;
+        }
+        g_trace[k] = rec;
+      }
+      dsh.t_flag = 0;
+    }
+#endif
   }
   if (tid == 0) {
     __threadfence();
@@ -271,6 +311,19 @@ void decode_split_plan(int pairs, int max_tiles, int num_ctas, int* nsplit) {
   if (ns < 1) ns = 1;
   *nsplit = ns;
 }
+
+#ifdef NOSA_TRACE
+extern "C" __attribute__((visibility("default"))) int nosa_trace_read(void* host, int max_records) {
+  uint32_t n = 0;
+  if (cudaMemcpyFromSymbol(&n, g_trace_count, sizeof n) != cudaSuccess) return -1;
+  if (n > static_cast<uint32_t>(max_records)) n = static_cast<uint32_t>(max_records);
+  if (n > kTraceCapacity) n = kTraceCapacity;
+  if (n && cudaMemcpyFromSymbol(host, g_trace, n * sizeof(TraceRecord)) != cudaSuccess) return -1;
+  const uint32_t zero = 0;
+  cudaMemcpyToSymbol(g_trace_count, &zero, sizeof zero);
+  return static_cast<int>(n);
+}
+#endif
 
 cudaError_t launch_wait_selftest(uint32_t* status, uint32_t max_iters, cudaStream_t stream) {
   wait_selftest_kernel<<<1, 32, 0, stream>>>(status, max_iters);
