@@ -202,6 +202,35 @@ NOSA_API int nosa_decode_step_device(const nosa_params* p, const void* q, const 
                                      int32_t* sel_cnt, void* out, float* lse, void* ws,
                                      size_t ws_bytes, void* stream);
 
+/* The fused decode step for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a deployment variant of
+ * nosa_decode_step_device.  Some callers cannot provide a workspace -- a
+ * plugin inside an inference engine whose memory manager owns the whole
+ * device pool and offers no workspace hook, or a serving loop that must not
+ * call cudaMalloc once the KV cache has taken the free memory.  This entry
+ * point takes the same arguments without `ws` and keeps its scratch in an
+ * 8 MiB array that the library defines in device memory (every GPU that loads
+ * the library holds it until the process exits).  It allocates nothing and
+ * calls no allocating routine.
+ *  * A batch whose nosa_workspace_size exceeds 8 MiB is rejected with
+ *    NOSA_ERR_WORKSPACE (nothing is enqueued); use nosa_decode_step_device.
+ *  * The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  * Every call on a device shares the one array: the call clears its
+ *    counters and flags first (asynchronously, on `stream`), but calls that
+ *    overlap on the GPU race.  Order them on one stream.
+ *  * Device-side data checks land in the array's status word, which no entry
+ *    point reads back; callers that need those reports use the workspace
+ *    variant and nosa_read_device_status. */
+NOSA_API int nosa_decode_step_device_noalloc(const nosa_params* p, const void* q,
+                                             const void* k_new, const void* v_new,
+                                             void* k_cache, void* v_cache, int64_t cache_rows,
+                                             const int64_t* seq_start, const int32_t* seq_len,
+                                             int batch, int max_seq_len, float* pooled,
+                                             int nc_cap, int32_t* sel_idx, int32_t* sel_cnt,
+                                             void* out, float* lse, void* stream);
+
 /* One whole decode step from HOST buffers (the pages' per-token decode,
  * steps 1-4 above in order): copies q_host (bf16 [batch, Hq, D]) and the new
  * token's k_new_host / v_new_host (bf16 [batch, Hkv, D]) to the device,

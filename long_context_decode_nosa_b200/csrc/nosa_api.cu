@@ -414,6 +414,17 @@ int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new
 
 }  // namespace
 
+namespace nosa {
+
+size_t workspace_counter_bytes(const nosa_params* p, int batch, int max_seq_len) {
+  if (check_params(p) != NOSA_OK || batch < 0 || max_seq_len < 1) return 0;
+  return layout_of(p, batch, max_seq_len).bscores;
+}
+
+int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
+}  // namespace nosa
+
 extern "C" {
 
 void nosa_default_params(nosa_params* p) {

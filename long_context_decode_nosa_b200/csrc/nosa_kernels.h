@@ -8,6 +8,8 @@
 
 #include <utility>
 
+#include "nosa.h"
+
 namespace nosa {
 
 struct PoolArgs {
@@ -97,6 +99,13 @@ cudaError_t launch_pool_append(const PoolArgs& a, cudaStream_t stream);
 cudaError_t launch_step(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t stream);
 cudaError_t launch_select_only(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint32_t* status, uint32_t max_iters, cudaStream_t stream);
+
+// Bytes at the start of a workspace that must be zero before a call
+// (status word, work queue, tickets, ready flags); 0 for invalid parameters.
+size_t workspace_counter_bytes(const nosa_params* p, int batch, int max_seq_len);
+
+// Records `msg` as the calling thread's last error and returns `code`.
+int record_error(int code, const char* msg);
 
 // CTAs of the step kernel that fit on the current device at once.
 int step_resident_ctas(int group);

@@ -69,6 +69,7 @@ _SIGNATURES = {
     "nosa_block_select": (_I, [_P, _P, _P, _I, _P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "nosa_sparse_decode": (_I, [_P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "nosa_decode_step_device": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "nosa_decode_step_device_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
     "nosa_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "nosa_read_device_status": (_I, [_P, _SZ, _P]),
     "nosa_last_device_bits": (ctypes.c_uint32, []),
@@ -235,6 +236,27 @@ def nosa_decode_step_device(p: nosa_params, q: torch.Tensor, k_cache: torch.Tens
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"),
         ws.numel(), _stream(stream))
     _check(rc, "nosa_decode_step_device")
+
+
+def nosa_decode_step_device_noalloc(p: nosa_params, q: torch.Tensor, k_cache: torch.Tensor,
+                                    v_cache: torch.Tensor, seq_start: torch.Tensor, seq_len: torch.Tensor,
+                                    max_seq_len: int, pooled: torch.Tensor, sel_idx: torch.Tensor,
+                                    sel_cnt: torch.Tensor, out: torch.Tensor, *,
+                                    k_new: Optional[torch.Tensor] = None, v_new: Optional[torch.Tensor] = None,
+                                    lse: Optional[torch.Tensor] = None, stream=None):
+    """The fused decode step without a workspace: its scratch is the library's
+    own fixed device array (for callers that cannot allocate device memory)."""
+    if sel_idx.shape[-1] != p.topk:
+        raise ValueError("sel_idx's last dimension must equal params.topk")
+    batch = seq_len.shape[0]
+    rc = lib().nosa_decode_step_device_noalloc(
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
+        _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len, _ptr(pooled, torch.float32, "pooled"),
+        pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
+        _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _stream(stream))
+    _check(rc, "nosa_decode_step_device_noalloc")
 
 
 def nosa_decode_step(p: nosa_params, q_host: torch.Tensor, k_new_host: torch.Tensor,
