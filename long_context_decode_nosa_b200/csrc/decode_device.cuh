@@ -76,13 +76,14 @@ __device__ inline uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// 3-D tiled TMA load of one {64 dims, 1 head, 64 tokens} box, completing on `bar`.
+// 3-D tiled TMA load of one {64 dims, 1 head, 64 tokens} box, completing on
+// `bar`, with the given L2 cache policy.
 __device__ inline void tma_load_box(void* dst, const CUtensorMap* map, int dim0, int head, int row,
-                                    uint64_t* bar) {
+                                    uint64_t* bar, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
-      "l"(map), "r"(dim0), "r"(head), "r"(row), "r"(smem_addr(bar))
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(dim0), "r"(head), "r"(row), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
 }
 
@@ -105,18 +106,21 @@ __device__ inline bool wait_ready(const uint32_t* flag, uint32_t* status) {
       asm volatile("fence.proxy.async.global;" ::: "memory");
       return true;
     }
-    __nanosleep(64);
+    __nanosleep(200);
     if ((it & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) break;
   }
   set_status(status, NOSA_DEV_TIMEOUT);
   return false;
 }
 
+constexpr int kSelList = 128;  // selected block indices a split stages in shared memory
+
 struct DecodeShared {
   uint64_t full_bar[kStages];
   uint64_t empty_bar[kStages];
   int stage_blk[kStages];
   int last;
+  int sel_list[kSelList];
 #ifdef NOSA_TRACE
   uint64_t t_flag;  // instrumented builds: when the producer saw the selection
   uint64_t t_issue[8], t_full[8], t_done[8];  // per tile: TMA issued, landed, consumed (warp 0)
@@ -176,28 +180,48 @@ __device__ inline void decode_item(const DecodeArgs& a, const CUtensorMap* tm_k,
 
   if (warp == kDecConsumerWarps) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      bool have_sel = ready == nullptr;
-      bool sel_ok = have_sel;
-      int issued = 0;
-      for (int n = 0; n < my_n; ++n) {
-        const int t = t_begin + n;
-        // The selected tiles and the last local block (it holds the token
-        // appended by this launch) wait for the pair's selection flag.
-        if (!have_sel && t >= n_local - 1) {
-          sel_ok = wait_ready(ready, a.status);
-          have_sel = true;
+    // The whole warp walks the tiles; lane 0 waits and issues the copies.
+    // Once the selection is known, the warp fetches this split's selected
+    // block indices into shared memory in one parallel round trip.
+    const uint64_t policy = l2_evict_first_policy();
+    const int first_sel = max(t_begin, n_local);
+    const int n_sel = max(0, t_end - first_sel);
+    bool have_sel = ready == nullptr;
+    bool sel_ok = have_sel;
+    auto load_sel_list = [&]() {
+      for (int x = lane; x < min(n_sel, kSelList); x += 32) sh.sel_list[x] = __ldcg(sel + (first_sel - n_local) + x);
+      __syncwarp();
+    };
+    if (have_sel) load_sel_list();
+    int issued = 0;
+    for (int n = 0; n < my_n; ++n) {
+      const int t = t_begin + n;
+      // The selected tiles and the last local block (it holds the token
+      // appended by this launch) wait for the pair's selection flag.
+      if (!have_sel && t >= n_local - 1) {
+        int ok = 0;
+        if (lane == 0) {
+          ok = wait_ready(ready, a.status) ? 1 : 0;
 #ifdef NOSA_TRACE
           sh.t_flag = global_timer_ns();
 #endif
-          if (sel_ok && __ldcg(a.sel_cnt + pair) != cnt) set_status(a.status, NOSA_DEV_BAD_COUNT);
+          if (ok && __ldcg(a.sel_cnt + pair) != cnt) set_status(a.status, NOSA_DEV_BAD_COUNT);
         }
+        sel_ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+        have_sel = true;
+        if (sel_ok) load_sel_list();
+      }
+      int stop = 0;
+      if (lane == 0) {
         int blk;
         if (t < n_local) {
           blk = ncand + t;
+        } else if (!sel_ok) {
+          blk = -1;
         } else {
-          blk = sel_ok ? __ldcg(sel + (t - n_local)) : -1;
-          if (sel_ok && (blk < 0 || blk >= ncand)) {
+          const int x = t - first_sel;
+          blk = x < kSelList ? sh.sel_list[x] : __ldcg(sel + (t - n_local));
+          if (blk < 0 || blk >= ncand) {
             set_status(a.status, NOSA_DEV_BAD_INDEX);
             blk = -1;
           }
@@ -205,22 +229,27 @@ __device__ inline void decode_item(const DecodeArgs& a, const CUtensorMap* tm_k,
         const uint32_t r = ring_n + static_cast<uint32_t>(n);
         const int s = static_cast<int>(r % kStages);
         if (r >= static_cast<uint32_t>(kStages) &&
-            !mbar_wait(&sh.empty_bar[s], ((r / kStages) - 1) & 1u, a.status))
-          break;
-        sh.stage_blk[s] = blk;
-        const int row = static_cast<int>(seq_base + (blk < 0 ? 0 : static_cast<int64_t>(blk) * kBlock));
-        uint8_t* st = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(&sh.full_bar[s], kTileTxBytes);
-        tma_load_box(st, tm_k, 0, g, row, &sh.full_bar[s]);
-        tma_load_box(st + kHalfBytes, tm_k, 64, g, row, &sh.full_bar[s]);
-        tma_load_box(st + 2 * kHalfBytes, tm_v, 0, g, row, &sh.full_bar[s]);
-        tma_load_box(st + 3 * kHalfBytes, tm_v, 64, g, row, &sh.full_bar[s]);
+            !mbar_wait(&sh.empty_bar[s], ((r / kStages) - 1) & 1u, a.status)) {
+          stop = 1;
+        } else {
+          sh.stage_blk[s] = blk;
+          const int row = static_cast<int>(seq_base + (blk < 0 ? 0 : static_cast<int64_t>(blk) * kBlock));
+          uint8_t* st = smem + s * kStageBytes;
+          mbar_arrive_expect_tx(&sh.full_bar[s], kTileTxBytes);
+          tma_load_box(st, tm_k, 0, g, row, &sh.full_bar[s], policy);
+          tma_load_box(st + kHalfBytes, tm_k, 64, g, row, &sh.full_bar[s], policy);
+          tma_load_box(st + 2 * kHalfBytes, tm_v, 0, g, row, &sh.full_bar[s], policy);
+          tma_load_box(st + 3 * kHalfBytes, tm_v, 64, g, row, &sh.full_bar[s], policy);
 #ifdef NOSA_TRACE
-        if (n < 8) sh.t_issue[n] = global_timer_ns();
+          if (n < 8) sh.t_issue[n] = global_timer_ns();
 #endif
-        issued = n + 1;
+          issued = n + 1;
+        }
       }
-      // Every copy issued has landed before shared memory is reused.
+      if (__shfl_sync(0xffffffffu, stop, 0)) break;
+    }
+    // Every copy issued has landed before shared memory is reused.
+    if (lane == 0) {
       for (int n = max(0, issued - kStages); n < issued; ++n) {
         const uint32_t r = ring_n + static_cast<uint32_t>(n);
         mbar_wait(&sh.full_bar[r % kStages], (r / kStages) & 1u, a.status);

@@ -73,40 +73,54 @@ __device__ inline void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-__device__ inline bool mbar_test_parity(uint64_t* bar, uint32_t parity) {
+// Tests whether the phase with the given parity has completed.  A waiting
+// thread is suspended (it takes no issue slots) until the phase completes
+// or `suspend_ns` pass, so polling warps do not slow down the other warps
+// of their SM.
+__device__ inline bool mbar_test_parity(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(suspend_ns)
       : "memory");
   return done != 0;
 }
 
 // Waits until the phase with the given parity has completed.  Bounded by
-// `max_iters` polls and kWaitLimitNs of wall time; on giving up it sets
-// NOSA_DEV_TIMEOUT and returns false.
+// `max_iters` suspended polls of at most `suspend_ns` each and by
+// kWaitLimitNs of wall time; on giving up it sets NOSA_DEV_TIMEOUT and
+// returns false.
 __device__ inline bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                 uint32_t max_iters = kWaitLimitIters) {
-  if (mbar_test_parity(bar, parity)) return true;
+                                 uint32_t max_iters = kWaitLimitIters, uint32_t suspend_ns = 100000u) {
+  if (mbar_test_parity(bar, parity, suspend_ns)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1; it < max_iters; ++it) {
-    if (mbar_test_parity(bar, parity)) return true;
-    if ((it & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) break;
+    if (mbar_test_parity(bar, parity, suspend_ns)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) break;
   }
   set_status(status, NOSA_DEV_TIMEOUT);
   return false;
 }
 
-// 1-D bulk copy global -> shared through the TMA unit, completing on `bar`.
-// dst, src and bytes must be multiples of 16.
+// L2 policy for data read once per step (KV tiles, pooled keys): evict it
+// first, so streaming it does not push the kernels' code and small metadata
+// out of L2.
+__device__ inline uint64_t l2_evict_first_policy() {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  return policy;
+}
+
+// 1-D bulk copy global -> shared through the TMA unit, completing on `bar`,
+// with the evict-first L2 policy.  dst, src and bytes must be multiples of 16.
 __device__ inline void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
           smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(l2_evict_first_policy())
       : "memory");
 }
 

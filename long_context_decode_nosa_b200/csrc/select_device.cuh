@@ -77,17 +77,81 @@ struct TopkShared {
   uint32_t prefix, need, run_eq, run_pos;
 };
 
+// Exact top-k by one warp, for up to 32 * KPL candidates (candidate b lives
+// in lane b % 32, register b / 32).  The k-th largest order-preserving key T
+// is found bit by bit from the top (T = the largest value with at least k
+// keys >= T; each step counts with ballots), then an index-ordered ballot
+// compaction writes every key above T plus the lowest-index keys equal to T.
+// No block-wide barriers; the other warps are not involved.
+template <int KPL>
+__device__ void warp_topk(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
+                          int32_t* sel_cnt, int lane) {
+  const int k_eff = ncand < topk ? ncand : topk;
+  uint32_t key[KPL];
+#pragma unroll
+  for (int m = 0; m < KPL; ++m) {
+    const int b = m * 32 + lane;
+    key[m] = b < ncand ? order_key(coherent ? __ldcg(scores + b) : scores[b]) : 0u;  // valid keys are > 0
+  }
+  uint32_t T = 0u;
+  int need = 0;
+  if (k_eff < ncand) {
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      int c = 0;
+#pragma unroll
+      for (int m = 0; m < KPL; ++m) c += __popc(__ballot_sync(0xffffffffu, key[m] >= cand));
+      if (c >= k_eff) T = cand;
+    }
+    int above = 0;
+#pragma unroll
+    for (int m = 0; m < KPL; ++m) above += __popc(__ballot_sync(0xffffffffu, key[m] > T));
+    need = k_eff - above;
+  }
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int eq_seen = 0, pos = 0;
+#pragma unroll
+  for (int m = 0; m < KPL; ++m) {
+    const int b = m * 32 + lane;
+    const bool valid = b < ncand;
+    const bool eq = valid && k_eff < ncand && key[m] == T;
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    const bool take = valid && (key[m] > T || (eq && eq_seen + __popc(eb & lt_mask) < need));
+    const uint32_t tb = __ballot_sync(0xffffffffu, take);
+    const int p = pos + __popc(tb & lt_mask);
+    if (take && p < topk) sel_row[p] = b;
+    eq_seen += __popc(eb);
+    pos += __popc(tb);
+  }
+  for (int t = k_eff + lane; t < topk; t += 32) sel_row[t] = -1;
+  if (lane == 0) *sel_cnt = k_eff;
+}
+
+// Candidates up to which one warp selects (warp_topk); larger sets use the
+// block-wide radix select.
+constexpr int kWarpTopkMax = 1024;
+
 // Top-k of `ncand` scores (global; read with ld.global.cg when `coherent`) by
-// NT threads.  Exact 4 x 8-bit radix select of the k-th largest
-// order-preserving key, then an index-ordered ballot compaction: every key
-// above the threshold plus the lowest-index keys equal to it.  Writes the
-// pair's sel_idx row (ascending, -1 padded) and its count.  `ords` is
-// shared memory for ncand keys.
+// NT threads: one warp (warp_topk) for up to kWarpTopkMax candidates, else an
+// exact 4 x 8-bit radix select of the k-th largest order-preserving key and
+// an index-ordered ballot compaction (every key above it plus the
+// lowest-index keys equal to it).  Writes the pair's sel_idx row (ascending,
+// -1 padded) and its count.  `ords` is shared memory for ncand keys.
 template <int NT>
 __device__ void select_topk(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
                             int32_t* sel_cnt, uint32_t* ords, TopkShared& sh) {
   constexpr int kWarpsNT = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (ncand <= kWarpTopkMax) {
+    if (warp == 0) {
+      if (ncand <= 256)
+        warp_topk<8>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
+      else
+        warp_topk<32>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
+    }
+    return;
+  }
   const int k_eff = ncand < topk ? ncand : topk;
   for (int b = tid; b < ncand; b += NT) ords[b] = order_key(coherent ? __ldcg(scores + b) : scores[b]);
   if (tid == 0) {
@@ -194,7 +258,7 @@ __device__ bool score_chunk(const __nv_bfloat16* __restrict__ q, const float* __
                             int nc_cap, int hq, int hkv, int i, int g, float scale, const ScoreGeometry& geo,
                             float* __restrict__ bscratch_row, float* __restrict__ comp_out,
                             float* __restrict__ bs_out_row, uint8_t* smem, uint64_t* bar, uint32_t phase,
-                            uint32_t* status) {
+                            uint32_t* status, uint64_t* trace_landed = nullptr) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float* keys = reinterpret_cast<float*>(smem);
   float* ssm = reinterpret_cast<float*>(smem + kScoreKeysBytes);
@@ -216,22 +280,35 @@ __device__ bool score_chunk(const __nv_bfloat16* __restrict__ q, const float* __
                          __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u));
   }
   const bool ok = mbar_wait(bar, phase, status);
+#ifdef NOSA_TRACE
+  if (tid == 0 && trace_landed) *trace_landed = global_timer_ns();
+#endif
   if (ok) {
+    // Four windows per warp and iteration: four independent reduction chains
+    // keep the shuffle pipeline busy.
+    constexpr int kWin = 4;
     const int writer_mask = 32 / G - 1;
-    for (int jj = warp; jj < nwin; jj += NT / 32) {
-      const float4 kv = reinterpret_cast<const float4*>(keys + jj * kHeadDim)[lane];
-      float v[G];
+    for (int j0 = warp * kWin; j0 < nwin; j0 += (NT / 32) * kWin) {
+      float v[kWin][G];
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        float d = qv[hh].x * kv.x;
-        d = fmaf(qv[hh].y, kv.y, d);
-        d = fmaf(qv[hh].z, kv.z, d);
-        d = fmaf(qv[hh].w, kv.w, d);
-        v[hh] = d;
+      for (int w = 0; w < kWin; ++w) {
+        const int jj = min(j0 + w, nwin - 1);
+        const float4 kv = reinterpret_cast<const float4*>(keys + jj * kHeadDim)[lane];
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          float d = qv[hh].x * kv.x;
+          d = fmaf(qv[hh].y, kv.y, d);
+          d = fmaf(qv[hh].z, kv.z, d);
+          d = fmaf(qv[hh].w, kv.w, d);
+          v[w][hh] = d;
+        }
       }
-      int head;
-      const float s = group_warp_sum<G>(v, lane, &head);
-      if ((lane & writer_mask) == 0) ssm[head * kScoreStride + jj] = s * scale;
+#pragma unroll
+      for (int w = 0; w < kWin; ++w) {
+        int head;
+        const float s = group_warp_sum<G>(v[w], lane, &head);
+        if ((lane & writer_mask) == 0 && j0 + w < nwin) ssm[head * kScoreStride + j0 + w] = s * scale;
+      }
     }
   }
   __syncthreads();
@@ -247,13 +324,18 @@ __device__ bool score_chunk(const __nv_bfloat16* __restrict__ q, const float* __
     const int bend = min(geo.b1, geo.ncand);
     for (int t = tid; t < bend - geo.b0; t += NT) {
       const int b = geo.b0 + t;
-      const int j0 = max(0, kWindowsPerBlock * b - 1);
-      const int j1 = static_cast<int>(geo.nc < kWindowsPerBlock * b + 4 ? geo.nc : kWindowsPerBlock * b + 4);
+      // J(b) = {4b-1, ..., 4b+3} clipped to [0, nc): a fixed 5-step loop with
+      // predication keeps the shared-memory loads independent.
+      const int jb = kWindowsPerBlock * b - 1;
       float S = 0.0f;
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
         float m = -INFINITY;
-        for (int j = j0; j < j1; ++j) m = fmaxf(m, ssm[hh * kScoreStride + (j - geo.jlo)]);
+#pragma unroll
+        for (int w = 0; w < kWindowsPerBlock + 1; ++w) {
+          const int j = jb + w;
+          if (j >= 0 && j < geo.nc) m = fmaxf(m, ssm[hh * kScoreStride + (j - geo.jlo)]);
+        }
         S += m;
       }
       bscratch_row[b] = S;

@@ -30,7 +30,7 @@ namespace nosa {
 // Instrumented builds only (-DNOSA_TRACE): one record per work item of the
 // step kernel -- CTA, SM, item, start / selection-seen / end globaltimer.
 struct TraceRecord {
-  uint32_t cta, smid, item, pad;
+  uint32_t cta, smid, item, clk_delta;  // clk_delta: SM clock cycles spent in the item
   uint64_t t_start, t_flag, t_end;
   uint32_t issue[8], full[8], done[8];  // per tile, ns after t_start
 };
@@ -80,14 +80,26 @@ __device__ void append_and_pool(const PoolArgs& p, int pair, int L) {
   }
 }
 
+#ifdef NOSA_TRACE
+#define NOSA_STAMP(slot)                                      \
+  do {                                                        \
+    if (threadIdx.x == 0) stamps[slot] = global_timer_ns();   \
+  } while (0)
+#else
+#define NOSA_STAMP(slot) \
+  do {                   \
+  } while (0)
+#endif
+
 template <int G>
 __device__ void score_item(const StepArgs& a, int item, uint8_t* smem, uint64_t* key_bar, uint32_t& key_phase,
-                           TopkShared& tsh, int* sh_last) {
+                           TopkShared& tsh, int* sh_last, uint64_t* stamps) {
   const SelectArgs& s = a.sel;
   const int pair = item % a.pairs, chunk = item / a.pairs;
   const int i = pair / s.hkv, g = pair % s.hkv;
   const int tid = threadIdx.x;
   const int L = s.seq_len[i];
+  NOSA_STAMP(0);
   if (L < 1 || L > s.max_seq_len) {
     if (chunk == 0) {
       if (tid == 0) set_status(s.status, L < 1 ? NOSA_DEV_BAD_LENGTH : NOSA_DEV_MAX_LEN);
@@ -103,15 +115,17 @@ __device__ void score_item(const StepArgs& a, int item, uint8_t* smem, uint64_t*
   score_chunk<G, kDecThreads>(s.q, s.pooled, s.nc_cap, s.hq, s.hkv, i, g, s.scale, geo,
                               s.bscratch + static_cast<int64_t>(pair) * s.nb_ws, s.comp_out,
                               s.bs_out ? s.bs_out + static_cast<int64_t>(pair) * s.nb_out : nullptr, smem, key_bar,
-                              key_phase, s.status);
+                              key_phase, s.status, stamps ? stamps + 1 : nullptr);
   if (uses_keys) key_phase ^= 1u;
   __syncthreads();
+  NOSA_STAMP(2);
   if (tid == 0) {
     __threadfence();
     const uint32_t t = atomicAdd(&s.tickets[pair], 1u);
     *sh_last = (t == static_cast<uint32_t>(geo.nchunks - 1));
   }
   __syncthreads();
+  NOSA_STAMP(3);
   if (!*sh_last) return;
   __threadfence();
   // The pair's last chunk: every block score is written; select.
@@ -120,6 +134,7 @@ __device__ void score_item(const StepArgs& a, int item, uint8_t* smem, uint64_t*
                            s.sel_idx + static_cast<int64_t>(pair) * s.topk, s.sel_cnt + pair,
                            reinterpret_cast<uint32_t*>(smem), tsh);
   __syncthreads();
+  NOSA_STAMP(4);
   if (tid == 0) {
     s.tickets[pair] = 0u;
     if (a.mode & kStepDecode) {
@@ -172,9 +187,14 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     if (item >= a.n_items) break;
 #ifdef NOSA_TRACE
     const uint64_t tr_start = global_timer_ns();
+    const long long tr_clk0 = clock64();
 #endif
     if (item < a.n_score_items) {
-      score_item<G>(a, item, smem, &key_bar, key_phase, tsh, &sh_last);
+#ifdef NOSA_TRACE
+      score_item<G>(a, item, smem, &key_bar, key_phase, tsh, &sh_last, dsh.t_issue);
+#else
+      score_item<G>(a, item, smem, &key_bar, key_phase, tsh, &sh_last, nullptr);
+#endif
     } else {
       const int d = item - a.n_score_items;
       decode_item(a.dec, &tm_k, &tm_v, d % a.pairs, d / a.pairs, (a.mode & kStepScore) ? a.ready + d % a.pairs : nullptr,
@@ -189,7 +209,8 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
       if (k < kTraceCapacity) {
         uint32_t smid;
         asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-        TraceRecord rec{blockIdx.x, smid, static_cast<uint32_t>(item), 0u, tr_start, dsh.t_flag, global_timer_ns()};
+        TraceRecord rec{blockIdx.x, smid, static_cast<uint32_t>(item), static_cast<uint32_t>(clock64() - tr_clk0),
+                        tr_start, dsh.t_flag, global_timer_ns()};
         for (int n = 0; n < 8; ++n) {
           rec.issue[n] = dsh.t_issue[n] ? static_cast<uint32_t>(dsh.t_issue[n] - tr_start) : 0u;
           rec.full[n] = dsh.t_full[n] ? static_cast<uint32_t>(dsh.t_full[n] - tr_start) : 0u;
@@ -240,7 +261,7 @@ __global__ void wait_selftest_kernel(uint32_t* status, uint32_t max_iters) {
     fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) mbar_wait(&bar, 0, status, max_iters);
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, status, max_iters, 1000u);
 }
 
 constexpr int kStepSmem = kRingBytes + 1024;

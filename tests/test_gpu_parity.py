@@ -158,6 +158,27 @@ def test_select_only_bitexact_from_oracle_scores(nosa, seed):
         _status_ok(nosa, ws)
 
 
+@pytest.mark.parametrize("topk", [1, 64, 96, 700])
+def test_select_only_bitexact_many_candidates(nosa, topk):
+    """Candidate sets above 1024 (contexts past 66K, up to 128K) take the
+    block-wide radix path; 256-1024 the wide warp path; bit-exact either way."""
+    rng = np.random.default_rng(topk)
+    lens = np.array([131072, 64 * 1100 + 7, 64 * 700, 64 * 250, 5000], np.int32)
+    nb_cap = oracle.n_blocks(int(lens.max()))
+    S = rng.integers(-6, 7, size=(5, 2, nb_cap)).astype(np.float32)
+    S[0, 1] += rng.standard_normal(nb_cap).astype(np.float32)
+    idx, cnt = oracle.topk(S, lens, topk)
+    p = nosa.params(4, 2, topk=topk)
+    ws = nosa.workspace(p, 5, int(lens.max()))
+    sel = torch.full((5, 2, topk), -7, dtype=torch.int32, device=DEV)
+    sc = torch.zeros(5, 2, dtype=torch.int32, device=DEV)
+    nosa.nosa_block_select(p, None, None, torch.from_numpy(lens).to(DEV), int(lens.max()), sel, sc, ws,
+                           block_scores_in=torch.from_numpy(S).to(DEV))
+    np.testing.assert_array_equal(sel.cpu().numpy(), idx)
+    np.testing.assert_array_equal(sc.cpu().numpy(), cnt)
+    _status_ok(nosa, ws)
+
+
 def test_select_unplanted_ragged_valid(nosa):
     """N(0,1) keys, ragged lengths: scores within 1e-3 and the GPU's choice is a
     valid top-k of the oracle's scores (exact wherever the boundary is not a
