@@ -85,7 +85,7 @@ struct TopkShared {
 // No block-wide barriers; the other warps are not involved.
 template <int KPL>
 __device__ void warp_topk(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
-                          int32_t* sel_cnt, int lane) {
+                          int32_t* sel_cnt, int lane, uint64_t* trace_stamps = nullptr) {
   const int k_eff = ncand < topk ? ncand : topk;
   uint32_t key[KPL];
 #pragma unroll
@@ -93,22 +93,39 @@ __device__ void warp_topk(const float* scores, bool coherent, int ncand, int top
     const int b = m * 32 + lane;
     key[m] = b < ncand ? order_key(coherent ? __ldcg(scores + b) : scores[b]) : 0u;  // valid keys are > 0
   }
+#ifdef NOSA_TRACE
+  if (trace_stamps && lane == 0) trace_stamps[0] = global_timer_ns() + (key[0] & 0u);
+#endif
   uint32_t T = 0u;
   int need = 0;
   if (k_eff < ncand) {
+    // Two bits per step: count the keys >= each of the three thresholds
+    // T|01, T|10, T|11 (warp sums with redux.sync) and keep the largest one
+    // that still has at least k keys at or above it.
 #pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = T | (1u << bit);
-      int c = 0;
+    for (int bit = 30; bit >= 0; bit -= 2) {
+      const uint32_t c1 = T | (1u << bit), c2 = T | (2u << bit), c3 = T | (3u << bit);
+      uint32_t n1 = 0, n2 = 0, n3 = 0;
 #pragma unroll
-      for (int m = 0; m < KPL; ++m) c += __popc(__ballot_sync(0xffffffffu, key[m] >= cand));
-      if (c >= k_eff) T = cand;
+      for (int m = 0; m < KPL; ++m) {
+        n1 += key[m] >= c1;
+        n2 += key[m] >= c2;
+        n3 += key[m] >= c3;
+      }
+      n1 = __reduce_add_sync(0xffffffffu, n1);
+      n2 = __reduce_add_sync(0xffffffffu, n2);
+      n3 = __reduce_add_sync(0xffffffffu, n3);
+      const uint32_t k = static_cast<uint32_t>(k_eff);
+      T = n3 >= k ? c3 : n2 >= k ? c2 : n1 >= k ? c1 : T;
     }
-    int above = 0;
+    uint32_t above = 0;
 #pragma unroll
-    for (int m = 0; m < KPL; ++m) above += __popc(__ballot_sync(0xffffffffu, key[m] > T));
-    need = k_eff - above;
+    for (int m = 0; m < KPL; ++m) above += key[m] > T;
+    need = k_eff - static_cast<int>(__reduce_add_sync(0xffffffffu, above));
   }
+#ifdef NOSA_TRACE
+  if (trace_stamps && lane == 0) trace_stamps[1] = global_timer_ns() + (T & 0u);
+#endif
   const uint32_t lt_mask = (1u << lane) - 1u;
   int eq_seen = 0, pos = 0;
 #pragma unroll
@@ -126,6 +143,9 @@ __device__ void warp_topk(const float* scores, bool coherent, int ncand, int top
   }
   for (int t = k_eff + lane; t < topk; t += 32) sel_row[t] = -1;
   if (lane == 0) *sel_cnt = k_eff;
+#ifdef NOSA_TRACE
+  if (trace_stamps && lane == 0) trace_stamps[2] = global_timer_ns();
+#endif
 }
 
 // Candidates up to which one warp selects (warp_topk); larger sets use the
@@ -140,15 +160,15 @@ constexpr int kWarpTopkMax = 1024;
 // -1 padded) and its count.  `ords` is shared memory for ncand keys.
 template <int NT>
 __device__ void select_topk(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
-                            int32_t* sel_cnt, uint32_t* ords, TopkShared& sh) {
+                            int32_t* sel_cnt, uint32_t* ords, TopkShared& sh, uint64_t* trace_stamps = nullptr) {
   constexpr int kWarpsNT = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (ncand <= kWarpTopkMax) {
     if (warp == 0) {
       if (ncand <= 256)
-        warp_topk<8>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
+        warp_topk<8>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane, trace_stamps);
       else
-        warp_topk<32>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
+        warp_topk<32>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane, trace_stamps);
     }
     return;
   }
@@ -282,6 +302,8 @@ __device__ bool score_chunk(const __nv_bfloat16* __restrict__ q, const float* __
   const bool ok = mbar_wait(bar, phase, status);
 #ifdef NOSA_TRACE
   if (tid == 0 && trace_landed) *trace_landed = global_timer_ns();
+  if (lane == 0 && trace_landed) atomicMax(reinterpret_cast<unsigned long long*>(trace_landed + 3),
+                                           static_cast<unsigned long long>(global_timer_ns()));
 #endif
   if (ok) {
     // Four windows per warp and iteration: four independent reduction chains
@@ -294,13 +316,24 @@ __device__ bool score_chunk(const __nv_bfloat16* __restrict__ q, const float* __
       for (int w = 0; w < kWin; ++w) {
         const int jj = min(j0 + w, nwin - 1);
         const float4 kv = reinterpret_cast<const float4*>(keys + jj * kHeadDim)[lane];
+        if constexpr (G >= 2) {
+          // Two heads per packed fp32x2 FMA; each head's sum keeps the order
+          // x, y, z, w of the scalar form (same rounding).
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          float d = qv[hh].x * kv.x;
-          d = fmaf(qv[hh].y, kv.y, d);
-          d = fmaf(qv[hh].z, kv.z, d);
-          d = fmaf(qv[hh].w, kv.w, d);
-          v[w][hh] = d;
+          for (int hh = 0; hh < G; hh += 2) {
+            float2 d = __fmul2_rn(make_float2(qv[hh].x, qv[hh + 1].x), make_float2(kv.x, kv.x));
+            d = __ffma2_rn(make_float2(qv[hh].y, qv[hh + 1].y), make_float2(kv.y, kv.y), d);
+            d = __ffma2_rn(make_float2(qv[hh].z, qv[hh + 1].z), make_float2(kv.z, kv.z), d);
+            d = __ffma2_rn(make_float2(qv[hh].w, qv[hh + 1].w), make_float2(kv.w, kv.w), d);
+            v[w][hh] = d.x;
+            v[w][hh + 1] = d.y;
+          }
+        } else {
+          float d = qv[0].x * kv.x;
+          d = fmaf(qv[0].y, kv.y, d);
+          d = fmaf(qv[0].z, kv.z, d);
+          d = fmaf(qv[0].w, kv.w, d);
+          v[w][0] = d;
         }
       }
 #pragma unroll
@@ -310,6 +343,10 @@ __device__ bool score_chunk(const __nv_bfloat16* __restrict__ q, const float* __
         if ((lane & writer_mask) == 0 && j0 + w < nwin) ssm[head * kScoreStride + j0 + w] = s * scale;
       }
     }
+#ifdef NOSA_TRACE
+    if (lane == 0 && trace_landed) atomicMax(reinterpret_cast<unsigned long long*>(trace_landed + 4),
+                                             static_cast<unsigned long long>(global_timer_ns()));
+#endif
   }
   __syncthreads();
   if (ok) {

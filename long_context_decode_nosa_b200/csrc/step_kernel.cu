@@ -128,13 +128,13 @@ __device__ void score_item(const StepArgs& a, int item, uint8_t* smem, uint64_t*
   NOSA_STAMP(3);
   if (!*sh_last) return;
   __threadfence();
+  NOSA_STAMP(7);
   // The pair's last chunk: every block score is written; select.
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   select_topk<kDecThreads>(s.bscratch + static_cast<int64_t>(pair) * s.nb_ws, true, geo.ncand, s.topk,
                            s.sel_idx + static_cast<int64_t>(pair) * s.topk, s.sel_cnt + pair,
-                           reinterpret_cast<uint32_t*>(smem), tsh);
+                           reinterpret_cast<uint32_t*>(smem), tsh, stamps ? stamps + 4 : nullptr);
   __syncthreads();
-  NOSA_STAMP(4);
   if (tid == 0) {
     s.tickets[pair] = 0u;
     if (a.mode & kStepDecode) {
