@@ -118,12 +118,15 @@ constexpr int kSelList = 128;  // selected block indices a split stages in share
 struct DecodeShared {
   uint64_t full_bar[kStages];
   uint64_t empty_bar[kStages];
+  uint64_t merge_bar;     // bulk copies of the split partials (final merge)
+  uint32_t merge_phase;   // its current parity
   int stage_blk[kStages];
   int last;
   int sel_list[kSelList];
 #ifdef NOSA_TRACE
   uint64_t t_flag;  // instrumented builds: when the producer saw the selection
   uint64_t t_issue[8], t_full[8], t_done[8];  // per tile: TMA issued, landed, consumed (warp 0)
+  uint64_t t_merge[6];  // drained, warps merged, partial written, ticket taken, splits loaded, done
 #endif
 };
 
@@ -378,18 +381,33 @@ __device__ inline void decode_item(const DecodeArgs& a, const CUtensorMap* tm_k,
   }
   ring_n += static_cast<uint32_t>(my_n);
   __syncthreads();  // ring drained: reuse it for the cross-warp merge
+#ifdef NOSA_TRACE
+#define NOSA_MSTAMP(k) \
+  if (tid == 0) sh.t_merge[k] = global_timer_ns()
+#else
+#define NOSA_MSTAMP(k)
+#endif
+  NOSA_MSTAMP(0);
 
-  float* mo = reinterpret_cast<float*>(smem);                    // [4][G][128]
-  float* mm = mo + kDecConsumerWarps * G * kHeadDim;             // [4][G]
-  float* ml = mm + kDecConsumerWarps * G;                        // [4][G]
+  // Cross-warp merge in fixed warp order.  Each warp's O goes to shared
+  // memory as float2 pairs with a padded row stride (bank-conflict free);
+  // per-row weights are computed once.
+  constexpr int kMoStride = kHeadDim + 8;                         // floats per merge row
+  float* mo = reinterpret_cast<float*>(smem);                     // [4][G][kMoStride]
+  float* mm = mo + kDecConsumerWarps * G * kMoStride;             // [4][G] row max
+  float* ml = mm + kDecConsumerWarps * G;                         // [4][G] row sum
+  float* mw = ml + kDecConsumerWarps * G;                         // [4][G] weights
+  float* mrow = mw + kDecConsumerWarps * G;                       // [G] M, then [G] L
   if (warp < kDecConsumerWarps) {
     const int grp = lane >> 2, tig = lane & 3;
 #pragma unroll
     for (int d = 0; d < 16; ++d) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int row = grp + (e >> 1) * 8;
-        if (row < G) mo[(warp * G + row) * kHeadDim + d * 8 + 2 * tig + (e & 1)] = acc[d][e];
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int row = grp + h2 * 8;
+        if (row < G)
+          *reinterpret_cast<float2*>(mo + (warp * G + row) * kMoStride + d * 8 + 2 * tig) =
+              make_float2(acc[d][2 * h2], acc[d][2 * h2 + 1]);
       }
     }
     if (tig == 0) {
@@ -404,102 +422,175 @@ __device__ inline void decode_item(const DecodeArgs& a, const CUtensorMap* tm_k,
     }
   }
   __syncthreads();
+  for (int row = tid; row < G; row += kDecThreads) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, mm[w * G + row]);
+    float lsum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kDecConsumerWarps; ++w) {
+      const float m_w = mm[w * G + row];
+      const float f = m_w == -INFINITY ? 0.0f : exp2f(m_w - M);
+      mw[w * G + row] = f;
+      lsum += ml[w * G + row] * f;
+    }
+    mrow[row] = M;
+    mrow[G + row] = lsum;
+  }
+  __syncthreads();
+  NOSA_MSTAMP(1);
 
   const bool single = a.nsplit == 1;
   const int stride = part_stride(G);
   float* part = a.part + (static_cast<int64_t>(pair) * kMaxSplits + split) * stride;
-  for (int t = tid; t < G * kHeadDim; t += kDecThreads) {
-    const int row = t / kHeadDim, d = t % kHeadDim;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, mm[w * G + row]);
-    float lsum = 0.0f, o = 0.0f;
+  constexpr int kVec = kHeadDim / 4;
+  for (int t = tid; t < G * kVec; t += kDecThreads) {
+    const int row = t / kVec, d4 = t % kVec;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int w = 0; w < kDecConsumerWarps; ++w) {
-      const float mw = mm[w * G + row];
-      if (mw == -INFINITY) continue;
-      const float f = exp2f(mw - M);
-      lsum += ml[w * G + row] * f;
-      o += mo[(w * G + row) * kHeadDim + d] * f;
+      const float f = mw[w * G + row];
+      const float4 x = *reinterpret_cast<const float4*>(mo + (w * G + row) * kMoStride + 4 * d4);
+      o.x = fmaf(f, x.x, o.x);
+      o.y = fmaf(f, x.y, o.y);
+      o.z = fmaf(f, x.z, o.z);
+      o.w = fmaf(f, x.w, o.w);
     }
     if (single) {
-      a.out[(out_row0 + row) * kHeadDim + d] = __float2bfloat16_rn(lsum > 0.0f ? o / lsum : 0.0f);
-      if (a.lse && d == 0) a.lse[out_row0 + row] = lsum > 0.0f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
+      const float lsum = mrow[G + row];
+      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.out + (out_row0 + row) * kHeadDim + 4 * d4);
+      dst[0] = __floats2bfloat162_rn(o.x * inv, o.y * inv);
+      dst[1] = __floats2bfloat162_rn(o.z * inv, o.w * inv);
+      if (a.lse && d4 == 0) a.lse[out_row0 + row] = lsum > 0.0f ? (mrow[row] + log2f(lsum)) * kLn2 : -INFINITY;
     } else {
-      part[row * kHeadDim + d] = o;
-      if (d == 0) {
-        part[G * kHeadDim + row] = M;
-        part[G * kHeadDim + G + row] = lsum;
-      }
+      reinterpret_cast<float4*>(part + row * kHeadDim)[d4] = o;
     }
   }
+  if (!single)
+    for (int row = tid; row < G; row += kDecThreads) {
+      part[G * kHeadDim + row] = mrow[row];
+      part[G * kHeadDim + G + row] = mrow[G + row];
+    }
   if (single) {
     if (ready != nullptr && tid == 0) *ready = 0u;  // the pair's only item: re-arm the flag
     return;
   }
 
+  // Publish this split's partial, then take a ticket; the last split of the
+  // pair merges all of them.
+  __threadfence();
   __syncthreads();
+  NOSA_MSTAMP(2);
   if (tid == 0) {
-    __threadfence();
     const uint32_t t = atomicAdd(&a.tickets[pair], 1u);
     sh.last = (t == static_cast<uint32_t>(a.nsplit - 1));
   }
   __syncthreads();
+  NOSA_MSTAMP(3);
   if (!sh.last) return;
-  __threadfence();
-  // Merge the splits in split order: their (m, l) go to shared memory first
-  // (one parallel round trip), then each output float4 streams the splits'
-  // partial O with independent loads.
-  const float* pbase = a.part + static_cast<int64_t>(pair) * kMaxSplits * stride;
-  float* sm_w = reinterpret_cast<float*>(smem);       // [nsplit][G]: m, then weights
-  float* sm_l = sm_w + kMaxSplits * kMaxGroup;        // [nsplit][G]
-  float* sm_L = sm_l + kMaxSplits * kMaxGroup;        // [G]
-  float* sm_M = sm_L + kMaxGroup;                     // [G]
-  for (int t = tid; t < a.nsplit * G; t += kDecThreads) {
-    const int s = t / G, row = t % G;
-    sm_w[t] = __ldcg(pbase + s * stride + G * kHeadDim + row);
-    sm_l[t] = __ldcg(pbase + s * stride + G * kHeadDim + G + row);
-  }
+  if (tid == 0) __threadfence();  // acquire: the other splits' partials
   __syncthreads();
+  // Merge the splits in split order.  The partials (O, m, l of every split)
+  // are staged in shared memory by 1-D bulk (TMA) copies -- all of them in
+  // one copy when they fit -- then the weights and the weighted sums are
+  // computed from there.
+  const float* pbase = a.part + static_cast<int64_t>(pair) * kMaxSplits * stride;
+  float* sm_w = reinterpret_cast<float*>(smem + kRingBytes - (kMaxSplits * kMaxGroup + 2 * kMaxGroup) * 4);
+  float* sm_L = sm_w + kMaxSplits * kMaxGroup;                    // [G]
+  float* sm_M = sm_L + kMaxGroup;                                 // [G]
+  const int stage_bytes_max = kRingBytes - (kMaxSplits * kMaxGroup + 2 * kMaxGroup) * 4;
+  const int per_copy = max(1, stage_bytes_max / (stride * 4));
+  const bool one_copy = a.nsplit <= per_copy;
+  // The TMA unit reads next the other splits' partials (published by their
+  // tickets) and writes shared memory this CTA wrote with plain stores.
+  asm volatile("fence.proxy.async;" ::: "memory");
+  __syncthreads();
+  const float* stg = reinterpret_cast<const float*>(smem);
+  if (one_copy && tid == 0) {
+    const uint32_t bytes = static_cast<uint32_t>(a.nsplit * stride * 4);
+    mbar_arrive_expect_tx(&sh.merge_bar, bytes);
+    bulk_copy_g2s(smem, pbase, bytes, &sh.merge_bar);
+  }
+  // (m, l) of split sp, row r: from the staged copy, or from global memory.
+  auto m_of = [&](int sp, int r) {
+    return one_copy ? stg[sp * stride + G * kHeadDim + r] : __ldcg(pbase + sp * stride + G * kHeadDim + r);
+  };
+  auto l_of = [&](int sp, int r) {
+    return one_copy ? stg[sp * stride + G * kHeadDim + G + r] : __ldcg(pbase + sp * stride + G * kHeadDim + G + r);
+  };
+  if (one_copy) mbar_wait(&sh.merge_bar, sh.merge_phase, a.status);
   for (int row = tid; row < G; row += kDecThreads) {
     float M = -INFINITY;
-    for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, sm_w[s * G + row]);
-    float lsum = 0.0f;
-    for (int s = 0; s < a.nsplit; ++s) {
-      const float ms = sm_w[s * G + row];
-      const float w = ms == -INFINITY ? 0.0f : exp2f(ms - M);
-      sm_w[s * G + row] = w;
-      lsum += sm_l[s * G + row] * w;
-    }
-    sm_L[row] = lsum;
+    for (int sp = 0; sp < a.nsplit; ++sp) M = fmaxf(M, m_of(sp, row));
     sm_M[row] = M;
   }
   __syncthreads();
-  constexpr int kVec = kHeadDim / 4;
-  for (int t = tid; t < G * kVec; t += kDecThreads) {
-    const int row = t / kVec, d4 = t % kVec;
-    const float4* src = reinterpret_cast<const float4*>(pbase + row * kHeadDim) + d4;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-    for (int s = 0; s < a.nsplit; ++s) {
-      const float w = sm_w[s * G + row];
-      const float4 x = __ldcg(src + s * (stride / 4));
-      o.x = fmaf(w, x.x, o.x);
-      o.y = fmaf(w, x.y, o.y);
-      o.z = fmaf(w, x.z, o.z);
-      o.w = fmaf(w, x.w, o.w);
+  for (int t = tid; t < a.nsplit * G; t += kDecThreads) {
+    const int sp = t / G, row = t % G;
+    const float ms = m_of(sp, row);
+    sm_w[t] = ms == -INFINITY ? 0.0f : exp2f(ms - sm_M[row]);
+  }
+  __syncthreads();
+  for (int row = tid; row < G; row += kDecThreads) {
+    float lsum = 0.0f;
+    for (int sp = 0; sp < a.nsplit; ++sp) lsum += l_of(sp, row) * sm_w[sp * G + row];
+    sm_L[row] = lsum;
+  }
+  NOSA_MSTAMP(4);
+  // Each thread owns output float4s t = tid, tid + 160, ... (at most 4).
+  constexpr int kOwn = (kMaxGroup * kVec + kDecThreads - 1) / kDecThreads;
+  float4 o[kOwn];
+#pragma unroll
+  for (int k = 0; k < kOwn; ++k) o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sp0 = 0; sp0 < a.nsplit; sp0 += per_copy) {
+    const int nsp = min(per_copy, a.nsplit - sp0);
+    if (!one_copy) {
+      if (tid == 0) {
+        const uint32_t bytes = static_cast<uint32_t>(nsp * stride * 4);
+        mbar_arrive_expect_tx(&sh.merge_bar, bytes);
+        bulk_copy_g2s(smem, pbase + static_cast<int64_t>(sp0) * stride, bytes, &sh.merge_bar);
+      }
+      mbar_wait(&sh.merge_bar, sh.merge_phase, a.status);
     }
-    const float lsum = sm_L[row];
-    const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.out + (out_row0 + row) * kHeadDim + 4 * d4);
-    dst[0] = __floats2bfloat162_rn(o.x * inv, o.y * inv);
-    dst[1] = __floats2bfloat162_rn(o.z * inv, o.w * inv);
-    if (a.lse && d4 == 0) a.lse[out_row0 + row] = lsum > 0.0f ? (sm_M[row] + log2f(lsum)) * kLn2 : -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kOwn; ++k) {
+      const int t = tid + k * kDecThreads;
+      if (t < G * kVec) {
+        const int row = t / kVec, d4 = t % kVec;
+        for (int sp = 0; sp < nsp; ++sp) {
+          const float w = sm_w[(sp0 + sp) * G + row];
+          const float4 x = *reinterpret_cast<const float4*>(stg + sp * stride + row * kHeadDim + 4 * d4);
+          o[k].x = fmaf(w, x.x, o[k].x);
+          o[k].y = fmaf(w, x.y, o[k].y);
+          o[k].z = fmaf(w, x.z, o[k].z);
+          o[k].w = fmaf(w, x.w, o[k].w);
+        }
+      }
+    }
+    __syncthreads();  // everyone is done with the staged splits
+    if (tid == 0) sh.merge_phase ^= 1u;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+  }
+#pragma unroll
+  for (int k = 0; k < kOwn; ++k) {
+    const int t = tid + k * kDecThreads;
+    if (t < G * kVec) {
+      const int row = t / kVec, d4 = t % kVec;
+      const float lsum = sm_L[row];
+      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.out + (out_row0 + row) * kHeadDim + 4 * d4);
+      dst[0] = __floats2bfloat162_rn(o[k].x * inv, o[k].y * inv);
+      dst[1] = __floats2bfloat162_rn(o[k].z * inv, o[k].w * inv);
+      if (a.lse && d4 == 0) a.lse[out_row0 + row] = lsum > 0.0f ? (sm_M[row] + log2f(lsum)) * kLn2 : -INFINITY;
+    }
   }
   if (tid == 0) {
     a.tickets[pair] = 0u;
     if (ready != nullptr) *ready = 0u;  // every item of the pair has passed its wait
   }
+  NOSA_MSTAMP(5);
 }
 
 }  // namespace nosa

@@ -99,24 +99,51 @@ __device__ void warp_topk(const float* scores, bool coherent, int ncand, int top
   uint32_t T = 0u;
   int need = 0;
   if (k_eff < ncand) {
-    // Two bits per step: count the keys >= each of the three thresholds
-    // T|01, T|10, T|11 (warp sums with redux.sync) and keep the largest one
-    // that still has at least k keys at or above it.
-#pragma unroll 1
-    for (int bit = 30; bit >= 0; bit -= 2) {
-      const uint32_t c1 = T | (1u << bit), c2 = T | (2u << bit), c3 = T | (3u << bit);
-      uint32_t n1 = 0, n2 = 0, n3 = 0;
+    // The k-th largest key lies in [min, max]: its bits above their highest
+    // differing bit are theirs.  The rest is found two bits per step --
+    // count the keys >= each of T|01, T|10, T|11 (warp sums, redux.sync) and
+    // keep the largest threshold that still has at least k keys at or above.
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
 #pragma unroll
-      for (int m = 0; m < KPL; ++m) {
-        n1 += key[m] >= c1;
-        n2 += key[m] >= c2;
-        n3 += key[m] >= c3;
+    for (int m = 0; m < KPL; ++m) {
+      if (m * 32 + lane < ncand) {
+        lo = min(lo, key[m]);
+        hi = max(hi, key[m]);
       }
-      n1 = __reduce_add_sync(0xffffffffu, n1);
-      n2 = __reduce_add_sync(0xffffffffu, n2);
-      n3 = __reduce_add_sync(0xffffffffu, n3);
-      const uint32_t k = static_cast<uint32_t>(k_eff);
-      T = n3 >= k ? c3 : n2 >= k ? c2 : n1 >= k ? c1 : T;
+    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t k = static_cast<uint32_t>(k_eff);
+    if (lo != hi) {
+      const int top = 31 - __clz(lo ^ hi);                // highest differing bit
+      T = hi & ~((2u << top) - 1u);                       // common prefix (top == 31: shift by 32 avoided)
+      if (top == 31) T = 0u;
+      int bit = top;
+      if ((top & 1) == 0) {                               // odd number of bits left: one single-bit step
+        const uint32_t c1 = T | (1u << bit);
+        uint32_t n1 = 0;
+#pragma unroll
+        for (int m = 0; m < KPL; ++m) n1 += key[m] >= c1;
+        if (__reduce_add_sync(0xffffffffu, n1) >= k) T = c1;
+        --bit;
+      }
+#pragma unroll 1
+      for (bit -= 1; bit >= 0; bit -= 2) {
+        const uint32_t c1 = T | (1u << bit), c2 = T | (2u << bit), c3 = T | (3u << bit);
+        uint32_t n1 = 0, n2 = 0, n3 = 0;
+#pragma unroll
+        for (int m = 0; m < KPL; ++m) {
+          n1 += key[m] >= c1;
+          n2 += key[m] >= c2;
+          n3 += key[m] >= c3;
+        }
+        n1 = __reduce_add_sync(0xffffffffu, n1);
+        n2 = __reduce_add_sync(0xffffffffu, n2);
+        n3 = __reduce_add_sync(0xffffffffu, n3);
+        T = n3 >= k ? c3 : n2 >= k ? c2 : n1 >= k ? c1 : T;
+      }
+    } else {
+      T = hi;
     }
     uint32_t above = 0;
 #pragma unroll
@@ -127,19 +154,37 @@ __device__ void warp_topk(const float* scores, bool coherent, int ncand, int top
   if (trace_stamps && lane == 0) trace_stamps[1] = global_timer_ns() + (T & 0u);
 #endif
   const uint32_t lt_mask = (1u << lane) - 1u;
-  int eq_seen = 0, pos = 0;
+  uint32_t n_eq = 0;
 #pragma unroll
-  for (int m = 0; m < KPL; ++m) {
-    const int b = m * 32 + lane;
-    const bool valid = b < ncand;
-    const bool eq = valid && k_eff < ncand && key[m] == T;
-    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
-    const bool take = valid && (key[m] > T || (eq && eq_seen + __popc(eb & lt_mask) < need));
-    const uint32_t tb = __ballot_sync(0xffffffffu, take);
-    const int p = pos + __popc(tb & lt_mask);
-    if (take && p < topk) sel_row[p] = b;
-    eq_seen += __popc(eb);
-    pos += __popc(tb);
+  for (int m = 0; m < KPL; ++m) n_eq += (m * 32 + lane < ncand) && key[m] == T;
+  n_eq = __reduce_add_sync(0xffffffffu, n_eq);
+  int pos = 0;
+  if (k_eff == ncand || static_cast<uint32_t>(need) == n_eq) {
+    // Every key tied with the threshold is taken: key >= T decides alone.
+#pragma unroll
+    for (int m = 0; m < KPL; ++m) {
+      const int b = m * 32 + lane;
+      const bool take = b < ncand && key[m] >= T;
+      const uint32_t tb = __ballot_sync(0xffffffffu, take);
+      const int p = pos + __popc(tb & lt_mask);
+      if (take && p < topk) sel_row[p] = b;
+      pos += __popc(tb);
+    }
+  } else {
+    int eq_seen = 0;
+#pragma unroll
+    for (int m = 0; m < KPL; ++m) {
+      const int b = m * 32 + lane;
+      const bool valid = b < ncand;
+      const bool eq = valid && key[m] == T;
+      const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+      const bool take = valid && (key[m] > T || (eq && eq_seen + __popc(eb & lt_mask) < need));
+      const uint32_t tb = __ballot_sync(0xffffffffu, take);
+      const int p = pos + __popc(tb & lt_mask);
+      if (take && p < topk) sel_row[p] = b;
+      eq_seen += __popc(eb);
+      pos += __popc(tb);
+    }
   }
   for (int t = k_eff + lane; t < topk; t += 32) sel_row[t] = -1;
   if (lane == 0) *sel_cnt = k_eff;

@@ -33,6 +33,7 @@ struct TraceRecord {
   uint32_t cta, smid, item, clk_delta;  // clk_delta: SM clock cycles spent in the item
   uint64_t t_start, t_flag, t_end;
   uint32_t issue[8], full[8], done[8];  // per tile, ns after t_start
+  uint32_t merge[6];                     // decode merge phase, ns after t_start
 };
 constexpr int kTraceCapacity = 1 << 16;
 __device__ TraceRecord g_trace[kTraceCapacity];
@@ -127,7 +128,8 @@ __device__ void score_item(const StepArgs& a, int item, uint8_t* smem, uint64_t*
   __syncthreads();
   NOSA_STAMP(3);
   if (!*sh_last) return;
-  __threadfence();
+  if (tid == 0) __threadfence();  // acquire: the other chunks' block scores
+  __syncthreads();
   NOSA_STAMP(7);
   // The pair's last chunk: every block score is written; select.
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -164,6 +166,8 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
       mbar_init(&dsh.empty_bar[s], kDecConsumerWarps);
     }
     mbar_init(&key_bar, 1);
+    mbar_init(&dsh.merge_bar, 1);
+    dsh.merge_phase = 0;
     fence_barrier_init();
   }
   if (tid == kDecConsumerWarps * 32 && (a.mode & kStepDecode)) {
@@ -174,6 +178,7 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
   if (tid == 0) {
     dsh.t_flag = 0;
     for (int n = 0; n < 8; ++n) dsh.t_issue[n] = dsh.t_full[n] = dsh.t_done[n] = 0;
+    for (int n = 0; n < 6; ++n) dsh.t_merge[n] = 0;
   }
 #endif
   grid_dependency_wait();
@@ -216,6 +221,10 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
           rec.full[n] = dsh.t_full[n] ? static_cast<uint32_t>(dsh.t_full[n] - tr_start) : 0u;
           rec.done[n] = dsh.t_done[n] ? static_cast<uint32_t>(dsh.t_done[n] - tr_start) : 0u;
           dsh.t_issue[n] = dsh.t_full[n] = dsh.t_done[n] = 0;
+        }
+        for (int n = 0; n < 6; ++n) {
+          rec.merge[n] = dsh.t_merge[n] ? static_cast<uint32_t>(dsh.t_merge[n] - tr_start) : 0u;
+          dsh.t_merge[n] = 0;
         }
         g_trace[k] = rec;
       }
