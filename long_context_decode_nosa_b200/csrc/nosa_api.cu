@@ -71,31 +71,25 @@ float scale_of(const nosa_params* p) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace layout (all offsets 256-byte aligned).
+// Workspace layout (all offsets 256-byte aligned): the device status word;
+// block scores that do not fit in shared memory (pairs x candidates, only
+// when a sequence may have more than kSmemBlockScores candidates); staging
+// buffers of the host-buffer step (q, new K/V rows, out).
 struct Layout {
-  size_t status, work, sel_tickets, dec_tickets, ready, bscores, part, stage_q, stage_k, stage_v, stage_out, total;
-  int nb_ws;
+  size_t status, spill, stage_q, stage_k, stage_v, stage_out, total;
+  int nb_spill;  // candidates per pair in `spill` (0: block scores stay in shared memory)
 };
 
 Layout layout_of(const nosa_params* p, int batch, int max_seq_len) {
   Layout l{};
   const size_t pairs = static_cast<size_t>(batch) * p->num_kv_heads;
-  const int G = p->num_q_heads / p->num_kv_heads;
-  l.nb_ws = static_cast<int>(nosa::n_blocks(max_seq_len));
+  const int64_t ncand_max = nosa::n_candidates(max_seq_len, p->local_blocks);
+  l.nb_spill = ncand_max > nosa::kSmemBlockScores ? static_cast<int>(ncand_max) : 0;
   size_t off = 0;
   l.status = off;  // uint32 device status word
-  l.work = off + 16;  // uint32[2] work queue of the step kernel
   off += 256;
-  l.sel_tickets = off;
-  off = round_up(off + pairs * 4, 256);
-  l.dec_tickets = off;
-  off = round_up(off + pairs * 4, 256);
-  l.ready = off;
-  off = round_up(off + pairs * 4, 256);
-  l.bscores = off;
-  off = round_up(off + pairs * static_cast<size_t>(l.nb_ws) * 4, 256);
-  l.part = off;
-  off = round_up(off + pairs * nosa::kMaxSplits * static_cast<size_t>(nosa::part_stride(G)) * 4, 256);
+  l.spill = off;
+  off = round_up(off + pairs * static_cast<size_t>(l.nb_spill) * 4, 256);
   const size_t qbytes = static_cast<size_t>(batch) * p->num_q_heads * nosa::kHeadDim * 2;
   const size_t kvbytes = pairs * nosa::kHeadDim * 2;
   l.stage_q = off;
@@ -150,6 +144,26 @@ int encode_kv_map(CUtensorMap* map, const void* base, int hkv, int64_t rows) {
   return NOSA_OK;
 }
 
+// 2-D map over the pooled keys [batch * hkv * nc_cap rows, 128 fp32]: boxes of
+// {32 columns, 65 rows} (one 32-dimension slice of one scoring chunk),
+// 128-byte swizzle, zero fill past the last row.
+int encode_pooled_map(CUtensorMap* map, const float* pooled, int batch, int hkv, int nc_cap) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(NOSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t rows = static_cast<cuuint64_t>(batch) * hkv * nc_cap;
+  // TMA row coordinates are signed 32-bit.
+  if (rows >= (cuuint64_t{1} << 31)) return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads * nc_cap must be below 2^31");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(nosa::kHeadDim), rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(nosa::kHeadDim) * 4};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(nosa::kBoxCols), static_cast<cuuint32_t>(nosa::kBoxRows)};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pooled), dims, strides, box,
+                   elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NOSA_ERR_INVALID_ARG, "pooled tensor map encode failed (code %d)", static_cast<int>(r));
+  return NOSA_OK;
+}
+
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
@@ -192,78 +206,34 @@ int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t c
   return ok();
 }
 
-void fill_select_args(nosa::SelectArgs& a, const nosa_params* p, const void* q, const float* pooled, int nc_cap,
-                      const int32_t* seq_len, int batch, int max_seq_len, float* comp_out, float* bs_out,
-                      int nb_out, int32_t* sel_idx, int32_t* sel_cnt, void* ws, const Layout& l) {
+// Arguments of the step kernel common to its three uses.
+nosa::StepArgs step_args(const nosa_params* p, const void* q, const int32_t* seq_len, int batch, int max_seq_len,
+                         int32_t* sel_idx, int32_t* sel_cnt, void* ws, const Layout& l) {
+  nosa::StepArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
-  a.pooled = pooled;
   a.seq_len = seq_len;
-  a.bs_in = nullptr;
-  a.comp_out = comp_out;
-  a.bs_out = bs_out;
   a.sel_idx = sel_idx;
   a.sel_cnt = sel_cnt;
-  a.bscratch = at<float>(ws, l.bscores);
-  a.tickets = at<uint32_t>(ws, l.sel_tickets);
+  a.bs_spill = l.nb_spill > 0 ? at<float>(ws, l.spill) : nullptr;
+  a.nb_spill = l.nb_spill;
   a.status = at<uint32_t>(ws, l.status);
   a.batch = batch;
   a.hq = p->num_q_heads;
   a.hkv = p->num_kv_heads;
-  a.group = p->num_q_heads / p->num_kv_heads;
   a.local_blocks = p->local_blocks;
   a.topk = p->topk;
   a.max_seq_len = max_seq_len;
-  a.nc_cap = nc_cap;
-  a.nb_in = 0;
-  a.nb_out = nb_out;
-  a.nb_ws = l.nb_ws;
+  a.nc_cap = 1;
   a.scale = scale_of(p);
-}
-
-void fill_decode_args(nosa::DecodeArgs& a, const nosa_params* p, const void* q, const void* k_cache,
-                      const void* v_cache, int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len,
-                      int batch, int max_seq_len, const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
-                      float* lse, void* ws, const Layout& l) {
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.k_cache = static_cast<const __nv_bfloat16*>(k_cache);
-  a.v_cache = static_cast<const __nv_bfloat16*>(v_cache);
-  a.cache_rows = cache_rows;
-  a.seq_start = seq_start;
-  a.seq_len = seq_len;
-  a.sel_idx = sel_idx;
-  a.sel_cnt = sel_cnt;
-  a.out = static_cast<__nv_bfloat16*>(out);
-  a.lse = lse;
-  a.part = at<float>(ws, l.part);
-  a.tickets = at<uint32_t>(ws, l.dec_tickets);
-  a.status = at<uint32_t>(ws, l.status);
-  a.batch = batch;
-  a.hq = p->num_q_heads;
-  a.hkv = p->num_kv_heads;
-  a.group = p->num_q_heads / p->num_kv_heads;
-  a.local_blocks = p->local_blocks;
-  a.topk = p->topk;
-  a.max_seq_len = max_seq_len;
-  const int nb_max = static_cast<int>(nosa::n_blocks(max_seq_len));
-  const int ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
-  const int max_tiles = (p->topk < ncand_max ? p->topk : ncand_max) +
-                        (p->local_blocks < nb_max ? p->local_blocks : nb_max);
-  nosa::decode_split_plan(batch * p->num_kv_heads, max_tiles, nosa::step_resident_ctas(a.group), &a.nsplit);
-  a.scale_log2 = scale_of(p) * 1.4426950408889634f;
-}
-
-int scoring_items(const nosa_params* p, int batch, int max_seq_len, bool full) {
-  const int nbw = static_cast<int>(full ? nosa::n_blocks(max_seq_len) : nosa::n_candidates(max_seq_len, p->local_blocks));
-  const int chunks = nbw > 0 ? (nbw + nosa::kChunkBlocks - 1) / nosa::kChunkBlocks : 1;
-  return batch * p->num_kv_heads * chunks;
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  return a;
 }
 
 int check_common(const nosa_params* p, int batch, int max_seq_len) {
   if (batch < 0 || max_seq_len < 1) return fail(NOSA_ERR_INVALID_ARG, "batch >= 0 and max_seq_len >= 1 required");
   if (static_cast<int64_t>(batch) * p->num_kv_heads > (1 << 20))
     return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 2^20");
-  if (nosa::n_blocks(max_seq_len) * 4 > nosa::kRingBytes)
-    return fail(NOSA_ERR_UNSUPPORTED, "max_seq_len too long for the selector's shared memory");
+  if (max_seq_len > (1 << 30)) return fail(NOSA_ERR_UNSUPPORTED, "max_seq_len above 2^30");
   return NOSA_OK;
 }
 
@@ -277,15 +247,24 @@ int do_block_select(const nosa_params* p, const void* q, const float* pooled, in
   if (int rc = check_ws(ws, ws_bytes, l)) return rc;
   if (!seq_len || !sel_idx || !sel_cnt) return fail(NOSA_ERR_INVALID_ARG, "seq_len, sel_idx and sel_cnt must not be NULL");
   const int ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
-  nosa::SelectArgs a{};
   if (bs_in) {
     if (nb_in < ncand_max)
       return fail(NOSA_ERR_INVALID_ARG, "nb_cap_in %d below the %d candidates of max_seq_len", nb_in, ncand_max);
     if (static_cast<int64_t>(batch) * p->num_kv_heads > 65535)
       return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads above 65535");
-    fill_select_args(a, p, nullptr, nullptr, 0, seq_len, batch, max_seq_len, nullptr, nullptr, 0, sel_idx, sel_cnt,
-                     ws, l);
+    if (static_cast<int64_t>(nb_in) * 4 > 200 * 1024)
+      return fail(NOSA_ERR_UNSUPPORTED, "nb_cap_in %d above the selector's shared memory", nb_in);
+    nosa::SelectArgs a{};
+    a.seq_len = seq_len;
     a.bs_in = bs_in;
+    a.sel_idx = sel_idx;
+    a.sel_cnt = sel_cnt;
+    a.status = at<uint32_t>(ws, l.status);
+    a.batch = batch;
+    a.hkv = p->num_kv_heads;
+    a.local_blocks = p->local_blocks;
+    a.topk = p->topk;
+    a.max_seq_len = max_seq_len;
     a.nb_in = nb_in;
     cudaError_t e = nosa::launch_select_only(a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "block_select launch");
@@ -296,19 +275,17 @@ int do_block_select(const nosa_params* p, const void* q, const float* pooled, in
   if (nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "nc_cap must be >= 1");
   if (bs_out && nb_out < ncand_max)
     return fail(NOSA_ERR_INVALID_ARG, "nb_cap_out %d below the %d candidates of max_seq_len", nb_out, ncand_max);
-  nosa::StepArgs s{};
-  fill_select_args(s.sel, p, q, pooled, nc_cap, seq_len, batch, max_seq_len, comp_out, bs_out, nb_out, sel_idx,
-                   sel_cnt, ws, l);
-  s.dec.group = s.sel.group;
-  s.work = at<uint32_t>(ws, l.work);
-  s.ready = at<uint32_t>(ws, l.ready);
+  nosa::StepArgs s = step_args(p, q, seq_len, batch, max_seq_len, sel_idx, sel_cnt, ws, l);
+  s.pooled = const_cast<float*>(pooled);
+  s.nc_cap = nc_cap;
+  s.comp_out = comp_out;
+  s.bs_out = bs_out;
+  s.nb_out = nb_out;
   s.mode = nosa::kStepScore;
-  s.pairs = batch * p->num_kv_heads;
-  s.n_score_items = scoring_items(p, batch, max_seq_len, comp_out != nullptr);
-  s.n_items = s.n_score_items;
-  CUtensorMap none;
+  CUtensorMap none, tm_p;
   memset(&none, 0, sizeof none);
-  cudaError_t e = nosa::launch_step(s, none, none, stream);
+  if (int rc = encode_pooled_map(&tm_p, pooled, batch, p->num_kv_heads, nc_cap)) return rc;
+  cudaError_t e = nosa::launch_step(s, none, none, tm_p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "block_select launch");
   return ok();
 }
@@ -334,19 +311,18 @@ int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, c
   const Layout l = layout_of(p, batch, max_seq_len);
   if (int rc = check_ws(ws, ws_bytes, l)) return rc;
   if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, seq_start, seq_len, sel_idx, sel_cnt, out)) return rc;
-  nosa::StepArgs s{};
-  fill_decode_args(s.dec, p, q, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len, sel_idx,
-                   sel_cnt, out, lse, ws, l);
-  s.work = at<uint32_t>(ws, l.work);
-  s.ready = at<uint32_t>(ws, l.ready);
+  nosa::StepArgs s = step_args(p, q, seq_len, batch, max_seq_len, const_cast<int32_t*>(sel_idx),
+                               const_cast<int32_t*>(sel_cnt), ws, l);
+  s.seq_start = seq_start;
+  s.cache_rows = cache_rows;
+  s.out = static_cast<__nv_bfloat16*>(out);
+  s.lse = lse;
   s.mode = nosa::kStepDecode;
-  s.pairs = batch * p->num_kv_heads;
-  s.n_score_items = 0;
-  s.n_items = s.pairs * s.dec.nsplit;
-  CUtensorMap tm_k, tm_v;
+  CUtensorMap tm_k, tm_v, none;
+  memset(&none, 0, sizeof none);
   if (int rc = encode_kv_map(&tm_k, k_cache, p->num_kv_heads, cache_rows)) return rc;
   if (int rc = encode_kv_map(&tm_v, v_cache, p->num_kv_heads, cache_rows)) return rc;
-  cudaError_t e = nosa::launch_step(s, tm_k, tm_v, stream);
+  cudaError_t e = nosa::launch_step(s, tm_k, tm_v, none, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse_decode launch");
   return ok();
 }
@@ -379,35 +355,23 @@ int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new
                                    sel_idx, sel_cnt, out, lse, ws, ws_bytes, stream);
     return rc;
   }
-  nosa::StepArgs s{};
-  fill_select_args(s.sel, p, q, pooled, nc_cap, seq_len, batch, max_seq_len, nullptr, nullptr, 0, sel_idx, sel_cnt,
-                   ws, l);
-  fill_decode_args(s.dec, p, q, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len, sel_idx,
-                   sel_cnt, out, lse, ws, l);
-  s.pool.k_cache = static_cast<__nv_bfloat16*>(k_cache);
-  s.pool.v_cache = static_cast<__nv_bfloat16*>(v_cache);
-  s.pool.cache_rows = cache_rows;
-  s.pool.seq_start = seq_start;
-  s.pool.len_old = nullptr;
-  s.pool.len_new = seq_len;
-  s.pool.pooled = pooled;
-  s.pool.k_new = static_cast<const __nv_bfloat16*>(k_new);
-  s.pool.v_new = static_cast<const __nv_bfloat16*>(v_new);
-  s.pool.status = at<uint32_t>(ws, l.status);
-  s.pool.batch = batch;
-  s.pool.hkv = p->num_kv_heads;
-  s.pool.nc_cap = nc_cap;
-  s.pool.max_new_keys = 1;
-  s.work = at<uint32_t>(ws, l.work);
-  s.ready = at<uint32_t>(ws, l.ready);
+  nosa::StepArgs s = step_args(p, q, seq_len, batch, max_seq_len, sel_idx, sel_cnt, ws, l);
+  s.seq_start = seq_start;
+  s.cache_rows = cache_rows;
+  s.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  s.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  s.pooled = pooled;
+  s.nc_cap = nc_cap;
+  s.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  s.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  s.out = static_cast<__nv_bfloat16*>(out);
+  s.lse = lse;
   s.mode = nosa::kStepScore | nosa::kStepDecode | nosa::kStepAppend;
-  s.pairs = batch * p->num_kv_heads;
-  s.n_score_items = scoring_items(p, batch, max_seq_len, false);
-  s.n_items = s.n_score_items + s.pairs * s.dec.nsplit;
-  CUtensorMap tm_k, tm_v;
+  CUtensorMap tm_k, tm_v, tm_p;
   if (int rc = encode_kv_map(&tm_k, k_cache, p->num_kv_heads, cache_rows)) return rc;
   if (int rc = encode_kv_map(&tm_v, v_cache, p->num_kv_heads, cache_rows)) return rc;
-  cudaError_t e = nosa::launch_step(s, tm_k, tm_v, stream);
+  if (int rc = encode_pooled_map(&tm_p, pooled, batch, p->num_kv_heads, nc_cap)) return rc;
+  cudaError_t e = nosa::launch_step(s, tm_k, tm_v, tm_p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
   return ok();
 }
@@ -418,7 +382,7 @@ namespace nosa {
 
 size_t workspace_counter_bytes(const nosa_params* p, int batch, int max_seq_len) {
   if (check_params(p) != NOSA_OK || batch < 0 || max_seq_len < 1) return 0;
-  return layout_of(p, batch, max_seq_len).bscores;
+  return layout_of(p, batch, max_seq_len).spill;
 }
 
 int record_error(int code, const char* msg) { return fail(code, "%s", msg); }

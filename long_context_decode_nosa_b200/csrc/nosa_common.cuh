@@ -20,15 +20,18 @@ constexpr int kPoolKernel = 32;
 constexpr int kPoolStride = 16;
 constexpr int kBlock = 64;
 constexpr int kWindowsPerBlock = kBlock / kPoolStride;  // 4
+// A scoring chunk covers 15 blocks [b0, b0+15), i.e. pooled windows
+// [4*b0-1, 4*b0+60): 61 rows, fetched as TMA boxes of 32 fp32 columns
+// (128 bytes) each, so that a chunk's four boxes fill one 32 KB ring stage.
+constexpr int kChunkBlocks = 15;
+constexpr int kChunkWindows = kChunkBlocks * kWindowsPerBlock + 1;  // 61
+constexpr int kBoxCols = 32;
+constexpr int kBoxRows = kChunkWindows;
+constexpr int kMaxCluster = 16;  // CTAs per (sequence, KV head) cluster, at most
 constexpr int kMaxGroup = 16;
-constexpr int kMaxSplits = 64;
 constexpr int kMaxLocalBlocks = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint32_t kWaitLimitIters = 1u << 30;
-
-// Floats per (pair, split) partial softmax state: O[G][128], m[G], l[G],
-// padded to a multiple of 4 floats so every split's O starts 16-byte aligned.
-__host__ __device__ constexpr int part_stride(int G) { return G * kHeadDim + ((2 * G + 3) & ~3); }
 
 __host__ __device__ inline int64_t n_windows(int64_t L) {
   return L >= kPoolKernel ? (L - kPoolKernel) / kPoolStride + 1 : 0;
@@ -132,6 +135,90 @@ __device__ inline void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
 // prologue early.  Both are no-ops without a programmatic predecessor.
 __device__ inline void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ inline void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------- clusters
+// Thread-block cluster primitives (distributed shared memory).  Addresses
+// of another CTA's shared memory are 32-bit shared::cluster addresses from
+// mapa.
+
+__device__ inline uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ inline uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ inline uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+
+// The address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ inline uint32_t map_shared_rank(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+
+__device__ inline void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+__device__ inline float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ inline float4 ld_cluster_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Split cluster barrier: every thread of every CTA of the cluster arrives
+// once and waits once per phase (arrive publishes this thread's earlier
+// writes, wait acquires everyone's).
+__device__ inline void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ inline void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+
+__device__ inline void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
+// Arrive on an mbarrier of another CTA of the cluster, releasing this
+// thread's earlier writes at cluster scope.
+__device__ inline void mbar_remote_arrive(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+
+// As mbar_wait, acquiring at cluster scope: for phases completed by other
+// CTAs' remote arrivals.
+__device__ inline bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                         uint32_t max_iters = kWaitLimitIters, uint32_t suspend_ns = 100000u) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0; it < max_iters; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    if (done) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) break;
+  }
+  set_status(status, NOSA_DEV_TIMEOUT);
+  return false;
+}
 
 // Order-preserving map of an fp32 score to uint32, with -0.0 == +0.0 and NaN
 // ranked as -inf (ties are then broken by index by the caller).

@@ -26,54 +26,42 @@ struct PoolArgs {
   int batch, hkv, nc_cap, max_new_keys;
 };
 
-struct SelectArgs {
-  const __nv_bfloat16* q;
-  const float* pooled;
+struct SelectArgs {  // selection from given block scores (select_only_kernel)
   const int32_t* seq_len;
-  const float* bs_in;      // nullable: selection only
-  float* comp_out;         // nullable
-  float* bs_out;           // nullable
+  const float* bs_in;      // [pairs, nb_in]
   int32_t* sel_idx;
   int32_t* sel_cnt;
-  float* bscratch;         // [pairs, nb_ws] block scores of the scoring pass
-  uint32_t* tickets;       // [pairs]
   uint32_t* status;
-  int batch, hq, hkv, group, local_blocks, topk, max_seq_len;
-  int nc_cap, nb_in, nb_out, nb_ws;
-  float scale;
+  int batch, hkv, local_blocks, topk, max_seq_len, nb_in;
 };
 
-struct DecodeArgs {
-  const __nv_bfloat16* q;
-  const __nv_bfloat16* k_cache;
-  const __nv_bfloat16* v_cache;
-  int64_t cache_rows;
-  const int64_t* seq_start;
-  const int32_t* seq_len;
-  const int32_t* sel_idx;
-  const int32_t* sel_cnt;
-  __nv_bfloat16* out;
-  float* lse;        // nullable
-  float* part;       // [pairs, kMaxSplits, part_stride(group)] partial softmax state
-  uint32_t* tickets; // [pairs]
-  uint32_t* status;
-  int batch, hq, hkv, group, local_blocks, topk, max_seq_len;
-  int nsplit;
-  float scale_log2;  // softmax scale * log2(e)
-};
-
-// Work mix of one launch of the persistent step kernel.
-constexpr int kStepScore = 1;   // scoring items (+ top-k of each pair)
-constexpr int kStepDecode = 2;  // decode items
-constexpr int kStepAppend = 4;  // the first scoring item of a pair appends the new token and pools
+// Work of one launch of the decode-step kernel (any of the three parts).
+constexpr int kStepScore = 1;   // compressed scores, block scores and top-k of every pair
+constexpr int kStepDecode = 2;  // attention over the local window and the selected blocks
+constexpr int kStepAppend = 4;  // write the new token's K/V rows and pool the window it completes
 
 struct StepArgs {
-  SelectArgs sel;
-  DecodeArgs dec;
-  PoolArgs pool;
-  uint32_t* work;   // [2]: queue position, CTAs finished (zero between launches)
-  uint32_t* ready;  // [pairs]: selection published (zero between launches)
-  int mode, pairs, n_score_items, n_items;
+  const __nv_bfloat16* q;        // [batch, hq, 128]
+  const int32_t* seq_len;        // [batch]
+  const int64_t* seq_start;      // [batch] (decode / append)
+  int64_t cache_rows;
+  __nv_bfloat16* k_cache;        // [cache_rows, hkv, 128] (append writes; tiles come through tensor maps)
+  __nv_bfloat16* v_cache;
+  float* pooled;                 // [batch, hkv, nc_cap, 128] (append writes; scoring reads through a tensor map)
+  const __nv_bfloat16* k_new;    // [batch, hkv, 128], nullable (append)
+  const __nv_bfloat16* v_new;
+  int32_t* sel_idx;              // [pairs, topk]: written when scoring, read otherwise
+  int32_t* sel_cnt;              // [pairs]
+  float* comp_out;               // nullable: [batch, hq, nc_cap] compressed scores
+  float* bs_out;                 // nullable: [pairs, nb_out] block scores
+  float* bs_spill;               // nullable: [pairs, nb_spill] block scores kept in global memory
+  __nv_bfloat16* out;            // [batch, hq, 128] (decode)
+  float* lse;                    // nullable: [batch, hq]
+  uint32_t* status;
+  int batch, hq, hkv, local_blocks, topk, max_seq_len, nc_cap, nb_out, nb_spill;
+  int mode;
+  float scale;       // softmax scale
+  float scale_log2;  // softmax scale * log2(e)
 };
 
 // Launches `kernel` with programmatic stream serialization, so that it can be
@@ -96,22 +84,21 @@ cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 cudaError_t launch_pool_append(const PoolArgs& a, cudaStream_t stream);
-cudaError_t launch_step(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t stream);
+cudaError_t launch_step(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
+                        cudaStream_t stream);
 cudaError_t launch_select_only(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint32_t* status, uint32_t max_iters, cudaStream_t stream);
 
-// Bytes at the start of a workspace that must be zero before a call
-// (status word, work queue, tickets, ready flags); 0 for invalid parameters.
+// Block scores of a pair stay in shared memory up to this many candidates
+// (64 * 2048 tokens before the local window); beyond, they live in a
+// workspace region of pairs x candidates floats.
+constexpr int kSmemBlockScores = 2048;
+
+// Bytes at the start of a workspace that must be zero before a call (the
+// device status word); 0 for invalid parameters.
 size_t workspace_counter_bytes(const nosa_params* p, int batch, int max_seq_len);
 
 // Records `msg` as the calling thread's last error and returns `code`.
 int record_error(int code, const char* msg);
-
-// CTAs of the step kernel that fit on the current device at once.
-int step_resident_ctas(int group);
-
-// Splits per (sequence, KV head) for the decode items: about one item per
-// resident CTA, at most one per tile and kMaxSplits.
-void decode_split_plan(int pairs, int max_tiles, int num_ctas, int* nsplit);
 
 }  // namespace nosa

@@ -1,5 +1,5 @@
-// Compressed scores, block scores and top-k selection: device routines shared
-// by the selection-only kernel and the persistent decode-step kernel.
+// Compressed scores, block scores and top-k selection: device routines of the
+// selection-only kernel and the decode-step kernel.
 //
 // "NOSA-1B 模型家族全景" (demingchina.com), 核心原理: compressed attention
 // screens the history for the TopK blocks; "NOSA-1B 性能基准全解析" (wmrh.cn)
@@ -13,62 +13,11 @@
 //             ascending, -1 padded.
 #pragma once
 
+#include <cuda.h>
+
 #include "nosa_common.cuh"
 
 namespace nosa {
-
-constexpr int kChunkBlocks = 16;                                     // blocks per scoring item
-constexpr int kChunkWindows = kChunkBlocks * kWindowsPerBlock + 1;   // 65 pooled rows
-constexpr int kScoreStride = 68;                                     // floats per head row
-constexpr int kKeyBytes = kHeadDim * 4;                              // one fp32 pooled key
-constexpr int kScoreKeysBytes = kChunkWindows * kKeyBytes;           // 33,280
-constexpr int kScoreSmemBytes = kScoreKeysBytes + kMaxGroup * kScoreStride * 4;
-
-// Exchange half of `v` (N values) with lane ^ off; keep the half this lane's
-// side owns, added to the partner's copy of it.
-template <int N>
-__device__ inline void xpose_step(float* v, int lane, int off) {
-  const bool upper = (lane & off) != 0;
-#pragma unroll
-  for (int k = 0; k < N / 2; ++k) {
-    const float send = upper ? v[k] : v[k + N / 2];
-    const float keep = upper ? v[k + N / 2] : v[k];
-    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-  }
-}
-
-template <int G>
-__host__ __device__ constexpr int log2_of() {
-  return G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
-}
-
-// Sum over the 32 lanes of v[h] for the head h this lane ends up owning:
-// log2(G) halving exchanges, then 5 - log2(G) plain butterfly steps.
-template <int G>
-__device__ inline float group_warp_sum(float (&v)[G], int lane, int* head) {
-  int h = 0;
-  if constexpr (G >= 2) {
-    xpose_step<G>(v, lane, 16);
-    h += (lane & 16) ? G / 2 : 0;
-  }
-  if constexpr (G >= 4) {
-    xpose_step<G / 2>(v, lane, 8);
-    h += (lane & 8) ? G / 4 : 0;
-  }
-  if constexpr (G >= 8) {
-    xpose_step<G / 4>(v, lane, 4);
-    h += (lane & 4) ? G / 8 : 0;
-  }
-  if constexpr (G >= 16) {
-    xpose_step<G / 8>(v, lane, 2);
-    h += (lane & 2) ? G / 16 : 0;
-  }
-  float s = v[0];
-#pragma unroll
-  for (int o = 16 >> log2_of<G>(); o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  *head = h;
-  return s;
-}
 
 struct TopkShared {
   uint32_t hist[256];
@@ -306,145 +255,223 @@ __device__ void select_topk(const float* scores, bool coherent, int ncand, int t
   if (tid == 0) *sel_cnt = k_eff;
 }
 
-struct ScoreGeometry {
-  int L, nb, ncand, nchunks, b0, b1, jlo, jhi;
-  int64_t nc;
-};
-
-// Scores one chunk of 16 blocks of one (sequence i, KV head g) with NT
-// threads: one 1-D bulk (TMA) copy stages the chunk's pooled rows
-// [4*b0-1, 4*b1) in shared memory (`keys`), each warp scores one window at a
-// time with the group's queries in registers, and the block rule runs from
-// shared memory (`ssm`).  Writes block scores to `bscratch` (and the optional
-// outputs).  `bar` is this CTA's key barrier, `phase` its current parity.
-// Returns false when a bounded wait gave up.
-template <int G, int NT>
-__device__ bool score_chunk(const __nv_bfloat16* __restrict__ q, const float* __restrict__ pooled,
-                            int nc_cap, int hq, int hkv, int i, int g, float scale, const ScoreGeometry& geo,
-                            float* __restrict__ bscratch_row, float* __restrict__ comp_out,
-                            float* __restrict__ bs_out_row, uint8_t* smem, uint64_t* bar, uint32_t phase,
-                            uint32_t* status, uint64_t* trace_landed = nullptr) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* keys = reinterpret_cast<float*>(smem);
-  float* ssm = reinterpret_cast<float*>(smem + kScoreKeysBytes);
-  const int nwin = geo.jhi - geo.jlo;
-  if (geo.b1 <= geo.b0 || nwin <= 0) return true;
-  if (tid == 0) {
-    const uint32_t bytes = static_cast<uint32_t>(nwin) * kKeyBytes;
-    mbar_arrive_expect_tx(bar, bytes);
-    const float* src = pooled + ((static_cast<int64_t>(i) * hkv + g) * nc_cap + geo.jlo) * kHeadDim;
-    bulk_copy_g2s(keys, src, bytes, bar);
-  }
-  // The group's queries, dims 4*lane .. 4*lane+3, widened to fp32.
-  float4 qv[G];
-  const __nv_bfloat16* qbase = q + (static_cast<int64_t>(i) * hq + g * G) * kHeadDim;
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(qbase + hh * kHeadDim) + lane);
-    qv[hh] = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
-                         __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u));
-  }
-  const bool ok = mbar_wait(bar, phase, status);
-#ifdef NOSA_TRACE
-  if (tid == 0 && trace_landed) *trace_landed = global_timer_ns();
-  if (lane == 0 && trace_landed) atomicMax(reinterpret_cast<unsigned long long*>(trace_landed + 3),
-                                           static_cast<unsigned long long>(global_timer_ns()));
-#endif
-  if (ok) {
-    // Four windows per warp and iteration: four independent reduction chains
-    // keep the shuffle pipeline busy.
-    constexpr int kWin = 4;
-    const int writer_mask = 32 / G - 1;
-    for (int j0 = warp * kWin; j0 < nwin; j0 += (NT / 32) * kWin) {
-      float v[kWin][G];
-#pragma unroll
-      for (int w = 0; w < kWin; ++w) {
-        const int jj = min(j0 + w, nwin - 1);
-        const float4 kv = reinterpret_cast<const float4*>(keys + jj * kHeadDim)[lane];
-        if constexpr (G >= 2) {
-          // Two heads per packed fp32x2 FMA; each head's sum keeps the order
-          // x, y, z, w of the scalar form (same rounding).
-#pragma unroll
-          for (int hh = 0; hh < G; hh += 2) {
-            float2 d = __fmul2_rn(make_float2(qv[hh].x, qv[hh + 1].x), make_float2(kv.x, kv.x));
-            d = __ffma2_rn(make_float2(qv[hh].y, qv[hh + 1].y), make_float2(kv.y, kv.y), d);
-            d = __ffma2_rn(make_float2(qv[hh].z, qv[hh + 1].z), make_float2(kv.z, kv.z), d);
-            d = __ffma2_rn(make_float2(qv[hh].w, qv[hh + 1].w), make_float2(kv.w, kv.w), d);
-            v[w][hh] = d.x;
-            v[w][hh + 1] = d.y;
-          }
-        } else {
-          float d = qv[0].x * kv.x;
-          d = fmaf(qv[0].y, kv.y, d);
-          d = fmaf(qv[0].z, kv.z, d);
-          d = fmaf(qv[0].w, kv.w, d);
-          v[w][0] = d;
+// Exact top-k by one warp over any number of candidates held in memory
+// (shared, or global when `coherent`): warp_topk's threshold search and
+// compaction, with the keys re-read on every step instead of kept in
+// registers.  For candidate sets beyond warp_topk's register capacity.
+__device__ inline void warp_topk_mem(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
+                                     int32_t* sel_cnt, int lane) {
+  auto key_at = [&](int b) { return order_key(coherent ? __ldcg(scores + b) : scores[b]); };
+  const int k_eff = ncand < topk ? ncand : topk;
+  uint32_t T = 0u;
+  uint32_t need = 0u;
+  if (k_eff < ncand) {
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (int b = lane; b < ncand; b += 32) {
+      const uint32_t k = key_at(b);
+      lo = min(lo, k);
+      hi = max(hi, k);
+    }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t k = static_cast<uint32_t>(k_eff);
+    if (lo != hi) {
+      const int top = 31 - __clz(lo ^ hi);
+      T = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+      int bit = top;
+      if ((top & 1) == 0) {
+        const uint32_t c1 = T | (1u << bit);
+        uint32_t n1 = 0;
+        for (int b = lane; b < ncand; b += 32) n1 += key_at(b) >= c1;
+        if (__reduce_add_sync(0xffffffffu, n1) >= k) T = c1;
+        --bit;
+      }
+      for (bit -= 1; bit >= 0; bit -= 2) {
+        const uint32_t c1 = T | (1u << bit), c2 = T | (2u << bit), c3 = T | (3u << bit);
+        uint32_t n1 = 0, n2 = 0, n3 = 0;
+        for (int b = lane; b < ncand; b += 32) {
+          const uint32_t key = key_at(b);
+          n1 += key >= c1;
+          n2 += key >= c2;
+          n3 += key >= c3;
         }
+        n1 = __reduce_add_sync(0xffffffffu, n1);
+        n2 = __reduce_add_sync(0xffffffffu, n2);
+        n3 = __reduce_add_sync(0xffffffffu, n3);
+        T = n3 >= k ? c3 : n2 >= k ? c2 : n1 >= k ? c1 : T;
       }
-#pragma unroll
-      for (int w = 0; w < kWin; ++w) {
-        int head;
-        const float s = group_warp_sum<G>(v[w], lane, &head);
-        if ((lane & writer_mask) == 0 && j0 + w < nwin) ssm[head * kScoreStride + j0 + w] = s * scale;
-      }
+    } else {
+      T = hi;
     }
-#ifdef NOSA_TRACE
-    if (lane == 0 && trace_landed) atomicMax(reinterpret_cast<unsigned long long*>(trace_landed + 4),
-                                             static_cast<unsigned long long>(global_timer_ns()));
-#endif
+    uint32_t above = 0;
+    for (int b = lane; b < ncand; b += 32) above += key_at(b) > T;
+    need = k - __reduce_add_sync(0xffffffffu, above);
   }
-  __syncthreads();
-  if (ok) {
-    if (comp_out) {
-      const int jo0 = kWindowsPerBlock * geo.b0, jo1 = geo.jhi;
-      const int span = jo1 - jo0;
-      for (int t = tid; t < G * span; t += NT) {
-        const int hh = t / span, j = jo0 + t % span;
-        comp_out[(static_cast<int64_t>(i) * hq + g * G + hh) * nc_cap + j] = ssm[hh * kScoreStride + (j - geo.jlo)];
-      }
-    }
-    const int bend = min(geo.b1, geo.ncand);
-    for (int t = tid; t < bend - geo.b0; t += NT) {
-      const int b = geo.b0 + t;
-      // J(b) = {4b-1, ..., 4b+3} clipped to [0, nc): a fixed 5-step loop with
-      // predication keeps the shared-memory loads independent.
-      const int jb = kWindowsPerBlock * b - 1;
-      float S = 0.0f;
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        float m = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kWindowsPerBlock + 1; ++w) {
-          const int j = jb + w;
-          if (j >= 0 && j < geo.nc) m = fmaxf(m, ssm[hh * kScoreStride + (j - geo.jlo)]);
-        }
-        S += m;
-      }
-      bscratch_row[b] = S;
-      if (bs_out_row) bs_out_row[b] = S;
-    }
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int pos = 0;
+  uint32_t eq_seen = 0;
+  for (int base = 0; base < ncand; base += 32) {
+    const int b = base + lane;
+    const bool valid = b < ncand;
+    const uint32_t key = valid ? key_at(b) : 0u;
+    const bool eq = valid && k_eff < ncand && key == T;
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    const bool take = valid && (key > T || (k_eff == ncand) || (eq && eq_seen + __popc(eb & lt_mask) < need));
+    const uint32_t tb = __ballot_sync(0xffffffffu, take);
+    const int p = pos + __popc(tb & lt_mask);
+    if (take && p < topk) sel_row[p] = b;
+    eq_seen += __popc(eb);
+    pos += __popc(tb);
   }
-  return ok;
+  for (int t = k_eff + lane; t < topk; t += 32) sel_row[t] = -1;
+  if (lane == 0) *sel_cnt = k_eff;
 }
 
-// Geometry of scoring item `chunk` of a sequence of length L (L valid).
-// `full` = scores wanted for every window (comp_out) rather than only the
-// windows the selection reads.
-__device__ inline ScoreGeometry score_geometry(int L, int nc_cap, int local_blocks, bool full, int chunk) {
-  ScoreGeometry g;
-  g.L = L;
-  g.nc = n_windows(L);
-  if (g.nc > nc_cap) g.nc = nc_cap;
-  g.nb = static_cast<int>(n_blocks(L));
-  g.ncand = static_cast<int>(n_candidates(L, local_blocks));
-  const int nbw = full ? g.nb : g.ncand;
-  g.nchunks = nbw > 0 ? (nbw + kChunkBlocks - 1) / kChunkBlocks : 1;
-  g.b0 = chunk * kChunkBlocks;
-  g.b1 = min(g.b0 + kChunkBlocks, nbw);
-  g.jlo = max(0, kWindowsPerBlock * g.b0 - 1);
-  const int64_t jh = static_cast<int64_t>(kWindowsPerBlock) * g.b1;
-  g.jhi = static_cast<int>(g.nc < jh ? g.nc : jh);
-  return g;
+// Top-k by one warp: register-resident keys up to kWarpTopkMax candidates,
+// memory-resident beyond.
+__device__ inline void warp_select(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
+                                   int32_t* sel_cnt, int lane) {
+  if (ncand <= 256)
+    warp_topk<8>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
+  else if (ncand <= kWarpTopkMax)
+    warp_topk<32>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
+  else
+    warp_topk_mem(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
+}
+
+// ---------------------------------------------------------------- scoring
+// A scoring chunk k of a (sequence, KV head) covers blocks [15k, 15k+15)
+// and pooled windows [60k-1, 60k+60) (61 rows; row r is window 60k-1+r).
+// Its rows arrive as four 2-D TMA boxes of {32 fp32 columns, 61 rows}
+// (128-byte swizzle), box c holding dimensions [32c, 32c+32), each in an
+// 8 KB slot (64 rows) of one ring stage.
+constexpr int kScoreSlotBytes = 64 * 128;                          // 8 KB
+constexpr uint32_t kScoreTxBytes = 4u * kBoxRows * kBoxCols * 4u;  // bytes landed per chunk
+constexpr int kScoreStride = 64 + 4;                               // floats per head row of window scores
+
+__device__ inline uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+__device__ inline void mma_tf32_1688(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// 2-D tiled TMA load of one {32 columns, 61 rows} fp32 box of the pooled keys.
+__device__ inline void tma_load_keys(void* dst, const CUtensorMap* map, int col, int row, uint64_t* bar,
+                                     uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(col), "r"(row), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+template <int G>
+struct ScoreQ {
+  static constexpr int kNTiles = G > 8 ? 2 : 1;  // n-tiles of 8 heads
+  uint32_t b[kNTiles][16][2];
+};
+
+// The group's queries as TF32 B fragments of mma m16n8k8 (k = dimension,
+// n = head; heads >= G are zero).  bf16 widens to TF32 exactly.
+template <int G>
+__device__ inline void load_score_q(ScoreQ<G>& f, const __nv_bfloat16* __restrict__ q_group, int lane) {
+  const int grp = lane >> 2, tig = lane & 3;
+  const uint16_t* bits = reinterpret_cast<const uint16_t*>(q_group);
+#pragma unroll
+  for (int nt = 0; nt < ScoreQ<G>::kNTiles; ++nt) {
+    const int head = nt * 8 + grp;
+#pragma unroll
+    for (int ks = 0; ks < 16; ++ks) {
+      f.b[nt][ks][0] = head < G ? static_cast<uint32_t>(__ldg(bits + head * kHeadDim + 8 * ks + tig)) << 16 : 0u;
+      f.b[nt][ks][1] = head < G ? static_cast<uint32_t>(__ldg(bits + head * kHeadDim + 8 * ks + tig + 4)) << 16 : 0u;
+    }
+  }
+}
+
+// Compressed scores of one chunk on the tensor cores: consumer warp w
+// computes rows [16w, 16w+16) of S^T = K * Q^T (mma.sync m16n8k8, TF32
+// inputs, fp32 accumulation) and stores scale * s into ssm[head][row] for
+// rows < 61.  Each fp32 pooled value x is split into hi (x with its low 13
+// mantissa bits cleared, exact in TF32) and lo = tf32(x - hi); the hi and lo
+// products go to separate fp32 accumulators that are added at the end, so
+// the only input rounding is that of lo, below 2^-21 of |x| ("NOSA-1B
+// 性能基准全解析" §三.3: scores of the pooled keys).
+template <int G>
+__device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* __restrict__ ssm, float scale,
+                                   int warp, int lane) {
+  constexpr int NT = ScoreQ<G>::kNTiles;
+  const int grp = lane >> 2, tig = lane & 3;
+  const int r0 = warp * 16;
+  const int ra = r0 + grp, rb = ra + 8;
+  float acc_hi[NT][4], acc_lo[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc_hi[nt][e] = acc_lo[nt][e] = 0.0f;
+#pragma unroll
+  for (int ks = 0; ks < 16; ++ks) {
+    const uint32_t box = stage + (ks >> 2) * kScoreSlotBytes;
+    const int unit = 2 * (ks & 3);  // 16-byte unit of dimension 8*(ks%4) within the 128-byte row
+    float x[4];
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(x[0]) : "r"(box + ra * 128 + ((unit ^ (ra & 7)) << 4) + tig * 4));
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(x[1]) : "r"(box + rb * 128 + ((unit ^ (rb & 7)) << 4) + tig * 4));
+    asm volatile("ld.shared.f32 %0, [%1];"
+                 : "=f"(x[2])
+                 : "r"(box + ra * 128 + (((unit + 1) ^ (ra & 7)) << 4) + tig * 4));
+    asm volatile("ld.shared.f32 %0, [%1];"
+                 : "=f"(x[3])
+                 : "r"(box + rb * 128 + (((unit + 1) ^ (rb & 7)) << 4) + tig * 4));
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      hi[e] = __float_as_uint(x[e]) & 0xffffe000u;
+      const float r = x[e] - __uint_as_float(hi[e]);  // exact; NaN only for infinite x
+      lo[e] = to_tf32(r == r ? r : 0.0f);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      mma_tf32_1688(acc_hi[nt], hi, qf.b[nt][ks][0], qf.b[nt][ks][1]);
+      mma_tf32_1688(acc_lo[nt], lo, qf.b[nt][ks][0], qf.b[nt][ks][1]);
+    }
+  }
+  // acc[nt][0..1]: row ra, heads nt*8 + 2*tig + {0,1}; [2..3]: row rb.
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int head = nt * 8 + 2 * tig + (e & 1);
+      const int row = (e >> 1) ? rb : ra;
+      if (head < G && row < kChunkWindows) ssm[head * kScoreStride + row] = (acc_hi[nt][e] + acc_lo[nt][e]) * scale;
+    }
+  }
+}
+
+// Block rule for block b = 15k + t of chunk k (t < 15) from the chunk's
+// window scores: S[b] = sum over the group's heads (ascending) of the max of
+// s over windows 4b-1 .. 4b+3 that exist (0 <= j < nc), i.e. rows 4t .. 4t+4.
+template <int G>
+__device__ inline float block_rule(const float* __restrict__ ssm, int k, int t, int64_t nc) {
+  const int64_t jb = static_cast<int64_t>(kWindowsPerBlock) * (kChunkBlocks * k + t) - 1;
+  float S = 0.0f;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWindowsPerBlock + 1; ++w) {
+      const int64_t j = jb + w;
+      if (j >= 0 && j < nc) m = fmaxf(m, ssm[h * kScoreStride + 4 * t + w]);
+    }
+    S += m;
+  }
+  return S;
 }
 
 }  // namespace nosa

@@ -1,244 +1,552 @@
-// Kernels for selection, sparse attention and the fused decode step.
+// The decode step: one kernel launch, one thread-block cluster of C CTAs per
+// (sequence, KV head) pair.
 //
-// One persistent kernel, `step_kernel<G>`, runs any mix of two kinds of work
-// items from an atomic work queue held in the workspace:
-//   * scoring items (sequence i, KV head g, chunk of 16 blocks): compressed
-//     scores and block scores of the chunk; the last chunk of a pair (atomic
-//     ticket) selects its top-k ("NOSA-1B 性能基准全解析" §三.2/§三.3);
-//   * decode items (i, g, split): exact attention over that split of the
-//     pair's tiles (§三.3 / §三.2 local window).
-// Scoring items are handed out first.  In the fused decode step the first
-// scoring item of each pair also appends the new token's K/V rows and pools
-// the window the token completes ("从论文到代码…" item 2), and each decode
-// item streams its local-window tiles at once but waits -- a bounded spin on
-// the pair's ready flag, published with a release store by the CTA that
-// selected the pair's blocks -- before its first tile that depends on the
-// selection or on the appended token.  Items are dispensed in index order to
-// resident CTAs only (the grid never exceeds what fits on the GPU), so every
-// scoring item a decode item waits for is already running: no deadlock.
-// The last CTA to leave resets the queue; tickets and flags are reset by
-// their last users, so the workspace is ready for the next launch.
+// What a step computes ("NOSA-1B 性能基准全解析" (wmrh.cn) §三.2 / §三.3;
+// "从论文到代码：手把手教你理解NOSA-8B的高效注意力机制实现" (nzsm.cn) item 2):
+// append the new token's K/V rows and pool the window it completes; score
+// the pooled keys with the group's queries and reduce them to block scores;
+// select the top-k blocks; attend exactly over the selected blocks and the
+// local window.  Any subset of the three parts runs (kStepScore,
+// kStepDecode, kStepAppend), so the same kernel serves the fused step and
+// the separate selection / attention entry points.
+//
+// Work split inside a cluster (rank r of C):
+//   * scoring chunks k = r, r + C, ... (15 blocks = 61 pooled rows each);
+//   * attention tiles t = r, r + C, ... of the pair's tile list (the local
+//     blocks, then the selected blocks in ascending order).
+// Roles inside a CTA (192 threads):
+//   * warps 0-3, consumers: tensor-core scoring of a staged chunk (block
+//     rule, block scores sent to every CTA of the cluster through
+//     distributed shared memory), then the attention tiles (online softmax
+//     per warp);
+//   * warp 4, producer: issues every TMA copy of the CTA in job order --
+//     scoring chunks, local tiles, selected tiles (after the selection) --
+//     into a 3-stage ring of 32 KB stages (full / empty mbarriers);
+//   * warp 5, selector: pools the window completed by the new token (rank
+//     0), waits until the block scores of the whole pair have arrived (one
+//     remote mbarrier arrival per CTA), runs the exact top-k (every CTA
+//     computes the same selection, so no second exchange is needed) and
+//     hands the selected blocks to the producer; rank 0 writes the
+//     selection out.
+// Merge: each CTA merges its four warps into one partial (O, m, l) in its
+// shared memory; after a cluster barrier, CTA r combines the partials of
+// all C CTAs (fixed order) for its share of the output elements; a last
+// cluster barrier keeps every CTA resident until its partial has been read.
+//
+// No global-memory flags, tickets or work queues: the only cross-CTA
+// traffic is inside the cluster, and every wait is bounded (status bit
+// NOSA_DEV_TIMEOUT), so a launch always finishes.
 #include "decode_device.cuh"
 #include "nosa_common.cuh"
 #include "nosa_kernels.h"
 #include "pool_device.cuh"
 #include "select_device.cuh"
 
+#include <mutex>
+
 namespace nosa {
 
 #ifdef NOSA_TRACE
-// Instrumented builds only (-DNOSA_TRACE): one record per work item of the
-// step kernel -- CTA, SM, item, start / selection-seen / end globaltimer.
+// Instrumented builds only (-DNOSA_TRACE): one record per CTA of the step
+// kernel with %globaltimer stamps of its phases.
 struct TraceRecord {
-  uint32_t cta, smid, item, clk_delta;  // clk_delta: SM clock cycles spent in the item
-  uint64_t t_start, t_flag, t_end;
-  uint32_t issue[8], full[8], done[8];  // per tile, ns after t_start
-  uint32_t merge[6];                     // decode merge phase, ns after t_start
+  uint32_t pair, rank, smid, csize;
+  uint64_t t[8];  // start, scoring issued, scores sent, scores gathered, selection done, tiles done, -, end
 };
 constexpr int kTraceCapacity = 1 << 16;
 __device__ TraceRecord g_trace[kTraceCapacity];
 __device__ uint32_t g_trace_count;
+#define NOSA_STAMP(k) (sh.tr[k] = global_timer_ns())
+#else
+#define NOSA_STAMP(k) ((void)0)
 #endif
 
 namespace {
 
-constexpr int kSelOnlyThreads = 256;
+constexpr int kProducerWarp = kConsumerWarps;            // 4
+constexpr int kSelectorWarp = kConsumerWarps + 1;        // 5
+constexpr int kStepThreads = (kConsumerWarps + 2) * 32;  // 192
+constexpr int kConsumerThreads = kConsumerWarps * 32;    // 128
 constexpr int kCtasPerSm = 2;
+constexpr int kSelOnlyThreads = 256;
+
+struct StepShared {
+  uint64_t full_bar[kStages];
+  uint64_t empty_bar[kStages];
+  uint64_t scores_bar;  // completes when every CTA of the cluster has sent its block scores
+  uint64_t sel_bar;     // completes when the selection is in shared memory (selector -> producer)
+  int stage_blk[kStages];
+  int sel_count;
+  float blk[kChunkBlocks];  // block scores of the chunk being sent
+#ifdef NOSA_TRACE
+  uint64_t tr[8];
+#endif
+};
+
+// Shared memory of the step kernel (dynamic, from a 1024-byte aligned base):
+//   ring  kRingBytes                      kStages stages of 32 KB
+//   ssm   G x kScoreStride floats         window scores of the chunk being scored
+//   sel   round16(4 * topk) bytes         the pair's selection (ascending block indices)
+//   bsm   4 * ncand_max bytes             the pair's block scores (unless kept in global memory)
+template <int G>
+__host__ __device__ constexpr int ssm_bytes() {
+  return G * kScoreStride * 4;
+}
+__host__ __device__ constexpr int round16(int x) { return (x + 15) & ~15; }
+
+// Named barrier of the four consumer warps.
+__device__ inline void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory"); }
+
+// Named barrier of the consumer warps that also returns whether `v` holds in
+// all of them (so that they leave a loop together).
+__device__ inline bool consumer_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kConsumerThreads)
+      : "memory");
+  return r != 0;
+}
+
+// Cross-warp merge scratch (in the drained ring): per warp O rows with a
+// padded stride (bank-conflict free float2 stores), row max / sum / weight,
+// then the CTA's partial that the other CTAs of the cluster read.
+constexpr int kMoStride = kHeadDim + 8;
+template <int G>
+struct MergeLayout {
+  static constexpr int kMo = 0;                                      // [4][G][kMoStride]
+  static constexpr int kMm = kMo + kConsumerWarps * G * kMoStride;   // [4][G]
+  static constexpr int kMl = kMm + kConsumerWarps * G;               // [4][G]
+  static constexpr int kMw = kMl + kConsumerWarps * G;               // [4][G]
+  static constexpr int kPart = (kMw + kConsumerWarps * G + 3) & ~3;  // [G][128] partial O
+  static constexpr int kPm = kPart + G * kHeadDim;                   // [G] partial row max
+  static constexpr int kPl = kPm + G;                                // [G] partial row sum
+};
+static_assert((MergeLayout<kMaxGroup>::kPl + kMaxGroup) * 4 <= kRingBytes, "merge scratch must fit in the ring");
+
+template <int G>
+__global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
+    step_kernel(const StepArgs a, const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const __grid_constant__ CUtensorMap tm_p) {
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte swizzled TMA boxes want 1024-byte aligned destinations.
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* ssm = reinterpret_cast<float*>(smem + kRingBytes);
+  int32_t* sel_list = reinterpret_cast<int32_t*>(smem + kRingBytes + ssm_bytes<G>());
+  float* bsm = reinterpret_cast<float*>(smem + kRingBytes + ssm_bytes<G>() + round16(4 * a.topk));
+  __shared__ StepShared sh;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t C = cluster_nctarank(), rank = cluster_ctarank();
+  const int pair = static_cast<int>(cluster_id_x());
+  const bool scoring = (a.mode & kStepScore) != 0;
+  const bool decoding = (a.mode & kStepDecode) != 0;
+  const bool appending = (a.mode & kStepAppend) != 0;
+  const bool spill = a.bs_spill != nullptr;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh.full_bar[s], 1);
+      mbar_init(&sh.empty_bar[s], kConsumerWarps);
+    }
+    mbar_init(&sh.scores_bar, C);
+    mbar_init(&sh.sel_bar, 1);
+    fence_barrier_init();
+#ifdef NOSA_TRACE
+    for (int k = 0; k < 8; ++k) sh.tr[k] = 0;
+    NOSA_STAMP(0);
+#endif
+  }
+  __syncthreads();
+  // Cluster barrier phase 1: this CTA's barriers exist.  Each thread waits
+  // on it before its first access to another CTA's shared memory.
+  cluster_arrive();
+  if (warp == kProducerWarp && lane == 0) {
+    if (scoring) asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_p) : "memory");
+    if (decoding) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_k) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_v) : "memory");
+    }
+  }
+  grid_dependency_wait();
+  allow_dependents();
+
+  // ---------------------------------------------------------------- geometry
+  // (identical in every CTA of the cluster)
+  const int i = pair / a.hkv, g = pair % a.hkv;
+  const int L = a.seq_len[i];
+  const bool bad_len = L < 1 || L > a.max_seq_len;
+  const bool uses_cache = decoding || appending;
+  const int64_t seq_base = uses_cache && !bad_len ? a.seq_start[i] : 0;
+  const bool bad_rows = uses_cache && !bad_len && (seq_base < 0 || seq_base + L > a.cache_rows);
+  const int Lv = bad_len ? 0 : L;
+  const int nb = static_cast<int>(n_blocks(Lv));
+  const int ncand = static_cast<int>(n_candidates(Lv, a.local_blocks));
+  const int nloc = nb - ncand;
+  const int64_t nc_all = n_windows(Lv);
+  const int64_t nc = nc_all < a.nc_cap ? nc_all : a.nc_cap;
+  const int cnt_max = min(a.topk, ncand);
+  const int nchunks = scoring ? ((a.comp_out ? nb : ncand) + kChunkBlocks - 1) / kChunkBlocks : 0;
+  int cnt = cnt_max;
+  if (decoding && !scoring && !bad_len) {
+    cnt = a.sel_cnt[pair];
+    if (cnt < 0 || cnt > cnt_max) {
+      if (rank == 0 && tid == 0) set_status(a.status, NOSA_DEV_BAD_COUNT);
+      cnt = cnt < 0 ? 0 : cnt_max;
+    }
+  }
+  const int ntiles = decoding && !bad_rows ? nloc + cnt : 0;
+  if (rank == 0 && tid == 0) {
+    if (bad_len) set_status(a.status, L < 1 ? NOSA_DEV_BAD_LENGTH : NOSA_DEV_MAX_LEN);
+    if (bad_rows) set_status(a.status, NOSA_DEV_CACHE_ROWS);
+    if (scoring && nc_all > a.nc_cap) set_status(a.status, NOSA_DEV_NC_CAP);
+  }
+  const __nv_bfloat16* q_group = a.q + (static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G) * kHeadDim;
+
+  AttnState att;
+  if (warp == kProducerWarp) {
+    // ---------------------------------------------------------------- producer
+    const uint64_t policy = l2_evict_first_policy();
+    uint32_t r = 0;  // jobs issued
+    bool ok = true;
+    // Lane 0 waits for the stage, then issues the job's boxes.
+    auto issue = [&](auto&& body) {
+      int good = 1;
+      if (lane == 0) {
+        const int s = static_cast<int>(r % kStages);
+        if (r >= static_cast<uint32_t>(kStages) && !mbar_wait(&sh.empty_bar[s], ((r / kStages) - 1) & 1u, a.status))
+          good = 0;
+        else
+          body(s, smem + s * kStageBytes);
+      }
+      ok = __shfl_sync(0xffffffffu, good, 0) != 0;
+      if (ok) ++r;
+    };
+    const int row_base = pair * a.nc_cap;  // first pooled row of the pair (host: rows < 2^31)
+    for (int k = static_cast<int>(rank); k < nchunks && ok; k += static_cast<int>(C)) {
+      issue([&](int s, uint8_t* st) {
+        const int row0 = row_base + kChunkBlocks * kWindowsPerBlock * k - 1;
+        mbar_arrive_expect_tx(&sh.full_bar[s], kScoreTxBytes);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tma_load_keys(st + c * kScoreSlotBytes, &tm_p, c * kBoxCols, row0, &sh.full_bar[s], policy);
+      });
+    }
+#ifdef NOSA_TRACE
+    if (lane == 0) NOSA_STAMP(1);
+#endif
+    bool have_sel = false, sel_ok = false;
+    for (int t = static_cast<int>(rank); t < ntiles && ok; t += static_cast<int>(C)) {
+      int blk = -1;
+      if (t < nloc) {
+        blk = ncand + t;
+      } else {
+        if (!have_sel) {
+          int got = 0;
+          if (lane == 0) got = mbar_wait(&sh.sel_bar, 0, a.status) ? 1 : 0;
+          sel_ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+          have_sel = true;
+        }
+        if (lane == 0 && sel_ok) {
+          blk = sel_list[t - nloc];
+          if (blk < 0 || blk >= ncand) {
+            set_status(a.status, NOSA_DEV_BAD_INDEX);
+            blk = -1;
+          }
+        }
+      }
+      if (appending && t == nloc - 1 && a.k_new != nullptr) {
+        // This tile holds token L-1: write the new K/V rows first and order
+        // them before the tile's TMA read (same CTA, async proxy).
+        const int64_t row = (seq_base + L - 1) * a.hkv + g;
+        const int64_t src = static_cast<int64_t>(i) * a.hkv + g;
+        reinterpret_cast<uint2*>(a.k_cache + row * kHeadDim)[lane] =
+            reinterpret_cast<const uint2*>(a.k_new + src * kHeadDim)[lane];
+        reinterpret_cast<uint2*>(a.v_cache + row * kHeadDim)[lane] =
+            reinterpret_cast<const uint2*>(a.v_new + src * kHeadDim)[lane];
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+      }
+      issue([&](int s, uint8_t* st) {
+        sh.stage_blk[s] = blk;
+        const int row = static_cast<int>(seq_base + (blk < 0 ? 0 : static_cast<int64_t>(blk) * kBlock));
+        mbar_arrive_expect_tx(&sh.full_bar[s], kTileTxBytes);
+        tma_load_box(st, &tm_k, 0, g, row, &sh.full_bar[s], policy);
+        tma_load_box(st + kHalfBytes, &tm_k, 64, g, row, &sh.full_bar[s], policy);
+        tma_load_box(st + 2 * kHalfBytes, &tm_v, 0, g, row, &sh.full_bar[s], policy);
+        tma_load_box(st + 3 * kHalfBytes, &tm_v, 64, g, row, &sh.full_bar[s], policy);
+      });
+    }
+    // Every copy issued has landed before the ring is reused for the merge.
+    if (lane == 0) {
+      const uint32_t first = r > static_cast<uint32_t>(kStages) ? r - kStages : 0u;
+      for (uint32_t n = first; n < r; ++n) mbar_wait(&sh.full_bar[n % kStages], (n / kStages) & 1u, a.status);
+    }
+    __syncwarp();
+    cluster_wait();
+  } else if (warp == kSelectorWarp) {
+    // ---------------------------------------------------------------- selector
+    cluster_wait();
+    if (appending && rank == 0 && !bad_len && !bad_rows) {
+      // Pool the window that token L-1 completes (it lies in the local
+      // window, so this step's selection never reads it).
+      const int64_t j = n_windows(L) - 1;
+      if (j >= 0 && j >= n_windows(L - 1)) {
+        if (j >= a.nc_cap) {
+          if (lane == 0) set_status(a.status, NOSA_DEV_NC_CAP);
+        } else {
+          const uint2* knew = a.k_new ? reinterpret_cast<const uint2*>(
+                                            a.k_new + (static_cast<int64_t>(i) * a.hkv + g) * kHeadDim)
+                                      : nullptr;
+          pool_window_warp(a.k_cache, a.hkv, seq_base, g, j, knew ? L - 1 : -1, knew,
+                           a.pooled + (static_cast<int64_t>(pair) * a.nc_cap + j) * kHeadDim, lane);
+        }
+      }
+    }
+    if (scoring) {
+      const bool ok = mbar_wait_cluster(&sh.scores_bar, 0, a.status);
+#ifdef NOSA_TRACE
+      if (lane == 0) NOSA_STAMP(3);
+#endif
+      if (ok) {
+        const float* src = spill ? a.bs_spill + static_cast<int64_t>(pair) * a.nb_spill : bsm;
+        warp_select(src, spill, ncand, a.topk, sel_list, &sh.sel_count, lane);
+      } else {
+        for (int t = lane; t < a.topk; t += 32) sel_list[t] = -1;
+        if (lane == 0) sh.sel_count = 0;
+      }
+      __syncwarp();
+      if (rank == 0) {
+        int32_t* dst = a.sel_idx + static_cast<int64_t>(pair) * a.topk;
+        for (int t = lane; t < a.topk; t += 32) dst[t] = sel_list[t];
+        if (lane == 0) a.sel_cnt[pair] = sh.sel_count;
+      }
+    } else if (decoding) {
+      const int32_t* src = a.sel_idx + static_cast<int64_t>(pair) * a.topk;
+      for (int t = lane; t < cnt; t += 32) sel_list[t] = src[t];
+    }
+    __syncwarp();
+#ifdef NOSA_TRACE
+    if (lane == 0) NOSA_STAMP(4);
+#endif
+    if (lane == 0) mbar_arrive(&sh.sel_bar);
+  } else {
+    // ---------------------------------------------------------------- consumers
+    cluster_wait();
+    uint32_t r = 0;  // jobs consumed
+    bool ok = true;
+    if (scoring) {
+      if (static_cast<int>(rank) < nchunks) {
+        ScoreQ<G> qf;
+        load_score_q<G>(qf, q_group, lane);
+        for (int k = static_cast<int>(rank); k < nchunks; k += static_cast<int>(C)) {
+          const int s = static_cast<int>(r % kStages);
+          const bool landed = consumer_all(mbar_wait(&sh.full_bar[s], (r / kStages) & 1u, a.status));
+          if (!landed) {
+            ok = false;
+            break;
+          }
+          score_stage<G>(qf, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
+          ++r;
+          consumer_sync();  // the chunk's window scores are complete
+          const int b0 = kChunkBlocks * k;
+          const int nblk = min(kChunkBlocks, ncand - b0);
+          if (tid < nblk) {
+            const float S = block_rule<G>(ssm, k, tid, nc);
+            sh.blk[tid] = S;
+            if (a.bs_out) a.bs_out[static_cast<int64_t>(pair) * a.nb_out + b0 + tid] = S;
+            if (spill) a.bs_spill[static_cast<int64_t>(pair) * a.nb_spill + b0 + tid] = S;
+          }
+          if (a.comp_out) {
+            // windows [60k, min(60k + 60, nc)); the row of window j is j - 60k + 1
+            const int64_t j0 = static_cast<int64_t>(kChunkBlocks) * kWindowsPerBlock * k;
+            constexpr int kWin = kChunkBlocks * kWindowsPerBlock;
+            for (int t = tid; t < G * kWin; t += kConsumerThreads) {
+              const int h = t / kWin, x = t % kWin;
+              if (j0 + x < nc)
+                a.comp_out[(static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G + h) * a.nc_cap + j0 + x] =
+                    ssm[h * kScoreStride + x + 1];
+            }
+          }
+          consumer_sync();  // sh.blk is complete; ssm may be overwritten
+          if (!spill)
+            for (int x = tid; x < nblk * static_cast<int>(C); x += kConsumerThreads) {
+              const int b = x / static_cast<int>(C);
+              const uint32_t dst = static_cast<uint32_t>(x % static_cast<int>(C));
+              st_cluster_f32(map_shared_rank(smem_addr(bsm + b0 + b), dst), sh.blk[b]);
+            }
+        }
+      }
+      // Tell every CTA of the cluster (this one included) that this CTA's
+      // block scores are in place.
+      fence_acq_rel_cluster();
+      consumer_sync();
+      if (tid == 0) {
+        for (uint32_t d = 0; d < C; ++d) mbar_remote_arrive(map_shared_rank(smem_addr(&sh.scores_bar), d));
+        NOSA_STAMP(2);
+      }
+    }
+    attn_init(att);
+    if (decoding && ok) {
+      const int my_tiles = ntiles > static_cast<int>(rank)
+                               ? (ntiles - static_cast<int>(rank) + static_cast<int>(C) - 1) / static_cast<int>(C)
+                               : 0;
+      if (my_tiles > 0) {
+        uint32_t qa[8][4];
+        load_attn_q(qa, q_group, G, lane);
+        for (int n = 0; n < my_tiles; ++n) {
+          const int s = static_cast<int>(r % kStages);
+          if (!mbar_wait(&sh.full_bar[s], (r / kStages) & 1u, a.status)) break;
+          attend_tile(att, qa, smem + s * kStageBytes, sh.stage_blk[s], L, a.scale_log2, warp, lane);
+          if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
+          ++r;
+        }
+      }
+      attn_finish(att);
+    }
+  }
+  __syncthreads();  // the ring is drained: reuse it for the merge
+#ifdef NOSA_TRACE
+  if (tid == 0) NOSA_STAMP(5);
+#endif
+
+  // ---------------------------------------------------------------- merge
+  using ML = MergeLayout<G>;
+  float* mf = reinterpret_cast<float*>(smem);
+  if (decoding) {
+    // The four warps' states, in warp order, into this CTA's partial.
+    if (warp < kConsumerWarps) {
+      const int grp = lane >> 2, tig = lane & 3;
+#pragma unroll
+      for (int d = 0; d < 16; ++d) {
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int row = grp + h2 * 8;
+          if (row < G)
+            *reinterpret_cast<float2*>(mf + ML::kMo + (warp * G + row) * kMoStride + d * 8 + 2 * tig) =
+                make_float2(att.acc[d][2 * h2], att.acc[d][2 * h2 + 1]);
+        }
+      }
+      if (tig == 0) {
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int row = grp + rr * 8;
+          if (row < G) {
+            mf[ML::kMm + warp * G + row] = att.m[rr];
+            mf[ML::kMl + warp * G + row] = att.l[rr];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    for (int row = tid; row < G; row += kStepThreads) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mf[ML::kMm + w * G + row]);
+      float lsum = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float m_w = mf[ML::kMm + w * G + row];
+        const float f = m_w == -INFINITY ? 0.0f : exp2f(m_w - M);
+        mf[ML::kMw + w * G + row] = f;
+        lsum += mf[ML::kMl + w * G + row] * f;
+      }
+      mf[ML::kPm + row] = M;
+      mf[ML::kPl + row] = lsum;
+    }
+    __syncthreads();
+    constexpr int kVec = kHeadDim / 4;
+    for (int t = tid; t < G * kVec; t += kStepThreads) {
+      const int row = t / kVec, d4 = t % kVec;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float f = mf[ML::kMw + w * G + row];
+        const float4 x = *reinterpret_cast<const float4*>(mf + ML::kMo + (w * G + row) * kMoStride + 4 * d4);
+        o.x = fmaf(f, x.x, o.x);
+        o.y = fmaf(f, x.y, o.y);
+        o.z = fmaf(f, x.z, o.z);
+        o.w = fmaf(f, x.w, o.w);
+      }
+      *reinterpret_cast<float4*>(mf + ML::kPart + row * kHeadDim + 4 * d4) = o;
+    }
+  }
+  // Cluster barrier phase 2: every CTA's partial is in its shared memory.
+  cluster_arrive();
+  cluster_wait();
+  if (decoding) {
+    // CTA r combines all C partials, in rank order, for its share of the
+    // G x 32 output float4s.
+    constexpr int kVec = kHeadDim / 4;
+    const int n_items = G * kVec;
+    const int f0 = static_cast<int>((static_cast<int64_t>(rank) * n_items) / C);
+    const int f1 = static_cast<int>((static_cast<int64_t>(rank + 1) * n_items) / C);
+    const uint32_t base = smem_addr(mf);
+    for (int f = f0 + tid; f < f1; f += kStepThreads) {
+      const int row = f / kVec, d4 = f % kVec;
+      float mk[kMaxCluster];
+      float M = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kMaxCluster; ++k) {
+        if (k < static_cast<int>(C)) {
+          mk[k] = ld_cluster_f32(map_shared_rank(base + 4 * (ML::kPm + row), k));
+          M = fmaxf(M, mk[k]);
+        }
+      }
+      float lsum = 0.0f;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < kMaxCluster; ++k) {
+        if (k < static_cast<int>(C)) {
+          const float w = mk[k] == -INFINITY ? 0.0f : exp2f(mk[k] - M);
+          lsum += ld_cluster_f32(map_shared_rank(base + 4 * (ML::kPl + row), k)) * w;
+          const float4 x = ld_cluster_f32x4(map_shared_rank(base + 4 * (ML::kPart + row * kHeadDim + 4 * d4), k));
+          o.x = fmaf(w, x.x, o.x);
+          o.y = fmaf(w, x.y, o.y);
+          o.z = fmaf(w, x.z, o.z);
+          o.w = fmaf(w, x.w, o.w);
+        }
+      }
+      const int64_t orow = static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G + row;
+      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(a.out + orow * kHeadDim + 4 * d4);
+      dst[0] = __floats2bfloat162_rn(o.x * inv, o.y * inv);
+      dst[1] = __floats2bfloat162_rn(o.z * inv, o.w * inv);
+      if (a.lse && d4 == 0) a.lse[orow] = lsum > 0.0f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
+    }
+  }
+  // Cluster barrier phase 3: no CTA leaves while its partial may be read.
+  cluster_arrive();
+  cluster_wait();
+#ifdef NOSA_TRACE
+  if (tid == 0) {
+    NOSA_STAMP(7);
+    const uint32_t k = atomicAdd(&g_trace_count, 1u);
+    if (k < kTraceCapacity) {
+      uint32_t smid;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+      TraceRecord rec;
+      rec.pair = pair;
+      rec.rank = rank;
+      rec.smid = smid;
+      rec.csize = C;
+      for (int n = 0; n < 8; ++n) rec.t[n] = sh.tr[n];
+      g_trace[k] = rec;
+    }
+  }
+#endif
+}
 
 __device__ void write_empty_selection(const SelectArgs& a, int pair, int nthreads) {
   for (int t = threadIdx.x; t < a.topk; t += nthreads) a.sel_idx[static_cast<int64_t>(pair) * a.topk + t] = -1;
   if (threadIdx.x == 0) a.sel_cnt[pair] = 0;
-}
-
-// Append the new token's K/V rows and pool the window it completes, for one
-// (sequence, KV head) of length L (the new token is token L-1).  Warp 0
-// stores the rows, warp 1 pools (reading the new K row from k_new).
-__device__ void append_and_pool(const PoolArgs& p, int pair, int L) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = pair / p.hkv, h = pair % p.hkv;
-  const int64_t base = p.seq_start[i];
-  if (base < 0 || base + L > p.cache_rows) {
-    if (threadIdx.x == 0) set_status(p.status, NOSA_DEV_CACHE_ROWS);
-    return;
-  }
-  const int64_t len_old = L - 1;
-  const uint2* knew =
-      p.k_new ? reinterpret_cast<const uint2*>(p.k_new + (static_cast<int64_t>(i) * p.hkv + h) * kHeadDim) : nullptr;
-  if (warp == 0 && knew) {
-    const int64_t row = (base + len_old) * p.hkv + h;
-    const uint2* vnew = reinterpret_cast<const uint2*>(p.v_new + (static_cast<int64_t>(i) * p.hkv + h) * kHeadDim);
-    reinterpret_cast<uint2*>(p.k_cache + row * kHeadDim)[lane] = knew[lane];
-    reinterpret_cast<uint2*>(p.v_cache + row * kHeadDim)[lane] = vnew[lane];
-  }
-  const int64_t j = n_windows(L) - 1;
-  if (warp == 1 && j >= 0 && j >= n_windows(len_old)) {
-    if (j >= p.nc_cap) {
-      if (lane == 0) set_status(p.status, NOSA_DEV_NC_CAP);
-    } else {
-      pool_window_warp(p.k_cache, p.hkv, base, h, j, knew ? len_old : -1, knew,
-                       p.pooled + ((static_cast<int64_t>(i) * p.hkv + h) * p.nc_cap + j) * kHeadDim, lane);
-    }
-  }
-}
-
-#ifdef NOSA_TRACE
-#define NOSA_STAMP(slot)                                      \
-  do {                                                        \
-    if (threadIdx.x == 0) stamps[slot] = global_timer_ns();   \
-  } while (0)
-#else
-#define NOSA_STAMP(slot) \
-  do {                   \
-  } while (0)
-#endif
-
-template <int G>
-__device__ void score_item(const StepArgs& a, int item, uint8_t* smem, uint64_t* key_bar, uint32_t& key_phase,
-                           TopkShared& tsh, int* sh_last, uint64_t* stamps) {
-  const SelectArgs& s = a.sel;
-  const int pair = item % a.pairs, chunk = item / a.pairs;
-  const int i = pair / s.hkv, g = pair % s.hkv;
-  const int tid = threadIdx.x;
-  const int L = s.seq_len[i];
-  NOSA_STAMP(0);
-  if (L < 1 || L > s.max_seq_len) {
-    if (chunk == 0) {
-      if (tid == 0) set_status(s.status, L < 1 ? NOSA_DEV_BAD_LENGTH : NOSA_DEV_MAX_LEN);
-      write_empty_selection(s, pair, kDecThreads);
-    }
-    return;
-  }
-  const ScoreGeometry geo = score_geometry(L, s.nc_cap, s.local_blocks, s.comp_out != nullptr, chunk);
-  if (chunk >= geo.nchunks) return;
-  if (chunk == 0 && n_windows(L) > s.nc_cap && tid == 0) set_status(s.status, NOSA_DEV_NC_CAP);
-  if ((a.mode & kStepAppend) && chunk == 0) append_and_pool(a.pool, pair, L);
-  const bool uses_keys = geo.b1 > geo.b0 && geo.jhi > geo.jlo;
-  score_chunk<G, kDecThreads>(s.q, s.pooled, s.nc_cap, s.hq, s.hkv, i, g, s.scale, geo,
-                              s.bscratch + static_cast<int64_t>(pair) * s.nb_ws, s.comp_out,
-                              s.bs_out ? s.bs_out + static_cast<int64_t>(pair) * s.nb_out : nullptr, smem, key_bar,
-                              key_phase, s.status, stamps ? stamps + 1 : nullptr);
-  if (uses_keys) key_phase ^= 1u;
-  __syncthreads();
-  NOSA_STAMP(2);
-  if (tid == 0) {
-    __threadfence();
-    const uint32_t t = atomicAdd(&s.tickets[pair], 1u);
-    *sh_last = (t == static_cast<uint32_t>(geo.nchunks - 1));
-  }
-  __syncthreads();
-  NOSA_STAMP(3);
-  if (!*sh_last) return;
-  if (tid == 0) __threadfence();  // acquire: the other chunks' block scores
-  __syncthreads();
-  NOSA_STAMP(7);
-  // The pair's last chunk: every block score is written; select.
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  select_topk<kDecThreads>(s.bscratch + static_cast<int64_t>(pair) * s.nb_ws, true, geo.ncand, s.topk,
-                           s.sel_idx + static_cast<int64_t>(pair) * s.topk, s.sel_cnt + pair,
-                           reinterpret_cast<uint32_t*>(smem), tsh, stamps ? stamps + 4 : nullptr);
-  __syncthreads();
-  if (tid == 0) {
-    s.tickets[pair] = 0u;
-    if (a.mode & kStepDecode) {
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      __threadfence();
-      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.ready + pair), "r"(1u) : "memory");
-    }
-  }
-}
-
-template <int G>
-__global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
-    step_kernel(const StepArgs a, const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
-  extern __shared__ uint8_t smem_raw[];
-  // 128-byte swizzled TMA boxes want 1024-byte aligned destinations.
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ DecodeShared dsh;
-  __shared__ TopkShared tsh;
-  __shared__ __align__(8) uint64_t key_bar;
-  __shared__ int sh_item;
-  __shared__ int sh_last;
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&dsh.full_bar[s], 1);
-      mbar_init(&dsh.empty_bar[s], kDecConsumerWarps);
-    }
-    mbar_init(&key_bar, 1);
-    mbar_init(&dsh.merge_bar, 1);
-    dsh.merge_phase = 0;
-    fence_barrier_init();
-  }
-  if (tid == kDecConsumerWarps * 32 && (a.mode & kStepDecode)) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_k) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_v) : "memory");
-  }
-#ifdef NOSA_TRACE
-  if (tid == 0) {
-    dsh.t_flag = 0;
-    for (int n = 0; n < 8; ++n) dsh.t_issue[n] = dsh.t_full[n] = dsh.t_done[n] = 0;
-    for (int n = 0; n < 6; ++n) dsh.t_merge[n] = 0;
-  }
-#endif
-  grid_dependency_wait();
-  allow_dependents();
-  __syncthreads();
-  uint32_t ring_n = 0, key_phase = 0;
-  for (;;) {
-    if (tid == 0) sh_item = static_cast<int>(atomicAdd(a.work, 1u));
-    __syncthreads();
-    const int item = sh_item;
-    if (item >= a.n_items) break;
-#ifdef NOSA_TRACE
-    const uint64_t tr_start = global_timer_ns();
-    const long long tr_clk0 = clock64();
-#endif
-    if (item < a.n_score_items) {
-#ifdef NOSA_TRACE
-      score_item<G>(a, item, smem, &key_bar, key_phase, tsh, &sh_last, dsh.t_issue);
-#else
-      score_item<G>(a, item, smem, &key_bar, key_phase, tsh, &sh_last, nullptr);
-#endif
-    } else {
-      const int d = item - a.n_score_items;
-      decode_item(a.dec, &tm_k, &tm_v, d % a.pairs, d / a.pairs, (a.mode & kStepScore) ? a.ready + d % a.pairs : nullptr,
-                  ring_n, smem, dsh);
-    }
-    // Shared memory written by this item's threads may next be written by TMA.
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-#ifdef NOSA_TRACE
-    if (tid == 0) {
-      const uint32_t k = atomicAdd(&g_trace_count, 1u);
-      if (k < kTraceCapacity) {
-        uint32_t smid;
-        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-        TraceRecord rec{blockIdx.x, smid, static_cast<uint32_t>(item), static_cast<uint32_t>(clock64() - tr_clk0),
-                        tr_start, dsh.t_flag, global_timer_ns()};
-        for (int n = 0; n < 8; ++n) {
-          rec.issue[n] = dsh.t_issue[n] ? static_cast<uint32_t>(dsh.t_issue[n] - tr_start) : 0u;
-          rec.full[n] = dsh.t_full[n] ? static_cast<uint32_t>(dsh.t_full[n] - tr_start) : 0u;
-          rec.done[n] = dsh.t_done[n] ? static_cast<uint32_t>(dsh.t_done[n] - tr_start) : 0u;
-          dsh.t_issue[n] = dsh.t_full[n] = dsh.t_done[n] = 0;
-        }
-        for (int n = 0; n < 6; ++n) {
-          rec.merge[n] = dsh.t_merge[n] ? static_cast<uint32_t>(dsh.t_merge[n] - tr_start) : 0u;
-          dsh.t_merge[n] = 0;
-        }
-        g_trace[k] = rec;
-      }
-      dsh.t_flag = 0;
-    }
-#endif
-  }
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(a.work + 1, 1u) == gridDim.x - 1) {
-      a.work[0] = 0u;
-      a.work[1] = 0u;
-    }
-  }
 }
 
 // Selection only, from caller-provided block scores: one CTA per pair.
@@ -273,54 +581,119 @@ __global__ void wait_selftest_kernel(uint32_t* status, uint32_t max_iters) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, status, max_iters, 1000u);
 }
 
-constexpr int kStepSmem = kRingBytes + 1024;
+template <int G>
+size_t step_smem_bytes(const StepArgs& a) {
+  const int ncand_max = static_cast<int>(n_candidates(a.max_seq_len, a.local_blocks));
+  return 1024 + kRingBytes + ssm_bytes<G>() + round16(4 * a.topk) + (a.bs_spill ? 0 : round16(4 * max(ncand_max, 1)));
+}
+
+// Cluster size for `pairs` clusters: the largest power of two up to
+// kMaxCluster with pairs * C CTAs resident at once (then every pair's
+// cluster runs in the first wave); 1 when even that does not fit.
+struct ClusterPlanCache {
+  int dev = -1;
+  size_t smem = 0;
+  int slots = 0;
+  int max_clusters[5] = {0, 0, 0, 0, 0};  // C = 1, 2, 4, 8, 16
+};
+std::mutex g_plan_mu;
+ClusterPlanCache g_plan[5];  // per group size
 
 template <int G>
-int resident_ctas() {
-  static int cached[64] = {0};
+cudaError_t plan_cluster(int pairs, size_t smem, int* csize) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (cached[dev] == 0) {
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  constexpr int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
+  std::lock_guard<std::mutex> lock(g_plan_mu);
+  ClusterPlanCache& c = g_plan[gi];
+  if (c.dev != dev || c.smem != smem) {
+    // The attribute is an upper bound: set to the largest size the device
+    // allows next to the kernel's static shared memory, so that concurrent
+    // launches of different sizes never undercut each other.
+    int optin = 0;
+    cudaFuncAttributes fa;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa, step_kernel<G>)) != cudaSuccess) return e;
+    const int max_dyn = optin - static_cast<int>(fa.sharedSizeBytes);
+    if (static_cast<int>(smem) > max_dyn) return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(step_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaFuncSetAttribute(step_kernel<G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
+      return e;
     int per_sm = 0, sms = 0;
-    cudaFuncSetAttribute(step_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<G>, kDecThreads, kStepSmem) != cudaSuccess ||
-        per_sm < 1)
-      per_sm = 1;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 1;
-    cached[dev] = per_sm * sms;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<G>, kStepThreads, smem)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    c.slots = per_sm * sms;
+    for (int x = 0; x < 5; ++x) {
+      const int cs = 1 << x;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(cs);
+      cfg.blockDim = dim3(kStepThreads);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = cs;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, step_kernel<G>, &cfg) != cudaSuccess) {
+        cudaGetLastError();  // a size the device cannot co-schedule: never chosen
+        n = 0;
+      }
+      c.max_clusters[x] = n;
+    }
+    c.dev = dev;
+    c.smem = smem;
   }
-  return cached[dev];
+  int x = 0;
+  while (x < 4 && static_cast<int64_t>(pairs) * (2 << x) <= c.slots) ++x;
+  while (x > 0 && c.max_clusters[x] < pairs) --x;
+  *csize = 1 << x;
+  return cudaSuccess;
 }
 
 template <int G>
-cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t stream) {
-  if (a.n_items <= 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(step_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStepSmem);
+cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
+                          cudaStream_t stream) {
+  const int pairs = a.batch * a.hkv;
+  if (pairs <= 0) return cudaSuccess;
+  const size_t smem = step_smem_bytes<G>(a);
+  int csize = 1;
+  cudaError_t e = plan_cluster<G>(pairs, smem, &csize);
   if (e != cudaSuccess) return e;
-  const int grid = min(a.n_items, resident_ctas<G>());
-  return launch_overlapped(step_kernel<G>, dim3(grid), dim3(kDecThreads), kStepSmem, stream, a, tm_k, tm_v);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pairs) * csize);
+  cfg.blockDim = dim3(kStepThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, step_kernel<G>, a, tm_k, tm_v, tm_p);
 }
 
 }  // namespace
 
-int step_resident_ctas(int group) {
-  switch (group) {
-    case 1: return resident_ctas<1>();
-    case 2: return resident_ctas<2>();
-    case 4: return resident_ctas<4>();
-    case 8: return resident_ctas<8>();
-    case 16: return resident_ctas<16>();
-    default: return 0;
-  }
-}
-
-cudaError_t launch_step(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, cudaStream_t stream) {
-  switch (a.dec.group) {
-    case 1: return launch_step_g<1>(a, tm_k, tm_v, stream);
-    case 2: return launch_step_g<2>(a, tm_k, tm_v, stream);
-    case 4: return launch_step_g<4>(a, tm_k, tm_v, stream);
-    case 8: return launch_step_g<8>(a, tm_k, tm_v, stream);
-    case 16: return launch_step_g<16>(a, tm_k, tm_v, stream);
+cudaError_t launch_step(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
+                        cudaStream_t stream) {
+  switch (a.hq / a.hkv) {
+    case 1: return launch_step_g<1>(a, tm_k, tm_v, tm_p, stream);
+    case 2: return launch_step_g<2>(a, tm_k, tm_v, tm_p, stream);
+    case 4: return launch_step_g<4>(a, tm_k, tm_v, tm_p, stream);
+    case 8: return launch_step_g<8>(a, tm_k, tm_v, tm_p, stream);
+    case 16: return launch_step_g<16>(a, tm_k, tm_v, tm_p, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -331,15 +704,6 @@ cudaError_t launch_select_only(const SelectArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(select_only_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return launch_overlapped(select_only_kernel, dim3(1, a.batch * a.hkv), dim3(kSelOnlyThreads), smem, stream, a);
-}
-
-void decode_split_plan(int pairs, int max_tiles, int num_ctas, int* nsplit) {
-  if (max_tiles < 1) max_tiles = 1;
-  int ns = pairs > 0 ? num_ctas / pairs : 1;
-  if (ns > max_tiles) ns = max_tiles;
-  if (ns > kMaxSplits) ns = kMaxSplits;
-  if (ns < 1) ns = 1;
-  *nsplit = ns;
 }
 
 #ifdef NOSA_TRACE

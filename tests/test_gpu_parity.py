@@ -203,6 +203,31 @@ def test_select_unplanted_ragged_valid(nosa):
     _status_ok(nosa, st.ws)
 
 
+@pytest.mark.parametrize("hq,hkv,key_dist", [(2, 2, "normal"), (4, 2, "student_t"), (8, 2, "normal"),
+                                             (16, 2, "student_t"), (32, 2, "normal"), (32, 8, "student_t")])
+def test_select_scores_every_group_size(nosa, hq, hkv, key_dist):
+    """Compressed and block scores for group sizes 1..16 (the tensor-core
+    scoring tiles the group's heads as the n dimension) on ragged lengths whose
+    chunks end mid-tile; heavy-tailed keys exercise the split of each pooled
+    value into two TF32 parts."""
+    lens = [64 * 16 + 64 * 16 * 3 + 64 * 5 + 9, 2100, 64 * 17, 4097]
+    b = inputs.make_batch(lens, num_q_heads=hq, num_kv_heads=hkv, seed=hq + 7 * hkv, key_dist=key_dist)
+    ref = oracle_step(b, 64)
+    g = b.to(DEV)
+    p, st = _gpu_state(nosa, b, 64)
+    st.rebuild_pooled(g.k_cache, g.seq_start, g.seq_len)
+    comp = torch.full((b.batch, hq, st.nc_cap), float("nan"), device=DEV)
+    bsc = torch.full((b.batch, hkv, nosa.n_blocks(max(lens))), float("nan"), device=DEV)
+    nosa.nosa_block_select(p, g.q, st.pooled, g.seq_len, max(lens), st.sel_idx, st.sel_cnt, st.ws,
+                           comp_scores_out=comp, block_scores_out=bsc)
+    got_c, got_S = comp.cpu().numpy(), bsc.cpu().numpy()
+    for i, L in enumerate(lens):
+        nc, ncand = oracle.n_windows(L), oracle.n_candidates(L)
+        assert_scores_close(got_c[i, :, :nc], ref["comp_scores"][i, :, :nc])
+        assert_scores_close(got_S[i, :, :ncand], ref["block_scores"][i, :, :ncand])
+    _status_ok(nosa, st.ws)
+
+
 # ----------------------------------------------------------------------------- K3 attention
 
 @pytest.mark.parametrize("hq,hkv", [(2, 2), (4, 2), (16, 2), (32, 2), (32, 8)])
@@ -284,6 +309,34 @@ def test_determinism_bitwise(nosa):
     l1 = st.lse.clone()
     o2 = st.step(b.q, b.k_cache, b.v_cache, b.seq_start, b.seq_len, append=False, with_lse=True)
     assert torch.equal(o1, o2) and torch.equal(l1, st.lse)
+    _status_ok(nosa, st.ws)
+
+
+def test_step_long_context_block_scores_in_workspace(nosa):
+    """A 150K-token sequence has 2328 candidates: more than shared memory keeps,
+    so its block scores go through the workspace and the selector runs the
+    memory-resident top-k.  Planted blocks make the selection exact; one short
+    sequence rides along in the same launch."""
+    lens = [150_000, 3000]
+    b = inputs.make_batch(lens, num_q_heads=16, num_kv_heads=2, seed=31)
+    inputs.plant_blocks(b, seed=131)
+    ref = oracle_step(b, 64)
+    g = b.to(DEV)
+    p, st = _gpu_state(nosa, b, 64)
+    assert oracle.n_candidates(150_000) > 2048
+    st.rebuild_pooled(g.k_cache, g.seq_start, g.seq_len)
+    bsc = torch.full((2, 2, nosa.n_blocks(150_000)), float("nan"), device=DEV)
+    nosa.nosa_block_select(p, g.q, st.pooled, g.seq_len, 150_000, st.sel_idx, st.sel_cnt, st.ws,
+                           block_scores_out=bsc)
+    for i, L in enumerate(lens):
+        nc = oracle.n_candidates(L)
+        assert_scores_close(bsc.cpu().numpy()[i, :, :nc], ref["block_scores"][i, :, :nc])
+    np.testing.assert_array_equal(st.sel_idx.cpu().numpy(), ref["sel_idx"])
+    np.testing.assert_array_equal(st.sel_cnt.cpu().numpy(), ref["sel_cnt"])
+    st.step(g.q, g.k_cache, g.v_cache, g.seq_start, g.seq_len, append=False, with_lse=True)
+    np.testing.assert_array_equal(st.sel_idx.cpu().numpy(), ref["sel_idx"])
+    assert_out_close(st.out.float().cpu().numpy(), ref["out"])
+    np.testing.assert_allclose(st.lse.cpu().numpy(), ref["lse"], atol=1e-3, rtol=0)
     _status_ok(nosa, st.ws)
 
 

@@ -61,18 +61,20 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(nosa):
 
 
 def test_noalloc_rejects_a_batch_beyond_its_scratch(nosa):
-    # 512 sequences of 64K tokens need far more than the built-in 8 MiB.
+    # 64 sequences of up to 2^20 tokens keep their block scores in scratch
+    # (16368 candidates each, beyond what shared memory holds): more than the
+    # built-in 8 MiB.  The call is refused before anything is launched.
     p = nosa.params(16, 2, topk=64)
-    assert nosa.workspace_size(p, 512, 65536) > 8 << 20
+    assert nosa.workspace_size(p, 64, 1 << 20) > 8 << 20
     one = torch.zeros(1, dtype=torch.bfloat16, device=DEV)
-    i64 = torch.zeros(512, dtype=torch.int64, device=DEV)
-    i32 = torch.ones(512, dtype=torch.int32, device=DEV)
+    i64 = torch.zeros(64, dtype=torch.int64, device=DEV)
+    i32 = torch.ones(64, dtype=torch.int32, device=DEV)
     with pytest.raises(nosa.NosaError) as err:
         nosa.nosa_decode_step_device_noalloc(
-            p, one.expand(512, 16, 128).contiguous(), one.expand(8, 2, 128).contiguous(),
-            one.expand(8, 2, 128).contiguous(), i64, i32, 65536,
-            torch.zeros(512, 2, 1, 128, device=DEV), torch.zeros(512, 2, 64, dtype=torch.int32, device=DEV),
-            torch.zeros(512, 2, dtype=torch.int32, device=DEV),
-            torch.zeros(512, 16, 128, dtype=torch.bfloat16, device=DEV))
+            p, one.expand(64, 16, 128).contiguous(), one.expand(8, 2, 128).contiguous(),
+            one.expand(8, 2, 128).contiguous(), i64, i32, 1 << 20,
+            torch.zeros(64, 2, 1, 128, device=DEV), torch.zeros(64, 2, 64, dtype=torch.int32, device=DEV),
+            torch.zeros(64, 2, dtype=torch.int32, device=DEV),
+            torch.zeros(64, 16, 128, dtype=torch.bfloat16, device=DEV))
     assert err.value.code == nosa.NOSA_ERR_WORKSPACE
     assert "8388608" in str(err.value)
