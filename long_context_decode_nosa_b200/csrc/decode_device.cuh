@@ -136,19 +136,22 @@ __device__ inline void attend_tile(AttnState& s, const uint32_t (&qa)[8][4], uin
     }
     __syncwarp();
   }
-  // S = Q K^T over this warp's 16 tokens (two n-tiles of 8).
+  // S = Q K^T over this warp's 16 tokens (two n-tiles of 8), even and odd
+  // k-steps in separate accumulators (two short chains instead of one long).
   float sc[2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.0f;
+    float s0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, s1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     const int row = wrow + nt * 8 + (lane & 7);
 #pragma unroll
     for (int kp = 0; kp < 4; ++kp) {
       uint32_t b0, b1, b2, b3;
       ldsm_x4(swz(k_lo + (kp >> 1) * kHalfBytes, row, (kp & 1) * 4 + (lane >> 3)), b0, b1, b2, b3);
-      mma_bf16_16816(sc[nt], qa[2 * kp], b0, b1);
-      mma_bf16_16816(sc[nt], qa[2 * kp + 1], b2, b3);
+      mma_bf16_16816(s0, qa[2 * kp], b0, b1);
+      mma_bf16_16816(s1, qa[2 * kp + 1], b2, b3);
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[nt][e] = s0[e] + s1[e];
   }
   // Scale into the exp2 domain and mask tokens outside [0, L) / rejected tiles.
   float mx[2] = {-INFINITY, -INFINITY};

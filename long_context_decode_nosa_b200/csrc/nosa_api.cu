@@ -223,6 +223,7 @@ nosa::StepArgs step_args(const nosa_params* p, const void* q, const int32_t* seq
   a.local_blocks = p->local_blocks;
   a.topk = p->topk;
   a.max_seq_len = max_seq_len;
+  a.ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
   a.nc_cap = 1;
   a.scale = scale_of(p);
   a.scale_log2 = a.scale * 1.4426950408889634f;

@@ -59,6 +59,7 @@ struct StepArgs {
   float* lse;                    // nullable: [batch, hq]
   uint32_t* status;
   int batch, hq, hkv, local_blocks, topk, max_seq_len, nc_cap, nb_out, nb_spill;
+  int ncand_max;  // candidates of a sequence of max_seq_len tokens
   int mode;
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)

@@ -330,11 +330,11 @@ __device__ inline void warp_topk_mem(const float* scores, bool coherent, int nca
 // Top-k by one warp: register-resident keys up to kWarpTopkMax candidates,
 // memory-resident beyond.
 __device__ inline void warp_select(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
-                                   int32_t* sel_cnt, int lane) {
+                                   int32_t* sel_cnt, int lane, uint64_t* trace_stamps = nullptr) {
   if (ncand <= 256)
-    warp_topk<8>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
+    warp_topk<8>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane, trace_stamps);
   else if (ncand <= kWarpTopkMax)
-    warp_topk<32>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
+    warp_topk<32>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane, trace_stamps);
   else
     warp_topk_mem(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
 }
@@ -401,8 +401,9 @@ __device__ inline void load_score_q(ScoreQ<G>& f, const __nv_bfloat16* __restric
 // inputs, fp32 accumulation) and stores scale * s into ssm[head][row] for
 // rows < 61.  Each fp32 pooled value x is split into hi (x with its low 13
 // mantissa bits cleared, exact in TF32) and lo = tf32(x - hi); the hi and lo
-// products go to separate fp32 accumulators that are added at the end, so
-// the only input rounding is that of lo, below 2^-21 of |x| ("NOSA-1B
+// products go to separate fp32 accumulators (even and odd k-steps apart)
+// that are added at the end, so the only input rounding is that of lo,
+// below 2^-21 of |x| ("NOSA-1B
 // 性能基准全解析" §三.3: scores of the pooled keys).
 template <int G>
 __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* __restrict__ ssm, float scale,
@@ -411,11 +412,15 @@ __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* _
   const int grp = lane >> 2, tig = lane & 3;
   const int r0 = warp * 16;
   const int ra = r0 + grp, rb = ra + 8;
-  float acc_hi[NT][4], acc_lo[NT][4];
+  // Four independent accumulation chains per n-tile (hi / lo x even / odd
+  // k-step) keep the tensor pipe busy instead of waiting on one chain.
+  float acc_hi[2][NT][4], acc_lo[2][NT][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  for (int c = 0; c < 2; ++c)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc_hi[nt][e] = acc_lo[nt][e] = 0.0f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc_hi[c][nt][e] = acc_lo[c][nt][e] = 0.0f;
 #pragma unroll
   for (int ks = 0; ks < 16; ++ks) {
     const uint32_t box = stage + (ks >> 2) * kScoreSlotBytes;
@@ -438,8 +443,8 @@ __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* _
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      mma_tf32_1688(acc_hi[nt], hi, qf.b[nt][ks][0], qf.b[nt][ks][1]);
-      mma_tf32_1688(acc_lo[nt], lo, qf.b[nt][ks][0], qf.b[nt][ks][1]);
+      mma_tf32_1688(acc_hi[ks & 1][nt], hi, qf.b[nt][ks][0], qf.b[nt][ks][1]);
+      mma_tf32_1688(acc_lo[ks & 1][nt], lo, qf.b[nt][ks][0], qf.b[nt][ks][1]);
     }
   }
   // acc[nt][0..1]: row ra, heads nt*8 + 2*tig + {0,1}; [2..3]: row rb.
@@ -449,7 +454,9 @@ __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* _
     for (int e = 0; e < 4; ++e) {
       const int head = nt * 8 + 2 * tig + (e & 1);
       const int row = (e >> 1) ? rb : ra;
-      if (head < G && row < kChunkWindows) ssm[head * kScoreStride + row] = (acc_hi[nt][e] + acc_lo[nt][e]) * scale;
+      if (head < G && row < kChunkWindows)
+        ssm[head * kScoreStride + row] =
+            ((acc_hi[0][nt][e] + acc_hi[1][nt][e]) + (acc_lo[0][nt][e] + acc_lo[1][nt][e])) * scale;
     }
   }
 }

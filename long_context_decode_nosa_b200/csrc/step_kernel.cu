@@ -28,10 +28,10 @@
 //     computes the same selection, so no second exchange is needed) and
 //     hands the selected blocks to the producer; rank 0 writes the
 //     selection out.
-// Merge: each CTA merges its four warps into one partial (O, m, l) in its
-// shared memory; after a cluster barrier, CTA r combines the partials of
-// all C CTAs (fixed order) for its share of the output elements; a last
-// cluster barrier keeps every CTA resident until its partial has been read.
+// Merge: each CTA merges its four warps into one partial (O, m, l) and
+// pushes it, slice by slice, into the receive buffers of the cluster's CTAs
+// (CTA r owns output slice r); after one cluster barrier, CTA r combines
+// the C partials of its slice from its own shared memory, in rank order.
 //
 // No global-memory flags, tickets or work queues: the only cross-CTA
 // traffic is inside the cluster, and every wait is bounded (status bit
@@ -42,6 +42,8 @@
 #include "pool_device.cuh"
 #include "select_device.cuh"
 
+#include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 namespace nosa {
@@ -51,7 +53,7 @@ namespace nosa {
 // kernel with %globaltimer stamps of its phases.
 struct TraceRecord {
   uint32_t pair, rank, smid, csize;
-  uint64_t t[8];  // start, scoring issued, scores sent, scores gathered, selection done, tiles done, -, end
+  uint64_t t[16];  // see the NOSA_STAMP call sites
 };
 constexpr int kTraceCapacity = 1 << 16;
 __device__ TraceRecord g_trace[kTraceCapacity];
@@ -79,7 +81,7 @@ struct StepShared {
   int sel_count;
   float blk[kChunkBlocks];  // block scores of the chunk being sent
 #ifdef NOSA_TRACE
-  uint64_t tr[8];
+  uint64_t tr[16];
 #endif
 };
 
@@ -88,11 +90,24 @@ struct StepShared {
 //   ssm   G x kScoreStride floats         window scores of the chunk being scored
 //   sel   round16(4 * topk) bytes         the pair's selection (ascending block indices)
 //   bsm   4 * ncand_max bytes             the pair's block scores (unless kept in global memory)
+//   recv  recv_bytes<G>()                 the partials the cluster's CTAs push for this CTA's
+//                                         share of the output (see the merge)
 template <int G>
 __host__ __device__ constexpr int ssm_bytes() {
   return G * kScoreStride * 4;
 }
 __host__ __device__ constexpr int round16(int x) { return (x + 15) & ~15; }
+// Output float4s of a pair and the receive buffer that holds, for any
+// cluster size C <= 16, C x ceil(items / C) pushed float4s plus C x G row
+// maxima and C x G row sums.
+template <int G>
+__host__ __device__ constexpr int out_items() {
+  return G * kHeadDim / 4;
+}
+template <int G>
+__host__ __device__ constexpr int recv_bytes() {
+  return (out_items<G>() + kMaxCluster) * 16 + 2 * kMaxCluster * G * 4;
+}
 
 // Named barrier of the four consumer warps.
 __device__ inline void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory"); }
@@ -114,7 +129,7 @@ __device__ inline bool consumer_all(bool v) {
 
 // Cross-warp merge scratch (in the drained ring): per warp O rows with a
 // padded stride (bank-conflict free float2 stores), row max / sum / weight,
-// then the CTA's partial that the other CTAs of the cluster read.
+// then the CTA's row max / sum.
 constexpr int kMoStride = kHeadDim + 8;
 template <int G>
 struct MergeLayout {
@@ -122,9 +137,8 @@ struct MergeLayout {
   static constexpr int kMm = kMo + kConsumerWarps * G * kMoStride;   // [4][G]
   static constexpr int kMl = kMm + kConsumerWarps * G;               // [4][G]
   static constexpr int kMw = kMl + kConsumerWarps * G;               // [4][G]
-  static constexpr int kPart = (kMw + kConsumerWarps * G + 3) & ~3;  // [G][128] partial O
-  static constexpr int kPm = kPart + G * kHeadDim;                   // [G] partial row max
-  static constexpr int kPl = kPm + G;                                // [G] partial row sum
+  static constexpr int kPm = kMw + kConsumerWarps * G;               // [G] the CTA's row max
+  static constexpr int kPl = kPm + G;                                // [G] the CTA's row sum
 };
 static_assert((MergeLayout<kMaxGroup>::kPl + kMaxGroup) * 4 <= kRingBytes, "merge scratch must fit in the ring");
 
@@ -158,7 +172,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     mbar_init(&sh.sel_bar, 1);
     fence_barrier_init();
 #ifdef NOSA_TRACE
-    for (int k = 0; k < 8; ++k) sh.tr[k] = 0;
+    for (int k = 0; k < 16; ++k) sh.tr[k] = 0;
     NOSA_STAMP(0);
 #endif
   }
@@ -179,10 +193,11 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   // ---------------------------------------------------------------- geometry
   // (identical in every CTA of the cluster)
   const int i = pair / a.hkv, g = pair % a.hkv;
-  const int L = a.seq_len[i];
-  const bool bad_len = L < 1 || L > a.max_seq_len;
   const bool uses_cache = decoding || appending;
-  const int64_t seq_base = uses_cache && !bad_len ? a.seq_start[i] : 0;
+  const int L = a.seq_len[i];
+  const int64_t start_i = uses_cache ? a.seq_start[i] : 0;  // issued with the length load
+  const bool bad_len = L < 1 || L > a.max_seq_len;
+  const int64_t seq_base = bad_len ? 0 : start_i;
   const bool bad_rows = uses_cache && !bad_len && (seq_base < 0 || seq_base + L > a.cache_rows);
   const int Lv = bad_len ? 0 : L;
   const int nb = static_cast<int>(n_blocks(Lv));
@@ -315,7 +330,11 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 #endif
       if (ok) {
         const float* src = spill ? a.bs_spill + static_cast<int64_t>(pair) * a.nb_spill : bsm;
+#ifdef NOSA_TRACE
+        warp_select(src, spill, ncand, a.topk, sel_list, &sh.sel_count, lane, &sh.tr[8]);
+#else
         warp_select(src, spill, ncand, a.topk, sel_list, &sh.sel_count, lane);
+#endif
       } else {
         for (int t = lane; t < a.topk; t += 32) sel_list[t] = -1;
         if (lane == 0) sh.sel_count = 0;
@@ -420,6 +439,8 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   // ---------------------------------------------------------------- merge
   using ML = MergeLayout<G>;
   float* mf = reinterpret_cast<float*>(smem);
+  float* recv = reinterpret_cast<float*>(smem + kRingBytes + ssm_bytes<G>() + round16(4 * a.topk) +
+                                         (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))));
   if (decoding) {
     // The four warps' states, in warp order, into this CTA's partial.
     if (warp < kConsumerWarps) {
@@ -462,57 +483,72 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       mf[ML::kPl + row] = lsum;
     }
     __syncthreads();
+    // Push: output float4 f of this CTA's partial goes to CTA f / slice of
+    // the cluster (slot [rank][f % slice] of its receive buffer), and this
+    // CTA's row maxima and sums go to every CTA.
     constexpr int kVec = kHeadDim / 4;
-    for (int t = tid; t < G * kVec; t += kStepThreads) {
-      const int row = t / kVec, d4 = t % kVec;
+    const int slice = (out_items<G>() + static_cast<int>(C) - 1) / static_cast<int>(C);
+    float* recv_m = recv + 4 * static_cast<int>(C) * slice;  // [C][G]
+    float* recv_l = recv_m + static_cast<int>(C) * G;         // [C][G]
+    for (int f = tid; f < out_items<G>(); f += kStepThreads) {
+      const int row = f / kVec, d4 = f % kVec;
       float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) {
-        const float f = mf[ML::kMw + w * G + row];
+        const float fw = mf[ML::kMw + w * G + row];
         const float4 x = *reinterpret_cast<const float4*>(mf + ML::kMo + (w * G + row) * kMoStride + 4 * d4);
-        o.x = fmaf(f, x.x, o.x);
-        o.y = fmaf(f, x.y, o.y);
-        o.z = fmaf(f, x.z, o.z);
-        o.w = fmaf(f, x.w, o.w);
+        o.x = fmaf(fw, x.x, o.x);
+        o.y = fmaf(fw, x.y, o.y);
+        o.z = fmaf(fw, x.z, o.z);
+        o.w = fmaf(fw, x.w, o.w);
       }
-      *reinterpret_cast<float4*>(mf + ML::kPart + row * kHeadDim + 4 * d4) = o;
+      const int dst = f / slice;
+      st_cluster_f32x4(map_shared_rank(smem_addr(recv + 4 * (static_cast<int>(rank) * slice + (f - dst * slice))),
+                                       static_cast<uint32_t>(dst)),
+                       o);
+    }
+    for (int t = tid; t < G * static_cast<int>(C); t += kStepThreads) {
+      const int row = t % G;
+      const uint32_t dst = static_cast<uint32_t>(t / G);
+      st_cluster_f32(map_shared_rank(smem_addr(recv_m + static_cast<int>(rank) * G + row), dst), mf[ML::kPm + row]);
+      st_cluster_f32(map_shared_rank(smem_addr(recv_l + static_cast<int>(rank) * G + row), dst), mf[ML::kPl + row]);
     }
   }
-  // Cluster barrier phase 2: every CTA's partial is in its shared memory.
+  // Cluster barrier phase 2: every CTA's pushes have landed.  Nothing
+  // touches another CTA's shared memory after it, so no CTA needs to wait
+  // for the others before leaving.
+#ifdef NOSA_TRACE
+  if (tid == 0) NOSA_STAMP(11);
+#endif
   cluster_arrive();
   cluster_wait();
+#ifdef NOSA_TRACE
+  if (tid == 0) NOSA_STAMP(12);
+#endif
   if (decoding) {
-    // CTA r combines all C partials, in rank order, for its share of the
-    // G x 32 output float4s.
+    // This CTA's slice of the output: all C partials from the receive
+    // buffer, combined in rank order.
     constexpr int kVec = kHeadDim / 4;
-    const int n_items = G * kVec;
-    const int f0 = static_cast<int>((static_cast<int64_t>(rank) * n_items) / C);
-    const int f1 = static_cast<int>((static_cast<int64_t>(rank + 1) * n_items) / C);
-    const uint32_t base = smem_addr(mf);
+    const int slice = (out_items<G>() + static_cast<int>(C) - 1) / static_cast<int>(C);
+    const float* recv_m = recv + 4 * static_cast<int>(C) * slice;
+    const float* recv_l = recv_m + static_cast<int>(C) * G;
+    const int f0 = static_cast<int>(rank) * slice;
+    const int f1 = min(f0 + slice, out_items<G>());
     for (int f = f0 + tid; f < f1; f += kStepThreads) {
       const int row = f / kVec, d4 = f % kVec;
-      float mk[kMaxCluster];
       float M = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < kMaxCluster; ++k) {
-        if (k < static_cast<int>(C)) {
-          mk[k] = ld_cluster_f32(map_shared_rank(base + 4 * (ML::kPm + row), k));
-          M = fmaxf(M, mk[k]);
-        }
-      }
+      for (int k = 0; k < static_cast<int>(C); ++k) M = fmaxf(M, recv_m[k * G + row]);
       float lsum = 0.0f;
       float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < kMaxCluster; ++k) {
-        if (k < static_cast<int>(C)) {
-          const float w = mk[k] == -INFINITY ? 0.0f : exp2f(mk[k] - M);
-          lsum += ld_cluster_f32(map_shared_rank(base + 4 * (ML::kPl + row), k)) * w;
-          const float4 x = ld_cluster_f32x4(map_shared_rank(base + 4 * (ML::kPart + row * kHeadDim + 4 * d4), k));
-          o.x = fmaf(w, x.x, o.x);
-          o.y = fmaf(w, x.y, o.y);
-          o.z = fmaf(w, x.z, o.z);
-          o.w = fmaf(w, x.w, o.w);
-        }
+      for (int k = 0; k < static_cast<int>(C); ++k) {
+        const float mk = recv_m[k * G + row];
+        const float w = mk == -INFINITY ? 0.0f : exp2f(mk - M);
+        lsum += recv_l[k * G + row] * w;
+        const float4 x = *reinterpret_cast<const float4*>(recv + 4 * (k * slice + (f - f0)));
+        o.x = fmaf(w, x.x, o.x);
+        o.y = fmaf(w, x.y, o.y);
+        o.z = fmaf(w, x.z, o.z);
+        o.w = fmaf(w, x.w, o.w);
       }
       const int64_t orow = static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G + row;
       const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
@@ -522,9 +558,6 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       if (a.lse && d4 == 0) a.lse[orow] = lsum > 0.0f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
     }
   }
-  // Cluster barrier phase 3: no CTA leaves while its partial may be read.
-  cluster_arrive();
-  cluster_wait();
 #ifdef NOSA_TRACE
   if (tid == 0) {
     NOSA_STAMP(7);
@@ -537,7 +570,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       rec.rank = rank;
       rec.smid = smid;
       rec.csize = C;
-      for (int n = 0; n < 8; ++n) rec.t[n] = sh.tr[n];
+      for (int n = 0; n < 16; ++n) rec.t[n] = sh.tr[n];
       g_trace[k] = rec;
     }
   }
@@ -583,24 +616,23 @@ __global__ void wait_selftest_kernel(uint32_t* status, uint32_t max_iters) {
 
 template <int G>
 size_t step_smem_bytes(const StepArgs& a) {
-  const int ncand_max = static_cast<int>(n_candidates(a.max_seq_len, a.local_blocks));
-  return 1024 + kRingBytes + ssm_bytes<G>() + round16(4 * a.topk) + (a.bs_spill ? 0 : round16(4 * max(ncand_max, 1)));
+  return 1024 + kRingBytes + ssm_bytes<G>() + round16(4 * a.topk) + (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))) +
+         recv_bytes<G>();
 }
 
-// Cluster size for `pairs` clusters: the largest power of two up to
-// kMaxCluster with pairs * C CTAs resident at once (then every pair's
-// cluster runs in the first wave); 1 when even that does not fit.
+// Cluster size and launch mode for `pairs` clusters (see the rules below);
+// C = 1 when no larger cluster fits (then clusters run in waves).
 struct ClusterPlanCache {
   int dev = -1;
   size_t smem = 0;
   int slots = 0;
-  int max_clusters[5] = {0, 0, 0, 0, 0};  // C = 1, 2, 4, 8, 16
+  int max_clusters[kMaxCluster + 1] = {};  // co-resident clusters of C CTAs, C = 1..16
 };
 std::mutex g_plan_mu;
 ClusterPlanCache g_plan[5];  // per group size
 
 template <int G>
-cudaError_t plan_cluster(int pairs, size_t smem, int* csize) {
+cudaError_t plan_cluster(int pairs, int units, size_t smem, int* csize, bool* pdl) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -628,8 +660,7 @@ cudaError_t plan_cluster(int pairs, size_t smem, int* csize) {
       return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     c.slots = per_sm * sms;
-    for (int x = 0; x < 5; ++x) {
-      const int cs = 1 << x;
+    for (int cs = 1; cs <= kMaxCluster; ++cs) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(cs);
       cfg.blockDim = dim3(kStepThreads);
@@ -646,15 +677,41 @@ cudaError_t plan_cluster(int pairs, size_t smem, int* csize) {
         cudaGetLastError();  // a size the device cannot co-schedule: never chosen
         n = 0;
       }
-      c.max_clusters[x] = n;
+      c.max_clusters[cs] = n;
     }
     c.dev = dev;
     c.smem = smem;
   }
-  int x = 0;
-  while (x < 4 && static_cast<int64_t>(pairs) * (2 << x) <= c.slots) ++x;
-  while (x > 0 && c.max_clusters[x] < pairs) --x;
-  *csize = 1 << x;
+  // Among the cluster sizes whose pairs x C CTAs are all resident at once,
+  // the smallest C with the fewest scoring chunks per CTA: a larger cluster
+  // would not shorten the longest CTA's scoring and only costs wider
+  // exchanges.  The environment variable
+  // NOSA_CLUSTER_SIZE (1..16) overrides the choice.
+  int best = 1, best_units = units;
+  for (int cs = 2; cs <= kMaxCluster; ++cs) {
+    if (static_cast<int64_t>(pairs) * cs > c.slots || c.max_clusters[cs] < pairs) continue;
+    const int per_cta = (units + cs - 1) / cs;
+    if (per_cta < best_units) {
+      best = cs;
+      best_units = per_cta;
+    }
+  }
+  static const int forced = [] {
+    const char* v = getenv("NOSA_CLUSTER_SIZE");
+    const int n = v ? atoi(v) : 0;
+    return n >= 1 && n <= kMaxCluster ? n : 0;
+  }();
+  if (forced && c.max_clusters[forced] > 0) best = forced;
+  // Programmatic dependent launch only when the grid leaves at least half of
+  // the slots free: the next launch's clusters then become resident and run
+  // their prologue early.  When the grid fills the GPU, early-resident
+  // clusters of the next launch only skew where the rest are placed.
+  *pdl = static_cast<int64_t>(pairs) * best * 2 <= c.slots;
+#ifdef NOSA_TRACE
+  fprintf(stderr, "plan G=%d smem=%zu slots=%d pairs=%d units=%d -> C=%d pdl=%d (max clusters %d)\n", G, smem,
+          c.slots, pairs, units, best, static_cast<int>(*pdl), c.max_clusters[best]);
+#endif
+  *csize = best;
   return cudaSuccess;
 }
 
@@ -664,8 +721,14 @@ cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUte
   const int pairs = a.batch * a.hkv;
   if (pairs <= 0) return cudaSuccess;
   const size_t smem = step_smem_bytes<G>(a);
+  // Work units of the longest pair: its selection's scoring chunks.  The
+  // same in every mode, so the separate selection and attention launches
+  // split a pair's tiles exactly as the fused step does (bit-identical
+  // results).
+  const int units = (a.ncand_max + kChunkBlocks - 1) / kChunkBlocks;
   int csize = 1;
-  cudaError_t e = plan_cluster<G>(pairs, smem, &csize);
+  bool pdl = false;
+  cudaError_t e = plan_cluster<G>(pairs, max(units, 1), smem, &csize, &pdl);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pairs) * csize);
@@ -680,7 +743,7 @@ cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUte
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, step_kernel<G>, a, tm_k, tm_v, tm_p);
 }
 
