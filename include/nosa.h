@@ -56,7 +56,8 @@
  *    writes zeros where it owns output, and sets a bit in the workspace's
  *    device status word, which nosa_read_device_status returns and clears.
  *  * Calls that share one workspace must not overlap on the GPU (order them
- *    on one stream): the workspace holds per-call counters and partials.
+ *    on one stream): the workspace holds the status word, block scores of
+ *    very long sequences and the host-buffer step's staging.
  */
 #ifndef NOSA_B200_H
 #define NOSA_B200_H
@@ -114,12 +115,15 @@ NOSA_API void nosa_default_params(nosa_params* p);
 
 /* Bytes of device workspace that nosa_block_select / nosa_sparse_decode /
  * nosa_decode_step need for `batch` sequences of at most `max_seq_len`
- * tokens.  Returns 0 if the parameters are invalid.  The workspace must be
- * 256-byte aligned and zeroed once with nosa_workspace_init before first use;
- * afterwards every call leaves its counters at zero again. */
+ * tokens: the device status word; block scores [batch * Hkv, ncand] fp32
+ * when a sequence of max_seq_len tokens has more than 2048 candidates (fewer
+ * stay in shared memory); the staging buffers of nosa_decode_step (q, new
+ * K/V rows, out).  Returns 0 if the parameters are invalid.  The workspace
+ * must be 256-byte aligned and zeroed once with nosa_workspace_init before
+ * first use. */
 NOSA_API size_t nosa_workspace_size(const nosa_params* p, int batch, int max_seq_len);
 
-/* Zeroes the workspace (counters and device status word) on `stream`. */
+/* Zeroes the workspace (device status word included) on `stream`. */
 NOSA_API int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Step 1 -- CIS mean pooling of keys, appended incrementally
@@ -136,7 +140,7 @@ NOSA_API int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * len_old may be NULL, meaning len_new[i] - 1 for every i.
  * At most max_new_keys windows per (sequence, KV head) are produced; more sets
  * NOSA_DEV_MAX_NEW_KEYS.  A window past nc_cap sets NOSA_DEV_NC_CAP.
- * Does not use the workspace's counters; `ws` may be NULL (then device data
+ * Uses only the workspace's status word; `ws` may be NULL (then device data
  * errors are not reported). */
 NOSA_API int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache,
                      int64_t cache_rows, const int64_t* seq_start, const int32_t* len_old,
@@ -182,18 +186,19 @@ NOSA_API int nosa_sparse_decode(const nosa_params* p, const void* q, const void*
                        void* out, float* lse, void* ws, size_t ws_bytes,
                        void* stream);
 
-/* One whole decode step on DEVICE buffers, fused into a single launch of a
- * persistent kernel (steps 1-4 above, in the pages' order): appends the new
+/* One whole decode step on DEVICE buffers, fused into a single launch
+ * (steps 1-4 above, in the pages' order): appends the new
  * token's K/V rows (k_new / v_new, bf16 [batch, Hkv, D], nullable: then the
  * rows must already be in the caches) at seq_start[i] + seq_len[i] - 1, pools
  * the window it completes, scores and selects blocks (sel_idx / sel_cnt
  * receive the selection) and attends, writing out (bf16 [batch, Hq, D]) and
  * lse (nullable).  Results are bit-identical to nosa_pool_append +
- * nosa_block_select + nosa_sparse_decode on the same inputs.  Work items are
- * taken from a queue in the workspace by resident CTAs; the attention items
- * of a sequence wait (bounded, NOSA_DEV_TIMEOUT on expiry) for that
- * sequence's selection, published by the CTA that computed it.  With fewer
- * than two local blocks the three separate launches run instead. */
+ * nosa_block_select + nosa_sparse_decode on the same inputs.  Each
+ * (sequence, KV head) is one thread-block cluster: its CTAs score the
+ * pooled keys, exchange block scores through distributed shared memory,
+ * select, attend over their share of the tiles and merge in the cluster;
+ * every wait is bounded (NOSA_DEV_TIMEOUT on expiry).  With fewer than two
+ * local blocks the three separate launches run instead. */
 NOSA_API int nosa_decode_step_device(const nosa_params* p, const void* q, const void* k_new,
                                      const void* v_new, void* k_cache, void* v_cache,
                                      int64_t cache_rows, const int64_t* seq_start,
@@ -218,7 +223,7 @@ NOSA_API int nosa_decode_step_device(const nosa_params* p, const void* q, const 
  *    that device current) and caches it; make that first call before any
  *    stream capture.
  *  * Every call on a device shares the one array: the call clears its
- *    counters and flags first (asynchronously, on `stream`), but calls that
+ *    status word first (asynchronously, on `stream`), but calls that
  *    overlap on the GPU race.  Order them on one stream.
  *  * Device-side data checks land in the array's status word, which no entry
  *    point reads back; callers that need those reports use the workspace

@@ -1,7 +1,7 @@
 // The decode step for callers that cannot allocate device memory.
 //
-// nosa_decode_step_device needs a caller-provided workspace (counters, flags,
-// block scores, split partials).  Some callers have no way to provide one:
+// nosa_decode_step_device needs a caller-provided workspace (device status
+// word, block scores of very long sequences, staging).  Some callers have no way to provide one:
 // a plugin loaded into an inference engine whose memory manager owns the
 // whole device pool and exposes no workspace hook, or a serving loop that
 // must not call cudaMalloc once the KV cache has claimed the free memory
@@ -18,8 +18,8 @@
 namespace {
 
 // The library's own scratch for nosa_decode_step_device_noalloc: 8 MiB per
-// device (the NOSA-1B attention shape at batch 8 and 16K tokens needs about
-// 4.4 MB).
+// device (the NOSA-1B attention shape at batch 8 and 16K tokens needs 74 KB;
+// sequences beyond 2048 candidates keep their block scores here too).
 constexpr size_t kNoAllocScratchBytes = size_t{8} << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -64,8 +64,8 @@ int nosa_decode_step_device_noalloc(const nosa_params* p, const void* q, const v
     }
     scratch = g_scratch_addr[dev];
   }
-  // The array keeps whatever the previous call left; the counters, tickets
-  // and flags must start at zero.
+  // The array keeps whatever the previous call left; the status word starts
+  // at zero.
   const size_t zero_bytes = nosa::workspace_counter_bytes(p, batch, max_seq_len);
   const cudaError_t e = cudaMemsetAsync(scratch, 0, zero_bytes, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return nosa::record_error(NOSA_ERR_CUDA, cudaGetErrorString(e));
