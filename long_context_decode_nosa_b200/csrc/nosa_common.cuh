@@ -175,6 +175,16 @@ __device__ inline void st_cluster_f32x4(uint32_t addr, float4 v) {
                : "memory");
 }
 
+// Asynchronous store of one fp32 into another CTA's shared memory that
+// completes `bytes` (4) of transaction count on that CTA's mbarrier (both
+// addresses are shared::cluster addresses): the receiver's wait on the
+// barrier then sees the value, with no fence on the sender's side.
+__device__ inline void st_async_f32(uint32_t addr, float v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr),
+               "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
+
 __device__ inline float ld_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");

@@ -327,6 +327,185 @@ __device__ inline void warp_topk_mem(const float* scores, bool coherent, int nca
   if (lane == 0) *sel_cnt = k_eff;
 }
 
+// Exact top-k by a group of NT threads (a multiple of 32, synchronised with
+// named barrier `bar_id`) over up to NT * kGroupKeys candidates in memory
+// (shared, or global when `coherent`).  Thread t holds the contiguous keys
+// [t * kpt, (t + 1) * kpt).  The k-th largest order-preserving key T is
+// found by a radix select on 8-bit digits (a shared-memory histogram per
+// pass) below the common prefix of the min and max keys; one prefix scan of
+// the per-thread (greater, equal) counts then places every key above T and
+// the lowest-index keys equal to T in ascending order.  Same result as
+// warp_topk.  Every thread of the group must call it with the same
+// arguments; `tid` is the thread's index in the group.
+constexpr int kGroupKeys = 16;
+
+struct GroupTopkShared {
+  uint32_t hist[256];
+  uint32_t red[2][8][2];  // per-warp partials, double-buffered
+  uint32_t prefix, need;
+};
+
+__device__ inline void group_bar(int bar_id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthreads) : "memory");
+}
+
+template <int NT>
+__device__ void group_topk(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
+                           int32_t* sel_cnt, int tid, GroupTopkShared& sh, int bar_id,
+                           uint64_t* trace_stamps = nullptr) {
+#ifdef NOSA_TRACE
+#define GTK_STAMP(k) \
+  if (trace_stamps && tid == 0) trace_stamps[k] = global_timer_ns()
+#else
+#define GTK_STAMP(k)
+#endif
+  constexpr int kWarps = NT / 32;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int k_eff = ncand < topk ? ncand : topk;
+  const int kpt = (ncand + NT - 1) / NT;
+  const int b0 = tid * kpt;
+  uint32_t key[kGroupKeys];
+#pragma unroll
+  for (int m = 0; m < kGroupKeys; ++m) {
+    const int b = b0 + m;
+    key[m] = (m < kpt && b < ncand) ? order_key(coherent ? __ldcg(scores + b) : scores[b]) : 0u;  // valid keys > 0
+  }
+  GTK_STAMP(0);
+  uint32_t T = 0u, need = 0u;
+  if (k_eff < ncand) {
+    // Common prefix of the min and max valid keys.
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+    for (int m = 0; m < kGroupKeys; ++m)
+      if (m < kpt && b0 + m < ncand) {
+        lo = min(lo, key[m]);
+        hi = max(hi, key[m]);
+      }
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) {
+      sh.red[0][warp][0] = lo;
+      sh.red[0][warp][1] = hi;
+    }
+    group_bar(bar_id, NT);
+    GTK_STAMP(1);
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      lo = min(lo, sh.red[0][w][0]);
+      hi = max(hi, sh.red[0][w][1]);
+    }
+    need = static_cast<uint32_t>(k_eff);
+    if (lo == hi) {
+      T = hi;
+    } else {
+      const int top = 31 - __clz(lo ^ hi);
+      uint32_t P = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+      int r = top + 1;  // bits of T still open: [0, r)
+      while (r > 0) {   // the same pass count in every thread
+        const int w = r < 8 ? r : 8;
+        const int shift = r - w;
+        for (int x = tid; x < 256; x += NT) sh.hist[x] = 0u;
+        group_bar(bar_id, NT);
+#pragma unroll
+        for (int m = 0; m < kGroupKeys; ++m) {
+          const uint32_t kk = key[m];
+          if (m < kpt && b0 + m < ncand && (r == 32 || (kk >> r) == (P >> r)))
+            atomicAdd(&sh.hist[(kk >> shift) & ((1u << w) - 1u)], 1u);
+        }
+        group_bar(bar_id, NT);
+        if (warp == 0) {
+          // Lane l owns digits [8l, 8l+8); the digit holding the need-th
+          // largest key is where the count from the top first reaches need.
+          uint32_t c[8], sum = 0;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            c[q] = sh.hist[8 * lane + q];
+            sum += c[q];
+          }
+          uint32_t suf = sum;  // sum over lanes >= this lane
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += y;
+          }
+          const uint32_t above = suf - sum;
+          if (above < need && need <= suf) {
+            uint32_t acc = above;
+#pragma unroll
+            for (int q = 7; q >= 0; --q) {
+              if (acc + c[q] >= need) {
+                sh.prefix = P | (static_cast<uint32_t>(8 * lane + q) << shift);
+                sh.need = need - acc;
+                break;
+              }
+              acc += c[q];
+            }
+          }
+        }
+        group_bar(bar_id, NT);
+        P = sh.prefix;
+        need = sh.need;
+        r = shift;
+        GTK_STAMP(2);
+      }
+      T = P;
+    }
+  }
+  // Placement: keys above T, then the first `need` keys equal to T in index
+  // order.  (gt << 16 | eq) per thread, scanned over the group.
+  uint32_t gt = 0, eq = 0;
+#pragma unroll
+  for (int m = 0; m < kGroupKeys; ++m)
+    if (m < kpt && b0 + m < ncand) {
+      gt += key[m] > T;
+      eq += key[m] == T;
+    }
+  if (k_eff == ncand) {  // everything is taken
+    gt += eq;
+    eq = 0;
+    need = 0;
+  }
+  const uint32_t mine = (gt << 16) | eq;
+  uint32_t incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sh.red[1][warp][0] = incl;
+  GTK_STAMP(3);
+  group_bar(bar_id, NT);
+  GTK_STAMP(4);
+  uint32_t before = incl - mine;
+  for (int w = 0; w < warp; ++w) before += sh.red[1][w][0];
+  const uint32_t gt_before = before >> 16, eq_before = before & 0xFFFFu;
+  int pos = static_cast<int>(gt_before + min(eq_before, need));
+  uint32_t eq_take = min(eq_before + eq, need) - min(eq_before, need);
+#pragma unroll
+  for (int m = 0; m < kGroupKeys; ++m) {
+    const int b = b0 + m;
+    if (m < kpt && b < ncand) {
+      bool take = key[m] > T || k_eff == ncand;
+      if (!take && key[m] == T && eq_take > 0) {
+        take = true;
+        --eq_take;
+      }
+      if (take) {
+        if (pos < topk) sel_row[pos] = b;
+        ++pos;
+      }
+    }
+  }
+  for (int x = k_eff + tid; x < topk; x += NT) sel_row[x] = -1;
+  if (tid == 0) *sel_cnt = k_eff;
+  GTK_STAMP(5);
+#undef GTK_STAMP
+}
+
+// Candidates up to which one warp selects faster than the selection group
+// (measured on B200: 240 candidates one warp, 1008 the group).
+constexpr int kWarpSelectMax = 256;
+
 // Top-k by one warp: register-resident keys up to kWarpTopkMax candidates,
 // memory-resident beyond.
 __device__ inline void warp_select(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,

@@ -53,7 +53,7 @@ namespace nosa {
 // kernel with %globaltimer stamps of its phases.
 struct TraceRecord {
   uint32_t pair, rank, smid, csize;
-  uint64_t t[16];  // see the NOSA_STAMP call sites
+  uint64_t t[24];  // see the NOSA_STAMP call sites
 };
 constexpr int kTraceCapacity = 1 << 16;
 __device__ TraceRecord g_trace[kTraceCapacity];
@@ -80,8 +80,9 @@ struct StepShared {
   int stage_blk[kStages];
   int sel_count;
   float blk[kChunkBlocks];  // block scores of the chunk being sent
+  GroupTopkShared gtk;      // the selection group's exchange (consumers + selector)
 #ifdef NOSA_TRACE
-  uint64_t tr[16];
+  uint64_t tr[24];
 #endif
 };
 
@@ -127,6 +128,24 @@ __device__ inline bool consumer_all(bool v) {
   return r != 0;
 }
 
+// The selection group: the consumer warps and the selector warp (160
+// threads, named barrier 2) select together once the block scores are in.
+constexpr int kSelectThreads = kConsumerThreads + 32;
+constexpr int kSelectBar = 2;
+
+__device__ inline bool select_group_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kSelectBar), "n"(kSelectThreads)
+      : "memory");
+  return r != 0;
+}
+
 // Cross-warp merge scratch (in the drained ring): per warp O rows with a
 // padded stride (bank-conflict free float2 stores), row max / sum / weight,
 // then the CTA's row max / sum.
@@ -168,18 +187,18 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       mbar_init(&sh.full_bar[s], 1);
       mbar_init(&sh.empty_bar[s], kConsumerWarps);
     }
-    mbar_init(&sh.scores_bar, C);
+    // Block scores in shared memory arrive as st.async transactions counted
+    // in bytes against the selector's one arrival; in global memory (spill)
+    // every CTA of the cluster arrives once.
+    mbar_init(&sh.scores_bar, spill ? C : 1);
     mbar_init(&sh.sel_bar, 1);
     fence_barrier_init();
 #ifdef NOSA_TRACE
-    for (int k = 0; k < 16; ++k) sh.tr[k] = 0;
+    for (int k = 0; k < 24; ++k) sh.tr[k] = 0;
     NOSA_STAMP(0);
 #endif
   }
   __syncthreads();
-  // Cluster barrier phase 1: this CTA's barriers exist.  Each thread waits
-  // on it before its first access to another CTA's shared memory.
-  cluster_arrive();
   if (warp == kProducerWarp && lane == 0) {
     if (scoring) asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_p) : "memory");
     if (decoding) {
@@ -222,6 +241,40 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     if (scoring && nc_all > a.nc_cap) set_status(a.status, NOSA_DEV_NC_CAP);
   }
   const __nv_bfloat16* q_group = a.q + (static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G) * kHeadDim;
+  // The selector expects the pair's block-score bytes before this CTA joins
+  // cluster barrier phase 1, so no other CTA can send one before.
+  if (scoring && !spill && warp == kSelectorWarp && lane == 0)
+    mbar_arrive_expect_tx(&sh.scores_bar, 4u * static_cast<uint32_t>(ncand));
+  // Cluster barrier phase 1: this CTA's barriers exist (and expect their
+  // bytes).  Each thread waits on it before its first access to another
+  // CTA's shared memory.
+  cluster_arrive();
+
+  // Who selects: one warp (the selector) for small candidate sets or block
+  // scores in global memory, else the selection group (uniform per pair).
+  const bool group_selects = scoring && !spill && ncand > kWarpSelectMax;
+  // Top-k of the pair by the selection group, from the block scores in
+  // shared memory; every member calls it (gtid = its index in the group).
+  // The decision to give up after a timed-out wait is taken together.
+  auto group_select = [&](int gtid) {
+    bool ok = mbar_wait_cluster(&sh.scores_bar, 0, a.status);
+    ok = select_group_all(ok);
+#ifdef NOSA_TRACE
+    if (gtid == kConsumerThreads) NOSA_STAMP(3);
+#endif
+    if (ok) {
+#ifdef NOSA_TRACE
+      group_topk<kSelectThreads>(bsm, false, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar,
+                                 &sh.tr[14]);
+#else
+      group_topk<kSelectThreads>(bsm, false, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
+#endif
+    } else {
+      for (int x = gtid; x < a.topk; x += kSelectThreads) sel_list[x] = -1;
+      if (gtid == 0) sh.sel_count = 0;
+    }
+    group_bar(kSelectBar, kSelectThreads);
+  };
 
   AttnState att;
   if (warp == kProducerWarp) {
@@ -324,22 +377,22 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       }
     }
     if (scoring) {
-      const bool ok = mbar_wait_cluster(&sh.scores_bar, 0, a.status);
-#ifdef NOSA_TRACE
-      if (lane == 0) NOSA_STAMP(3);
-#endif
-      if (ok) {
-        const float* src = spill ? a.bs_spill + static_cast<int64_t>(pair) * a.nb_spill : bsm;
-#ifdef NOSA_TRACE
-        warp_select(src, spill, ncand, a.topk, sel_list, &sh.sel_count, lane, &sh.tr[8]);
-#else
-        warp_select(src, spill, ncand, a.topk, sel_list, &sh.sel_count, lane);
-#endif
+      if (group_selects) {
+        group_select(kConsumerThreads + lane);
       } else {
-        for (int t = lane; t < a.topk; t += 32) sel_list[t] = -1;
-        if (lane == 0) sh.sel_count = 0;
+        const bool ok = mbar_wait_cluster(&sh.scores_bar, 0, a.status);
+#ifdef NOSA_TRACE
+        if (lane == 0) NOSA_STAMP(3);
+#endif
+        if (ok) {
+          warp_select(spill ? a.bs_spill + static_cast<int64_t>(pair) * a.nb_spill : bsm, spill, ncand, a.topk,
+                      sel_list, &sh.sel_count, lane);
+        } else {
+          for (int t = lane; t < a.topk; t += 32) sel_list[t] = -1;
+          if (lane == 0) sh.sel_count = 0;
+        }
+        __syncwarp();
       }
-      __syncwarp();
       if (rank == 0) {
         int32_t* dst = a.sel_idx + static_cast<int64_t>(pair) * a.topk;
         for (int t = lane; t < a.topk; t += 32) dst[t] = sel_list[t];
@@ -370,11 +423,18 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
             ok = false;
             break;
           }
+#ifdef NOSA_TRACE
+          const int cix = (k - static_cast<int>(rank)) / static_cast<int>(C);
+          if (tid == 0 && cix < 0) NOSA_STAMP(14 + 4 * cix);
+#endif
           score_stage<G>(qf, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
           ++r;
           consumer_sync();  // the chunk's window scores are complete
+#ifdef NOSA_TRACE
+          if (tid == 0 && cix < 0) NOSA_STAMP(15 + 4 * cix);
+#endif
           const int b0 = kChunkBlocks * k;
           const int nblk = min(kChunkBlocks, ncand - b0);
           if (tid < nblk) {
@@ -395,22 +455,33 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
             }
           }
           consumer_sync();  // sh.blk is complete; ssm may be overwritten
+#ifdef NOSA_TRACE
+          if (tid == 0 && cix < 0) NOSA_STAMP(16 + 4 * cix);
+#endif
           if (!spill)
             for (int x = tid; x < nblk * static_cast<int>(C); x += kConsumerThreads) {
               const int b = x / static_cast<int>(C);
               const uint32_t dst = static_cast<uint32_t>(x % static_cast<int>(C));
-              st_cluster_f32(map_shared_rank(smem_addr(bsm + b0 + b), dst), sh.blk[b]);
+              st_async_f32(map_shared_rank(smem_addr(bsm + b0 + b), dst), sh.blk[b],
+                           map_shared_rank(smem_addr(&sh.scores_bar), dst));
             }
+#ifdef NOSA_TRACE
+          if (tid == 0 && cix < 0) NOSA_STAMP(17 + 4 * cix);
+#endif
         }
       }
-      // Tell every CTA of the cluster (this one included) that this CTA's
-      // block scores are in place.
-      fence_acq_rel_cluster();
-      consumer_sync();
-      if (tid == 0) {
-        for (uint32_t d = 0; d < C; ++d) mbar_remote_arrive(map_shared_rank(smem_addr(&sh.scores_bar), d));
-        NOSA_STAMP(2);
+      if (spill) {
+        // Block scores in global memory: tell every CTA of the cluster (this
+        // one included) that this CTA's are in place.
+        fence_acq_rel_cluster();
+        consumer_sync();
+        if (tid == 0)
+          for (uint32_t d = 0; d < C; ++d) mbar_remote_arrive(map_shared_rank(smem_addr(&sh.scores_bar), d));
       }
+#ifdef NOSA_TRACE
+      if (tid == 0) NOSA_STAMP(2);
+#endif
+      if (group_selects) group_select(tid);
     }
     attn_init(att);
     if (decoding && ok) {
@@ -420,9 +491,18 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       if (my_tiles > 0) {
         uint32_t qa[8][4];
         load_attn_q(qa, q_group, G, lane);
+        // Tiles start once the selection is known (the consumers took part
+        // in it, or wait for the selector): the selection runs on a quiet
+        // SM, and the local tiles, already staged, are consumed while the
+        // first selected tiles are in flight.
+        if (scoring && !group_selects) mbar_wait(&sh.sel_bar, 0, a.status);
         for (int n = 0; n < my_tiles; ++n) {
           const int s = static_cast<int>(r % kStages);
           if (!mbar_wait(&sh.full_bar[s], (r / kStages) & 1u, a.status)) break;
+#ifdef NOSA_TRACE
+          if (tid == 0 && n == 0) NOSA_STAMP(22);
+          if (tid == 0 && n == 2) NOSA_STAMP(23);
+#endif
           attend_tile(att, qa, smem + s * kStageBytes, sh.stage_blk[s], L, a.scale_log2, warp, lane);
           if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
           ++r;
@@ -570,7 +650,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       rec.rank = rank;
       rec.smid = smid;
       rec.csize = C;
-      for (int n = 0; n < 16; ++n) rec.t[n] = sh.tr[n];
+      for (int n = 0; n < 24; ++n) rec.t[n] = sh.tr[n];
       g_trace[k] = rec;
     }
   }

@@ -203,6 +203,34 @@ def test_select_unplanted_ragged_valid(nosa):
     _status_ok(nosa, st.ws)
 
 
+@pytest.mark.parametrize("L", [16384, 65536, 132_000])
+def test_select_ties_resolved_to_lowest_index(nosa, L):
+    """All keys zero except 10 planted blocks per KV head: every other block
+    scores exactly 0, so 54 of the 64 picks are ties that the lowest block
+    index must win -- through the whole scoring path (240, 1008 and 2047
+    candidates: every key count per thread of the selection group)."""
+    b = inputs.make_batch(L, batch=1, num_q_heads=16, num_kv_heads=2, seed=41)
+    b.k_cache.zero_()
+    G = 8
+    rng = np.random.default_rng(41)
+    ncand = oracle.n_candidates(L)
+    for h in range(2):
+        u = b.q[0, h * G:(h + 1) * G].float().sum(0)
+        u = u / u.norm()
+        for c in rng.choice(ncand, size=10, replace=False):
+            t0 = int(b.seq_start[0]) + 64 * int(c) + 16
+            b.k_cache[t0:t0 + 32, h] = (u * float(rng.uniform(1.0, 3.0))).to(torch.bfloat16)
+    ref = oracle_step(b, 64)
+    g = b.to(DEV)
+    p, st = _gpu_state(nosa, b, 64)
+    st.rebuild_pooled(g.k_cache, g.seq_start, g.seq_len)
+    st.step(g.q, g.k_cache, g.v_cache, g.seq_start, g.seq_len, append=False)
+    np.testing.assert_array_equal(st.sel_idx.cpu().numpy(), ref["sel_idx"])
+    np.testing.assert_array_equal(st.sel_cnt.cpu().numpy(), ref["sel_cnt"])
+    assert_out_close(st.out.float().cpu().numpy(), ref["out"])
+    _status_ok(nosa, st.ws)
+
+
 @pytest.mark.parametrize("hq,hkv,key_dist", [(2, 2, "normal"), (4, 2, "student_t"), (8, 2, "normal"),
                                              (16, 2, "student_t"), (32, 2, "normal"), (32, 8, "student_t")])
 def test_select_scores_every_group_size(nosa, hq, hkv, key_dist):
