@@ -33,10 +33,11 @@
 namespace nosa {
 
 constexpr int kConsumerWarps = 4;                          // warps that own 16 tokens of a tile each
-constexpr int kStages = 3;
 constexpr int kHalfBytes = kBlock * 128;                   // one 64-token x 64-dim box: 8 KB
 constexpr int kStageBytes = 4 * kHalfBytes;                // K lo/hi, V lo/hi: 32 KB
-constexpr int kRingBytes = kStages * kStageBytes;          // 96 KB
+constexpr int kMinStages = 3;                              // ring of 2 CTAs per SM
+constexpr int kMaxStages = 6;                              // ring of 1 CTA per SM
+constexpr int kRingBytes = kMinStages * kStageBytes;       // 96 KB: the smallest ring
 constexpr uint32_t kTileTxBytes = kStageBytes;
 constexpr float kLn2 = 0.69314718055994530942f;
 

@@ -73,11 +73,11 @@ constexpr int kCtasPerSm = 2;
 constexpr int kSelOnlyThreads = 256;
 
 struct StepShared {
-  uint64_t full_bar[kStages];
-  uint64_t empty_bar[kStages];
+  uint64_t full_bar[kMaxStages];
+  uint64_t empty_bar[kMaxStages];
   uint64_t scores_bar;  // completes when every CTA of the cluster has sent its block scores
   uint64_t sel_bar;     // completes when the selection is in shared memory (selector -> producer)
-  int stage_blk[kStages];
+  int stage_blk[kMaxStages];
   int sel_count;
   float blk[kChunkBlocks];  // block scores of the chunk being sent
   GroupTopkShared gtk;      // the selection group's exchange (consumers + selector)
@@ -161,16 +161,19 @@ struct MergeLayout {
 };
 static_assert((MergeLayout<kMaxGroup>::kPl + kMaxGroup) * 4 <= kRingBytes, "merge scratch must fit in the ring");
 
-template <int G>
+// S = ring stages: 3 (two CTAs per SM) or 6 (one CTA per SM, twice the
+// bytes in flight per CTA).
+template <int G, int S>
 __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     step_kernel(const StepArgs a, const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_p) {
+  constexpr int kRing = S * kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled TMA boxes want 1024-byte aligned destinations.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* ssm = reinterpret_cast<float*>(smem + kRingBytes);
-  int32_t* sel_list = reinterpret_cast<int32_t*>(smem + kRingBytes + ssm_bytes<G>());
-  float* bsm = reinterpret_cast<float*>(smem + kRingBytes + ssm_bytes<G>() + round16(4 * a.topk));
+  float* ssm = reinterpret_cast<float*>(smem + kRing);
+  int32_t* sel_list = reinterpret_cast<int32_t*>(smem + kRing + ssm_bytes<G>());
+  float* bsm = reinterpret_cast<float*>(smem + kRing + ssm_bytes<G>() + round16(4 * a.topk));
   __shared__ StepShared sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -183,7 +186,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 
   if (tid == 0) {
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&sh.full_bar[s], 1);
       mbar_init(&sh.empty_bar[s], kConsumerWarps);
     }
@@ -286,8 +289,8 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     auto issue = [&](auto&& body) {
       int good = 1;
       if (lane == 0) {
-        const int s = static_cast<int>(r % kStages);
-        if (r >= static_cast<uint32_t>(kStages) && !mbar_wait(&sh.empty_bar[s], ((r / kStages) - 1) & 1u, a.status))
+        const int s = static_cast<int>(r % S);
+        if (r >= static_cast<uint32_t>(S) && !mbar_wait(&sh.empty_bar[s], ((r / S) - 1) & 1u, a.status))
           good = 0;
         else
           body(s, smem + s * kStageBytes);
@@ -352,8 +355,8 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     }
     // Every copy issued has landed before the ring is reused for the merge.
     if (lane == 0) {
-      const uint32_t first = r > static_cast<uint32_t>(kStages) ? r - kStages : 0u;
-      for (uint32_t n = first; n < r; ++n) mbar_wait(&sh.full_bar[n % kStages], (n / kStages) & 1u, a.status);
+      const uint32_t first = r > static_cast<uint32_t>(S) ? r - S : 0u;
+      for (uint32_t n = first; n < r; ++n) mbar_wait(&sh.full_bar[n % S], (n / S) & 1u, a.status);
     }
     __syncwarp();
     cluster_wait();
@@ -417,8 +420,8 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
         ScoreQ<G> qf;
         load_score_q<G>(qf, q_group, lane);
         for (int k = static_cast<int>(rank); k < nchunks; k += static_cast<int>(C)) {
-          const int s = static_cast<int>(r % kStages);
-          const bool landed = consumer_all(mbar_wait(&sh.full_bar[s], (r / kStages) & 1u, a.status));
+          const int s = static_cast<int>(r % S);
+          const bool landed = consumer_all(mbar_wait(&sh.full_bar[s], (r / S) & 1u, a.status));
           if (!landed) {
             ok = false;
             break;
@@ -438,10 +441,10 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           const int b0 = kChunkBlocks * k;
           const int nblk = min(kChunkBlocks, ncand - b0);
           if (tid < nblk) {
-            const float S = block_rule<G>(ssm, k, tid, nc);
-            sh.blk[tid] = S;
-            if (a.bs_out) a.bs_out[static_cast<int64_t>(pair) * a.nb_out + b0 + tid] = S;
-            if (spill) a.bs_spill[static_cast<int64_t>(pair) * a.nb_spill + b0 + tid] = S;
+            const float bscore = block_rule<G>(ssm, k, tid, nc);
+            sh.blk[tid] = bscore;
+            if (a.bs_out) a.bs_out[static_cast<int64_t>(pair) * a.nb_out + b0 + tid] = bscore;
+            if (spill) a.bs_spill[static_cast<int64_t>(pair) * a.nb_spill + b0 + tid] = bscore;
           }
           if (a.comp_out) {
             // windows [60k, min(60k + 60, nc)); the row of window j is j - 60k + 1
@@ -497,8 +500,8 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
         // first selected tiles are in flight.
         if (scoring && !group_selects) mbar_wait(&sh.sel_bar, 0, a.status);
         for (int n = 0; n < my_tiles; ++n) {
-          const int s = static_cast<int>(r % kStages);
-          if (!mbar_wait(&sh.full_bar[s], (r / kStages) & 1u, a.status)) break;
+          const int s = static_cast<int>(r % S);
+          if (!mbar_wait(&sh.full_bar[s], (r / S) & 1u, a.status)) break;
 #ifdef NOSA_TRACE
           if (tid == 0 && n == 0) NOSA_STAMP(22);
           if (tid == 0 && n == 2) NOSA_STAMP(23);
@@ -519,7 +522,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   // ---------------------------------------------------------------- merge
   using ML = MergeLayout<G>;
   float* mf = reinterpret_cast<float*>(smem);
-  float* recv = reinterpret_cast<float*>(smem + kRingBytes + ssm_bytes<G>() + round16(4 * a.topk) +
+  float* recv = reinterpret_cast<float*>(smem + kRing + ssm_bytes<G>() + round16(4 * a.topk) +
                                          (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))));
   if (decoding) {
     // The four warps' states, in warp order, into this CTA's partial.
@@ -649,7 +652,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       rec.pair = pair;
       rec.rank = rank;
       rec.smid = smid;
-      rec.csize = C;
+      rec.csize = C | (S << 8);
       for (int n = 0; n < 24; ++n) rec.t[n] = sh.tr[n];
       g_trace[k] = rec;
     }
@@ -695,30 +698,29 @@ __global__ void wait_selftest_kernel(uint32_t* status, uint32_t max_iters) {
 }
 
 template <int G>
-size_t step_smem_bytes(const StepArgs& a) {
-  return 1024 + kRingBytes + ssm_bytes<G>() + round16(4 * a.topk) + (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))) +
-         recv_bytes<G>();
+size_t step_smem_bytes(const StepArgs& a, int stages) {
+  return 1024 + static_cast<size_t>(stages) * kStageBytes + ssm_bytes<G>() + round16(4 * a.topk) +
+         (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))) + recv_bytes<G>();
 }
 
-// Cluster size and launch mode for `pairs` clusters (see the rules below);
-// C = 1 when no larger cluster fits (then clusters run in waves).
-struct ClusterPlanCache {
+// Residency of the step kernel at a given shared-memory size: resident
+// CTAs and co-resident clusters of each size (cached per kernel and size).
+struct Capacity {
   int dev = -1;
   size_t smem = 0;
-  int slots = 0;
-  int max_clusters[kMaxCluster + 1] = {};  // co-resident clusters of C CTAs, C = 1..16
+  int slots = 0, sms = 0;
+  int max_clusters[kMaxCluster + 1] = {};  // C = 1..16
 };
 std::mutex g_plan_mu;
-ClusterPlanCache g_plan[5];  // per group size
+Capacity g_cap[5][2];  // [group size][ring: 3 or 6 stages]
 
-template <int G>
-cudaError_t plan_cluster(int pairs, int units, size_t smem, int* csize, bool* pdl) {
+template <int G, int S>
+cudaError_t capacity(size_t smem, const Capacity** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   constexpr int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
-  std::lock_guard<std::mutex> lock(g_plan_mu);
-  ClusterPlanCache& c = g_plan[gi];
+  Capacity& c = g_cap[gi][S == kMinStages ? 0 : 1];
   if (c.dev != dev || c.smem != smem) {
     // The attribute is an upper bound: set to the largest size the device
     // allows next to the kernel's static shared memory, so that concurrent
@@ -726,20 +728,22 @@ cudaError_t plan_cluster(int pairs, int units, size_t smem, int* csize, bool* pd
     int optin = 0;
     cudaFuncAttributes fa;
     if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-    if ((e = cudaFuncGetAttributes(&fa, step_kernel<G>)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa, step_kernel<G, S>)) != cudaSuccess) return e;
     const int max_dyn = optin - static_cast<int>(fa.sharedSizeBytes);
     if (static_cast<int>(smem) > max_dyn) return cudaErrorInvalidValue;
-    if ((e = cudaFuncSetAttribute(step_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn)) !=
+    if ((e = cudaFuncSetAttribute(step_kernel<G, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn)) !=
         cudaSuccess)
       return e;
-    if ((e = cudaFuncSetAttribute(step_kernel<G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(step_kernel<G, S>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
+        cudaSuccess)
       return e;
     int per_sm = 0, sms = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<G>, kStepThreads, smem)) !=
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<G, S>, kStepThreads, smem)) !=
         cudaSuccess)
       return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     c.slots = per_sm * sms;
+    c.sms = sms;
     for (int cs = 1; cs <= kMaxCluster; ++cs) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(cs);
@@ -753,7 +757,7 @@ cudaError_t plan_cluster(int pairs, int units, size_t smem, int* csize, bool* pd
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, step_kernel<G>, &cfg) != cudaSuccess) {
+      if (cudaOccupancyMaxActiveClusters(&n, step_kernel<G, S>, &cfg) != cudaSuccess) {
         cudaGetLastError();  // a size the device cannot co-schedule: never chosen
         n = 0;
       }
@@ -762,11 +766,16 @@ cudaError_t plan_cluster(int pairs, int units, size_t smem, int* csize, bool* pd
     c.dev = dev;
     c.smem = smem;
   }
-  // Among the cluster sizes whose pairs x C CTAs are all resident at once,
-  // the smallest C with the fewest scoring chunks per CTA: a larger cluster
-  // would not shorten the longest CTA's scoring and only costs wider
-  // exchanges.  The environment variable
-  // NOSA_CLUSTER_SIZE (1..16) overrides the choice.
+  *out = &c;
+  return cudaSuccess;
+}
+
+// Among the cluster sizes whose pairs x C CTAs are all resident at once,
+// the smallest C with the fewest scoring chunks per CTA (`units` of the
+// longest pair): a larger cluster would not shorten the longest CTA's
+// scoring and only costs wider exchanges.  1 when no larger cluster fits
+// (then clusters run in waves).
+int choose_cluster(const Capacity& c, int pairs, int units) {
   int best = 1, best_units = units;
   for (int cs = 2; cs <= kMaxCluster; ++cs) {
     if (static_cast<int64_t>(pairs) * cs > c.slots || c.max_clusters[cs] < pairs) continue;
@@ -776,42 +785,14 @@ cudaError_t plan_cluster(int pairs, int units, size_t smem, int* csize, bool* pd
       best_units = per_cta;
     }
   }
-  static const int forced = [] {
-    const char* v = getenv("NOSA_CLUSTER_SIZE");
-    const int n = v ? atoi(v) : 0;
-    return n >= 1 && n <= kMaxCluster ? n : 0;
-  }();
-  if (forced && c.max_clusters[forced] > 0) best = forced;
-  // Programmatic dependent launch only when the grid leaves at least half of
-  // the slots free: the next launch's clusters then become resident and run
-  // their prologue early.  When the grid fills the GPU, early-resident
-  // clusters of the next launch only skew where the rest are placed.
-  *pdl = static_cast<int64_t>(pairs) * best * 2 <= c.slots;
-#ifdef NOSA_TRACE
-  fprintf(stderr, "plan G=%d smem=%zu slots=%d pairs=%d units=%d -> C=%d pdl=%d (max clusters %d)\n", G, smem,
-          c.slots, pairs, units, best, static_cast<int>(*pdl), c.max_clusters[best]);
-#endif
-  *csize = best;
-  return cudaSuccess;
+  return best;
 }
 
-template <int G>
-cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
-                          cudaStream_t stream) {
-  const int pairs = a.batch * a.hkv;
-  if (pairs <= 0) return cudaSuccess;
-  const size_t smem = step_smem_bytes<G>(a);
-  // Work units of the longest pair: its selection's scoring chunks.  The
-  // same in every mode, so the separate selection and attention launches
-  // split a pair's tiles exactly as the fused step does (bit-identical
-  // results).
-  const int units = (a.ncand_max + kChunkBlocks - 1) / kChunkBlocks;
-  int csize = 1;
-  bool pdl = false;
-  cudaError_t e = plan_cluster<G>(pairs, max(units, 1), smem, &csize, &pdl);
-  if (e != cudaSuccess) return e;
+template <int G, int S>
+cudaError_t launch_with(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
+                        size_t smem, int csize, bool pdl, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(pairs) * csize);
+  cfg.gridDim = dim3(static_cast<unsigned>(a.batch * a.hkv) * csize);
   cfg.blockDim = dim3(kStepThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -824,7 +805,63 @@ cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUte
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, step_kernel<G>, a, tm_k, tm_v, tm_p);
+  return cudaLaunchKernelEx(&cfg, step_kernel<G, S>, a, tm_k, tm_v, tm_p);
+}
+
+// Launch plan: the cluster size (choose_cluster) on the 3-stage ring, two
+// CTAs per SM.  When the whole grid then fits one CTA per SM, the 6-stage
+// ring (one CTA per SM, twice the bytes in flight) runs instead, if the
+// same cluster size is still co-resident.  Programmatic dependent launch
+// only when the grid leaves at least half of the resident slots free: the
+// next launch's clusters then become resident and run their prologue early;
+// when the grid fills the GPU, early-resident clusters of the next launch
+// only skew where the rest are placed.  NOSA_CLUSTER_SIZE (1..16) and
+// NOSA_RING_STAGES (3 or 6) override the choices.
+template <int G>
+cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
+                          cudaStream_t stream) {
+  const int pairs = a.batch * a.hkv;
+  if (pairs <= 0) return cudaSuccess;
+  // Work units of the longest pair: its selection's scoring chunks.  The
+  // same in every mode, so the separate selection and attention launches
+  // split a pair's tiles exactly as the fused step does (bit-identical
+  // results).
+  const int units = max((a.ncand_max + kChunkBlocks - 1) / kChunkBlocks, 1);
+  static const int forced_c = [] {
+    const char* v = getenv("NOSA_CLUSTER_SIZE");
+    const int n = v ? atoi(v) : 0;
+    return n >= 1 && n <= kMaxCluster ? n : 0;
+  }();
+  static const int forced_s = [] {
+    const char* v = getenv("NOSA_RING_STAGES");
+    const int n = v ? atoi(v) : 0;
+    return n == kMinStages || n == kMaxStages ? n : 0;
+  }();
+  const size_t smem3 = step_smem_bytes<G>(a, kMinStages), smem6 = step_smem_bytes<G>(a, kMaxStages);
+  int csize, stages = kMinStages;
+  bool pdl;
+  {
+    std::lock_guard<std::mutex> lock(g_plan_mu);
+    const Capacity* c3 = nullptr;
+    cudaError_t e = capacity<G, kMinStages>(smem3, &c3);
+    if (e != cudaSuccess) return e;
+    csize = choose_cluster(*c3, pairs, units);
+    if (forced_c && c3->max_clusters[forced_c] > 0) csize = forced_c;
+    pdl = static_cast<int64_t>(pairs) * csize * 2 <= c3->slots;
+    const Capacity* c6 = nullptr;
+    const bool want6 = forced_s ? forced_s == kMaxStages : static_cast<int64_t>(pairs) * csize <= c3->sms;
+    if (want6 && capacity<G, kMaxStages>(smem6, &c6) == cudaSuccess && c6->max_clusters[csize] >= pairs) {
+      stages = kMaxStages;
+      pdl = static_cast<int64_t>(pairs) * csize * 2 <= c6->slots;
+    }
+    cudaGetLastError();  // a 6-stage ring the device cannot host is simply not used
+#ifdef NOSA_TRACE
+    fprintf(stderr, "plan G=%d pairs=%d units=%d -> C=%d stages=%d pdl=%d (3-stage slots %d, 6-stage clusters of C: %d)\n",
+            G, pairs, units, csize, stages, static_cast<int>(pdl), c3->slots, c6 ? c6->max_clusters[csize] : -1);
+#endif
+  }
+  if (stages == kMaxStages) return launch_with<G, kMaxStages>(a, tm_k, tm_v, tm_p, smem6, csize, pdl, stream);
+  return launch_with<G, kMinStages>(a, tm_k, tm_v, tm_p, smem3, csize, pdl, stream);
 }
 
 }  // namespace
