@@ -528,12 +528,6 @@ constexpr int kScoreSlotBytes = 64 * 128;                          // 8 KB
 constexpr uint32_t kScoreTxBytes = 4u * kBoxRows * kBoxCols * 4u;  // bytes landed per chunk
 constexpr int kScoreStride = 64 + 4;                               // floats per head row of window scores
 
-__device__ inline uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
-
 __device__ inline void mma_tf32_1688(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
@@ -579,10 +573,10 @@ __device__ inline void load_score_q(ScoreQ<G>& f, const __nv_bfloat16* __restric
 // computes rows [16w, 16w+16) of S^T = K * Q^T (mma.sync m16n8k8, TF32
 // inputs, fp32 accumulation) and stores scale * s into ssm[head][row] for
 // rows < 61.  Each fp32 pooled value x is split into hi (x with its low 13
-// mantissa bits cleared, exact in TF32) and lo = tf32(x - hi); the hi and lo
-// products go to separate fp32 accumulators (even and odd k-steps apart)
-// that are added at the end, so the only input rounding is that of lo,
-// below 2^-21 of |x| ("NOSA-1B
+// mantissa bits cleared, exact in TF32) and lo (x - hi, exact in fp32, with
+// its low 13 mantissa bits cleared too); the hi and lo products go to
+// separate fp32 accumulators (even and odd k-steps apart) that are added at
+// the end, so the only input rounding is that of lo, below 2^-20 of |x| ("NOSA-1B
 // 性能基准全解析" §三.3: scores of the pooled keys).
 template <int G>
 __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* __restrict__ ssm, float scale,
@@ -618,7 +612,7 @@ __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* _
     for (int e = 0; e < 4; ++e) {
       hi[e] = __float_as_uint(x[e]) & 0xffffe000u;
       const float r = x[e] - __uint_as_float(hi[e]);  // exact; NaN only for infinite x
-      lo[e] = to_tf32(r == r ? r : 0.0f);
+      lo[e] = __float_as_uint(r == r ? r : 0.0f) & 0xffffe000u;
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -640,24 +634,37 @@ __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* _
   }
 }
 
-// Block rule for block b = 15k + t of chunk k (t < 15) from the chunk's
-// window scores: S[b] = sum over the group's heads (ascending) of the max of
-// s over windows 4b-1 .. 4b+3 that exist (0 <= j < nc), i.e. rows 4t .. 4t+4.
+// Block rule for the blocks of chunk k, from the chunk's window scores:
+// S[b] = sum over the group's heads of the max of s over windows
+// 4b-1 .. 4b+3 that exist (0 <= j < nc), i.e. rows 4t .. 4t+4 for block
+// b = 15k + t.  Spread over the consumer threads: min(G, 8) lanes per block,
+// each taking the window max of G / min(G, 8) heads, then a fixed shuffle
+// tree sums the heads.  Every thread of the (full) warps calls it; lane
+// `hl == 0` of block t's lanes returns S[b] in *out and true.
 template <int G>
-__device__ inline float block_rule(const float* __restrict__ ssm, int k, int t, int64_t nc) {
+__device__ inline bool block_rule(const float* __restrict__ ssm, int k, int nblk, int64_t nc, int tid, float* out) {
+  constexpr int kLanes = G < 8 ? G : 8;   // lanes per block
+  constexpr int kHeads = G / kLanes;      // heads per lane
+  const int t = tid / kLanes, hl = tid % kLanes;
   const int64_t jb = static_cast<int64_t>(kWindowsPerBlock) * (kChunkBlocks * k + t) - 1;
-  float S = 0.0f;
+  float part = 0.0f;
+  if (t < nblk) {
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float m = -INFINITY;
+    for (int hh = 0; hh < kHeads; ++hh) {
+      const int h = hl * kHeads + hh;
+      float m = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWindowsPerBlock + 1; ++w) {
-      const int64_t j = jb + w;
-      if (j >= 0 && j < nc) m = fmaxf(m, ssm[h * kScoreStride + 4 * t + w]);
+      for (int w = 0; w < kWindowsPerBlock + 1; ++w) {
+        const int64_t j = jb + w;
+        if (j >= 0 && j < nc) m = fmaxf(m, ssm[h * kScoreStride + 4 * t + w]);
+      }
+      part += m;
     }
-    S += m;
   }
-  return S;
+#pragma unroll
+  for (int o = kLanes / 2; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  *out = part;
+  return t < nblk && hl == 0;
 }
 
 }  // namespace nosa

@@ -440,11 +440,15 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 #endif
           const int b0 = kChunkBlocks * k;
           const int nblk = min(kChunkBlocks, ncand - b0);
-          if (tid < nblk) {
-            const float bscore = block_rule<G>(ssm, k, tid, nc);
-            sh.blk[tid] = bscore;
-            if (a.bs_out) a.bs_out[static_cast<int64_t>(pair) * a.nb_out + b0 + tid] = bscore;
-            if (spill) a.bs_spill[static_cast<int64_t>(pair) * a.nb_spill + b0 + tid] = bscore;
+          {
+            float bscore;
+            if (block_rule<G>(ssm, k, nblk, nc, tid, &bscore)) {
+              constexpr int kLanes = G < 8 ? G : 8;
+              const int t = tid / kLanes;
+              sh.blk[t] = bscore;
+              if (a.bs_out) a.bs_out[static_cast<int64_t>(pair) * a.nb_out + b0 + t] = bscore;
+              if (spill) a.bs_spill[static_cast<int64_t>(pair) * a.nb_spill + b0 + t] = bscore;
+            }
           }
           if (a.comp_out) {
             // windows [60k, min(60k + 60, nc)); the row of window j is j - 60k + 1
