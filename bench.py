@@ -77,6 +77,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--settle-ms", type=float, default=300.0,
                     help="untimed repeated steps before timing, so clocks settle")
+    ap.add_argument("--sweep", action="store_true",
+                    help="NOSA-1B shape over context x batch x top-k (one JSON line per point)")
     return ap.parse_args()
 
 
@@ -284,6 +286,17 @@ def oracle_steps(wl: Workload, b_host, n_steps: int, threads: int, budget_s: flo
     return done, time.perf_counter() - t0
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def host_batch(wl: Workload, seed: int):
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     return inputs.make_batch(wl.lens, num_q_heads=wl.hq, num_kv_heads=wl.hkv, seed=seed,
@@ -429,10 +442,13 @@ def run_ours(args):
         threads = os.cpu_count() or 1
         n, secs = oracle_steps(wl, b_host, 10 ** 6, threads, args.cpu_seconds)
         cpu_ms = secs / n * wl.layers * 1e3
+        n1, secs1 = oracle_steps(wl, b_host, 10 ** 6, 1, min(3.0, args.cpu_seconds))
         cpu = {"value": queries_per_step / (cpu_ms / 1e3), "unit": UNIT, "cores": threads,
                "kind": "oracle",
                "sample": f"{n} one-layer decode steps of this workload (all {wl.batch} sequences) on the "
-                         f"fp64 C oracle in {secs:.1f} s" + (f", scaled x{wl.layers} layers" if wl.layers > 1 else "")}
+                         f"fp64 C oracle in {secs:.1f} s" + (f", scaled x{wl.layers} layers" if wl.layers > 1 else ""),
+               "value_single_thread": queries_per_step / (secs1 / n1 * wl.layers),
+               "cpu_model": cpu_model()}
 
     if rank == 0:
         line = {
@@ -498,12 +514,90 @@ def measure_e2e(nosa, wl: Workload, r: Replica, args, stream, info, device):
             "d2h_bytes_per_step": o_h.numel() * 2, "steps": n, "ms_per_step": ms / n}
 
 
+# ----------------------------------------------------------------------------- sweep
+
+SWEEP_CONTEXTS = (4096, 8192, 16384, 32768, 65536, 131072)
+SWEEP_BATCHES = (1, 8, 32, 64)
+SWEEP_TOPK = (32, 64, 96)          # 2048 / 4096 / 6144 selected tokens
+SWEEP_MEMORY_BYTES = 60e9          # points whose replicas would exceed this are skipped
+
+
+def run_sweep(args):
+    """The NOSA-1B attention shape over context x batch x top-k, one GPU.
+    Per point: fused steps captured as one CUDA graph over cache replicas
+    larger than L2 (CUDA events on the launching stream), and the three
+    standalone launches with events between them for the pool / select /
+    decode split.  One JSON line per point."""
+    from long_context_decode_nosa_b200 import nosa
+    nosa.lib()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peak, peak_kind = peak_hbm()
+    stream = torch.cuda.Stream(device)
+    for L in SWEEP_CONTEXTS:
+        for B in SWEEP_BATCHES:
+            for K in SWEEP_TOPK:
+                a = argparse.Namespace(workload="nosa1b_b8_16k", context=L, batch=B, topk=K)
+                wl = Workload(a, 0)
+                layer_bytes = B * L * wl.hkv * 128 * 2 * 2
+                R = max(2, min(16, math.ceil(1.0e9 / layer_bytes)))
+                point = {"context": L, "batch": B, "topk": K, "replicas": R}
+                if R * layer_bytes * 1.5 > SWEEP_MEMORY_BYTES:
+                    point["skipped"] = f"{R} replicas of {layer_bytes / 1e9:.1f} GB exceed the sweep's memory budget"
+                    print(json.dumps({"sweep_point": point}), flush=True)
+                    continue
+                reps = [Replica(nosa, wl, 1000 + 10 * r, device) for r in range(R)]
+                torch.cuda.synchronize()
+                steps = 100
+                with torch.cuda.stream(stream):
+                    for r in reps:
+                        step(nosa, r)
+                        step(nosa, r, fused=False)
+                stream.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for n in range(steps):
+                        step(nosa, reps[n % R])
+                evs = []
+                g_split = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g_split, stream=stream):
+                    for n in range(max(R, 20)):
+                        e = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+                        step(nosa, reps[n % R], e, fused=False)
+                        evs.append(e)
+                with torch.cuda.stream(stream):
+                    for _ in range(3):
+                        g.replay()
+                    stream.synchronize()
+                    start = torch.cuda.Event(enable_timing=True)
+                    stop = torch.cuda.Event(enable_timing=True)
+                    start.record(stream)
+                    g.replay()
+                    stop.record(stream)
+                    g_split.replay()
+                stream.synchronize()
+                us = start.elapsed_time(stop) * 1e3 / steps
+                split = {k: 1e3 * statistics.fmean(e[j].elapsed_time(e[j + 1]) for e in evs)
+                         for j, k in enumerate(("pool_append", "block_select", "sparse_decode"))}
+                step_bytes = sum(wl.bytes_model().values())
+                gbs = step_bytes / (us * 1e-6) / 1e9
+                point.update({"us_per_step": us, "queries_per_s": B / (us * 1e-6), "gb_per_s": gbs,
+                              "frac_of_peak": gbs / peak, "peak_kind": peak_kind,
+                              "algorithmic_bytes_per_step": step_bytes, "unfused_us": split})
+                print(json.dumps({"sweep_point": point}), flush=True)
+                del g, g_split, reps
+                torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (B200); the CUDA path has no CPU fallback")
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args)
 
 

@@ -307,6 +307,68 @@ def test_decode_dense_equivalence(nosa):
     _status_ok(nosa, st.ws)
 
 
+def test_decode_invariant_to_selection_order(nosa):
+    """Attention over a set: permuting each pair's selected indices (which
+    moves blocks between the cluster's CTAs and changes the merge order)
+    changes the result only by fp32 rounding."""
+    lens = [16384, 9000, 5000]
+    b = inputs.make_batch(lens, num_q_heads=16, num_kv_heads=2, seed=51).to(DEV)
+    p, st = _gpu_state(nosa, b, 64)
+    st.rebuild_pooled(b.k_cache, b.seq_start, b.seq_len)
+    st.step(b.q, b.k_cache, b.v_cache, b.seq_start, b.seq_len, append=False, with_lse=True)
+    out0, lse0 = st.out.float().clone(), st.lse.clone()
+    sel = st.sel_idx.clone()
+    rng = np.random.default_rng(51)
+    cnt = st.sel_cnt.cpu().numpy()
+    for i in range(len(lens)):
+        for h in range(2):
+            perm = torch.from_numpy(rng.permutation(int(cnt[i, h]))).to(DEV)
+            sel[i, h, :cnt[i, h]] = sel[i, h, perm]
+    out = torch.empty_like(st.out)
+    lse = torch.empty_like(st.lse)
+    nosa.nosa_sparse_decode(p, b.q, b.k_cache, b.v_cache, b.seq_start, b.seq_len, st.max_seq_len, sel,
+                            st.sel_cnt, out, st.ws, lse=lse)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(out.float().cpu().numpy(), out0.cpu().numpy(), atol=2e-3, rtol=8e-3)
+    np.testing.assert_allclose(lse.cpu().numpy(), lse0.cpu().numpy(), atol=1e-5, rtol=1e-6)
+    _status_ok(nosa, st.ws)
+
+
+_PARTITION_SCRIPT = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+from long_context_decode_nosa_b200 import inputs, nosa
+b = inputs.make_batch([16384, 6000], num_q_heads=16, num_kv_heads=2, seed=52, device="cuda")
+p = nosa.params(16, 2, topk=64)
+st = nosa.DecodeState(p, b.batch, b.max_seq_len)
+st.rebuild_pooled(b.k_cache, b.seq_start, b.seq_len)
+st.step(b.q, b.k_cache, b.v_cache, b.seq_start, b.seq_len, append=False, with_lse=True)
+torch.cuda.synchronize()
+np.savez(sys.argv[2], out=st.out.float().cpu().numpy(), lse=st.lse.cpu().numpy(),
+         sel=st.sel_idx.cpu().numpy())
+"""
+
+
+def test_attention_invariant_to_cluster_partition(nosa, tmp_path):
+    """Split-K merge of any partition equals one pass: the same step with one
+    CTA per (sequence, KV head) and with clusters of 8 (each CTA a different
+    share of the tiles, merged through distributed shared memory) agrees to
+    fp32 rounding, and selects the same blocks."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = {}
+    for c in (1, 8):
+        env = dict(os.environ, NOSA_CLUSTER_SIZE=str(c))
+        path = str(tmp_path / f"c{c}.npz")
+        subprocess.run([sys.executable, "-c", _PARTITION_SCRIPT, root, path], env=env, check=True, timeout=300)
+        res[c] = np.load(path)
+    np.testing.assert_array_equal(res[1]["sel"], res[8]["sel"])
+    np.testing.assert_allclose(res[1]["lse"], res[8]["lse"], atol=1e-5, rtol=1e-6)
+    np.testing.assert_allclose(res[1]["out"], res[8]["out"], atol=2e-3, rtol=8e-3)
+
+
 def test_full_step_edge_lengths(nosa):
     """Lengths at every geometric edge in one ragged batch, whole step."""
     lens = [1, 2, 31, 32, 33, 63, 64, 65, 1023, 1024, 1025, 1088, 1089, 64 * 17 + 63, 2049, 4096]
