@@ -79,13 +79,29 @@ def n_candidates(L: int, bs: int = 64, local_blocks: int = 16) -> int:
     return max(0, n_blocks(L, bs) - local_blocks)
 
 
+def round_bf16(x):
+    """fp32 values rounded to the nearest bfloat16, ties to even, returned as
+    fp32 (the bf16 pooled-key variant keeps its pooled keys this way).  On the
+    fp32 bit pattern: add 0x7FFF plus the lowest kept bit, then clear the 16
+    dropped bits; NaN stays NaN, infinities stay infinite, and finite values
+    past the largest bf16 round to infinity."""
+    x = np.asarray(x, np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) & 0xFFFF0000).astype(np.uint32)
+    out = r.view(np.float32).copy()
+    out[np.isnan(x)] = np.nan
+    return out
+
+
 def pool(k_cache, seq_start, len_new, nc_cap, *, len_old=None, pooled=None,
-         kernel=32, stride=16):
+         kernel=32, stride=16, bf16=False):
     """Mean-pooled keys: windows [nc(len_old), nc(len_new)) of every (seq, KV head).
 
     k_cache: uint16 [T, Hkv, D] (bf16 bits).  Returns fp32 [B, Hkv, nc_cap, D];
     windows that were not (re)computed keep the contents of ``pooled`` (zeros
-    when ``pooled`` is None)."""
+    when ``pooled`` is None).  ``bf16``: every pooled key rounded to bfloat16
+    (round_bf16), the bf16 pooled-key variant."""
     k_cache = _c(k_cache, np.uint16)
     T, hkv, d = k_cache.shape
     seq_start = _c(seq_start, np.int64)
@@ -96,7 +112,7 @@ def pool(k_cache, seq_start, len_new, nc_cap, *, len_old=None, pooled=None,
     rc = _load().nosa_oracle_pool(_ptr(k_cache), _ptr(seq_start), _ptr(len_old), _ptr(len_new),
                                   B, hkv, d, kernel, stride, _ptr(out), nc_cap)
     _check(rc, "pool")
-    return out
+    return round_bf16(out) if bf16 else out
 
 
 def comp_scores(q, pooled, seq_len, *, num_kv_heads, scale=None, kernel=32, stride=16):

@@ -34,12 +34,12 @@ def sub_batch(b: inputs.DecodeBatch, seqs) -> inputs.DecodeBatch:
                               b.num_q_heads, b.num_kv_heads, b.head_dim)
 
 
-def oracle_step(b: inputs.DecodeBatch, topk: int, *, local_blocks: int = 16, scale=None):
+def oracle_step(b: inputs.DecodeBatch, topk: int, *, local_blocks: int = 16, scale=None, pooled_bf16=False):
     """Pool every window, then the whole selection + attention, on the oracle."""
     kb = inputs.bf16_bits(b.k_cache)
     lens = b.seq_len.cpu().numpy()
     nc_cap = max(1, oracle.n_windows(int(lens.max())))
-    pooled = oracle.pool(kb, b.seq_start.cpu().numpy(), lens, nc_cap)
+    pooled = oracle.pool(kb, b.seq_start.cpu().numpy(), lens, nc_cap, bf16=pooled_bf16)
     nb_cap = oracle.n_blocks(int(lens.max()))
     s = oracle.comp_scores(inputs.bf16_bits(b.q), pooled, lens, num_kv_heads=b.num_kv_heads,
                            scale=scale)

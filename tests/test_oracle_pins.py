@@ -319,3 +319,45 @@ def test_planted_blocks_are_selected_with_a_clear_gap(oracle_mod):
         S = np.sort(r["block_scores"][0, g, :112])[::-1]
         gap = S[47] - S[48]
         assert gap > 1e-3 * max(1.0, abs(S[47])), gap
+
+
+# ----------------------------------------------------------------------------- bf16 pooled keys
+
+def test_round_bf16_matches_torch_conversion(oracle_mod):
+    """The oracle's own round-to-nearest-even against torch's fp32 -> bfloat16
+    conversion: random values over many magnitudes, exact halfway cases with
+    an even and an odd kept bit, subnormals, the largest finite values and
+    the infinities."""
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-40, 40, 20000))).astype(np.float32)
+    kept = rng.integers(0, 1 << 16, 4000, dtype=np.uint32) << 16
+    kept = kept[(kept & 0x7F800000) != 0x7F800000]                   # no NaN / infinity patterns
+    halves = (kept | 0x8000).view(np.float32)                       # exactly halfway
+    sub = (rng.integers(1, 1 << 23, 2000, dtype=np.uint32)).view(np.float32)
+    special = np.array([0.0, -0.0, np.inf, -np.inf, 3.3895314e38, -3.3895314e38, 3.4028235e38,
+                        1.0, 1.00390625, 1.005859375], np.float32)
+    allx = np.concatenate([x, halves, sub, special])
+    want = torch.from_numpy(allx).to(torch.bfloat16).float().numpy()
+    got = oracle_mod.round_bf16(allx)
+    np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32))
+    nan = oracle_mod.round_bf16(np.array([np.nan], np.float32))
+    assert np.isnan(nan).all()
+
+
+def test_pool_bf16_within_half_ulp_of_window_mean(oracle_mod):
+    """bf16 pooled keys are bfloat16 values within half a bf16 ulp (plus the
+    fp32 rounding of the mean) of the exact fp64 mean of the window's keys."""
+    b = inputs.make_batch([300, 77], num_q_heads=4, num_kv_heads=2, seed=6)
+    kb = inputs.bf16_bits(b.k_cache)
+    lens = b.seq_len.numpy()
+    nc_cap = oracle_mod.n_windows(300)
+    pb = oracle_mod.pool(kb, b.seq_start.numpy(), lens, nc_cap, bf16=True)
+    assert np.array_equal(pb.view(np.uint32) & 0xFFFF, np.zeros_like(pb.view(np.uint32)))
+    k = b.k_cache.double().numpy()
+    for i, L in enumerate(lens):
+        s0 = int(b.seq_start[i])
+        for j in range(oracle_mod.n_windows(int(L))):
+            exact = k[s0 + 16 * j:s0 + 16 * j + 32].mean(axis=0)       # [Hkv, D]
+            ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact), 1e-30))) - 7)
+            err = np.abs(pb[i, :, j] - exact)
+            assert (err <= 0.5 * ulp * (1 + 2 ** -20) + 2.0 ** -126).all(), (i, j)
