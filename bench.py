@@ -77,6 +77,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--settle-ms", type=float, default=300.0,
                     help="untimed repeated steps before timing, so clocks settle")
+    ap.add_argument("--pooled", choices=["fp32", "bf16"], default="fp32",
+                    help="pooled-key precision (bf16: the half-size variant)")
     ap.add_argument("--sweep", action="store_true",
                     help="NOSA-1B shape over context x batch x top-k (one JSON line per point)")
     return ap.parse_args()
@@ -104,7 +106,8 @@ class Workload:
         self.layers = layers
         self.key_dist = kdist
         self.local_blocks = 16
-        self.desc = desc
+        self.pooled_bf16 = getattr(args, "pooled", "fp32") == "bf16"
+        self.desc = desc + (", bf16 pooled keys" if self.pooled_bf16 else "")
         if args.context or args.batch or args.topk:
             self.desc += f" [overridden: batch {self.batch}, context {max(self.lens)}, top-k {self.topk}]"
         self.max_len = max(self.lens)
@@ -121,9 +124,10 @@ class Workload:
             windows = min(nc, 4 * ncand)
             attended = k_eff * 64 + (L - 64 * ncand)
             new_window = _n_windows(L) - _n_windows(L - 1)
+            pk = 256 if self.pooled_bf16 else 512                     # bytes per pooled key
             for _ in range(self.hkv):
-                pool += 2 * 256 * 2 + new_window * (31 * 256 + 512)   # new K/V row in + out, window
-                select += windows * 512 + G * 256 + self.topk * 4 + 4
+                pool += 2 * 256 * 2 + new_window * (31 * 256 + pk)     # new K/V row in + out, window
+                select += windows * pk + G * 256 + self.topk * 4 + 4
                 decode += attended * 512 + 2 * G * 256 + self.topk * 4 + 4
         return {"pool_append": pool * self.layers, "block_select": select * self.layers,
                 "sparse_decode": decode * self.layers}
@@ -135,7 +139,7 @@ class Replica:
     def __init__(self, nosa, wl: Workload, seed: int, device):
         self.b = inputs.make_batch(wl.lens, num_q_heads=wl.hq, num_kv_heads=wl.hkv, seed=seed,
                                    key_dist=wl.key_dist, device=device)
-        self.p = nosa.params(wl.hq, wl.hkv, topk=wl.topk, local_blocks=wl.local_blocks)
+        self.p = nosa.params(wl.hq, wl.hkv, topk=wl.topk, local_blocks=wl.local_blocks, pooled_bf16=wl.pooled_bf16)
         self.st = nosa.DecodeState(self.p, wl.batch, wl.max_len, device=device)
         self.st.rebuild_pooled(self.b.k_cache, self.b.seq_start, self.b.seq_len)
         self.k_new, self.v_new = inputs.random_kv_rows(wl.batch, wl.hkv, 128, seed=seed + 7,
@@ -275,10 +279,10 @@ def oracle_steps(wl: Workload, b_host, n_steps: int, threads: int, budget_s: flo
     lens = b_host.seq_len.numpy()
     starts = b_host.seq_start.numpy()
     nc_cap = max(1, oracle.n_windows(int(lens.max())))
-    pooled = oracle.pool(kb, starts, lens - 1, nc_cap)          # state before the step (untimed)
+    pooled = oracle.pool(kb, starts, lens - 1, nc_cap, bf16=wl.pooled_bf16)   # state before the step (untimed)
     done, t0 = 0, time.perf_counter()
     while done < n_steps:
-        pooled = oracle.pool(kb, starts, lens, nc_cap, len_old=lens - 1, pooled=pooled)
+        pooled = oracle.pool(kb, starts, lens, nc_cap, len_old=lens - 1, pooled=pooled, bf16=wl.pooled_bf16)
         oracle.decode_step(qb, kb, vb, starts, lens, pooled, wl.topk, local_blocks=wl.local_blocks)
         done += 1
         if time.perf_counter() - t0 > budget_s:
@@ -537,7 +541,7 @@ def run_sweep(args):
     for L in SWEEP_CONTEXTS:
         for B in SWEEP_BATCHES:
             for K in SWEEP_TOPK:
-                a = argparse.Namespace(workload="nosa1b_b8_16k", context=L, batch=B, topk=K)
+                a = argparse.Namespace(workload="nosa1b_b8_16k", context=L, batch=B, topk=K, pooled=args.pooled)
                 wl = Workload(a, 0)
                 layer_bytes = B * L * wl.hkv * 128 * 2 * 2
                 R = max(2, min(16, math.ceil(1.0e9 / layer_bytes)))

@@ -35,7 +35,8 @@
  *                   < 2^31; sequence i occupies rows seq_start[i] ..
  *                   seq_start[i] + len - 1 (varlen packing as with
  *                   cu_seqlens: seq_start[i] = cu_seqlens[i]).
- *      pooled       fp32 [batch, num_kv_heads, nc_cap, head_dim]
+ *      pooled       fp32 (or bf16 when p->pooled_bf16) [batch, num_kv_heads, nc_cap,
+ *                   head_dim]
  *      sel_idx      int32 [batch, num_kv_heads, topk] (ascending, -1 padded)
  *      sel_cnt      int32 [batch, num_kv_heads]
  *      out          bf16 [batch, num_q_heads, head_dim]
@@ -107,10 +108,13 @@ typedef struct {
   int local_blocks;    /* forced local window in blocks (16 = 1024 tokens); 0..256 */
   int topk;            /* selected blocks per (sequence, KV head); 1..1024 */
   float softmax_scale; /* 0 => 1/sqrt(head_dim); used for scores and attention */
+  int pooled_bf16;     /* 0: pooled keys fp32 (default); 1: pooled keys bf16, each the
+                          round-to-nearest-even of the fp32 mean (half the selection bytes) */
 } nosa_params;
 
 /* Fills `p` with the NOSA-1B attention defaults: 16 q / 2 KV heads, head_dim
- * 128, kernel 32 / stride 16, block 64, 16 local blocks, topk 64, scale 0. */
+ * 128, kernel 32 / stride 16, block 64, 16 local blocks, topk 64, scale 0,
+ * fp32 pooled keys. */
 NOSA_API void nosa_default_params(nosa_params* p);
 
 /* Bytes of device workspace that nosa_block_select / nosa_sparse_decode /
@@ -132,7 +136,8 @@ NOSA_API int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * nc(len_old[i]) <= j < nc(len_new[i]):
  *     pooled[i][h][j][:] = (1/32) * sum_{t=16j}^{16j+31} K[seq_start[i]+t][h][:]
  * summed in fp32 in ascending t (so rebuilding and appending give identical
- * bits).  Windows outside that range are not touched.
+ * bits), then stored as fp32, or rounded to bf16 (nearest, ties to even) when
+ * p->pooled_bf16.  Windows outside that range are not touched.
  * Optional fused append: when k_new/v_new (bf16 [batch, Hkv, head_dim]) are
  * non-NULL, len_new[i] must equal len_old[i] + 1 and the row is first written
  * to k_cache/v_cache at seq_start[i] + len_old[i] (the new token's K is read
@@ -144,7 +149,7 @@ NOSA_API int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * errors are not reported). */
 NOSA_API int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache,
                      int64_t cache_rows, const int64_t* seq_start, const int32_t* len_old,
-                     const int32_t* len_new, int batch, float* pooled,
+                     const int32_t* len_new, int batch, void* pooled,
                      int nc_cap, int max_new_keys, const void* k_new,
                      const void* v_new, void* ws, size_t ws_bytes, void* stream);
 
@@ -163,7 +168,7 @@ NOSA_API int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache
  * receives S for every candidate block.  Other entries are not written.
  * seq_len[i] must not exceed max_seq_len (else NOSA_DEV_MAX_LEN, the pair is
  * skipped with sel_cnt = 0). */
-NOSA_API int nosa_block_select(const nosa_params* p, const void* q, const float* pooled,
+NOSA_API int nosa_block_select(const nosa_params* p, const void* q, const void* pooled,
                       int nc_cap, const int32_t* seq_len, int batch,
                       int max_seq_len, const float* block_scores_in,
                       int nb_cap_in, float* comp_scores_out,
@@ -203,7 +208,7 @@ NOSA_API int nosa_decode_step_device(const nosa_params* p, const void* q, const 
                                      const void* v_new, void* k_cache, void* v_cache,
                                      int64_t cache_rows, const int64_t* seq_start,
                                      const int32_t* seq_len, int batch, int max_seq_len,
-                                     float* pooled, int nc_cap, int32_t* sel_idx,
+                                     void* pooled, int nc_cap, int32_t* sel_idx,
                                      int32_t* sel_cnt, void* out, float* lse, void* ws,
                                      size_t ws_bytes, void* stream);
 
@@ -232,7 +237,7 @@ NOSA_API int nosa_decode_step_device_noalloc(const nosa_params* p, const void* q
                                              const void* k_new, const void* v_new,
                                              void* k_cache, void* v_cache, int64_t cache_rows,
                                              const int64_t* seq_start, const int32_t* seq_len,
-                                             int batch, int max_seq_len, float* pooled,
+                                             int batch, int max_seq_len, void* pooled,
                                              int nc_cap, int32_t* sel_idx, int32_t* sel_cnt,
                                              void* out, float* lse, void* stream);
 
@@ -252,7 +257,7 @@ NOSA_API int nosa_decode_step(const nosa_params* p, const void* q_host,
                      const void* k_new_host, const void* v_new_host,
                      void* out_host, void* k_cache, void* v_cache,
                      int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len,
-                     int batch, int max_seq_len, float* pooled, int nc_cap,
+                     int batch, int max_seq_len, void* pooled, int nc_cap,
                      int32_t* sel_idx, int32_t* sel_cnt, void* ws,
                      size_t ws_bytes, void* stream);
 

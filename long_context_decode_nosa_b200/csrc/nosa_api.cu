@@ -62,6 +62,7 @@ int check_params(const nosa_params* p) {
   if (p->topk < 1 || p->topk > 1024) return fail(NOSA_ERR_UNSUPPORTED, "topk %d outside 1..1024", p->topk);
   if (!(p->softmax_scale >= 0.0f) || std::isinf(p->softmax_scale))
     return fail(NOSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  if (p->pooled_bf16 != 0 && p->pooled_bf16 != 1) return fail(NOSA_ERR_INVALID_ARG, "pooled_bf16 must be 0 or 1");
   return NOSA_OK;
 }
 
@@ -144,20 +145,23 @@ int encode_kv_map(CUtensorMap* map, const void* base, int hkv, int64_t rows) {
   return NOSA_OK;
 }
 
-// 2-D map over the pooled keys [batch * hkv * nc_cap rows, 128 fp32]: boxes of
-// {32 columns, 65 rows} (one 32-dimension slice of one scoring chunk),
-// 128-byte swizzle, zero fill past the last row.
-int encode_pooled_map(CUtensorMap* map, const float* pooled, int batch, int hkv, int nc_cap) {
+// 2-D map over the pooled keys [batch * hkv * nc_cap rows, 128 fp32 or bf16]:
+// boxes of 128-byte rows ({32 fp32 or 64 bf16 columns, 61 rows}: one slice of
+// one scoring chunk), 128-byte swizzle, zero fill past the last row.
+int encode_pooled_map(CUtensorMap* map, const void* pooled, int batch, int hkv, int nc_cap, bool bf16) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(NOSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const cuuint64_t rows = static_cast<cuuint64_t>(batch) * hkv * nc_cap;
   // TMA row coordinates are signed 32-bit.
   if (rows >= (cuuint64_t{1} << 31)) return fail(NOSA_ERR_UNSUPPORTED, "batch * num_kv_heads * nc_cap must be below 2^31");
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(nosa::kHeadDim), rows};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(nosa::kHeadDim) * 4};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(nosa::kBoxCols), static_cast<cuuint32_t>(nosa::kBoxRows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(nosa::kHeadDim) * (bf16 ? 2 : 4)};
+  // 128-byte box rows: 32 fp32 or 64 bf16 columns.
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(bf16 ? 64 : nosa::kBoxCols),
+                             static_cast<cuuint32_t>(nosa::kBoxRows)};
   const cuuint32_t elem_strides[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pooled), dims, strides, box,
+  CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                   const_cast<void*>(pooled), dims, strides, box,
                    elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NOSA_ERR_INVALID_ARG, "pooled tensor map encode failed (code %d)", static_cast<int>(r));
@@ -170,7 +174,7 @@ T* at(void* ws, size_t off) {
 }
 
 int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t cache_rows, const int64_t* seq_start,
-                   const int32_t* len_old, const int32_t* len_new, int batch, float* pooled, int nc_cap,
+                   const int32_t* len_old, const int32_t* len_new, int batch, void* pooled, int nc_cap,
                    int max_new_keys, const void* k_new, const void* v_new, uint32_t* status,
                    cudaStream_t stream) {
   if (batch < 0 || nc_cap < 0 || max_new_keys < 0 || cache_rows < 0)
@@ -194,6 +198,7 @@ int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t c
   a.len_old = len_old;
   a.len_new = len_new;
   a.pooled = pooled;
+  a.pooled_bf16 = p->pooled_bf16;
   a.k_new = static_cast<const __nv_bfloat16*>(k_new);
   a.v_new = static_cast<const __nv_bfloat16*>(v_new);
   a.status = status;
@@ -224,6 +229,7 @@ nosa::StepArgs step_args(const nosa_params* p, const void* q, const int32_t* seq
   a.topk = p->topk;
   a.max_seq_len = max_seq_len;
   a.ncand_max = static_cast<int>(nosa::n_candidates(max_seq_len, p->local_blocks));
+  a.pooled_bf16 = p->pooled_bf16;
   a.nc_cap = 1;
   a.scale = scale_of(p);
   a.scale_log2 = a.scale * 1.4426950408889634f;
@@ -238,7 +244,7 @@ int check_common(const nosa_params* p, int batch, int max_seq_len) {
   return NOSA_OK;
 }
 
-int do_block_select(const nosa_params* p, const void* q, const float* pooled, int nc_cap,
+int do_block_select(const nosa_params* p, const void* q, const void* pooled, int nc_cap,
                     const int32_t* seq_len, int batch, int max_seq_len, const float* bs_in, int nb_in,
                     float* comp_out, float* bs_out, int nb_out, int32_t* sel_idx, int32_t* sel_cnt,
                     void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -277,7 +283,7 @@ int do_block_select(const nosa_params* p, const void* q, const float* pooled, in
   if (bs_out && nb_out < ncand_max)
     return fail(NOSA_ERR_INVALID_ARG, "nb_cap_out %d below the %d candidates of max_seq_len", nb_out, ncand_max);
   nosa::StepArgs s = step_args(p, q, seq_len, batch, max_seq_len, sel_idx, sel_cnt, ws, l);
-  s.pooled = const_cast<float*>(pooled);
+  s.pooled = const_cast<void*>(pooled);
   s.nc_cap = nc_cap;
   s.comp_out = comp_out;
   s.bs_out = bs_out;
@@ -285,7 +291,7 @@ int do_block_select(const nosa_params* p, const void* q, const float* pooled, in
   s.mode = nosa::kStepScore;
   CUtensorMap none, tm_p;
   memset(&none, 0, sizeof none);
-  if (int rc = encode_pooled_map(&tm_p, pooled, batch, p->num_kv_heads, nc_cap)) return rc;
+  if (int rc = encode_pooled_map(&tm_p, pooled, batch, p->num_kv_heads, nc_cap, p->pooled_bf16 != 0)) return rc;
   cudaError_t e = nosa::launch_step(s, none, none, tm_p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "block_select launch");
   return ok();
@@ -334,7 +340,7 @@ int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, c
 // separate launches run.
 int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new, const void* v_new, void* k_cache,
                           void* v_cache, int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len,
-                          int batch, int max_seq_len, float* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt,
+                          int batch, int max_seq_len, void* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt,
                           void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (int rc = check_common(p, batch, max_seq_len)) return rc;
   if (batch == 0) return ok();
@@ -371,7 +377,7 @@ int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new
   CUtensorMap tm_k, tm_v, tm_p;
   if (int rc = encode_kv_map(&tm_k, k_cache, p->num_kv_heads, cache_rows)) return rc;
   if (int rc = encode_kv_map(&tm_v, v_cache, p->num_kv_heads, cache_rows)) return rc;
-  if (int rc = encode_pooled_map(&tm_p, pooled, batch, p->num_kv_heads, nc_cap)) return rc;
+  if (int rc = encode_pooled_map(&tm_p, pooled, batch, p->num_kv_heads, nc_cap, p->pooled_bf16 != 0)) return rc;
   cudaError_t e = nosa::launch_step(s, tm_k, tm_v, tm_p, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
   return ok();
@@ -403,6 +409,7 @@ void nosa_default_params(nosa_params* p) {
   p->local_blocks = 16;
   p->topk = 64;
   p->softmax_scale = 0.0f;
+  p->pooled_bf16 = 0;
 }
 
 size_t nosa_workspace_size(const nosa_params* p, int batch, int max_seq_len) {
@@ -419,7 +426,7 @@ int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 }
 
 int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t cache_rows, const int64_t* seq_start,
-                     const int32_t* len_old, const int32_t* len_new, int batch, float* pooled, int nc_cap,
+                     const int32_t* len_old, const int32_t* len_new, int batch, void* pooled, int nc_cap,
                      int max_new_keys, const void* k_new, const void* v_new, void* ws, size_t ws_bytes,
                      void* stream) {
   if (int rc = check_params(p)) return rc;
@@ -432,7 +439,7 @@ int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t
                         max_new_keys, k_new, v_new, status, static_cast<cudaStream_t>(stream));
 }
 
-int nosa_block_select(const nosa_params* p, const void* q, const float* pooled, int nc_cap,
+int nosa_block_select(const nosa_params* p, const void* q, const void* pooled, int nc_cap,
                       const int32_t* seq_len, int batch, int max_seq_len, const float* block_scores_in,
                       int nb_cap_in, float* comp_scores_out, float* block_scores_out, int nb_cap_out,
                       int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes, void* stream) {
@@ -453,7 +460,7 @@ int nosa_sparse_decode(const nosa_params* p, const void* q, const void* k_cache,
 
 int nosa_decode_step_device(const nosa_params* p, const void* q, const void* k_new, const void* v_new,
                             void* k_cache, void* v_cache, int64_t cache_rows, const int64_t* seq_start,
-                            const int32_t* seq_len, int batch, int max_seq_len, float* pooled, int nc_cap,
+                            const int32_t* seq_len, int batch, int max_seq_len, void* pooled, int nc_cap,
                             int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* ws, size_t ws_bytes,
                             void* stream) {
   if (int rc = check_params(p)) return rc;
@@ -465,7 +472,7 @@ int nosa_decode_step_device(const nosa_params* p, const void* q, const void* k_n
 int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new_host,
                      const void* v_new_host, void* out_host, void* k_cache, void* v_cache,
                      int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
-                     float* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* ws,
+                     void* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* ws,
                      size_t ws_bytes, void* stream) {
   if (int rc = check_params(p)) return rc;
   if (int rc = check_common(p, batch, max_seq_len)) return rc;

@@ -19,11 +19,12 @@ struct PoolArgs {
   const int64_t* seq_start;
   const int32_t* len_old;  // nullable: len_new - 1
   const int32_t* len_new;
-  float* pooled;
+  void* pooled;                // fp32, or bf16 when pooled_bf16
   const __nv_bfloat16* k_new;  // nullable
   const __nv_bfloat16* v_new;
   uint32_t* status;            // nullable
   int batch, hkv, nc_cap, max_new_keys;
+  int pooled_bf16;
 };
 
 struct SelectArgs {  // selection from given block scores (select_only_kernel)
@@ -47,7 +48,8 @@ struct StepArgs {
   int64_t cache_rows;
   __nv_bfloat16* k_cache;        // [cache_rows, hkv, 128] (append writes; tiles come through tensor maps)
   __nv_bfloat16* v_cache;
-  float* pooled;                 // [batch, hkv, nc_cap, 128] (append writes; scoring reads through a tensor map)
+  void* pooled;                  // [batch, hkv, nc_cap, 128] fp32 or bf16 (append writes; scoring reads
+                                 // through a tensor map)
   const __nv_bfloat16* k_new;    // [batch, hkv, 128], nullable (append)
   const __nv_bfloat16* v_new;
   int32_t* sel_idx;              // [pairs, topk]: written when scoring, read otherwise
@@ -60,6 +62,7 @@ struct StepArgs {
   uint32_t* status;
   int batch, hq, hkv, local_blocks, topk, max_seq_len, nc_cap, nb_out, nb_spill;
   int ncand_max;  // candidates of a sequence of max_seq_len tokens
+  int pooled_bf16;
   int mode;
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)

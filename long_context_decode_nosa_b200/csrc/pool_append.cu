@@ -63,8 +63,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
     if (lane == 0) set_status(a.status, NOSA_DEV_NC_CAP);
     return;
   }
-  pool_window_warp(a.k_cache, a.hkv, base, h, j, append ? len_old : -1, knew_row,
-                   a.pooled + ((static_cast<int64_t>(i) * a.hkv + h) * a.nc_cap + j) * kHeadDim, lane);
+  const int64_t at = ((static_cast<int64_t>(i) * a.hkv + h) * a.nc_cap + j) * kHeadDim;
+  void* dst = a.pooled_bf16 ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.pooled) + at)
+                            : static_cast<void*>(static_cast<float*>(a.pooled) + at);
+  pool_window_warp(a.k_cache, a.hkv, base, h, j, append ? len_old : -1, knew_row, dst, a.pooled_bf16 != 0, lane);
 }
 
 }  // namespace

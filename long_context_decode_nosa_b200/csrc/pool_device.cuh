@@ -25,11 +25,12 @@ __device__ inline float4 bf16x4_to_float4(uint2 raw) {
 // instead of the cache -- the token being appended by the same launch.  The
 // fp32 sum runs in ascending token order, then x 1/32 (exact), so appending
 // and rebuilding give identical bits.  Rows [16j, 16j+32) must lie inside
-// the cache (the caller checks the sequence against cache_rows).
+// the cache (the caller checks the sequence against cache_rows).  The mean
+// is stored as fp32, or as bf16 (nearest, ties to even) when `bf16`.
 __device__ inline void pool_window_warp(const __nv_bfloat16* __restrict__ k_cache, int hkv,
                                         int64_t seq_base, int h, int64_t j, int64_t fresh_tok,
-                                        const uint2* __restrict__ fresh, float* __restrict__ dst,
-                                        int lane) {
+                                        const uint2* __restrict__ fresh, void* __restrict__ dst,
+                                        bool bf16, int lane) {
   const int64_t t0 = j * kPoolStride;
   const uint2* src = reinterpret_cast<const uint2*>(k_cache + ((seq_base + t0) * hkv + h) * kHeadDim) + lane;
   const int64_t row_stride = static_cast<int64_t>(hkv) * kHeadDim / 4;  // in uint2
@@ -53,7 +54,16 @@ __device__ inline void pool_window_warp(const __nv_bfloat16* __restrict__ k_cach
     acc.w += f.w;
   }
   constexpr float inv = 1.0f / kPoolKernel;
-  reinterpret_cast<float4*>(dst)[lane] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  const float4 m = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (bf16) {  // round to nearest, ties to even
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y), hi = __floats2bfloat162_rn(m.z, m.w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(dst)[lane] = packed;
+  } else {
+    reinterpret_cast<float4*>(dst)[lane] = m;
+  }
 }
 
 }  // namespace nosa

@@ -15,6 +15,7 @@
 
 #include <cuda.h>
 
+#include "decode_device.cuh"
 #include "nosa_common.cuh"
 
 namespace nosa {
@@ -630,6 +631,74 @@ __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* _
       if (head < G && row < kChunkWindows)
         ssm[head * kScoreStride + row] =
             ((acc_hi[0][nt][e] + acc_hi[1][nt][e]) + (acc_lo[0][nt][e] + acc_lo[1][nt][e])) * scale;
+    }
+  }
+}
+
+// bf16 pooled keys: a chunk's rows arrive as two 2-D TMA boxes of {64 bf16
+// columns, 61 rows} (128-byte swizzle), box c holding dimensions
+// [64c, 64c+64), in the first two 8 KB slots of the stage.
+constexpr uint32_t kScoreTxBytesBf16 = 2u * kBoxRows * 128u;  // bytes landed per chunk
+
+template <int G>
+struct ScoreQBf16 {
+  static constexpr int kNTiles = G > 8 ? 2 : 1;  // n-tiles of 8 heads
+  uint32_t b[kNTiles][8][2];
+};
+
+// The group's queries as bf16 B fragments of mma m16n8k16 (k = dimension,
+// n = head; heads >= G are zero).
+template <int G>
+__device__ inline void load_score_q_bf16(ScoreQBf16<G>& f, const __nv_bfloat16* __restrict__ q_group, int lane) {
+  const int grp = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < ScoreQBf16<G>::kNTiles; ++nt) {
+    const int head = nt * 8 + grp;
+    const uint32_t* row = reinterpret_cast<const uint32_t*>(q_group + head * kHeadDim);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      f.b[nt][ks][0] = head < G ? __ldg(row + ks * 8 + tig) : 0u;      // dims 16ks + 2tig, +1
+      f.b[nt][ks][1] = head < G ? __ldg(row + ks * 8 + tig + 4) : 0u;  // dims 16ks + 2tig + 8, +9
+    }
+  }
+}
+
+// Compressed scores of one chunk of bf16 pooled keys: S^T = K * Q^T on
+// mma.sync m16n8k16 (bf16 inputs, exact products, fp32 accumulation), the A
+// fragments read with ldmatrix from the swizzled boxes.  Warp w computes rows
+// [16w, 16w+16) and stores scale * s into ssm[head][row] for rows < 61, as
+// score_stage does.
+template <int G>
+__device__ inline void score_stage_bf16(const ScoreQBf16<G>& qf, uint32_t stage, float* __restrict__ ssm, float scale,
+                                        int warp, int lane) {
+  constexpr int NT = ScoreQBf16<G>::kNTiles;
+  const int grp = lane >> 2, tig = lane & 3;
+  const int r0 = warp * 16;
+  const int mat = lane >> 3;                             // ldmatrix: which 8x8 matrix this lane addresses
+  const int arow = r0 + (mat & 1) * 8 + (lane & 7);
+  float acc[2][NT][4];
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[c][nt][e] = 0.0f;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int k8 = 2 * ks + (mat >> 1);                  // 8-dimension chunk 0..15
+    uint32_t a[4];
+    ldsm_x4(swz(stage + (k8 >> 3) * kScoreSlotBytes, arow, k8 & 7), a[0], a[1], a[2], a[3]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc[ks & 1][nt], a, qf.b[nt][ks][0], qf.b[nt][ks][1]);
+  }
+  const int ra = r0 + grp, rb = ra + 8;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int head = nt * 8 + 2 * tig + (e & 1);
+      const int row = (e >> 1) ? rb : ra;
+      if (head < G && row < kChunkWindows) ssm[head * kScoreStride + row] = (acc[0][nt][e] + acc[1][nt][e]) * scale;
     }
   }
 }

@@ -36,7 +36,7 @@ extern "C" {
 
 int nosa_decode_step_device_noalloc(const nosa_params* p, const void* q, const void* k_new, const void* v_new,
                                     void* k_cache, void* v_cache, int64_t cache_rows, const int64_t* seq_start,
-                                    const int32_t* seq_len, int batch, int max_seq_len, float* pooled, int nc_cap,
+                                    const int32_t* seq_len, int batch, int max_seq_len, void* pooled, int nc_cap,
                                     int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* stream) {
   const size_t need = nosa_workspace_size(p, batch, max_seq_len);
   if (need == 0)  // invalid parameters: let the regular entry point report them

@@ -302,10 +302,16 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     for (int k = static_cast<int>(rank); k < nchunks && ok; k += static_cast<int>(C)) {
       issue([&](int s, uint8_t* st) {
         const int row0 = row_base + kChunkBlocks * kWindowsPerBlock * k - 1;
-        mbar_arrive_expect_tx(&sh.full_bar[s], kScoreTxBytes);
+        if (a.pooled_bf16) {
+          mbar_arrive_expect_tx(&sh.full_bar[s], kScoreTxBytesBf16);
+          tma_load_keys(st, &tm_p, 0, row0, &sh.full_bar[s], policy);
+          tma_load_keys(st + kScoreSlotBytes, &tm_p, 64, row0, &sh.full_bar[s], policy);
+        } else {
+          mbar_arrive_expect_tx(&sh.full_bar[s], kScoreTxBytes);
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tma_load_keys(st + c * kScoreSlotBytes, &tm_p, c * kBoxCols, row0, &sh.full_bar[s], policy);
+          for (int c = 0; c < 4; ++c)
+            tma_load_keys(st + c * kScoreSlotBytes, &tm_p, c * kBoxCols, row0, &sh.full_bar[s], policy);
+        }
       });
     }
 #ifdef NOSA_TRACE
@@ -374,8 +380,10 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           const uint2* knew = a.k_new ? reinterpret_cast<const uint2*>(
                                             a.k_new + (static_cast<int64_t>(i) * a.hkv + g) * kHeadDim)
                                       : nullptr;
-          pool_window_warp(a.k_cache, a.hkv, seq_base, g, j, knew ? L - 1 : -1, knew,
-                           a.pooled + (static_cast<int64_t>(pair) * a.nc_cap + j) * kHeadDim, lane);
+          const int64_t at = (static_cast<int64_t>(pair) * a.nc_cap + j) * kHeadDim;
+          void* dst = a.pooled_bf16 ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.pooled) + at)
+                                    : static_cast<void*>(static_cast<float*>(a.pooled) + at);
+          pool_window_warp(a.k_cache, a.hkv, seq_base, g, j, knew ? L - 1 : -1, knew, dst, a.pooled_bf16 != 0, lane);
         }
       }
     }
@@ -417,8 +425,13 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     bool ok = true;
     if (scoring) {
       if (static_cast<int>(rank) < nchunks) {
+        const bool bf16 = a.pooled_bf16 != 0;
         ScoreQ<G> qf;
-        load_score_q<G>(qf, q_group, lane);
+        ScoreQBf16<G> qfb;
+        if (bf16)
+          load_score_q_bf16<G>(qfb, q_group, lane);
+        else
+          load_score_q<G>(qf, q_group, lane);
         for (int k = static_cast<int>(rank); k < nchunks; k += static_cast<int>(C)) {
           const int s = static_cast<int>(r % S);
           const bool landed = consumer_all(mbar_wait(&sh.full_bar[s], (r / S) & 1u, a.status));
@@ -430,7 +443,10 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           const int cix = (k - static_cast<int>(rank)) / static_cast<int>(C);
           if (tid == 0 && cix < 0) NOSA_STAMP(14 + 4 * cix);
 #endif
-          score_stage<G>(qf, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
+          if (bf16)
+            score_stage_bf16<G>(qfb, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
+          else
+            score_stage<G>(qf, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
           ++r;

@@ -48,11 +48,16 @@ class nosa_params(ctypes.Structure):
                 ("head_dim", ctypes.c_int), ("pool_kernel", ctypes.c_int),
                 ("pool_stride", ctypes.c_int), ("block_size", ctypes.c_int),
                 ("local_blocks", ctypes.c_int), ("topk", ctypes.c_int),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("pooled_bf16", ctypes.c_int)]
 
     @property
     def group(self) -> int:
         return self.num_q_heads // self.num_kv_heads
+
+    @property
+    def pooled_dtype(self):
+        """torch dtype of the pooled keys: float32, or bfloat16 when pooled_bf16."""
+        return torch.bfloat16 if self.pooled_bf16 else torch.float32
 
 
 _lib = None
@@ -109,9 +114,10 @@ def _check(rc: int, func: str):
 
 def params(num_q_heads: int = 16, num_kv_heads: int = 2, *, topk: int = 64,
            local_blocks: int = 16, softmax_scale: float = 0.0, head_dim: int = 128,
-           pool_kernel: int = 32, pool_stride: int = 16, block_size: int = 64) -> nosa_params:
+           pool_kernel: int = 32, pool_stride: int = 16, block_size: int = 64,
+           pooled_bf16: bool = False) -> nosa_params:
     return nosa_params(num_q_heads, num_kv_heads, head_dim, pool_kernel, pool_stride, block_size,
-                       local_blocks, topk, softmax_scale)
+                       local_blocks, topk, softmax_scale, int(pooled_bf16))
 
 
 def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor", cuda=True):
@@ -172,7 +178,7 @@ def nosa_pool_append(p: nosa_params, k_cache: torch.Tensor, v_cache: Optional[to
     rc = lib().nosa_pool_append(
         ctypes.byref(p), _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
         k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"), _ptr(len_old, torch.int32, "len_old"),
-        _ptr(len_new, torch.int32, "len_new"), batch, _ptr(pooled, torch.float32, "pooled"),
+        _ptr(len_new, torch.int32, "len_new"), batch, _ptr(pooled, p.pooled_dtype, "pooled"),
         pooled.shape[2], max_new_keys, _ptr(k_new, torch.bfloat16, "k_new"),
         _ptr(v_new, torch.bfloat16, "v_new"), _ptr(ws, torch.uint8, "ws"),
         0 if ws is None else ws.numel(), _stream(stream))
@@ -188,7 +194,7 @@ def nosa_block_select(p: nosa_params, q: Optional[torch.Tensor], pooled: Optiona
     batch = seq_len.shape[0]
     nc_cap = pooled.shape[2] if pooled is not None else (comp_scores_out.shape[2] if comp_scores_out is not None else 0)
     rc = lib().nosa_block_select(
-        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(pooled, torch.float32, "pooled"), nc_cap,
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(pooled, p.pooled_dtype, "pooled"), nc_cap,
         _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len,
         _ptr(block_scores_in, torch.float32, "block_scores_in"),
         0 if block_scores_in is None else block_scores_in.shape[2],
@@ -231,7 +237,7 @@ def nosa_decode_step_device(p: nosa_params, q: torch.Tensor, k_cache: torch.Tens
         ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
         _ptr(v_new, torch.bfloat16, "v_new"), _ptr(k_cache, torch.bfloat16, "k_cache"),
         _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
-        _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len, _ptr(pooled, torch.float32, "pooled"),
+        _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len, _ptr(pooled, p.pooled_dtype, "pooled"),
         pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"),
         ws.numel(), _stream(stream))
@@ -253,7 +259,7 @@ def nosa_decode_step_device_noalloc(p: nosa_params, q: torch.Tensor, k_cache: to
         ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
         _ptr(v_new, torch.bfloat16, "v_new"), _ptr(k_cache, torch.bfloat16, "k_cache"),
         _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
-        _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len, _ptr(pooled, torch.float32, "pooled"),
+        _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len, _ptr(pooled, p.pooled_dtype, "pooled"),
         pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _stream(stream))
     _check(rc, "nosa_decode_step_device_noalloc")
@@ -274,7 +280,7 @@ def nosa_decode_step(p: nosa_params, q_host: torch.Tensor, k_new_host: torch.Ten
         _ptr(out_host, torch.bfloat16, "out_host", cuda=False),
         _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
         k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"), _ptr(seq_len, torch.int32, "seq_len"),
-        batch, max_seq_len, _ptr(pooled, torch.float32, "pooled"), pooled.shape[2],
+        batch, max_seq_len, _ptr(pooled, p.pooled_dtype, "pooled"), pooled.shape[2],
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(rc, "nosa_decode_step")
@@ -301,7 +307,7 @@ class DecodeState:
         self.batch = batch
         self.max_seq_len = max_seq_len
         self.nc_cap = max(1, n_windows(max_seq_len))
-        self.pooled = torch.zeros(batch, p.num_kv_heads, self.nc_cap, 128, dtype=torch.float32, device=device)
+        self.pooled = torch.zeros(batch, p.num_kv_heads, self.nc_cap, 128, dtype=p.pooled_dtype, device=device)
         self.sel_idx = torch.full((batch, p.num_kv_heads, p.topk), -1, dtype=torch.int32, device=device)
         self.sel_cnt = torch.zeros(batch, p.num_kv_heads, dtype=torch.int32, device=device)
         self.out = torch.empty(batch, p.num_q_heads, 128, dtype=torch.bfloat16, device=device)
