@@ -241,6 +241,35 @@ NOSA_API int nosa_decode_step_device_noalloc(const nosa_params* p, const void* q
                                              int nc_cap, int32_t* sel_idx, int32_t* sel_cnt,
                                              void* out, float* lse, void* stream);
 
+/* Paged KV cache (a deployment layout; the pages have no counterpart).
+ * The caches are a pool of 64-token pages, k_cache / v_cache bf16
+ * [num_pages * 64, Hkv, head_dim]; token t of sequence i lives in row
+ *     page_table[i * max_pages + t / 64] * 64 + t % 64,
+ * page_table int32 [batch, max_pages].  The page size equals the block size,
+ * so a selected block is exactly one page.  These three calls are
+ * nosa_pool_append, nosa_sparse_decode and nosa_decode_step_device with
+ * (num_pages, page_table, max_pages) in place of (cache_rows, seq_start);
+ * the results are bit-identical to the contiguous calls on the same tokens.
+ * A sequence longer than max_pages * 64 sets NOSA_DEV_CACHE_ROWS; a page
+ * index outside [0, num_pages) sets NOSA_DEV_BAD_INDEX (that tile, window or
+ * row is skipped; nothing traps).  num_pages must be below 2^31 / 64. */
+NOSA_API int nosa_pool_append_paged(const nosa_params* p, void* k_cache, void* v_cache, int64_t num_pages,
+                                    const int32_t* page_table, int max_pages, const int32_t* len_old,
+                                    const int32_t* len_new, int batch, void* pooled, int nc_cap,
+                                    int max_new_keys, const void* k_new, const void* v_new, void* ws,
+                                    size_t ws_bytes, void* stream);
+NOSA_API int nosa_sparse_decode_paged(const nosa_params* p, const void* q, const void* k_cache,
+                                      const void* v_cache, int64_t num_pages, const int32_t* page_table,
+                                      int max_pages, const int32_t* seq_len, int batch, int max_seq_len,
+                                      const int32_t* sel_idx, const int32_t* sel_cnt, void* out, float* lse,
+                                      void* ws, size_t ws_bytes, void* stream);
+NOSA_API int nosa_decode_step_device_paged(const nosa_params* p, const void* q, const void* k_new,
+                                           const void* v_new, void* k_cache, void* v_cache, int64_t num_pages,
+                                           const int32_t* page_table, int max_pages, const int32_t* seq_len,
+                                           int batch, int max_seq_len, void* pooled, int nc_cap,
+                                           int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* ws,
+                                           size_t ws_bytes, void* stream);
+
 /* One whole decode step from HOST buffers (the pages' per-token decode,
  * steps 1-4 above in order): copies q_host (bf16 [batch, Hq, D]) and the new
  * token's k_new_host / v_new_host (bf16 [batch, Hkv, D]) to the device,

@@ -168,20 +168,41 @@ int encode_pooled_map(CUtensorMap* map, const void* pooled, int batch, int hkv, 
   return NOSA_OK;
 }
 
+// Where sequences live in the K/V caches: contiguous rows from seq_start[i],
+// or 64-token pages through page_table[i * max_pages + block].
+struct KvLayout {
+  const int64_t* seq_start;
+  const int32_t* page_table;
+  int max_pages;
+};
+
+int check_layout(const KvLayout& kv, int64_t cache_rows) {
+  if ((kv.seq_start == nullptr) == (kv.page_table == nullptr))
+    return fail(NOSA_ERR_INVALID_ARG, "exactly one of seq_start and page_table must be given");
+  if (kv.page_table) {
+    if (kv.max_pages < 1) return fail(NOSA_ERR_INVALID_ARG, "max_pages must be >= 1");
+    if (!aligned(kv.page_table, 4)) return fail(NOSA_ERR_INVALID_ARG, "page_table must be 4-byte aligned");
+    if (cache_rows % nosa::kPageTokens != 0)
+      return fail(NOSA_ERR_INVALID_ARG, "a paged cache holds whole 64-token pages");
+  }
+  return NOSA_OK;
+}
+
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t cache_rows, const int64_t* seq_start,
+int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t cache_rows, const KvLayout& kvl,
                    const int32_t* len_old, const int32_t* len_new, int batch, void* pooled, int nc_cap,
                    int max_new_keys, const void* k_new, const void* v_new, uint32_t* status,
                    cudaStream_t stream) {
   if (batch < 0 || nc_cap < 0 || max_new_keys < 0 || cache_rows < 0)
     return fail(NOSA_ERR_INVALID_ARG, "batch, nc_cap, max_new_keys and cache_rows must be >= 0");
   if (batch == 0) return ok();
-  if (!k_cache || !seq_start || !len_new || !pooled)
-    return fail(NOSA_ERR_INVALID_ARG, "k_cache, seq_start, len_new and pooled must not be NULL");
+  if (!k_cache || !len_new || !pooled)
+    return fail(NOSA_ERR_INVALID_ARG, "k_cache, len_new and pooled must not be NULL");
+  if (int rc = check_layout(kvl, cache_rows)) return rc;
   if ((k_new == nullptr) != (v_new == nullptr))
     return fail(NOSA_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
   if (k_new && !v_cache) return fail(NOSA_ERR_INVALID_ARG, "v_cache must not be NULL when appending");
@@ -194,7 +215,9 @@ int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t c
   a.k_cache = static_cast<__nv_bfloat16*>(k_cache);
   a.v_cache = static_cast<__nv_bfloat16*>(v_cache);
   a.cache_rows = cache_rows;
-  a.seq_start = seq_start;
+  a.seq_start = kvl.seq_start;
+  a.page_table = kvl.page_table;
+  a.max_pages = kvl.max_pages;
   a.len_old = len_old;
   a.len_new = len_new;
   a.pooled = pooled;
@@ -298,29 +321,31 @@ int do_block_select(const nosa_params* p, const void* q, const void* pooled, int
 }
 
 int check_decode_ptrs(const void* q, const void* k_cache, const void* v_cache, int64_t cache_rows,
-                      const int64_t* seq_start, const int32_t* seq_len, const int32_t* sel_idx,
+                      const KvLayout& kvl, const int32_t* seq_len, const int32_t* sel_idx,
                       const int32_t* sel_cnt, const void* out) {
-  if (!q || !k_cache || !v_cache || !seq_start || !seq_len || !sel_idx || !sel_cnt || !out)
-    return fail(NOSA_ERR_INVALID_ARG, "q, caches, seq_start, seq_len, sel_idx, sel_cnt and out must not be NULL");
+  if (!q || !k_cache || !v_cache || !seq_len || !sel_idx || !sel_cnt || !out)
+    return fail(NOSA_ERR_INVALID_ARG, "q, caches, seq_len, sel_idx, sel_cnt and out must not be NULL");
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 8))
     return fail(NOSA_ERR_INVALID_ARG, "caches must be 16-byte and q 8-byte aligned");
   if (cache_rows < 1 || cache_rows >= (int64_t{1} << 31))
     return fail(NOSA_ERR_UNSUPPORTED, "cache_rows must be in [1, 2^31)");
-  return NOSA_OK;
+  return check_layout(kvl, cache_rows);
 }
 
 int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
-                     int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
+                     int64_t cache_rows, const KvLayout& kvl, const int32_t* seq_len, int batch, int max_seq_len,
                      const int32_t* sel_idx, const int32_t* sel_cnt, void* out, float* lse, void* ws,
                      size_t ws_bytes, cudaStream_t stream) {
   if (int rc = check_common(p, batch, max_seq_len)) return rc;
   if (batch == 0) return ok();
   const Layout l = layout_of(p, batch, max_seq_len);
   if (int rc = check_ws(ws, ws_bytes, l)) return rc;
-  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, seq_start, seq_len, sel_idx, sel_cnt, out)) return rc;
+  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, kvl, seq_len, sel_idx, sel_cnt, out)) return rc;
   nosa::StepArgs s = step_args(p, q, seq_len, batch, max_seq_len, const_cast<int32_t*>(sel_idx),
                                const_cast<int32_t*>(sel_cnt), ws, l);
-  s.seq_start = seq_start;
+  s.seq_start = kvl.seq_start;
+  s.page_table = kvl.page_table;
+  s.max_pages = kvl.max_pages;
   s.cache_rows = cache_rows;
   s.out = static_cast<__nv_bfloat16*>(out);
   s.lse = lse;
@@ -339,14 +364,14 @@ int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, c
 // completes is never read by the same step's selection); otherwise the three
 // separate launches run.
 int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new, const void* v_new, void* k_cache,
-                          void* v_cache, int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len,
+                          void* v_cache, int64_t cache_rows, const KvLayout& kvl, const int32_t* seq_len,
                           int batch, int max_seq_len, void* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt,
                           void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (int rc = check_common(p, batch, max_seq_len)) return rc;
   if (batch == 0) return ok();
   const Layout l = layout_of(p, batch, max_seq_len);
   if (int rc = check_ws(ws, ws_bytes, l)) return rc;
-  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, seq_start, seq_len, sel_idx, sel_cnt, out)) return rc;
+  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, kvl, seq_len, sel_idx, sel_cnt, out)) return rc;
   if (!pooled || nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "pooled must not be NULL and nc_cap >= 1");
   if (!aligned(pooled, 16)) return fail(NOSA_ERR_INVALID_ARG, "pooled must be 16-byte aligned");
   if ((k_new == nullptr) != (v_new == nullptr))
@@ -354,16 +379,18 @@ int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new
   if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16)))
     return fail(NOSA_ERR_INVALID_ARG, "new-row pointers must be 16-byte aligned");
   if (p->local_blocks < 2) {
-    int rc = do_pool_append(p, k_cache, v_cache, cache_rows, seq_start, nullptr, seq_len, batch, pooled, nc_cap, 1,
+    int rc = do_pool_append(p, k_cache, v_cache, cache_rows, kvl, nullptr, seq_len, batch, pooled, nc_cap, 1,
                             k_new, v_new, at<uint32_t>(ws, l.status), stream);
     if (!rc) rc = do_block_select(p, q, pooled, nc_cap, seq_len, batch, max_seq_len, nullptr, 0, nullptr, nullptr, 0,
                                   sel_idx, sel_cnt, ws, ws_bytes, stream);
-    if (!rc) rc = do_sparse_decode(p, q, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len,
+    if (!rc) rc = do_sparse_decode(p, q, k_cache, v_cache, cache_rows, kvl, seq_len, batch, max_seq_len,
                                    sel_idx, sel_cnt, out, lse, ws, ws_bytes, stream);
     return rc;
   }
   nosa::StepArgs s = step_args(p, q, seq_len, batch, max_seq_len, sel_idx, sel_cnt, ws, l);
-  s.seq_start = seq_start;
+  s.seq_start = kvl.seq_start;
+  s.page_table = kvl.page_table;
+  s.max_pages = kvl.max_pages;
   s.cache_rows = cache_rows;
   s.k_cache = static_cast<__nv_bfloat16*>(k_cache);
   s.v_cache = static_cast<__nv_bfloat16*>(v_cache);
@@ -435,8 +462,26 @@ int nosa_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t
     if (ws_bytes < 256 || !aligned(ws, 256)) return fail(NOSA_ERR_WORKSPACE, "workspace must be 256-byte aligned and >= 256 bytes");
     status = at<uint32_t>(ws, 0);
   }
-  return do_pool_append(p, k_cache, v_cache, cache_rows, seq_start, len_old, len_new, batch, pooled, nc_cap,
-                        max_new_keys, k_new, v_new, status, static_cast<cudaStream_t>(stream));
+  return do_pool_append(p, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, len_old, len_new, batch,
+                        pooled, nc_cap, max_new_keys, k_new, v_new, status, static_cast<cudaStream_t>(stream));
+}
+
+int nosa_pool_append_paged(const nosa_params* p, void* k_cache, void* v_cache, int64_t num_pages,
+                           const int32_t* page_table, int max_pages, const int32_t* len_old,
+                           const int32_t* len_new, int batch, void* pooled, int nc_cap, int max_new_keys,
+                           const void* k_new, const void* v_new, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_params(p)) return rc;
+  if (!page_table) return fail(NOSA_ERR_INVALID_ARG, "page_table must not be NULL");
+  if (num_pages < 1 || num_pages >= (int64_t{1} << 31) / nosa::kPageTokens)
+    return fail(NOSA_ERR_UNSUPPORTED, "num_pages must be in [1, 2^31 / 64)");
+  uint32_t* status = nullptr;
+  if (ws) {
+    if (ws_bytes < 256 || !aligned(ws, 256)) return fail(NOSA_ERR_WORKSPACE, "workspace must be 256-byte aligned and >= 256 bytes");
+    status = at<uint32_t>(ws, 0);
+  }
+  return do_pool_append(p, k_cache, v_cache, num_pages * nosa::kPageTokens, KvLayout{nullptr, page_table, max_pages},
+                        len_old, len_new, batch, pooled, nc_cap, max_new_keys, k_new, v_new, status,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int nosa_block_select(const nosa_params* p, const void* q, const void* pooled, int nc_cap,
@@ -454,8 +499,21 @@ int nosa_sparse_decode(const nosa_params* p, const void* q, const void* k_cache,
                        const int32_t* sel_idx, const int32_t* sel_cnt, void* out, float* lse, void* ws,
                        size_t ws_bytes, void* stream) {
   if (int rc = check_params(p)) return rc;
-  return do_sparse_decode(p, q, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len, sel_idx,
-                          sel_cnt, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+  return do_sparse_decode(p, q, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, seq_len, batch,
+                          max_seq_len, sel_idx, sel_cnt, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int nosa_sparse_decode_paged(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                             int64_t num_pages, const int32_t* page_table, int max_pages, const int32_t* seq_len,
+                             int batch, int max_seq_len, const int32_t* sel_idx, const int32_t* sel_cnt, void* out,
+                             float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_params(p)) return rc;
+  if (!page_table) return fail(NOSA_ERR_INVALID_ARG, "page_table must not be NULL");
+  if (num_pages < 1 || num_pages >= (int64_t{1} << 31) / nosa::kPageTokens)
+    return fail(NOSA_ERR_UNSUPPORTED, "num_pages must be in [1, 2^31 / 64)");
+  return do_sparse_decode(p, q, k_cache, v_cache, num_pages * nosa::kPageTokens,
+                          KvLayout{nullptr, page_table, max_pages}, seq_len, batch, max_seq_len, sel_idx, sel_cnt, out,
+                          lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int nosa_decode_step_device(const nosa_params* p, const void* q, const void* k_new, const void* v_new,
@@ -464,9 +522,23 @@ int nosa_decode_step_device(const nosa_params* p, const void* q, const void* k_n
                             int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* ws, size_t ws_bytes,
                             void* stream) {
   if (int rc = check_params(p)) return rc;
-  return do_decode_step_device(p, q, k_new, v_new, k_cache, v_cache, cache_rows, seq_start, seq_len, batch,
-                               max_seq_len, pooled, nc_cap, sel_idx, sel_cnt, out, lse, ws, ws_bytes,
+  return do_decode_step_device(p, q, k_new, v_new, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0},
+                               seq_len, batch, max_seq_len, pooled, nc_cap, sel_idx, sel_cnt, out, lse, ws, ws_bytes,
                                static_cast<cudaStream_t>(stream));
+}
+
+int nosa_decode_step_device_paged(const nosa_params* p, const void* q, const void* k_new, const void* v_new,
+                                  void* k_cache, void* v_cache, int64_t num_pages, const int32_t* page_table,
+                                  int max_pages, const int32_t* seq_len, int batch, int max_seq_len, void* pooled,
+                                  int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  if (int rc = check_params(p)) return rc;
+  if (!page_table) return fail(NOSA_ERR_INVALID_ARG, "page_table must not be NULL");
+  if (num_pages < 1 || num_pages >= (int64_t{1} << 31) / nosa::kPageTokens)
+    return fail(NOSA_ERR_UNSUPPORTED, "num_pages must be in [1, 2^31 / 64)");
+  return do_decode_step_device(p, q, k_new, v_new, k_cache, v_cache, num_pages * nosa::kPageTokens,
+                               KvLayout{nullptr, page_table, max_pages}, seq_len, batch, max_seq_len, pooled, nc_cap,
+                               sel_idx, sel_cnt, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new_host,
@@ -492,7 +564,8 @@ int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new
   if ((e = cudaMemcpyAsync(dq, q_host, qbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy q");
   if ((e = cudaMemcpyAsync(dk, k_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy k_new");
   if ((e = cudaMemcpyAsync(dv, v_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy v_new");
-  int rc = do_decode_step_device(p, dq, dk, dv, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len,
+  int rc = do_decode_step_device(p, dq, dk, dv, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, seq_len,
+                                 batch, max_seq_len,
                                  pooled, nc_cap, sel_idx, sel_cnt, dout, nullptr, ws, ws_bytes, s);
   if (rc) return rc;
   if ((e = cudaMemcpyAsync(out_host, dout, qbytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess) return cuda_fail(e, "copy out");

@@ -136,6 +136,29 @@ __device__ inline void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
 __device__ inline void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ inline void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// ---------------------------------------------------------------- KV rows
+// Where the tokens of one sequence live in the K/V caches: contiguous rows
+// from `base` (seq_start[i]), or 64-token pages through the sequence's row
+// of a page table (token t in row pages[t / 64] * 64 + t % 64).  The page
+// size equals the block size, so an attention tile is exactly one page.
+constexpr int kPageTokens = kBlock;
+
+struct KvRows {
+  int64_t base;          // contiguous: the sequence's first row
+  const int32_t* pages;  // paged: the sequence's page-table row (nullptr: contiguous)
+  int64_t num_pages;     // paged: valid page indices are [0, num_pages)
+  __device__ int64_t row(int64_t t) const {
+    return pages ? static_cast<int64_t>(pages[t / kPageTokens]) * kPageTokens + t % kPageTokens : base + t;
+  }
+  // Whether token t's page index is valid (always, for contiguous caches,
+  // whose range the caller checks once).
+  __device__ bool page_ok(int64_t t) const {
+    if (!pages) return true;
+    const int32_t pg = pages[t / kPageTokens];
+    return pg >= 0 && pg < num_pages;
+  }
+};
+
 // ---------------------------------------------------------------- clusters
 // Thread-block cluster primitives (distributed shared memory).  Addresses
 // of another CTA's shared memory are 32-bit shared::cluster addresses from

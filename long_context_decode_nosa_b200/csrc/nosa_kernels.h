@@ -16,7 +16,9 @@ struct PoolArgs {
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
   int64_t cache_rows;
-  const int64_t* seq_start;
+  const int64_t* seq_start;    // contiguous caches (nullptr when paged)
+  const int32_t* page_table;   // paged caches: [batch, max_pages] 64-token page indices (nullptr: contiguous)
+  int max_pages;
   const int32_t* len_old;  // nullable: len_new - 1
   const int32_t* len_new;
   void* pooled;                // fp32, or bf16 when pooled_bf16
@@ -44,7 +46,9 @@ constexpr int kStepAppend = 4;  // write the new token's K/V rows and pool the w
 struct StepArgs {
   const __nv_bfloat16* q;        // [batch, hq, 128]
   const int32_t* seq_len;        // [batch]
-  const int64_t* seq_start;      // [batch] (decode / append)
+  const int64_t* seq_start;      // [batch] (decode / append, contiguous caches; nullptr when paged)
+  const int32_t* page_table;     // [batch, max_pages] (paged caches; nullptr: contiguous)
+  int max_pages;
   int64_t cache_rows;
   __nv_bfloat16* k_cache;        // [cache_rows, hkv, 128] (append writes; tiles come through tensor maps)
   __nv_bfloat16* v_cache;

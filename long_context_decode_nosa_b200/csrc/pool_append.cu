@@ -10,7 +10,7 @@
 // 1/32 (exact).  A fixed order makes an incremental append bit-identical to a
 // rebuild.  With k_new/v_new given, warp 0 of chunk 0 also stores the new
 // token's K/V rows into the caches; pooling reads that token from k_new, so
-// no cross-warp ordering is needed.
+// no cross-warp ordering is needed.  Contiguous or paged caches (KvRows).
 #include "nosa_common.cuh"
 #include "nosa_kernels.h"
 #include "pool_device.cuh"
@@ -30,12 +30,17 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
   allow_dependents();
   const int32_t len_new = a.len_new[i];
   const int32_t len_old = a.len_old ? a.len_old[i] : len_new - 1;
-  const int64_t base = a.seq_start[i];
+  KvRows kv;
+  kv.pages = a.page_table ? a.page_table + static_cast<int64_t>(i) * a.max_pages : nullptr;
+  kv.base = kv.pages ? 0 : a.seq_start[i];
+  kv.num_pages = a.cache_rows / kPageTokens;
   if (len_old < 0 || len_new < len_old) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, NOSA_DEV_BAD_LENGTH);
     return;
   }
-  if (base < 0 || base + len_new > a.cache_rows) {
+  const bool fits = kv.pages ? static_cast<int64_t>(len_new) <= static_cast<int64_t>(a.max_pages) * kPageTokens
+                             : kv.base >= 0 && kv.base + len_new <= a.cache_rows;
+  if (!fits) {
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(a.status, NOSA_DEV_CACHE_ROWS);
     return;
   }
@@ -48,7 +53,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
       append ? reinterpret_cast<const uint2*>(a.k_new + (static_cast<int64_t>(i) * a.hkv + h) * kHeadDim)
              : nullptr;
   if (append && blockIdx.x == 0 && warp == 0) {
-    const int64_t row = (base + len_old) * a.hkv + h;
+    if (!kv.page_ok(len_old)) {
+      if (lane == 0) set_status(a.status, NOSA_DEV_BAD_INDEX);
+      return;
+    }
+    const int64_t row = kv.row(len_old) * a.hkv + h;
     const uint2* vnew_row =
         reinterpret_cast<const uint2*>(a.v_new + (static_cast<int64_t>(i) * a.hkv + h) * kHeadDim);
     reinterpret_cast<uint2*>(a.k_cache + row * kHeadDim)[lane] = knew_row[lane];
@@ -66,7 +75,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
   const int64_t at = ((static_cast<int64_t>(i) * a.hkv + h) * a.nc_cap + j) * kHeadDim;
   void* dst = a.pooled_bf16 ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.pooled) + at)
                             : static_cast<void*>(static_cast<float*>(a.pooled) + at);
-  pool_window_warp(a.k_cache, a.hkv, base, h, j, append ? len_old : -1, knew_row, dst, a.pooled_bf16 != 0, lane);
+  if (!kv.page_ok(j * kPoolStride) || !kv.page_ok(j * kPoolStride + kPoolKernel - 1)) {
+    if (lane == 0) set_status(a.status, NOSA_DEV_BAD_INDEX);
+    return;
+  }
+  pool_window_warp(a.k_cache, a.hkv, kv, h, j, append ? len_old : -1, knew_row, dst, a.pooled_bf16 != 0, lane);
 }
 
 }  // namespace

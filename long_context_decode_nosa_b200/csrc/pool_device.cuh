@@ -24,19 +24,26 @@ __device__ inline float4 bf16x4_to_float4(uint2 raw) {
 // trip); the row of token `fresh_tok` (when >= 0) is taken from `fresh`
 // instead of the cache -- the token being appended by the same launch.  The
 // fp32 sum runs in ascending token order, then x 1/32 (exact), so appending
-// and rebuilding give identical bits.  Rows [16j, 16j+32) must lie inside
-// the cache (the caller checks the sequence against cache_rows).  The mean
-// is stored as fp32, or as bf16 (nearest, ties to even) when `bf16`.
-__device__ inline void pool_window_warp(const __nv_bfloat16* __restrict__ k_cache, int hkv,
-                                        int64_t seq_base, int h, int64_t j, int64_t fresh_tok,
-                                        const uint2* __restrict__ fresh, void* __restrict__ dst,
-                                        bool bf16, int lane) {
+// and rebuilding give identical bits.  The window's tokens [16j, 16j+32) are
+// found through `kv` (in a paged cache they span at most two pages); the
+// caller checks that they lie inside the cache.  The mean is stored as fp32,
+// or as bf16 (nearest, ties to even) when `bf16`.
+__device__ inline void pool_window_warp(const __nv_bfloat16* __restrict__ k_cache, int hkv, const KvRows& kv,
+                                        int h, int64_t j, int64_t fresh_tok, const uint2* __restrict__ fresh,
+                                        void* __restrict__ dst, bool bf16, int lane) {
   const int64_t t0 = j * kPoolStride;
-  const uint2* src = reinterpret_cast<const uint2*>(k_cache + ((seq_base + t0) * hkv + h) * kHeadDim) + lane;
+  // Tokens [t0, t0+split) are consecutive rows from row_a, the rest from row_b.
+  const int split = kv.pages ? min(kPoolKernel, static_cast<int>(kPageTokens - t0 % kPageTokens)) : kPoolKernel;
+  const int64_t row_a = kv.row(t0);
+  const int64_t row_b = split < kPoolKernel ? kv.row(t0 + split) : 0;
+  const uint2* src = reinterpret_cast<const uint2*>(k_cache) + static_cast<int64_t>(h) * (kHeadDim / 4) + lane;
   const int64_t row_stride = static_cast<int64_t>(hkv) * kHeadDim / 4;  // in uint2
   uint2 raw[kPoolKernel];
 #pragma unroll
-  for (int t = 0; t < kPoolKernel; ++t) raw[t] = __ldcg(src + t * row_stride);
+  for (int t = 0; t < kPoolKernel; ++t) {
+    const int64_t row = t < split ? row_a + t : row_b + (t - split);
+    raw[t] = __ldcg(src + row * row_stride);
+  }
   const int64_t r = fresh_tok - t0;
   if (fresh != nullptr && r >= 0 && r < kPoolKernel) {
     const uint2 f = fresh[lane];

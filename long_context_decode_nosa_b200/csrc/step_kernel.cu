@@ -217,10 +217,17 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   const int i = pair / a.hkv, g = pair % a.hkv;
   const bool uses_cache = decoding || appending;
   const int L = a.seq_len[i];
-  const int64_t start_i = uses_cache ? a.seq_start[i] : 0;  // issued with the length load
+  const bool paged = a.page_table != nullptr;
+  const int64_t start_i = uses_cache && !paged ? a.seq_start[i] : 0;  // issued with the length load
   const bool bad_len = L < 1 || L > a.max_seq_len;
   const int64_t seq_base = bad_len ? 0 : start_i;
-  const bool bad_rows = uses_cache && !bad_len && (seq_base < 0 || seq_base + L > a.cache_rows);
+  KvRows kv;
+  kv.base = seq_base;
+  kv.pages = paged ? a.page_table + static_cast<int64_t>(i) * a.max_pages : nullptr;
+  kv.num_pages = a.cache_rows / kPageTokens;
+  const bool bad_rows = uses_cache && !bad_len &&
+                        (paged ? static_cast<int64_t>(L) > static_cast<int64_t>(a.max_pages) * kPageTokens
+                               : seq_base < 0 || seq_base + L > a.cache_rows);
   const int Lv = bad_len ? 0 : L;
   const int nb = static_cast<int>(n_blocks(Lv));
   const int ncand = static_cast<int>(n_candidates(Lv, a.local_blocks));
@@ -317,47 +324,83 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 #ifdef NOSA_TRACE
     if (lane == 0) NOSA_STAMP(1);
 #endif
-    bool have_sel = false, sel_ok = false;
-    for (int t = static_cast<int>(rank); t < ntiles && ok; t += static_cast<int>(C)) {
-      int blk = -1;
-      if (t < nloc) {
-        blk = ncand + t;
-      } else {
-        if (!have_sel) {
-          int got = 0;
-          if (lane == 0) got = mbar_wait(&sh.sel_bar, 0, a.status) ? 1 : 0;
-          sel_ok = __shfl_sync(0xffffffffu, got, 0) != 0;
-          have_sel = true;
-        }
-        if (lane == 0 && sel_ok) {
-          blk = sel_list[t - nloc];
-          if (blk < 0 || blk >= ncand) {
-            set_status(a.status, NOSA_DEV_BAD_INDEX);
-            blk = -1;
-          }
-        }
+    // The first row of a tile: in a paged cache its page's, read from the
+    // page table (an invalid page rejects the tile).  Resolved by the whole
+    // warp, 32 tiles at a time (one parallel round trip for the table).
+    auto tile_row = [&](int blk, int& out_blk) -> int {
+      out_blk = blk;
+      if (blk < 0) return 0;
+      if (!paged) return static_cast<int>(seq_base + static_cast<int64_t>(blk) * kBlock);
+      const int32_t pg = kv.pages[blk];
+      if (pg < 0 || pg >= kv.num_pages) {
+        set_status(a.status, NOSA_DEV_BAD_INDEX);
+        out_blk = -1;
+        return 0;
       }
-      if (appending && t == nloc - 1 && a.k_new != nullptr) {
-        // This tile holds token L-1: write the new K/V rows first and order
-        // them before the tile's TMA read (same CTA, async proxy).
-        const int64_t row = (seq_base + L - 1) * a.hkv + g;
-        const int64_t src = static_cast<int64_t>(i) * a.hkv + g;
-        reinterpret_cast<uint2*>(a.k_cache + row * kHeadDim)[lane] =
-            reinterpret_cast<const uint2*>(a.k_new + src * kHeadDim)[lane];
-        reinterpret_cast<uint2*>(a.v_cache + row * kHeadDim)[lane] =
-            reinterpret_cast<const uint2*>(a.v_new + src * kHeadDim)[lane];
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        __syncwarp();
-      }
+      return pg * kPageTokens;
+    };
+    auto issue_tile = [&](int blk, int row) {
       issue([&](int s, uint8_t* st) {
         sh.stage_blk[s] = blk;
-        const int row = static_cast<int>(seq_base + (blk < 0 ? 0 : static_cast<int64_t>(blk) * kBlock));
         mbar_arrive_expect_tx(&sh.full_bar[s], kTileTxBytes);
         tma_load_box(st, &tm_k, 0, g, row, &sh.full_bar[s], policy);
         tma_load_box(st + kHalfBytes, &tm_k, 64, g, row, &sh.full_bar[s], policy);
         tma_load_box(st + 2 * kHalfBytes, &tm_v, 0, g, row, &sh.full_bar[s], policy);
         tma_load_box(st + 3 * kHalfBytes, &tm_v, 64, g, row, &sh.full_bar[s], policy);
       });
+    };
+    const int Ci = static_cast<int>(C), ri = static_cast<int>(rank);
+    // Local tiles t = rank, rank + C, ... < nloc: known at once.
+    {
+      int my_blk = -1, my_row = 0, n = 0;
+      for (int t = ri; t < min(nloc, ntiles) && ok; t += Ci, ++n) {
+        if ((n & 31) == 0) {
+          const int tl = t + Ci * lane;
+          my_row = tile_row(tl < min(nloc, ntiles) ? ncand + tl : -1, my_blk);
+        }
+        const int blk = __shfl_sync(0xffffffffu, my_blk, n & 31);
+        const int row = __shfl_sync(0xffffffffu, my_row, n & 31);
+        if (appending && t == nloc - 1 && a.k_new != nullptr) {
+          // This tile holds token L-1: write the new K/V rows first and order
+          // them before the tile's TMA read (same CTA, async proxy).
+          if (kv.page_ok(L - 1)) {
+            const int64_t row_w = kv.row(L - 1) * a.hkv + g;
+            const int64_t src = static_cast<int64_t>(i) * a.hkv + g;
+            reinterpret_cast<uint2*>(a.k_cache + row_w * kHeadDim)[lane] =
+                reinterpret_cast<const uint2*>(a.k_new + src * kHeadDim)[lane];
+            reinterpret_cast<uint2*>(a.v_cache + row_w * kHeadDim)[lane] =
+                reinterpret_cast<const uint2*>(a.v_new + src * kHeadDim)[lane];
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+          }
+          __syncwarp();
+        }
+        issue_tile(blk, row);
+      }
+    }
+    // Selected tiles t = nloc + x, t = rank (mod C): after the selection.
+    {
+      const int t0 = nloc + ((ri - nloc % Ci) % Ci + Ci) % Ci;
+      if (t0 < ntiles && ok) {
+        int got = 0;
+        if (lane == 0) got = mbar_wait(&sh.sel_bar, 0, a.status) ? 1 : 0;
+        const bool sel_ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+        int my_blk = -1, my_row = 0, n = 0;
+        for (int t = t0; t < ntiles && ok; t += Ci, ++n) {
+          if ((n & 31) == 0) {
+            const int tl = t + Ci * lane;
+            int blk = -1;
+            if (tl < ntiles && sel_ok) {
+              blk = sel_list[tl - nloc];
+              if (blk < 0 || blk >= ncand) {
+                set_status(a.status, NOSA_DEV_BAD_INDEX);
+                blk = -1;
+              }
+            }
+            my_row = tile_row(blk, my_blk);
+          }
+          issue_tile(__shfl_sync(0xffffffffu, my_blk, n & 31), __shfl_sync(0xffffffffu, my_row, n & 31));
+        }
+      }
     }
     // Every copy issued has landed before the ring is reused for the merge.
     if (lane == 0) {
@@ -383,7 +426,10 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           const int64_t at = (static_cast<int64_t>(pair) * a.nc_cap + j) * kHeadDim;
           void* dst = a.pooled_bf16 ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.pooled) + at)
                                     : static_cast<void*>(static_cast<float*>(a.pooled) + at);
-          pool_window_warp(a.k_cache, a.hkv, seq_base, g, j, knew ? L - 1 : -1, knew, dst, a.pooled_bf16 != 0, lane);
+          if (kv.page_ok(j * kPoolStride) && kv.page_ok(j * kPoolStride + kPoolKernel - 1))
+            pool_window_warp(a.k_cache, a.hkv, kv, g, j, knew ? L - 1 : -1, knew, dst, a.pooled_bf16 != 0, lane);
+          else if (lane == 0)
+            set_status(a.status, NOSA_DEV_BAD_INDEX);
         }
       }
     }

@@ -75,6 +75,10 @@ _SIGNATURES = {
     "nosa_sparse_decode": (_I, [_P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "nosa_decode_step_device": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "nosa_decode_step_device_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P]),
+    "nosa_pool_append_paged": (_I, [_P, _P, _P, _I64, _P, _I, _P, _P, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
+    "nosa_sparse_decode_paged": (_I, [_P, _P, _P, _P, _I64, _P, _I, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "nosa_decode_step_device_paged": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _I, _P, _I, _I, _P, _I, _P, _P, _P,
+                                           _P, _P, _SZ, _P]),
     "nosa_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "nosa_read_device_status": (_I, [_P, _SZ, _P]),
     "nosa_last_device_bits": (ctypes.c_uint32, []),
@@ -242,6 +246,70 @@ def nosa_decode_step_device(p: nosa_params, q: torch.Tensor, k_cache: torch.Tens
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"),
         ws.numel(), _stream(stream))
     _check(rc, "nosa_decode_step_device")
+
+
+# ----------------------------------------------------------------------------- paged KV cache
+# Caches as pools of 64-token pages ([num_pages * 64, Hkv, 128]); page_table
+# int32 [batch, max_pages]: token t of sequence i in row
+# page_table[i, t // 64] * 64 + t % 64.
+
+def _pages(k_cache: torch.Tensor) -> int:
+    if k_cache.shape[0] % 64:
+        raise ValueError("a paged cache holds whole 64-token pages")
+    return k_cache.shape[0] // 64
+
+
+def nosa_pool_append_paged(p: nosa_params, k_cache: torch.Tensor, v_cache: Optional[torch.Tensor],
+                           page_table: torch.Tensor, len_new: torch.Tensor, pooled: torch.Tensor, *,
+                           len_old: Optional[torch.Tensor] = None, max_new_keys: int = 1,
+                           k_new: Optional[torch.Tensor] = None, v_new: Optional[torch.Tensor] = None,
+                           ws: Optional[torch.Tensor] = None, stream=None):
+    batch = len_new.shape[0]
+    rc = lib().nosa_pool_append_paged(
+        ctypes.byref(p), _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
+        _pages(k_cache), _ptr(page_table, torch.int32, "page_table"), page_table.shape[1],
+        _ptr(len_old, torch.int32, "len_old"), _ptr(len_new, torch.int32, "len_new"), batch,
+        _ptr(pooled, p.pooled_dtype, "pooled"), pooled.shape[2], max_new_keys,
+        _ptr(k_new, torch.bfloat16, "k_new"), _ptr(v_new, torch.bfloat16, "v_new"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel() if ws is not None else 0, _stream(stream))
+    _check(rc, "nosa_pool_append_paged")
+
+
+def nosa_sparse_decode_paged(p: nosa_params, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                             page_table: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int,
+                             sel_idx: torch.Tensor, sel_cnt: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, *,
+                             lse: Optional[torch.Tensor] = None, stream=None):
+    if sel_idx.shape[-1] != p.topk:
+        raise ValueError("sel_idx's last dimension must equal params.topk")
+    batch = seq_len.shape[0]
+    rc = lib().nosa_sparse_decode_paged(
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), _pages(k_cache), _ptr(page_table, torch.int32, "page_table"),
+        page_table.shape[1], _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len,
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
+        _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"),
+        ws.numel(), _stream(stream))
+    _check(rc, "nosa_sparse_decode_paged")
+
+
+def nosa_decode_step_device_paged(p: nosa_params, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                  page_table: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int,
+                                  pooled: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor,
+                                  out: torch.Tensor, ws: torch.Tensor, *, k_new: Optional[torch.Tensor] = None,
+                                  v_new: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                                  stream=None):
+    if sel_idx.shape[-1] != p.topk:
+        raise ValueError("sel_idx's last dimension must equal params.topk")
+    batch = seq_len.shape[0]
+    rc = lib().nosa_decode_step_device_paged(
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(k_cache, torch.bfloat16, "k_cache"),
+        _ptr(v_cache, torch.bfloat16, "v_cache"), _pages(k_cache), _ptr(page_table, torch.int32, "page_table"),
+        page_table.shape[1], _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len,
+        _ptr(pooled, p.pooled_dtype, "pooled"), pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"),
+        _ptr(sel_cnt, torch.int32, "sel_cnt"), _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(rc, "nosa_decode_step_device_paged")
 
 
 def nosa_decode_step_device_noalloc(p: nosa_params, q: torch.Tensor, k_cache: torch.Tensor,
