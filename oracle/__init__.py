@@ -42,8 +42,13 @@ def _load():
         lib.nosa_oracle_topk.argtypes = [P, i64, P, i32, i32, i32, i32, i32, P, P]
         lib.nosa_oracle_sparse_attention.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32,
                                                      P, P, i32, f64, P, P]
+        lib.nosa_oracle_quantize_int8.argtypes = [P, i64, i32, P, P]
+        lib.nosa_oracle_pool_int8.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, P, i64]
+        lib.nosa_oracle_sparse_attention_int8.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                                          i32, P, P, i32, f64, P, P]
         for name in ("nosa_oracle_pool", "nosa_oracle_comp_scores", "nosa_oracle_block_scores",
-                     "nosa_oracle_topk", "nosa_oracle_sparse_attention"):
+                     "nosa_oracle_topk", "nosa_oracle_sparse_attention", "nosa_oracle_quantize_int8",
+                     "nosa_oracle_pool_int8", "nosa_oracle_sparse_attention_int8"):
             getattr(lib, name).restype = i32
         _lib = lib
     return _lib
@@ -115,6 +120,40 @@ def pool(k_cache, seq_start, len_new, nc_cap, *, len_old=None, pooled=None,
     return round_bf16(out) if bf16 else out
 
 
+def quantize_int8(x):
+    """INT8 cache variant: rows of bf16 values (uint16 bits, [..., d]) to
+    (codes int8 [..., d], scales fp32 [...]), symmetric per row:
+    s = max|x| / 127, code = clamp(rint(x / s), -127, 127) in fp32, half to
+    even; s = 0 and zero codes for an all-zero row."""
+    x = _c(x, np.uint16)
+    d = x.shape[-1]
+    rows = x.size // d
+    codes = np.empty(x.shape, np.int8)
+    scales = np.empty(x.shape[:-1], np.float32)
+    rc = _load().nosa_oracle_quantize_int8(_ptr(x), rows, d, _ptr(codes), _ptr(scales))
+    _check(rc, "quantize_int8")
+    return codes, scales
+
+
+def pool_int8(k_codes, k_scales, seq_start, len_new, nc_cap, *, len_old=None, pooled=None,
+              kernel=32, stride=16, bf16=False):
+    """``pool`` over an INT8 key cache: codes int8 [T, Hkv, D], scales fp32
+    [T, Hkv]; each window's mean of the dequantized keys s_t * code_t."""
+    k_codes = _c(k_codes, np.int8)
+    k_scales = _c(k_scales, np.float32)
+    T, hkv, d = k_codes.shape
+    assert k_scales.shape == (T, hkv)
+    seq_start = _c(seq_start, np.int64)
+    len_new = _c(len_new, np.int32)
+    B = len_new.shape[0]
+    len_old = None if len_old is None else _c(len_old, np.int32)
+    out = np.zeros((B, hkv, nc_cap, d), np.float32) if pooled is None else _c(pooled, np.float32).copy()
+    rc = _load().nosa_oracle_pool_int8(_ptr(k_codes), _ptr(k_scales), _ptr(seq_start), _ptr(len_old),
+                                       _ptr(len_new), B, hkv, d, kernel, stride, _ptr(out), nc_cap)
+    _check(rc, "pool_int8")
+    return round_bf16(out) if bf16 else out
+
+
 def comp_scores(q, pooled, seq_len, *, num_kv_heads, scale=None, kernel=32, stride=16):
     """Compressed scores s[B, Hq, nc_cap] fp32 (-inf past nc(L_i))."""
     q = _c(q, np.uint16)
@@ -175,6 +214,29 @@ def sparse_attention(q, k_cache, v_cache, seq_start, seq_len, sel_idx, sel_cnt, 
         _ptr(_c(seq_len, np.int32)), B, hq, hkv, d, block_size, local_blocks,
         _ptr(sel_idx), _ptr(sel_cnt), tk, scale, _ptr(out), _ptr(lse))
     _check(rc, "sparse_attention")
+    return out, lse
+
+
+def sparse_attention_int8(q, k_codes, k_scales, v_codes, v_scales, seq_start, seq_len, sel_idx, sel_cnt, *,
+                          scale=None, block_size=64, local_blocks=16):
+    """``sparse_attention`` over INT8 caches (codes int8 [T, Hkv, D], scales
+    fp32 [T, Hkv]): keys and values are s_t * code_t."""
+    q = _c(q, np.uint16)
+    B, hq, d = q.shape
+    k_codes, v_codes = _c(k_codes, np.int8), _c(v_codes, np.int8)
+    k_scales, v_scales = _c(k_scales, np.float32), _c(v_scales, np.float32)
+    hkv = k_codes.shape[1]
+    sel_idx = _c(sel_idx, np.int32)
+    sel_cnt = _c(sel_cnt, np.int32)
+    tk = sel_idx.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = np.empty((B, hq, d), np.float64)
+    lse = np.empty((B, hq), np.float64)
+    rc = _load().nosa_oracle_sparse_attention_int8(
+        _ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
+        _ptr(_c(seq_start, np.int64)), _ptr(_c(seq_len, np.int32)), B, hq, hkv, d, block_size,
+        local_blocks, _ptr(sel_idx), _ptr(sel_cnt), tk, scale, _ptr(out), _ptr(lse))
+    _check(rc, "sparse_attention_int8")
     return out, lse
 
 

@@ -20,6 +20,8 @@
  *        stride 16, coarse scores, top-k, exact attention on the selected
  *        blocks), section 四 "NOSA-1B 模型配置速览" (table: 16 q / 2 KV heads,
  *        bfloat16, TopK64 / window 1024 / block 64 / kernel32 / stride16).
+ *   [P5] "NOSA 技术架构解析" (devpress.csdn.net), section "1.1 双阶段稀疏注意力设计"
+ *        ("关键技巧": 32-bit prefill, decode switchable to 16-bit or 8-bit integers).
  *
  * Conventions (all readings are listed in the design notes of the repo):
  *   * bf16 values are passed as their 16-bit patterns and widened exactly
@@ -40,6 +42,15 @@
  *     padded with -1.  -0.0 compares equal to +0.0; NaN ranks as -inf.
  *   * Attention: softmax over the token set (selected blocks) U [ncand*bs, L),
  *     clipped to [0, L), of scale * q.k, applied to v; fp64 throughout.
+ *   * INT8 cache variant (reading of [P5] "1.1 双阶段稀疏注意力设计",
+ *     "关键技巧": the decode stage may switch to 8-bit integers): each cache
+ *     row (token, KV head) of d bf16 values x is kept as d int8 codes and one
+ *     fp32 scale, symmetric per row:
+ *        amax = max_c |x_c|;  s = amax / 127;  code_c = clamp(rint(x_c / s), -127, 127)
+ *     with both divisions in fp32 (IEEE, round to nearest) and rint rounding
+ *     half to even; an all-zero row has s = 0 and zero codes.  The value the
+ *     method sees is s * code_c (exact in fp64); pooling and attention read
+ *     those values in place of the bf16 keys and values.
  *
  * Parity pins for every function live in the CPU test-suite (closed forms,
  * brute force on tiny inputs, dense-attention equivalence via a library
@@ -78,6 +89,49 @@ static double bf16_to_f64(uint16_t bits) {
   return (double)f;
 }
 
+/* A key or value cache as the oracle reads it: bf16 patterns [T, hkv, d], or
+ * INT8 codes [T, hkv, d] with one fp32 scale per (row, KV head), scales
+ * [T, hkv] (the INT8 cache variant). */
+typedef struct {
+  const uint16_t* bf16;
+  const int8_t* codes;
+  const float* scales;
+} kv_view;
+
+static double kv_at(const kv_view* v, int64_t row, int hkv, int h, int d, int c) {
+  int64_t at = (row * hkv + h) * d + c;
+  if (v->bf16) return bf16_to_f64(v->bf16[at]);
+  return (double)v->scales[row * hkv + h] * (double)v->codes[at];
+}
+
+static int kv_ok(const kv_view* v) { return v->bf16 || (v->codes && v->scales); }
+
+/* INT8 cache variant ([P5] 1.1 "关键技巧", reading in the header): quantizes
+ * `rows` rows of d bf16 values (x, [rows, d]) into codes [rows, d] and scales
+ * [rows]:  amax = max |x_c|, s = amax / 127, code_c = clamp(rint(x_c / s),
+ * -127, 127), divisions in fp32, half to even; s = 0 and zero codes for an
+ * all-zero row. */
+int nosa_oracle_quantize_int8(const uint16_t* x, int64_t rows, int d, int8_t* codes, float* scales) {
+  if (!x || !codes || !scales || rows < 0 || d < 1) return ORACLE_BAD_ARG;
+  for (int64_t r = 0; r < rows; ++r) {
+    float amax = 0.0f;
+    for (int c = 0; c < d; ++c) {
+      float v = (float)bf16_to_f64(x[r * d + c]);
+      if (fabsf(v) > amax) amax = fabsf(v);
+    }
+    float s = amax / 127.0f;
+    scales[r] = s;
+    for (int c = 0; c < d; ++c) {
+      float v = (float)bf16_to_f64(x[r * d + c]);
+      float code = s > 0.0f ? rintf(v / s) : 0.0f;
+      if (code > 127.0f) code = 127.0f;
+      if (code < -127.0f) code = -127.0f;
+      codes[r * d + c] = (int8_t)code;
+    }
+  }
+  return ORACLE_OK;
+}
+
 static int64_t n_windows(int64_t L, int kernel, int stride) {
   return L >= kernel ? (L - kernel) / stride + 1 : 0;
 }
@@ -94,11 +148,11 @@ static int64_t n_candidates(int64_t L, int bs, int local_blocks) {
  *   pooled[i][h][j][:] = (1/kernel) * sum_{t = j*stride}^{j*stride+kernel-1} K[seq_start[i]+t][h][:]
  * K is [T, hkv, d] bf16; pooled is [batch, hkv, nc_cap, d] fp32.
  * Windows outside [nc(len_old), nc(len_new)) are left untouched. */
-int nosa_oracle_pool(const uint16_t* k_cache, const int64_t* seq_start,
+static int pool_view(const kv_view* k, const int64_t* seq_start,
                      const int32_t* len_old, const int32_t* len_new, int batch,
                      int hkv, int d, int kernel, int stride, float* pooled,
                      int64_t nc_cap) {
-  if (!k_cache || !seq_start || !len_new || !pooled || batch < 0 || hkv < 1 ||
+  if (!kv_ok(k) || !seq_start || !len_new || !pooled || batch < 0 || hkv < 1 ||
       d < 1 || kernel < 1 || stride < 1)
     return ORACLE_BAD_ARG;
   int npairs = batch * hkv;
@@ -114,13 +168,30 @@ int nosa_oracle_pool(const uint16_t* k_cache, const int64_t* seq_start,
         double acc = 0.0;
         for (int t = 0; t < kernel; ++t) {
           int64_t row = seq_start[i] + j * stride + t;
-          acc += bf16_to_f64(k_cache[(row * hkv + h) * d + c]);
+          acc += kv_at(k, row, hkv, h, d, c);
         }
         dst[c] = (float)(acc / kernel);
       }
     }
   }
   return ORACLE_OK;
+}
+
+int nosa_oracle_pool(const uint16_t* k_cache, const int64_t* seq_start,
+                     const int32_t* len_old, const int32_t* len_new, int batch,
+                     int hkv, int d, int kernel, int stride, float* pooled,
+                     int64_t nc_cap) {
+  kv_view k = {k_cache, NULL, NULL};
+  return pool_view(&k, seq_start, len_old, len_new, batch, hkv, d, kernel, stride, pooled, nc_cap);
+}
+
+/* The same pooling over an INT8 cache: the mean of the dequantized keys
+ * s_t * code_t of the window (scales [T, hkv]). */
+int nosa_oracle_pool_int8(const int8_t* k_codes, const float* k_scales, const int64_t* seq_start,
+                          const int32_t* len_old, const int32_t* len_new, int batch, int hkv, int d,
+                          int kernel, int stride, float* pooled, int64_t nc_cap) {
+  kv_view k = {NULL, k_codes, k_scales};
+  return pool_view(&k, seq_start, len_old, len_new, batch, hkv, d, kernel, stride, pooled, nc_cap);
 }
 
 /* Compressed attention scores, [P3] 三.3 / [P2] 核心原理 (coarse screen):
@@ -260,14 +331,13 @@ int nosa_oracle_topk(const float* S, int64_t nb_cap, const int32_t* seq_len,
  * q is [batch, hq, d] bf16; K, V are [T_total, hkv, d] bf16 with sequence i
  * starting at row seq_start[i]; out is fp64 [batch, hq, d]; lse fp64 [batch, hq]
  * (nullable).  Indices outside [0, ncand) are rejected. */
-int nosa_oracle_sparse_attention(const uint16_t* q, const uint16_t* k_cache,
-                                 const uint16_t* v_cache,
-                                 const int64_t* seq_start, const int32_t* seq_len,
-                                 int batch, int hq, int hkv, int d, int bs,
-                                 int local_blocks, const int32_t* sel_idx,
-                                 const int32_t* sel_cnt, int topk, double scale,
-                                 double* out, double* lse) {
-  if (!q || !k_cache || !v_cache || !seq_start || !seq_len || !out ||
+static int attention_view(const uint16_t* q, const kv_view* kc, const kv_view* vc,
+                          const int64_t* seq_start, const int32_t* seq_len,
+                          int batch, int hq, int hkv, int d, int bs,
+                          int local_blocks, const int32_t* sel_idx,
+                          const int32_t* sel_cnt, int topk, double scale,
+                          double* out, double* lse) {
+  if (!q || !kv_ok(kc) || !kv_ok(vc) || !seq_start || !seq_len || !out ||
       hkv < 1 || hq % hkv != 0 || topk < 0 || (topk > 0 && (!sel_idx || !sel_cnt)))
     return ORACLE_BAD_ARG;
   int G = hq / hkv;
@@ -303,9 +373,8 @@ int nosa_oracle_sparse_attention(const uint16_t* q, const uint16_t* k_cache,
       double m = -INFINITY;
       for (int64_t tok = 0; tok < L; ++tok) {
         if (!in_set[tok]) continue;
-        const uint16_t* kv = k_cache + ((seq_start[i] + tok) * hkv + g) * d;
         double acc = 0.0;
-        for (int c = 0; c < d; ++c) acc += bf16_to_f64(qv[c]) * bf16_to_f64(kv[c]);
+        for (int c = 0; c < d; ++c) acc += bf16_to_f64(qv[c]) * kv_at(kc, seq_start[i] + tok, hkv, g, d, c);
         logit[tok] = scale * acc;
         if (logit[tok] > m) m = logit[tok];
       }
@@ -316,8 +385,7 @@ int nosa_oracle_sparse_attention(const uint16_t* q, const uint16_t* k_cache,
         if (!in_set[tok]) continue;
         double w = exp(logit[tok] - m);
         denom += w;
-        const uint16_t* vv = v_cache + ((seq_start[i] + tok) * hkv + g) * d;
-        for (int c = 0; c < d; ++c) o[c] += w * bf16_to_f64(vv[c]);
+        for (int c = 0; c < d; ++c) o[c] += w * kv_at(vc, seq_start[i] + tok, hkv, g, d, c);
       }
       for (int c = 0; c < d; ++c) o[c] = denom > 0.0 ? o[c] / denom : 0.0;
       if (lse) lse[(int64_t)i * hq + h] = denom > 0.0 ? m + log(denom) : -INFINITY;
@@ -326,4 +394,29 @@ int nosa_oracle_sparse_attention(const uint16_t* q, const uint16_t* k_cache,
     free(in_set);
   }
   return bad ? ORACLE_BAD_ARG : ORACLE_OK;
+}
+
+int nosa_oracle_sparse_attention(const uint16_t* q, const uint16_t* k_cache,
+                                 const uint16_t* v_cache,
+                                 const int64_t* seq_start, const int32_t* seq_len,
+                                 int batch, int hq, int hkv, int d, int bs,
+                                 int local_blocks, const int32_t* sel_idx,
+                                 const int32_t* sel_cnt, int topk, double scale,
+                                 double* out, double* lse) {
+  kv_view k = {k_cache, NULL, NULL}, v = {v_cache, NULL, NULL};
+  return attention_view(q, &k, &v, seq_start, seq_len, batch, hq, hkv, d, bs, local_blocks, sel_idx,
+                        sel_cnt, topk, scale, out, lse);
+}
+
+/* The same attention over INT8 caches: keys and values are s_t * code_t
+ * (scales [T, hkv]). */
+int nosa_oracle_sparse_attention_int8(const uint16_t* q, const int8_t* k_codes, const float* k_scales,
+                                      const int8_t* v_codes, const float* v_scales,
+                                      const int64_t* seq_start, const int32_t* seq_len, int batch,
+                                      int hq, int hkv, int d, int bs, int local_blocks,
+                                      const int32_t* sel_idx, const int32_t* sel_cnt, int topk,
+                                      double scale, double* out, double* lse) {
+  kv_view k = {NULL, k_codes, k_scales}, v = {NULL, v_codes, v_scales};
+  return attention_view(q, &k, &v, seq_start, seq_len, batch, hq, hkv, d, bs, local_blocks, sel_idx,
+                        sel_cnt, topk, scale, out, lse);
 }

@@ -361,3 +361,148 @@ def test_pool_bf16_within_half_ulp_of_window_mean(oracle_mod):
             ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact), 1e-30))) - 7)
             err = np.abs(pb[i, :, j] - exact)
             assert (err <= 0.5 * ulp * (1 + 2 ** -20) + 2.0 ** -126).all(), (i, j)
+
+
+# --------------------------------------------------------------------------- INT8 cache variant
+
+def _pow2_grid_rows(rng, rows, d):
+    """Rows k * 2^e (k integer in [-127, 127], one |k| = 127 per row): every
+    value has at most 7 significant bits, so it is an exact bfloat16."""
+    k = rng.integers(-127, 128, (rows, d))
+    k[np.arange(rows), rng.integers(0, d, rows)] = 127 * rng.choice([-1, 1], rows)
+    e = rng.integers(-30, 12, rows)
+    x = torch.from_numpy(k * np.exp2(e)[:, None]).to(torch.bfloat16)
+    assert torch.equal(x.double(), torch.from_numpy(k * np.exp2(e)[:, None]))
+    return x, k, e
+
+
+def test_quantize_int8_reproduces_a_power_of_two_grid(oracle_mod):
+    """A row k * 2^e with max |k| = 127 quantizes to scale 2^e and codes k
+    exactly (the scale divides out exactly, no rounding is involved)."""
+    rng = np.random.default_rng(21)
+    x, k, e = _pow2_grid_rows(rng, 300, 128)
+    codes, scales = oracle_mod.quantize_int8(_bits(x))
+    np.testing.assert_array_equal(scales, np.exp2(e).astype(np.float32))
+    np.testing.assert_array_equal(codes, k.astype(np.int8))
+
+
+def test_quantize_int8_rounds_half_to_even(oracle_mod):
+    """Values exactly halfway between two codes go to the even code: 2.5 -> 2,
+    3.5 -> 4, 126.5 -> 126, 125.5 -> 126 and the mirrored negatives (half away
+    from zero would give 3 and 127)."""
+    e = -3
+    halves = np.array([0.5, 1.5, 2.5, 3.5, 125.5, 126.5])
+    want = np.array([0, 2, 2, 4, 126, 126])
+    row = np.concatenate([[127.0], halves, -halves, np.zeros(128 - 13)]) * 2.0 ** e
+    x = torch.from_numpy(row[None]).to(torch.bfloat16)
+    assert torch.equal(x.double()[0], torch.from_numpy(row))
+    codes, scales = oracle_mod.quantize_int8(_bits(x))
+    assert scales[0] == np.float32(2.0 ** e)
+    np.testing.assert_array_equal(codes[0, 1:7], want)
+    np.testing.assert_array_equal(codes[0, 7:13], -want)
+
+
+def test_quantize_int8_properties_on_random_rows(oracle_mod):
+    """On Gaussian rows of many magnitudes, and an all-zero row: the largest
+    |code| is 127, codes keep the sign of their value and its order within a
+    row, every value lies within half a step (plus the fp32 rounding of x / s)
+    of s * code, and the zero row has scale 0 and zero codes."""
+    rng = np.random.default_rng(22)
+    x = rng.standard_normal((400, 128)) * np.exp(rng.uniform(-20, 20, (400, 1)))
+    x[7] = 0.0
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    codes, scales = oracle_mod.quantize_int8(_bits(xb))
+    xv = xb.double().numpy()
+    c = codes.astype(np.int64)
+    s = scales.astype(np.float64)
+    nz = np.abs(xv).max(1) > 0
+    assert (np.abs(c[nz]).max(1) == 127).all()
+    assert scales[7] == 0.0 and (codes[7] == 0).all()
+    assert ((np.sign(c) == np.sign(xv)) | (c == 0)).all()
+    assert (np.abs(xv - s[:, None] * c) <= s[:, None] * (0.5 + 2.0 ** -16)).all()
+    order = np.argsort(xv, axis=1, kind="stable")
+    assert (np.diff(np.take_along_axis(c, order, 1), axis=1) >= 0).all()
+    # the scale is the fp32 quotient of the row's largest magnitude by 127
+    amax = np.abs(xv).max(1)
+    assert (np.abs(s - amax / 127) <= np.spacing(np.float32(amax / 127)).astype(np.float64)).all()
+
+
+def _int8_cache(rng, T, hkv, d, pow2_scales):
+    codes = rng.integers(-127, 128, (T, hkv, d)).astype(np.int8)
+    if pow2_scales:
+        scales = np.exp2(rng.integers(-12, 4, (T, hkv))).astype(np.float32)
+    else:
+        scales = (rng.uniform(0.5, 2.0, (T, hkv)) * np.exp2(rng.integers(-10, 2, (T, hkv)))).astype(np.float32)
+    return codes, scales
+
+
+def _dequant_bf16(codes, scales):
+    """s * code as bfloat16 bits (exact when s is a power of two)."""
+    v = codes.astype(np.float64) * scales.astype(np.float64)[..., None]
+    t = torch.from_numpy(v).to(torch.bfloat16)
+    assert torch.equal(t.double(), torch.from_numpy(v))
+    return _bits(t)
+
+
+def test_pool_int8_equals_pool_of_dequantized_keys(oracle_mod):
+    """With power-of-two scales every s * code is an exact bfloat16, so pooling
+    the INT8 cache must give the bf16 pooling's bits; with general scales the
+    pooled key is the fp32 rounding of the window mean of s * code (numpy
+    sliding windows in fp64)."""
+    rng = np.random.default_rng(23)
+    lens = np.array([300, 77, 31], np.int32)
+    starts = np.array([0, 300, 377], np.int64)
+    nc_cap = oracle_mod.n_windows(300)
+    codes, scales = _int8_cache(rng, 408, 2, 128, True)
+    got = oracle_mod.pool_int8(codes, scales, starts, lens, nc_cap)
+    want = oracle_mod.pool(_dequant_bf16(codes, scales), starts, lens, nc_cap)
+    np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32))
+    codes, scales = _int8_cache(rng, 408, 2, 128, False)
+    got = oracle_mod.pool_int8(codes, scales, starts, lens, nc_cap)
+    v = codes.astype(np.float64) * scales.astype(np.float64)[..., None]
+    for i, L in enumerate(lens):
+        nc = oracle_mod.n_windows(int(L))
+        if nc == 0:
+            continue
+        win = np.lib.stride_tricks.sliding_window_view(v[starts[i]:starts[i] + L], 32, axis=0)[::16][:nc]
+        mean = win.mean(axis=-1).transpose(1, 0, 2)                     # [Hkv, nc, D]
+        np.testing.assert_allclose(got[i, :, :nc], mean, rtol=2.0 ** -23, atol=0)
+
+
+def test_attention_int8_equals_attention_of_dequantized_cache(oracle_mod):
+    """Power-of-two scales: INT8 attention == bf16 attention over the exact
+    dequantized cache, bit for bit (same fp64 values, same order).  General
+    scales: equal to torch's fp64 SDPA over s * code with the token mask of the
+    selection plus the local window."""
+    rng = np.random.default_rng(24)
+    L = 64 * 30 + 17                                                    # ncand = 15
+    b = inputs.make_batch(L, batch=1, num_q_heads=4, num_kv_heads=2, seed=25)
+    idx = np.array([[[0, 3, 14], [2, 7, -1]]], np.int32)
+    cnt = np.array([[3, 2]], np.int32)
+    for pow2 in (True, False):
+        kc, ks = _int8_cache(rng, L, 2, 128, pow2)
+        vc, vs = _int8_cache(rng, L, 2, 128, pow2)
+        out, lse = oracle_mod.sparse_attention_int8(_bits(b.q), kc, ks, vc, vs, b.seq_start.numpy(),
+                                                    b.seq_len.numpy(), idx, cnt)
+        if pow2:
+            o2, l2 = oracle_mod.sparse_attention(_bits(b.q), _dequant_bf16(kc, ks), _dequant_bf16(vc, vs),
+                                                 b.seq_start.numpy(), b.seq_len.numpy(), idx, cnt)
+            np.testing.assert_array_equal(out, o2)
+            np.testing.assert_array_equal(lse, l2)
+            continue
+        mask = np.zeros((2, L), bool)
+        for g in range(2):
+            for blk in idx[0, g, :cnt[0, g]]:
+                mask[g, 64 * blk:64 * blk + 64] = True
+            mask[g, 960:] = True
+        kd = torch.from_numpy(kc.astype(np.float64) * ks.astype(np.float64)[..., None])
+        vd = torch.from_numpy(vc.astype(np.float64) * vs.astype(np.float64)[..., None])
+        q = b.q[0].double().unsqueeze(1)
+        k = kd.permute(1, 0, 2).repeat_interleave(2, 0)
+        v = vd.permute(1, 0, 2).repeat_interleave(2, 0)
+        m = torch.from_numpy(mask).repeat_interleave(2, 0).unsqueeze(1)
+        o_ref = F.scaled_dot_product_attention(q, k, v, attn_mask=m)[:, 0].numpy()
+        logits = (q @ k.transpose(-1, -2)) / math.sqrt(128)
+        l_ref = torch.logsumexp(logits.masked_fill(~m, -math.inf), dim=-1)[:, 0].numpy()
+        np.testing.assert_allclose(out[0], o_ref, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(lse[0], l_ref, rtol=1e-12, atol=1e-12)
