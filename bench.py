@@ -79,6 +79,8 @@ def parse():
                     help="untimed repeated steps before timing, so clocks settle")
     ap.add_argument("--pooled", choices=["fp32", "bf16"], default="fp32",
                     help="pooled-key precision (bf16: the half-size variant)")
+    ap.add_argument("--kv", choices=["bf16", "int8"], default="bf16",
+                    help="K/V cache format (int8: codes + per-row scales, the 8-bit decode variant)")
     ap.add_argument("--sweep", action="store_true",
                     help="NOSA-1B shape over context x batch x top-k (one JSON line per point)")
     return ap.parse_args()
@@ -107,7 +109,9 @@ class Workload:
         self.key_dist = kdist
         self.local_blocks = 16
         self.pooled_bf16 = getattr(args, "pooled", "fp32") == "bf16"
-        self.desc = desc + (", bf16 pooled keys" if self.pooled_bf16 else "")
+        self.kv_int8 = getattr(args, "kv", "bf16") == "int8"
+        self.desc = desc + (", bf16 pooled keys" if self.pooled_bf16 else "") + (
+            ", INT8 K/V cache" if self.kv_int8 else "")
         if args.context or args.batch or args.topk:
             self.desc += f" [overridden: batch {self.batch}, context {max(self.lens)}, top-k {self.topk}]"
         self.max_len = max(self.lens)
@@ -125,10 +129,11 @@ class Workload:
             attended = k_eff * 64 + (L - 64 * ncand)
             new_window = _n_windows(L) - _n_windows(L - 1)
             pk = 256 if self.pooled_bf16 else 512                     # bytes per pooled key
+            row = 132 if self.kv_int8 else 256                        # bytes per cached K (or V) row
             for _ in range(self.hkv):
-                pool += 2 * 256 * 2 + new_window * (31 * 256 + pk)     # new K/V row in + out, window
+                pool += 2 * 256 + 2 * row + new_window * (31 * row + pk)  # new K/V row in + out, window
                 select += windows * pk + G * 256 + self.topk * 4 + 4
-                decode += attended * 512 + 2 * G * 256 + self.topk * 4 + 4
+                decode += attended * 2 * row + 2 * G * 256 + self.topk * 4 + 4
         return {"pool_append": pool * self.layers, "block_select": select * self.layers,
                 "sparse_decode": decode * self.layers}
 
@@ -139,9 +144,15 @@ class Replica:
     def __init__(self, nosa, wl: Workload, seed: int, device):
         self.b = inputs.make_batch(wl.lens, num_q_heads=wl.hq, num_kv_heads=wl.hkv, seed=seed,
                                    key_dist=wl.key_dist, device=device)
-        self.p = nosa.params(wl.hq, wl.hkv, topk=wl.topk, local_blocks=wl.local_blocks, pooled_bf16=wl.pooled_bf16)
+        self.p = nosa.params(wl.hq, wl.hkv, topk=wl.topk, local_blocks=wl.local_blocks, pooled_bf16=wl.pooled_bf16,
+                             kv_int8=wl.kv_int8)
+        if wl.kv_int8:   # the caches as the INT8 variant stores them (quantized on the GPU, untimed)
+            self.k_cache = nosa.Int8KvCache.from_bf16(self.p, self.b.k_cache)
+            self.v_cache = nosa.Int8KvCache.from_bf16(self.p, self.b.v_cache)
+        else:
+            self.k_cache, self.v_cache = self.b.k_cache, self.b.v_cache
         self.st = nosa.DecodeState(self.p, wl.batch, wl.max_len, device=device)
-        self.st.rebuild_pooled(self.b.k_cache, self.b.seq_start, self.b.seq_len)
+        self.st.rebuild_pooled(self.k_cache, self.b.seq_start, self.b.seq_len)
         self.k_new, self.v_new = inputs.random_kv_rows(wl.batch, wl.hkv, 128, seed=seed + 7,
                                                        device=device)
 
@@ -153,13 +164,13 @@ def step(nosa, r: Replica, events=None, fused=True):
     ``events`` (4 CUDA events) recorded before each kernel and after the last."""
     b, st, p = r.b, r.st, r.p
     if fused:
-        nosa.nosa_decode_step_device(p, b.q, b.k_cache, b.v_cache, b.seq_start, b.seq_len, st.max_seq_len,
+        nosa.nosa_decode_step_device(p, b.q, r.k_cache, r.v_cache, b.seq_start, b.seq_len, st.max_seq_len,
                                      st.pooled, st.sel_idx, st.sel_cnt, st.out, st.ws, k_new=r.k_new,
                                      v_new=r.v_new)
         return
     if events:
         events[0].record()
-    nosa.nosa_pool_append(p, b.k_cache, b.v_cache, b.seq_start, b.seq_len, st.pooled, max_new_keys=1,
+    nosa.nosa_pool_append(p, r.k_cache, r.v_cache, b.seq_start, b.seq_len, st.pooled, max_new_keys=1,
                           k_new=r.k_new, v_new=r.v_new, ws=st.ws)
     if events:
         events[1].record()
@@ -167,7 +178,7 @@ def step(nosa, r: Replica, events=None, fused=True):
                            st.ws)
     if events:
         events[2].record()
-    nosa.nosa_sparse_decode(p, b.q, b.k_cache, b.v_cache, b.seq_start, b.seq_len, st.max_seq_len,
+    nosa.nosa_sparse_decode(p, b.q, r.k_cache, r.v_cache, b.seq_start, b.seq_len, st.max_seq_len,
                             st.sel_idx, st.sel_cnt, st.out, st.ws)
     if events:
         events[3].record()
@@ -279,11 +290,25 @@ def oracle_steps(wl: Workload, b_host, n_steps: int, threads: int, budget_s: flo
     lens = b_host.seq_len.numpy()
     starts = b_host.seq_start.numpy()
     nc_cap = max(1, oracle.n_windows(int(lens.max())))
-    pooled = oracle.pool(kb, starts, lens - 1, nc_cap, bf16=wl.pooled_bf16)   # state before the step (untimed)
+    if wl.kv_int8:   # the INT8 variant: the oracle's own quantized caches (untimed)
+        kc, ks = oracle.quantize_int8(kb)
+        vc, vs = oracle.quantize_int8(vb)
+        pooled = oracle.pool_int8(kc, ks, starts, lens - 1, nc_cap, bf16=wl.pooled_bf16)
+    else:
+        pooled = oracle.pool(kb, starts, lens - 1, nc_cap, bf16=wl.pooled_bf16)   # state before the step (untimed)
+    nb_cap = oracle.n_blocks(int(lens.max()))
     done, t0 = 0, time.perf_counter()
     while done < n_steps:
-        pooled = oracle.pool(kb, starts, lens, nc_cap, len_old=lens - 1, pooled=pooled, bf16=wl.pooled_bf16)
-        oracle.decode_step(qb, kb, vb, starts, lens, pooled, wl.topk, local_blocks=wl.local_blocks)
+        if wl.kv_int8:
+            pooled = oracle.pool_int8(kc, ks, starts, lens, nc_cap, len_old=lens - 1, pooled=pooled,
+                                      bf16=wl.pooled_bf16)
+            sc = oracle.comp_scores(qb, pooled, lens, num_kv_heads=wl.hkv)
+            S = oracle.block_scores(sc, lens, nb_cap, num_kv_heads=wl.hkv, local_blocks=wl.local_blocks)
+            idx, cnt = oracle.topk(S, lens, wl.topk, local_blocks=wl.local_blocks)
+            oracle.sparse_attention_int8(qb, kc, ks, vc, vs, starts, lens, idx, cnt, local_blocks=wl.local_blocks)
+        else:
+            pooled = oracle.pool(kb, starts, lens, nc_cap, len_old=lens - 1, pooled=pooled, bf16=wl.pooled_bf16)
+            oracle.decode_step(qb, kb, vb, starts, lens, pooled, wl.topk, local_blocks=wl.local_blocks)
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
@@ -346,7 +371,7 @@ def run_ours(args):
     seed0 = multirank.rank_seed(0, info)
 
     # Replicas so that no step finds its inputs in L2 (126 MB).
-    layer_bytes = sum(wl.lens) * wl.hkv * 128 * 2 * 2
+    layer_bytes = sum(wl.lens) * wl.hkv * (132 if wl.kv_int8 else 256) * 2
     if wl.layers > 1:
         R = 1
         layers = [Replica(nosa, wl, seed0 + 10 * l, device) for l in range(wl.layers)]
@@ -458,7 +483,7 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "int8+bf16" if wl.kv_int8 else "bf16", "data": "synthetic",
             "config": {"workload": wl.desc, "batch": wl.batch, "seq_len": wl.max_len,
                        "topk": wl.topk, "local_blocks": wl.local_blocks, "layers": wl.layers,
                        "parallelism": f"dp{world}" if world > 1 else "single GPU",
@@ -497,7 +522,7 @@ def measure_e2e(nosa, wl: Workload, r: Replica, args, stream, info, device):
     n = max(10, min(args.steps, 500))
 
     def call():
-        nosa.nosa_decode_step(p, q_h, k_h, v_h, o_h, b.k_cache, b.v_cache, b.seq_start, b.seq_len,
+        nosa.nosa_decode_step(p, q_h, k_h, v_h, o_h, r.k_cache, r.v_cache, b.seq_start, b.seq_len,
                               st.max_seq_len, st.pooled, st.sel_idx, st.sel_cnt, st.ws, stream=stream)
 
     with torch.cuda.stream(stream):
@@ -541,7 +566,8 @@ def run_sweep(args):
     for L in SWEEP_CONTEXTS:
         for B in SWEEP_BATCHES:
             for K in SWEEP_TOPK:
-                a = argparse.Namespace(workload="nosa1b_b8_16k", context=L, batch=B, topk=K, pooled=args.pooled)
+                a = argparse.Namespace(workload="nosa1b_b8_16k", context=L, batch=B, topk=K, pooled=args.pooled,
+                                       kv=args.kv)
                 wl = Workload(a, 0)
                 layer_bytes = B * L * wl.hkv * 128 * 2 * 2
                 R = max(2, min(16, math.ceil(1.0e9 / layer_bytes)))

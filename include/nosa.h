@@ -34,7 +34,8 @@
  *      k_cache/v_cache bf16 [cache_rows, num_kv_heads, head_dim], cache_rows
  *                   < 2^31; sequence i occupies rows seq_start[i] ..
  *                   seq_start[i] + len - 1 (varlen packing as with
- *                   cu_seqlens: seq_start[i] = cu_seqlens[i]).
+ *                   cu_seqlens: seq_start[i] = cu_seqlens[i]).  With
+ *                   p->kv_int8: INT8 buffers (see nosa_kv_int8_bytes).
  *      pooled       fp32 (or bf16 when p->pooled_bf16) [batch, num_kv_heads, nc_cap,
  *                   head_dim]
  *      sel_idx      int32 [batch, num_kv_heads, topk] (ascending, -1 padded)
@@ -110,12 +111,35 @@ typedef struct {
   float softmax_scale; /* 0 => 1/sqrt(head_dim); used for scores and attention */
   int pooled_bf16;     /* 0: pooled keys fp32 (default); 1: pooled keys bf16, each the
                           round-to-nearest-even of the fp32 mean (half the selection bytes) */
+  int kv_int8;         /* 0: K/V caches bf16 (default); 1: INT8 caches (codes + per-row
+                          scales, see nosa_kv_int8_bytes): half the attention bytes */
 } nosa_params;
 
 /* Fills `p` with the NOSA-1B attention defaults: 16 q / 2 KV heads, head_dim
  * 128, kernel 32 / stride 16, block 64, 16 local blocks, topk 64, scale 0,
- * fp32 pooled keys. */
+ * fp32 pooled keys, bf16 caches. */
 NOSA_API void nosa_default_params(nosa_params* p);
+
+/* INT8 K/V caches (p->kv_int8 = 1; reading of "NOSA 技术架构解析"
+ * (devpress.csdn.net) §1.1 "关键技巧": the decode stage may switch to 8-bit
+ * integers).  Each cache row (token, KV head) of 128 bf16 values x is stored
+ * as 128 int8 codes and one fp32 scale, symmetric per row:
+ *     s = max|x| / 127,  code = clamp(rint(x / s), -127, 127)
+ * (IEEE fp32 divisions, rint half to even; s = 0 for an all-zero row), and
+ * read back as s * code.  With kv_int8 set, every k_cache / v_cache argument
+ * of the calls below is one such buffer (K and V separately):
+ *     codes  int8 [cache_rows, Hkv, 128]                at byte 0
+ *     scales fp32 [Hkv, scale_stride]                   at byte cache_rows * Hkv * 128
+ * with scale_stride = cache_rows rounded up to a multiple of 4 (for paged
+ * caches cache_rows = num_pages * 64).  The new token's k_new / v_new stay
+ * bf16: the calls quantize them on append.  Pooling reads s * code (the
+ * pooled keys are as in the bf16 case), attention uses s * code for K and V.
+ * nosa_kv_int8_bytes returns the buffer size (0 if the arguments are
+ * invalid); nosa_quantize_kv_int8 quantizes bf16 rows src [rows, Hkv, 128]
+ * into rows row0 .. row0 + rows - 1 of such a buffer (e.g. after a prefill). */
+NOSA_API size_t nosa_kv_int8_bytes(int64_t cache_rows, int num_kv_heads);
+NOSA_API int nosa_quantize_kv_int8(const nosa_params* p, const void* src, void* cache, int64_t cache_rows,
+                                   int64_t row0, int64_t rows, void* stream);
 
 /* Bytes of device workspace that nosa_block_select / nosa_sparse_decode /
  * nosa_decode_step need for `batch` sequences of at most `max_seq_len`

@@ -12,6 +12,7 @@
 #include "nosa_common.cuh"
 #include "nosa_kernels.h"
 #include "decode_device.cuh"
+#include "kv_int8.cuh"
 #include "select_device.cuh"
 
 namespace {
@@ -63,7 +64,14 @@ int check_params(const nosa_params* p) {
   if (!(p->softmax_scale >= 0.0f) || std::isinf(p->softmax_scale))
     return fail(NOSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
   if (p->pooled_bf16 != 0 && p->pooled_bf16 != 1) return fail(NOSA_ERR_INVALID_ARG, "pooled_bf16 must be 0 or 1");
+  if (p->kv_int8 != 0 && p->kv_int8 != 1) return fail(NOSA_ERR_INVALID_ARG, "kv_int8 must be 0 or 1");
   return NOSA_OK;
+}
+
+// The scale rows of an INT8 cache buffer (codes first, then scales).
+float* int8_scales(const void* cache, int64_t cache_rows, int hkv) {
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(const_cast<void*>(cache)) +
+                                  nosa::int8_scale_offset(cache_rows, hkv));
 }
 
 float scale_of(const nosa_params* p) {
@@ -127,22 +135,68 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 3-D map over a [rows, hkv, 128] bf16 cache: boxes of {64 dims, 1 head,
-// 64 tokens}, 128-byte swizzle, zero fill past `rows`.
-int encode_kv_map(CUtensorMap* map, const void* base, int hkv, int64_t rows) {
+// 3-D map over a [rows, hkv, 128] cache: bf16 boxes of {64 dims, 1 head,
+// 64 tokens}, or INT8 boxes of {128 codes, 1 head, 64 tokens}; 128-byte rows
+// with the 128-byte swizzle, zero fill past `rows`.
+int encode_kv_map(CUtensorMap* map, const void* base, int hkv, int64_t rows, bool int8) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(NOSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const cuuint64_t esize = int8 ? 1 : 2;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(nosa::kHeadDim), static_cast<cuuint64_t>(hkv),
                               static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(nosa::kHeadDim) * 2,
-                                 static_cast<cuuint64_t>(hkv) * nosa::kHeadDim * 2};
-  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(nosa::kBlock)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(nosa::kHeadDim) * esize,
+                                 static_cast<cuuint64_t>(hkv) * nosa::kHeadDim * esize};
+  const cuuint32_t box[3] = {int8 ? 128u : 64u, 1, static_cast<cuuint32_t>(nosa::kBlock)};
   const cuuint32_t elem_strides[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-                   elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NOSA_ERR_INVALID_ARG, "tensor map encode failed (code %d)", static_cast<int>(r));
   return NOSA_OK;
+}
+
+// 2-D map over the scale rows of an INT8 cache, fp32 [hkv, stride]: boxes of
+// 68 consecutive tokens of one head (a tile's 64 scales from the 16-byte
+// aligned token at or below its first row), no swizzle, zero fill past the
+// row.
+int encode_scale_map(CUtensorMap* map, const void* cache, int hkv, int64_t rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(NOSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const int64_t stride = nosa::int8_scale_stride(rows);
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(stride), static_cast<cuuint64_t>(hkv)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride) * 4};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(nosa::kScaleBox), 1};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, int8_scales(cache, rows, hkv), dims, strides, box,
+                   elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NOSA_ERR_INVALID_ARG, "scale tensor map encode failed (code %d)", static_cast<int>(r));
+  return NOSA_OK;
+}
+
+// The cache maps of a decode launch (K, V and, for INT8 caches, their
+// scale rows).
+int encode_cache_maps(nosa::StepMaps* m, const nosa_params* p, const void* k_cache, const void* v_cache,
+                      int64_t rows) {
+  const bool int8 = p->kv_int8 != 0;
+  if (int rc = encode_kv_map(&m->k, k_cache, p->num_kv_heads, rows, int8)) return rc;
+  if (int rc = encode_kv_map(&m->v, v_cache, p->num_kv_heads, rows, int8)) return rc;
+  if (int8) {
+    if (int rc = encode_scale_map(&m->ks, k_cache, p->num_kv_heads, rows)) return rc;
+    if (int rc = encode_scale_map(&m->vs, v_cache, p->num_kv_heads, rows)) return rc;
+  }
+  return NOSA_OK;
+}
+
+// INT8 fields of the kernel arguments.
+template <typename Args>
+void set_int8(Args& a, const nosa_params* p, void* k_cache, const void* v_cache, int64_t rows) {
+  a.kv_int8 = p->kv_int8;
+  if (p->kv_int8) {
+    a.k_scale = k_cache ? int8_scales(k_cache, rows, p->num_kv_heads) : nullptr;
+    a.v_scale = v_cache ? int8_scales(v_cache, rows, p->num_kv_heads) : nullptr;
+    a.scale_stride = nosa::int8_scale_stride(rows);
+  }
 }
 
 // 2-D map over the pooled keys [batch * hkv * nc_cap rows, 128 fp32 or bf16]:
@@ -229,6 +283,7 @@ int do_pool_append(const nosa_params* p, void* k_cache, void* v_cache, int64_t c
   a.hkv = p->num_kv_heads;
   a.nc_cap = nc_cap;
   a.max_new_keys = max_new_keys;
+  set_int8(a, p, k_cache, v_cache, cache_rows);
   cudaError_t e = nosa::launch_pool_append(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "pool_append launch");
   return ok();
@@ -312,10 +367,10 @@ int do_block_select(const nosa_params* p, const void* q, const void* pooled, int
   s.bs_out = bs_out;
   s.nb_out = nb_out;
   s.mode = nosa::kStepScore;
-  CUtensorMap none, tm_p;
-  memset(&none, 0, sizeof none);
-  if (int rc = encode_pooled_map(&tm_p, pooled, batch, p->num_kv_heads, nc_cap, p->pooled_bf16 != 0)) return rc;
-  cudaError_t e = nosa::launch_step(s, none, none, tm_p, stream);
+  nosa::StepMaps maps;
+  memset(&maps, 0, sizeof maps);
+  if (int rc = encode_pooled_map(&maps.p, pooled, batch, p->num_kv_heads, nc_cap, p->pooled_bf16 != 0)) return rc;
+  cudaError_t e = nosa::launch_step(s, maps, stream);
   if (e != cudaSuccess) return cuda_fail(e, "block_select launch");
   return ok();
 }
@@ -350,11 +405,11 @@ int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, c
   s.out = static_cast<__nv_bfloat16*>(out);
   s.lse = lse;
   s.mode = nosa::kStepDecode;
-  CUtensorMap tm_k, tm_v, none;
-  memset(&none, 0, sizeof none);
-  if (int rc = encode_kv_map(&tm_k, k_cache, p->num_kv_heads, cache_rows)) return rc;
-  if (int rc = encode_kv_map(&tm_v, v_cache, p->num_kv_heads, cache_rows)) return rc;
-  cudaError_t e = nosa::launch_step(s, tm_k, tm_v, none, stream);
+  set_int8(s, p, const_cast<void*>(k_cache), v_cache, cache_rows);
+  nosa::StepMaps maps;
+  memset(&maps, 0, sizeof maps);
+  if (int rc = encode_cache_maps(&maps, p, k_cache, v_cache, cache_rows)) return rc;
+  cudaError_t e = nosa::launch_step(s, maps, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse_decode launch");
   return ok();
 }
@@ -401,11 +456,12 @@ int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new
   s.out = static_cast<__nv_bfloat16*>(out);
   s.lse = lse;
   s.mode = nosa::kStepScore | nosa::kStepDecode | nosa::kStepAppend;
-  CUtensorMap tm_k, tm_v, tm_p;
-  if (int rc = encode_kv_map(&tm_k, k_cache, p->num_kv_heads, cache_rows)) return rc;
-  if (int rc = encode_kv_map(&tm_v, v_cache, p->num_kv_heads, cache_rows)) return rc;
-  if (int rc = encode_pooled_map(&tm_p, pooled, batch, p->num_kv_heads, nc_cap, p->pooled_bf16 != 0)) return rc;
-  cudaError_t e = nosa::launch_step(s, tm_k, tm_v, tm_p, stream);
+  set_int8(s, p, k_cache, v_cache, cache_rows);
+  nosa::StepMaps maps;
+  memset(&maps, 0, sizeof maps);
+  if (int rc = encode_cache_maps(&maps, p, k_cache, v_cache, cache_rows)) return rc;
+  if (int rc = encode_pooled_map(&maps.p, pooled, batch, p->num_kv_heads, nc_cap, p->pooled_bf16 != 0)) return rc;
+  cudaError_t e = nosa::launch_step(s, maps, stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode_step launch");
   return ok();
 }
@@ -437,6 +493,32 @@ void nosa_default_params(nosa_params* p) {
   p->topk = 64;
   p->softmax_scale = 0.0f;
   p->pooled_bf16 = 0;
+  p->kv_int8 = 0;
+}
+
+size_t nosa_kv_int8_bytes(int64_t cache_rows, int num_kv_heads) {
+  if (cache_rows < 1 || cache_rows >= (int64_t{1} << 31) || num_kv_heads < 1) return 0;
+  return static_cast<size_t>(nosa::int8_scale_offset(cache_rows, num_kv_heads)) +
+         static_cast<size_t>(num_kv_heads) * nosa::int8_scale_stride(cache_rows) * 4;
+}
+
+int nosa_quantize_kv_int8(const nosa_params* p, const void* src, void* cache, int64_t cache_rows, int64_t row0,
+                          int64_t rows, void* stream) {
+  if (int rc = check_params(p)) return rc;
+  if (!src || !cache) return fail(NOSA_ERR_INVALID_ARG, "src and cache must not be NULL");
+  if (!aligned(src, 8) || !aligned(cache, 16))
+    return fail(NOSA_ERR_INVALID_ARG, "src must be 8-byte and cache 16-byte aligned");
+  if (cache_rows < 1 || cache_rows >= (int64_t{1} << 31))
+    return fail(NOSA_ERR_UNSUPPORTED, "cache_rows must be in [1, 2^31)");
+  if (row0 < 0 || rows < 0 || row0 + rows > cache_rows)
+    return fail(NOSA_ERR_INVALID_ARG, "rows [%lld, %lld) outside the cache's %lld rows", static_cast<long long>(row0),
+                static_cast<long long>(row0 + rows), static_cast<long long>(cache_rows));
+  cudaError_t e = nosa::launch_quantize_int8(static_cast<const __nv_bfloat16*>(src), static_cast<int8_t*>(cache),
+                                             int8_scales(cache, cache_rows, p->num_kv_heads),
+                                             nosa::int8_scale_stride(cache_rows), row0, rows, p->num_kv_heads,
+                                             static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return ok();
 }
 
 size_t nosa_workspace_size(const nosa_params* p, int batch, int max_seq_len) {

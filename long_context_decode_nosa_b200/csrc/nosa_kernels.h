@@ -27,6 +27,10 @@ struct PoolArgs {
   uint32_t* status;            // nullable
   int batch, hkv, nc_cap, max_new_keys;
   int pooled_bf16;
+  int kv_int8;                 // INT8 caches: k_cache / v_cache hold int8 codes, scales below
+  float* k_scale;              // [hkv, scale_stride] (INT8 caches)
+  float* v_scale;
+  int64_t scale_stride;
 };
 
 struct SelectArgs {  // selection from given block scores (select_only_kernel)
@@ -67,6 +71,10 @@ struct StepArgs {
   int batch, hq, hkv, local_blocks, topk, max_seq_len, nc_cap, nb_out, nb_spill;
   int ncand_max;  // candidates of a sequence of max_seq_len tokens
   int pooled_bf16;
+  int kv_int8;         // INT8 caches: k_cache / v_cache hold int8 codes [cache_rows, hkv, 128]
+  float* k_scale;      // [hkv, scale_stride] per-row scales (INT8 caches)
+  float* v_scale;
+  int64_t scale_stride;
   int mode;
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)
@@ -92,8 +100,14 @@ cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 cudaError_t launch_pool_append(const PoolArgs& a, cudaStream_t stream);
-cudaError_t launch_step(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
-                        cudaStream_t stream);
+// Tensor maps of one step launch: K and V tiles, pooled keys, and (INT8
+// caches) the K and V scale rows.
+struct StepMaps {
+  CUtensorMap k, v, p, ks, vs;
+};
+cudaError_t launch_step(const StepArgs& a, const StepMaps& maps, cudaStream_t stream);
+cudaError_t launch_quantize_int8(const __nv_bfloat16* src, int8_t* codes, float* scales, int64_t scale_stride,
+                                 int64_t row0, int64_t rows, int hkv, cudaStream_t stream);
 cudaError_t launch_select_only(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint32_t* status, uint32_t max_iters, cudaStream_t stream);
 

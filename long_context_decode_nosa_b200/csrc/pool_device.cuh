@@ -6,6 +6,7 @@
 // (kernel_size 32, stride 16):  pooled[j] = (1/32) * sum_{t=16j}^{16j+31} K[t].
 #pragma once
 
+#include "kv_int8.cuh"
 #include "nosa_common.cuh"
 
 namespace nosa {
@@ -17,6 +18,22 @@ __device__ inline float4 bf16x4_to_float4(uint2 raw) {
   f.z = __uint_as_float(raw.y << 16);
   f.w = __uint_as_float(raw.y & 0xFFFF0000u);
   return f;
+}
+
+// The window sum `acc` (lane l: dims 4l..4l+3) x 1/32 (exact), stored as
+// fp32 or rounded to bf16 (nearest, ties to even).
+__device__ inline void store_pooled(float4 acc, void* __restrict__ dst, bool bf16, int lane) {
+  constexpr float inv = 1.0f / kPoolKernel;
+  const float4 m = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (bf16) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y), hi = __floats2bfloat162_rn(m.z, m.w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(dst)[lane] = packed;
+  } else {
+    reinterpret_cast<float4*>(dst)[lane] = m;
+  }
 }
 
 // One warp pools window j of one (sequence, KV head): lane l owns dims
@@ -60,17 +77,49 @@ __device__ inline void pool_window_warp(const __nv_bfloat16* __restrict__ k_cach
     acc.z += f.z;
     acc.w += f.w;
   }
-  constexpr float inv = 1.0f / kPoolKernel;
-  const float4 m = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (bf16) {  // round to nearest, ties to even
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(m.x, m.y), hi = __floats2bfloat162_rn(m.z, m.w);
-    uint2 packed;
-    packed.x = *reinterpret_cast<const uint32_t*>(&lo);
-    packed.y = *reinterpret_cast<const uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(dst)[lane] = packed;
-  } else {
-    reinterpret_cast<float4*>(dst)[lane] = m;
+  store_pooled(acc, dst, bf16, lane);
+}
+
+// The same window over an INT8 key cache: row t contributes s_t * code_t
+// (one fp32 product per value), summed in ascending token order.  The fresh
+// token's row is quantized here from `fresh` (bf16) exactly as the append
+// stores it, so appending and rebuilding still give identical bits.
+__device__ inline void pool_window_warp_int8(const Int8Cache& c, int hkv, const KvRows& kv, int h, int64_t j,
+                                             int64_t fresh_tok, const uint2* __restrict__ fresh,
+                                             void* __restrict__ dst, bool bf16, int lane) {
+  const int64_t t0 = j * kPoolStride;
+  const int split = kv.pages ? min(kPoolKernel, static_cast<int>(kPageTokens - t0 % kPageTokens)) : kPoolKernel;
+  const int64_t row_a = kv.row(t0);
+  const int64_t row_b = split < kPoolKernel ? kv.row(t0 + split) : 0;
+  uint32_t codes[kPoolKernel];
+  float sc[kPoolKernel];
+#pragma unroll
+  for (int t = 0; t < kPoolKernel; ++t) {
+    const int64_t row = t < split ? row_a + t : row_b + (t - split);
+    codes[t] = __ldcg(reinterpret_cast<const uint32_t*>(c.row(row, hkv, h)) + lane);
+    sc[t] = __ldcg(c.scale(row, h));
   }
+  const int64_t r = fresh_tok - t0;
+  if (fresh != nullptr && r >= 0 && r < kPoolKernel) {
+    float fs;
+    const uint32_t fc = quantize_row_warp(fresh[lane], fs);
+#pragma unroll
+    for (int t = 0; t < kPoolKernel; ++t)
+      if (t == r) {
+        codes[t] = fc;
+        sc[t] = fs;
+      }
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int t = 0; t < kPoolKernel; ++t) {
+    const float4 f = dequant4(codes[t], sc[t]);
+    acc.x += f.x;
+    acc.y += f.y;
+    acc.z += f.z;
+    acc.w += f.w;
+  }
+  store_pooled(acc, dst, bf16, lane);
 }
 
 }  // namespace nosa

@@ -21,7 +21,8 @@
 //     per warp);
 //   * warp 4, producer: issues every TMA copy of the CTA in job order --
 //     scoring chunks, local tiles, selected tiles (after the selection) --
-//     into a 3-stage ring of 32 KB stages (full / empty mbarriers);
+//     into a ring of 32 KB stages (full / empty mbarriers); with INT8 caches
+//     a stage carries two tiles (half the bytes each) and their scale rows;
 //   * warp 5, selector: pools the window completed by the new token (rank
 //     0), waits until the block scores of the whole pair have arrived (one
 //     remote mbarrier arrival per CTA), runs the exact top-k (every CTA
@@ -37,6 +38,7 @@
 // traffic is inside the cluster, and every wait is bounded (status bit
 // NOSA_DEV_TIMEOUT), so a launch always finishes.
 #include "decode_device.cuh"
+#include "kv_int8.cuh"
 #include "nosa_common.cuh"
 #include "nosa_kernels.h"
 #include "pool_device.cuh"
@@ -77,7 +79,8 @@ struct StepShared {
   uint64_t empty_bar[kMaxStages];
   uint64_t scores_bar;  // completes when every CTA of the cluster has sent its block scores
   uint64_t sel_bar;     // completes when the selection is in shared memory (selector -> producer)
-  int stage_blk[kMaxStages];
+  int stage_blk[kMaxStages][2];   // the stage's tiles (second: kAbsentTile when one)
+  int stage_soff[kMaxStages][2];  // INT8: position of the tile's first scale in its scale slot
   int sel_count;
   float blk[kChunkBlocks];  // block scores of the chunk being sent
   GroupTopkShared gtk;      // the selection group's exchange (consumers + selector)
@@ -86,6 +89,9 @@ struct StepShared {
 #endif
 };
 
+// A stage slot left empty (INT8 caches: a job with one tile).
+constexpr int kAbsentTile = -2;
+
 // Shared memory of the step kernel (dynamic, from a 1024-byte aligned base):
 //   ring  kRingBytes                      kStages stages of 32 KB
 //   ssm   G x kScoreStride floats         window scores of the chunk being scored
@@ -93,6 +99,7 @@ struct StepShared {
 //   bsm   4 * ncand_max bytes             the pair's block scores (unless kept in global memory)
 //   recv  recv_bytes<G>()                 the partials the cluster's CTAs push for this CTA's
 //                                         share of the output (see the merge)
+//   scl   S x kScaleStageBytes            INT8 caches: the scale rows of each stage's tiles
 template <int G>
 __host__ __device__ constexpr int ssm_bytes() {
   return G * kScoreStride * 4;
@@ -108,6 +115,15 @@ __host__ __device__ constexpr int out_items() {
 template <int G>
 __host__ __device__ constexpr int recv_bytes() {
   return (out_items<G>() + kMaxCluster) * 16 + 2 * kMaxCluster * G * 4;
+}
+
+// Offset (from the aligned base) of the INT8 scale slots: after the receive
+// buffer, 128-byte aligned.
+template <int G, int S>
+__host__ __device__ inline int step_scale_offset(const StepArgs& a) {
+  const int end = S * kStageBytes + ssm_bytes<G>() + round16(4 * a.topk) +
+                  (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))) + recv_bytes<G>();
+  return (end + 127) & ~127;
 }
 
 // Named barrier of the four consumer warps.
@@ -163,11 +179,14 @@ static_assert((MergeLayout<kMaxGroup>::kPl + kMaxGroup) * 4 <= kRingBytes, "merg
 
 // S = ring stages: 3 (two CTAs per SM) or 6 (one CTA per SM, twice the
 // bytes in flight per CTA).
-template <int G, int S>
+// Q8: the K/V caches are INT8 (codes + per-row scales).
+template <int G, int S, bool Q8>
 __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
-    step_kernel(const StepArgs a, const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                const __grid_constant__ CUtensorMap tm_p) {
+    step_kernel(const StepArgs a, const __grid_constant__ StepMaps maps) {
   constexpr int kRing = S * kStageBytes;
+  const CUtensorMap* tm_k = &maps.k;
+  const CUtensorMap* tm_v = &maps.v;
+  const CUtensorMap* tm_p = &maps.p;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled TMA boxes want 1024-byte aligned destinations.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -203,10 +222,14 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   }
   __syncthreads();
   if (warp == kProducerWarp && lane == 0) {
-    if (scoring) asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_p) : "memory");
+    if (scoring) asm volatile("prefetch.tensormap [%0];" ::"l"(tm_p) : "memory");
     if (decoding) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_k) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_v) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(tm_k) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(tm_v) : "memory");
+      if (Q8) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.ks) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.vs) : "memory");
+      }
     }
   }
   grid_dependency_wait();
@@ -311,13 +334,13 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
         const int row0 = row_base + kChunkBlocks * kWindowsPerBlock * k - 1;
         if (a.pooled_bf16) {
           mbar_arrive_expect_tx(&sh.full_bar[s], kScoreTxBytesBf16);
-          tma_load_keys(st, &tm_p, 0, row0, &sh.full_bar[s], policy);
-          tma_load_keys(st + kScoreSlotBytes, &tm_p, 64, row0, &sh.full_bar[s], policy);
+          tma_load_keys(st, tm_p, 0, row0, &sh.full_bar[s], policy);
+          tma_load_keys(st + kScoreSlotBytes, tm_p, 64, row0, &sh.full_bar[s], policy);
         } else {
           mbar_arrive_expect_tx(&sh.full_bar[s], kScoreTxBytes);
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            tma_load_keys(st + c * kScoreSlotBytes, &tm_p, c * kBoxCols, row0, &sh.full_bar[s], policy);
+            tma_load_keys(st + c * kScoreSlotBytes, tm_p, c * kBoxCols, row0, &sh.full_bar[s], policy);
         }
       });
     }
@@ -339,42 +362,78 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       }
       return pg * kPageTokens;
     };
-    auto issue_tile = [&](int blk, int row) {
+    // One job: a tile (bf16: four {64 dims, 1 head, 64 tokens} boxes), or
+    // with INT8 caches up to two tiles (a {128 bytes, 1 head, 64 tokens} box
+    // of K and of V each, plus their 68-scale rows).
+    auto issue_job = [&](int blk0, int row0, int blk1, int row1) {
       issue([&](int s, uint8_t* st) {
-        sh.stage_blk[s] = blk;
-        mbar_arrive_expect_tx(&sh.full_bar[s], kTileTxBytes);
-        tma_load_box(st, &tm_k, 0, g, row, &sh.full_bar[s], policy);
-        tma_load_box(st + kHalfBytes, &tm_k, 64, g, row, &sh.full_bar[s], policy);
-        tma_load_box(st + 2 * kHalfBytes, &tm_v, 0, g, row, &sh.full_bar[s], policy);
-        tma_load_box(st + 3 * kHalfBytes, &tm_v, 64, g, row, &sh.full_bar[s], policy);
+        sh.stage_blk[s][0] = blk0;
+        sh.stage_blk[s][1] = blk1;
+        if constexpr (Q8) {
+          uint8_t* scl = smem + step_scale_offset<G, S>(a) + s * kScaleStageBytes;
+          const int n = blk1 == kAbsentTile ? 1 : 2;
+          mbar_arrive_expect_tx(&sh.full_bar[s], n * kTileTxBytesInt8);
+          for (int x = 0; x < n; ++x) {
+            const int row = x ? row1 : row0;
+            sh.stage_soff[s][x] = row & 3;
+            tma_load_box(st + 2 * x * kTileBytesInt8, tm_k, 0, g, row, &sh.full_bar[s], policy);
+            tma_load_box(st + (2 * x + 1) * kTileBytesInt8, tm_v, 0, g, row, &sh.full_bar[s], policy);
+            tma_load_keys(scl + 2 * x * kScaleSlot, &maps.ks, row & ~3, g, &sh.full_bar[s], policy);
+            tma_load_keys(scl + (2 * x + 1) * kScaleSlot, &maps.vs, row & ~3, g, &sh.full_bar[s], policy);
+          }
+        } else {
+          (void)blk1;
+          (void)row1;
+          mbar_arrive_expect_tx(&sh.full_bar[s], kTileTxBytes);
+          tma_load_box(st, tm_k, 0, g, row0, &sh.full_bar[s], policy);
+          tma_load_box(st + kHalfBytes, tm_k, 64, g, row0, &sh.full_bar[s], policy);
+          tma_load_box(st + 2 * kHalfBytes, tm_v, 0, g, row0, &sh.full_bar[s], policy);
+          tma_load_box(st + 3 * kHalfBytes, tm_v, 64, g, row0, &sh.full_bar[s], policy);
+        }
       });
     };
+    constexpr int kPerJob = Q8 ? 2 : 1;
     const int Ci = static_cast<int>(C), ri = static_cast<int>(rank);
     // Local tiles t = rank, rank + C, ... < nloc: known at once.
     {
+      const int tend = min(nloc, ntiles);
       int my_blk = -1, my_row = 0, n = 0;
-      for (int t = ri; t < min(nloc, ntiles) && ok; t += Ci, ++n) {
+      for (int t = ri; t < tend && ok; t += kPerJob * Ci, n += kPerJob) {
         if ((n & 31) == 0) {
           const int tl = t + Ci * lane;
-          my_row = tile_row(tl < min(nloc, ntiles) ? ncand + tl : -1, my_blk);
+          my_row = tile_row(tl < tend ? ncand + tl : -1, my_blk);
         }
         const int blk = __shfl_sync(0xffffffffu, my_blk, n & 31);
         const int row = __shfl_sync(0xffffffffu, my_row, n & 31);
-        if (appending && t == nloc - 1 && a.k_new != nullptr) {
-          // This tile holds token L-1: write the new K/V rows first and order
+        const bool two = Q8 && t + Ci < tend;
+        int blk1 = kAbsentTile, row1 = 0;
+        if constexpr (Q8) {
+          blk1 = __shfl_sync(0xffffffffu, my_blk, (n + 1) & 31);
+          row1 = __shfl_sync(0xffffffffu, my_row, (n + 1) & 31);
+        }
+        if (appending && a.k_new != nullptr && (t == nloc - 1 || (two && t + Ci == nloc - 1))) {
+          // This job holds token L-1: write the new K/V rows first and order
           // them before the tile's TMA read (same CTA, async proxy).
           if (kv.page_ok(L - 1)) {
-            const int64_t row_w = kv.row(L - 1) * a.hkv + g;
             const int64_t src = static_cast<int64_t>(i) * a.hkv + g;
-            reinterpret_cast<uint2*>(a.k_cache + row_w * kHeadDim)[lane] =
-                reinterpret_cast<const uint2*>(a.k_new + src * kHeadDim)[lane];
-            reinterpret_cast<uint2*>(a.v_cache + row_w * kHeadDim)[lane] =
-                reinterpret_cast<const uint2*>(a.v_new + src * kHeadDim)[lane];
+            if constexpr (Q8) {
+              const int64_t r = kv.row(L - 1);
+              store_int8_row_warp(Int8Cache{reinterpret_cast<int8_t*>(a.k_cache), a.k_scale, a.scale_stride}, a.hkv,
+                                  r, g, reinterpret_cast<const uint2*>(a.k_new + src * kHeadDim), lane);
+              store_int8_row_warp(Int8Cache{reinterpret_cast<int8_t*>(a.v_cache), a.v_scale, a.scale_stride}, a.hkv,
+                                  r, g, reinterpret_cast<const uint2*>(a.v_new + src * kHeadDim), lane);
+            } else {
+              const int64_t row_w = kv.row(L - 1) * a.hkv + g;
+              reinterpret_cast<uint2*>(a.k_cache + row_w * kHeadDim)[lane] =
+                  reinterpret_cast<const uint2*>(a.k_new + src * kHeadDim)[lane];
+              reinterpret_cast<uint2*>(a.v_cache + row_w * kHeadDim)[lane] =
+                  reinterpret_cast<const uint2*>(a.v_new + src * kHeadDim)[lane];
+            }
             asm volatile("fence.proxy.async.global;" ::: "memory");
           }
           __syncwarp();
         }
-        issue_tile(blk, row);
+        issue_job(blk, row, two ? blk1 : kAbsentTile, row1);
       }
     }
     // Selected tiles t = nloc + x, t = rank (mod C): after the selection.
@@ -385,7 +444,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
         if (lane == 0) got = mbar_wait(&sh.sel_bar, 0, a.status) ? 1 : 0;
         const bool sel_ok = __shfl_sync(0xffffffffu, got, 0) != 0;
         int my_blk = -1, my_row = 0, n = 0;
-        for (int t = t0; t < ntiles && ok; t += Ci, ++n) {
+        for (int t = t0; t < ntiles && ok; t += kPerJob * Ci, n += kPerJob) {
           if ((n & 31) == 0) {
             const int tl = t + Ci * lane;
             int blk = -1;
@@ -398,7 +457,15 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
             }
             my_row = tile_row(blk, my_blk);
           }
-          issue_tile(__shfl_sync(0xffffffffu, my_blk, n & 31), __shfl_sync(0xffffffffu, my_row, n & 31));
+          const bool two = Q8 && t + Ci < ntiles;
+          const int blk0 = __shfl_sync(0xffffffffu, my_blk, n & 31);
+          const int row0 = __shfl_sync(0xffffffffu, my_row, n & 31);
+          int blk1 = kAbsentTile, row1 = 0;
+          if constexpr (Q8) {
+            blk1 = __shfl_sync(0xffffffffu, my_blk, (n + 1) & 31);
+            row1 = __shfl_sync(0xffffffffu, my_row, (n + 1) & 31);
+          }
+          issue_job(blk0, row0, two ? blk1 : kAbsentTile, row1);
         }
       }
     }
@@ -426,9 +493,13 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           const int64_t at = (static_cast<int64_t>(pair) * a.nc_cap + j) * kHeadDim;
           void* dst = a.pooled_bf16 ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.pooled) + at)
                                     : static_cast<void*>(static_cast<float*>(a.pooled) + at);
-          if (kv.page_ok(j * kPoolStride) && kv.page_ok(j * kPoolStride + kPoolKernel - 1))
-            pool_window_warp(a.k_cache, a.hkv, kv, g, j, knew ? L - 1 : -1, knew, dst, a.pooled_bf16 != 0, lane);
-          else if (lane == 0)
+          if (kv.page_ok(j * kPoolStride) && kv.page_ok(j * kPoolStride + kPoolKernel - 1)) {
+            if constexpr (Q8)
+              pool_window_warp_int8(Int8Cache{reinterpret_cast<int8_t*>(a.k_cache), a.k_scale, a.scale_stride}, a.hkv,
+                                    kv, g, j, knew ? L - 1 : -1, knew, dst, a.pooled_bf16 != 0, lane);
+            else
+              pool_window_warp(a.k_cache, a.hkv, kv, g, j, knew ? L - 1 : -1, knew, dst, a.pooled_bf16 != 0, lane);
+          } else if (lane == 0)
             set_status(a.status, NOSA_DEV_BAD_INDEX);
         }
       }
@@ -554,12 +625,22 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     }
     attn_init(att);
     if (decoding && ok) {
-      const int my_tiles = ntiles > static_cast<int>(rank)
-                               ? (ntiles - static_cast<int>(rank) + static_cast<int>(C) - 1) / static_cast<int>(C)
-                               : 0;
+      // This CTA's tiles: local t = rank, rank + C, ... < min(nloc, ntiles),
+      // then selected t = rank (mod C) in [nloc, ntiles); with INT8 caches
+      // each phase is issued two tiles per job.
+      const int Ci = static_cast<int>(C), ri = static_cast<int>(rank);
+      const int tend = min(nloc, ntiles);
+      const int my_local = tend > ri ? (tend - ri + Ci - 1) / Ci : 0;
+      const int t0 = nloc + ((ri - nloc % Ci) % Ci + Ci) % Ci;
+      const int my_sel = ntiles > t0 ? (ntiles - t0 + Ci - 1) / Ci : 0;
+      const int my_tiles = Q8 ? (my_local + 1) / 2 + (my_sel + 1) / 2 : my_local + my_sel;
       if (my_tiles > 0) {
         uint32_t qa[8][4];
-        load_attn_q(qa, q_group, G, lane);
+        float qpow = 1.0f;
+        if constexpr (Q8)
+          qpow = load_attn_q_int8(qa, q_group, G, lane);
+        else
+          load_attn_q(qa, q_group, G, lane);
         // Tiles start once the selection is known (the consumers took part
         // in it, or wait for the selector): the selection runs on a quiet
         // SM, and the local tiles, already staged, are consumed while the
@@ -572,7 +653,35 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           if (tid == 0 && n == 0) NOSA_STAMP(22);
           if (tid == 0 && n == 2) NOSA_STAMP(23);
 #endif
-          attend_tile(att, qa, smem + s * kStageBytes, sh.stage_blk[s], L, a.scale_log2, warp, lane);
+          if constexpr (Q8) {
+            const uint8_t* st = smem + s * kStageBytes;
+            const float* scl = reinterpret_cast<const float*>(smem + step_scale_offset<G, S>(a) + s * kScaleStageBytes);
+            const int blk[2] = {sh.stage_blk[s][0], sh.stage_blk[s][1]};
+            const float* const ksc[2] = {scl + sh.stage_soff[s][0], scl + 2 * (kScaleSlot / 4) + sh.stage_soff[s][1]};
+            const float* const vsc[2] = {scl + (kScaleSlot / 4) + sh.stage_soff[s][0],
+                                         scl + 3 * (kScaleSlot / 4) + sh.stage_soff[s][1]};
+#ifdef NOSA_TRACE
+            uint64_t* stamps = tid == 0 && n == 1 ? &sh.tr[14] : nullptr;
+            if (stamps) NOSA_STAMP(8);
+#else
+            uint64_t* stamps = nullptr;
+#endif
+            if (blk[1] == kAbsentTile)
+              attend_stage_int8<1>(att, qa, qpow, st, ksc, vsc, blk, L, a.scale_log2, warp, lane, stamps);
+            else
+              attend_stage_int8<2>(att, qa, qpow, st, ksc, vsc, blk, L, a.scale_log2, warp, lane, stamps);
+          } else {
+#ifdef NOSA_TRACE
+            if (tid == 0 && n == 1) NOSA_STAMP(8);
+#endif
+            attend_tile(att, qa, smem + s * kStageBytes, sh.stage_blk[s][0], L, a.scale_log2, warp, lane);
+          }
+#ifdef NOSA_TRACE
+          if (tid == 0 && n == 1) {
+            asm volatile("" ::"f"(att.acc[0][0]), "f"(att.acc[15][3]));
+            NOSA_STAMP(13);
+          }
+#endif
           if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
           ++r;
         }
@@ -599,9 +708,15 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int row = grp + h2 * 8;
-          if (row < G)
-            *reinterpret_cast<float2*>(mf + ML::kMo + (warp * G + row) * kMoStride + d * 8 + 2 * tig) =
-                make_float2(att.acc[d][2 * h2], att.acc[d][2 * h2 + 1]);
+          if (row < G) {
+            float* o = mf + ML::kMo + (warp * G + row) * kMoStride;
+            if constexpr (Q8) {  // acc[d][e]: dim 32 tig + 16 (e & 1) + d, scaled by 1 / U
+              o[32 * tig + d] = att.acc[d][2 * h2] * att.vscale;
+              o[32 * tig + 16 + d] = att.acc[d][2 * h2 + 1] * att.vscale;
+            } else {
+              *reinterpret_cast<float2*>(o + d * 8 + 2 * tig) = make_float2(att.acc[d][2 * h2], att.acc[d][2 * h2 + 1]);
+            }
+          }
         }
       }
       if (tig == 0) {
@@ -763,10 +878,9 @@ __global__ void wait_selftest_kernel(uint32_t* status, uint32_t max_iters) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, status, max_iters, 1000u);
 }
 
-template <int G>
-size_t step_smem_bytes(const StepArgs& a, int stages) {
-  return 1024 + static_cast<size_t>(stages) * kStageBytes + ssm_bytes<G>() + round16(4 * a.topk) +
-         (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))) + recv_bytes<G>();
+template <int G, int S, bool Q8>
+size_t step_smem_bytes(const StepArgs& a) {
+  return 1024 + step_scale_offset<G, S>(a) + (Q8 ? static_cast<size_t>(S) * kScaleStageBytes : 0);
 }
 
 // Residency of the step kernel at a given shared-memory size: resident
@@ -778,15 +892,15 @@ struct Capacity {
   int max_clusters[kMaxCluster + 1] = {};  // C = 1..16
 };
 std::mutex g_plan_mu;
-Capacity g_cap[5][2];  // [group size][ring: 3 or 6 stages]
+Capacity g_cap[5][2][2];  // [group size][ring: 3 or 6 stages][bf16 / INT8 caches]
 
-template <int G, int S>
+template <int G, int S, bool Q8>
 cudaError_t capacity(size_t smem, const Capacity** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   constexpr int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
-  Capacity& c = g_cap[gi][S == kMinStages ? 0 : 1];
+  Capacity& c = g_cap[gi][S == kMinStages ? 0 : 1][Q8 ? 1 : 0];
   if (c.dev != dev || c.smem != smem) {
     // The attribute is an upper bound: set to the largest size the device
     // allows next to the kernel's static shared memory, so that concurrent
@@ -794,17 +908,17 @@ cudaError_t capacity(size_t smem, const Capacity** out) {
     int optin = 0;
     cudaFuncAttributes fa;
     if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
-    if ((e = cudaFuncGetAttributes(&fa, step_kernel<G, S>)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa, step_kernel<G, S, Q8>)) != cudaSuccess) return e;
     const int max_dyn = optin - static_cast<int>(fa.sharedSizeBytes);
     if (static_cast<int>(smem) > max_dyn) return cudaErrorInvalidValue;
-    if ((e = cudaFuncSetAttribute(step_kernel<G, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn)) !=
+    if ((e = cudaFuncSetAttribute(step_kernel<G, S, Q8>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn)) !=
         cudaSuccess)
       return e;
-    if ((e = cudaFuncSetAttribute(step_kernel<G, S>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
+    if ((e = cudaFuncSetAttribute(step_kernel<G, S, Q8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
         cudaSuccess)
       return e;
     int per_sm = 0, sms = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<G, S>, kStepThreads, smem)) !=
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<G, S, Q8>, kStepThreads, smem)) !=
         cudaSuccess)
       return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
@@ -823,7 +937,7 @@ cudaError_t capacity(size_t smem, const Capacity** out) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, step_kernel<G, S>, &cfg) != cudaSuccess) {
+      if (cudaOccupancyMaxActiveClusters(&n, step_kernel<G, S, Q8>, &cfg) != cudaSuccess) {
         cudaGetLastError();  // a size the device cannot co-schedule: never chosen
         n = 0;
       }
@@ -854,9 +968,9 @@ int choose_cluster(const Capacity& c, int pairs, int units) {
   return best;
 }
 
-template <int G, int S>
-cudaError_t launch_with(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
-                        size_t smem, int csize, bool pdl, cudaStream_t stream) {
+template <int G, int S, bool Q8>
+cudaError_t launch_with(const StepArgs& a, const StepMaps& maps, size_t smem, int csize, bool pdl,
+                        cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.batch * a.hkv) * csize);
   cfg.blockDim = dim3(kStepThreads);
@@ -871,7 +985,7 @@ cudaError_t launch_with(const StepArgs& a, const CUtensorMap& tm_k, const CUtens
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, step_kernel<G, S>, a, tm_k, tm_v, tm_p);
+  return cudaLaunchKernelEx(&cfg, step_kernel<G, S, Q8>, a, maps);
 }
 
 // Launch plan: the cluster size (choose_cluster) on the 3-stage ring, two
@@ -883,9 +997,8 @@ cudaError_t launch_with(const StepArgs& a, const CUtensorMap& tm_k, const CUtens
 // when the grid fills the GPU, early-resident clusters of the next launch
 // only skew where the rest are placed.  NOSA_CLUSTER_SIZE (1..16) and
 // NOSA_RING_STAGES (3 or 6) override the choices.
-template <int G>
-cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
-                          cudaStream_t stream) {
+template <int G, bool Q8>
+cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t stream) {
   const int pairs = a.batch * a.hkv;
   if (pairs <= 0) return cudaSuccess;
   // Work units of the longest pair: its selection's scoring chunks.  The
@@ -903,20 +1016,20 @@ cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUte
     const int n = v ? atoi(v) : 0;
     return n == kMinStages || n == kMaxStages ? n : 0;
   }();
-  const size_t smem3 = step_smem_bytes<G>(a, kMinStages), smem6 = step_smem_bytes<G>(a, kMaxStages);
+  const size_t smem3 = step_smem_bytes<G, kMinStages, Q8>(a), smem6 = step_smem_bytes<G, kMaxStages, Q8>(a);
   int csize, stages = kMinStages;
   bool pdl;
   {
     std::lock_guard<std::mutex> lock(g_plan_mu);
     const Capacity* c3 = nullptr;
-    cudaError_t e = capacity<G, kMinStages>(smem3, &c3);
+    cudaError_t e = capacity<G, kMinStages, Q8>(smem3, &c3);
     if (e != cudaSuccess) return e;
     csize = choose_cluster(*c3, pairs, units);
     if (forced_c && c3->max_clusters[forced_c] > 0) csize = forced_c;
     pdl = static_cast<int64_t>(pairs) * csize * 2 <= c3->slots;
     const Capacity* c6 = nullptr;
     const bool want6 = forced_s ? forced_s == kMaxStages : static_cast<int64_t>(pairs) * csize <= c3->sms;
-    if (want6 && capacity<G, kMaxStages>(smem6, &c6) == cudaSuccess && c6->max_clusters[csize] >= pairs) {
+    if (want6 && capacity<G, kMaxStages, Q8>(smem6, &c6) == cudaSuccess && c6->max_clusters[csize] >= pairs) {
       stages = kMaxStages;
       pdl = static_cast<int64_t>(pairs) * csize * 2 <= c6->slots;
     }
@@ -926,20 +1039,27 @@ cudaError_t launch_step_g(const StepArgs& a, const CUtensorMap& tm_k, const CUte
             G, pairs, units, csize, stages, static_cast<int>(pdl), c3->slots, c6 ? c6->max_clusters[csize] : -1);
 #endif
   }
-  if (stages == kMaxStages) return launch_with<G, kMaxStages>(a, tm_k, tm_v, tm_p, smem6, csize, pdl, stream);
-  return launch_with<G, kMinStages>(a, tm_k, tm_v, tm_p, smem3, csize, pdl, stream);
+  if (stages == kMaxStages) return launch_with<G, kMaxStages, Q8>(a, maps, smem6, csize, pdl, stream);
+  return launch_with<G, kMinStages, Q8>(a, maps, smem3, csize, pdl, stream);
+}
+
+template <int G>
+cudaError_t launch_step_q(const StepArgs& a, const StepMaps& maps, cudaStream_t stream) {
+  // The INT8 kernels only differ in what the attention tiles hold: scoring
+  // and selection alone use the bf16 instance.
+  if (a.kv_int8 && (a.mode & (kStepDecode | kStepAppend))) return launch_step_g<G, true>(a, maps, stream);
+  return launch_step_g<G, false>(a, maps, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_step(const StepArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v, const CUtensorMap& tm_p,
-                        cudaStream_t stream) {
+cudaError_t launch_step(const StepArgs& a, const StepMaps& maps, cudaStream_t stream) {
   switch (a.hq / a.hkv) {
-    case 1: return launch_step_g<1>(a, tm_k, tm_v, tm_p, stream);
-    case 2: return launch_step_g<2>(a, tm_k, tm_v, tm_p, stream);
-    case 4: return launch_step_g<4>(a, tm_k, tm_v, tm_p, stream);
-    case 8: return launch_step_g<8>(a, tm_k, tm_v, tm_p, stream);
-    case 16: return launch_step_g<16>(a, tm_k, tm_v, tm_p, stream);
+    case 1: return launch_step_q<1>(a, maps, stream);
+    case 2: return launch_step_q<2>(a, maps, stream);
+    case 4: return launch_step_q<4>(a, maps, stream);
+    case 8: return launch_step_q<8>(a, maps, stream);
+    case 16: return launch_step_q<16>(a, maps, stream);
     default: return cudaErrorInvalidValue;
   }
 }

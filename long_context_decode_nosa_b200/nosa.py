@@ -48,7 +48,8 @@ class nosa_params(ctypes.Structure):
                 ("head_dim", ctypes.c_int), ("pool_kernel", ctypes.c_int),
                 ("pool_stride", ctypes.c_int), ("block_size", ctypes.c_int),
                 ("local_blocks", ctypes.c_int), ("topk", ctypes.c_int),
-                ("softmax_scale", ctypes.c_float), ("pooled_bf16", ctypes.c_int)]
+                ("softmax_scale", ctypes.c_float), ("pooled_bf16", ctypes.c_int),
+                ("kv_int8", ctypes.c_int)]
 
     @property
     def group(self) -> int:
@@ -68,6 +69,8 @@ _I64 = ctypes.c_int64
 
 _SIGNATURES = {
     "nosa_default_params": (None, [_P]),
+    "nosa_kv_int8_bytes": (_SZ, [_I64, _I]),
+    "nosa_quantize_kv_int8": (_I, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "nosa_workspace_size": (_SZ, [_P, _I, _I]),
     "nosa_workspace_init": (_I, [_P, _SZ, _P]),
     "nosa_pool_append": (_I, [_P, _P, _P, _I64, _P, _P, _P, _I, _P, _I, _I, _P, _P, _P, _SZ, _P]),
@@ -119,9 +122,9 @@ def _check(rc: int, func: str):
 def params(num_q_heads: int = 16, num_kv_heads: int = 2, *, topk: int = 64,
            local_blocks: int = 16, softmax_scale: float = 0.0, head_dim: int = 128,
            pool_kernel: int = 32, pool_stride: int = 16, block_size: int = 64,
-           pooled_bf16: bool = False) -> nosa_params:
+           pooled_bf16: bool = False, kv_int8: bool = False) -> nosa_params:
     return nosa_params(num_q_heads, num_kv_heads, head_dim, pool_kernel, pool_stride, block_size,
-                       local_blocks, topk, softmax_scale, int(pooled_bf16))
+                       local_blocks, topk, softmax_scale, int(pooled_bf16), int(kv_int8))
 
 
 def _ptr(t: Optional[torch.Tensor], dtype=None, name="tensor", cuda=True):
@@ -142,6 +145,82 @@ def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Int8KvCache:
+    """An INT8 K or V cache (params kv_int8) in the buffer layout of nosa.h:
+    int8 codes [rows, Hkv, 128], then fp32 scales [Hkv, scale_stride]
+    (scale_stride = rows rounded up to 4).  Row r of head h holds the values
+    scales[h, r] * codes[r, h, :].  Pass it wherever a call takes k_cache or
+    v_cache."""
+
+    def __init__(self, rows: int, num_kv_heads: int, device="cuda"):
+        n = lib().nosa_kv_int8_bytes(rows, num_kv_heads)
+        if n == 0:
+            raise NosaError(NOSA_ERR_INVALID_ARG, "nosa_kv_int8_bytes", "invalid rows / heads")
+        self.rows, self.num_kv_heads = rows, num_kv_heads
+        self.scale_stride = (rows + 3) // 4 * 4
+        self.buffer = torch.zeros(n, dtype=torch.uint8, device=device)
+
+    @property
+    def shape(self):
+        return (self.rows, self.num_kv_heads, 128)
+
+    @property
+    def is_cuda(self) -> bool:
+        return self.buffer.is_cuda
+
+    @property
+    def codes(self) -> torch.Tensor:
+        n = self.rows * self.num_kv_heads * 128
+        return self.buffer[:n].view(torch.int8).view(self.rows, self.num_kv_heads, 128)
+
+    @property
+    def scales(self) -> torch.Tensor:
+        off = self.rows * self.num_kv_heads * 128
+        n = self.num_kv_heads * self.scale_stride * 4
+        return self.buffer[off:off + n].view(torch.float32).view(self.num_kv_heads, self.scale_stride)
+
+    def row_scales(self) -> torch.Tensor:
+        """Scales as [rows, Hkv] (the token-major view)."""
+        return self.scales[:, :self.rows].t()
+
+    def clone(self) -> "Int8KvCache":
+        c = Int8KvCache.__new__(Int8KvCache)
+        c.rows, c.num_kv_heads, c.scale_stride = self.rows, self.num_kv_heads, self.scale_stride
+        c.buffer = self.buffer.clone()
+        return c
+
+    @classmethod
+    def from_bf16(cls, p: nosa_params, cache: torch.Tensor, stream=None) -> "Int8KvCache":
+        """Quantizes a whole bf16 cache [rows, Hkv, 128] on the GPU."""
+        c = cls(cache.shape[0], cache.shape[1], device=cache.device)
+        nosa_quantize_kv_int8(p, cache, c, stream=stream)
+        return c
+
+
+def nosa_quantize_kv_int8(p: nosa_params, src: torch.Tensor, cache: Int8KvCache, *, row0: int = 0, stream=None):
+    """Quantizes bf16 rows src [n, Hkv, 128] into rows row0 .. row0 + n - 1."""
+    if src.shape[1:] != (cache.num_kv_heads, 128):
+        raise ValueError("src must be [n, Hkv, 128] with the cache's Hkv")
+    rc = lib().nosa_quantize_kv_int8(ctypes.byref(p), _ptr(src, torch.bfloat16, "src"),
+                                     _ptr(cache.buffer, torch.uint8, "cache"), cache.rows, row0, src.shape[0],
+                                     _stream(stream))
+    _check(rc, "nosa_quantize_kv_int8")
+
+
+def _cache(p: nosa_params, c, name: str):
+    """Pointer of a K/V cache argument: a bf16 tensor, or an Int8KvCache when
+    params.kv_int8."""
+    if c is None:
+        return None
+    if p.kv_int8:
+        if not isinstance(c, Int8KvCache):
+            raise TypeError(f"{name} must be an Int8KvCache when params.kv_int8 is set")
+        return _ptr(c.buffer, torch.uint8, name)
+    if isinstance(c, Int8KvCache):
+        raise TypeError(f"{name} is an Int8KvCache but params.kv_int8 is not set")
+    return _ptr(c, torch.bfloat16, name)
 
 
 def n_windows(L: int) -> int:
@@ -180,7 +259,7 @@ def nosa_pool_append(p: nosa_params, k_cache: torch.Tensor, v_cache: Optional[to
                      ws: Optional[torch.Tensor] = None, stream=None):
     batch = len_new.shape[0]
     rc = lib().nosa_pool_append(
-        ctypes.byref(p), _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
+        ctypes.byref(p), _cache(p, k_cache, "k_cache"), _cache(p, v_cache, "v_cache"),
         k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"), _ptr(len_old, torch.int32, "len_old"),
         _ptr(len_new, torch.int32, "len_new"), batch, _ptr(pooled, p.pooled_dtype, "pooled"),
         pooled.shape[2], max_new_keys, _ptr(k_new, torch.bfloat16, "k_new"),
@@ -218,8 +297,8 @@ def nosa_sparse_decode(p: nosa_params, q: torch.Tensor, k_cache: torch.Tensor, v
         raise ValueError("sel_idx's last dimension must equal params.topk")
     batch = seq_len.shape[0]
     rc = lib().nosa_sparse_decode(
-        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
-        _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _cache(p, k_cache, "k_cache"),
+        _cache(p, v_cache, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
         _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len,
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
@@ -239,8 +318,8 @@ def nosa_decode_step_device(p: nosa_params, q: torch.Tensor, k_cache: torch.Tens
     batch = seq_len.shape[0]
     rc = lib().nosa_decode_step_device(
         ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
-        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(k_cache, torch.bfloat16, "k_cache"),
-        _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _cache(p, k_cache, "k_cache"),
+        _cache(p, v_cache, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
         _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len, _ptr(pooled, p.pooled_dtype, "pooled"),
         pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"),
@@ -266,7 +345,7 @@ def nosa_pool_append_paged(p: nosa_params, k_cache: torch.Tensor, v_cache: Optio
                            ws: Optional[torch.Tensor] = None, stream=None):
     batch = len_new.shape[0]
     rc = lib().nosa_pool_append_paged(
-        ctypes.byref(p), _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
+        ctypes.byref(p), _cache(p, k_cache, "k_cache"), _cache(p, v_cache, "v_cache"),
         _pages(k_cache), _ptr(page_table, torch.int32, "page_table"), page_table.shape[1],
         _ptr(len_old, torch.int32, "len_old"), _ptr(len_new, torch.int32, "len_new"), batch,
         _ptr(pooled, p.pooled_dtype, "pooled"), pooled.shape[2], max_new_keys,
@@ -283,8 +362,8 @@ def nosa_sparse_decode_paged(p: nosa_params, q: torch.Tensor, k_cache: torch.Ten
         raise ValueError("sel_idx's last dimension must equal params.topk")
     batch = seq_len.shape[0]
     rc = lib().nosa_sparse_decode_paged(
-        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_cache, torch.bfloat16, "k_cache"),
-        _ptr(v_cache, torch.bfloat16, "v_cache"), _pages(k_cache), _ptr(page_table, torch.int32, "page_table"),
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _cache(p, k_cache, "k_cache"),
+        _cache(p, v_cache, "v_cache"), _pages(k_cache), _ptr(page_table, torch.int32, "page_table"),
         page_table.shape[1], _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len,
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"),
@@ -303,8 +382,8 @@ def nosa_decode_step_device_paged(p: nosa_params, q: torch.Tensor, k_cache: torc
     batch = seq_len.shape[0]
     rc = lib().nosa_decode_step_device_paged(
         ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
-        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(k_cache, torch.bfloat16, "k_cache"),
-        _ptr(v_cache, torch.bfloat16, "v_cache"), _pages(k_cache), _ptr(page_table, torch.int32, "page_table"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _cache(p, k_cache, "k_cache"),
+        _cache(p, v_cache, "v_cache"), _pages(k_cache), _ptr(page_table, torch.int32, "page_table"),
         page_table.shape[1], _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len,
         _ptr(pooled, p.pooled_dtype, "pooled"), pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"),
         _ptr(sel_cnt, torch.int32, "sel_cnt"), _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
@@ -325,8 +404,8 @@ def nosa_decode_step_device_noalloc(p: nosa_params, q: torch.Tensor, k_cache: to
     batch = seq_len.shape[0]
     rc = lib().nosa_decode_step_device_noalloc(
         ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _ptr(k_new, torch.bfloat16, "k_new"),
-        _ptr(v_new, torch.bfloat16, "v_new"), _ptr(k_cache, torch.bfloat16, "k_cache"),
-        _ptr(v_cache, torch.bfloat16, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
+        _ptr(v_new, torch.bfloat16, "v_new"), _cache(p, k_cache, "k_cache"),
+        _cache(p, v_cache, "v_cache"), k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"),
         _ptr(seq_len, torch.int32, "seq_len"), batch, max_seq_len, _ptr(pooled, p.pooled_dtype, "pooled"),
         pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _stream(stream))
@@ -346,7 +425,7 @@ def nosa_decode_step(p: nosa_params, q_host: torch.Tensor, k_new_host: torch.Ten
         _ptr(k_new_host, torch.bfloat16, "k_new_host", cuda=False),
         _ptr(v_new_host, torch.bfloat16, "v_new_host", cuda=False),
         _ptr(out_host, torch.bfloat16, "out_host", cuda=False),
-        _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
+        _cache(p, k_cache, "k_cache"), _cache(p, v_cache, "v_cache"),
         k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"), _ptr(seq_len, torch.int32, "seq_len"),
         batch, max_seq_len, _ptr(pooled, p.pooled_dtype, "pooled"), pooled.shape[2],
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),

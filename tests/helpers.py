@@ -34,21 +34,40 @@ def sub_batch(b: inputs.DecodeBatch, seqs) -> inputs.DecodeBatch:
                               b.num_q_heads, b.num_kv_heads, b.head_dim)
 
 
-def oracle_step(b: inputs.DecodeBatch, topk: int, *, local_blocks: int = 16, scale=None, pooled_bf16=False):
-    """Pool every window, then the whole selection + attention, on the oracle."""
+def oracle_int8_caches(b: inputs.DecodeBatch):
+    """The oracle's own INT8 quantization of b's caches: (k_codes, k_scales,
+    v_codes, v_scales), scales [T, Hkv]."""
+    kc, ks = oracle.quantize_int8(inputs.bf16_bits(b.k_cache))
+    vc, vs = oracle.quantize_int8(inputs.bf16_bits(b.v_cache))
+    return kc, ks, vc, vs
+
+
+def oracle_step(b: inputs.DecodeBatch, topk: int, *, local_blocks: int = 16, scale=None, pooled_bf16=False,
+                kv_int8=None):
+    """Pool every window, then the whole selection + attention, on the oracle.
+    ``kv_int8``: the caches as (k_codes, k_scales, v_codes, v_scales) (the
+    INT8 cache variant) instead of b's bf16 caches."""
     kb = inputs.bf16_bits(b.k_cache)
     lens = b.seq_len.cpu().numpy()
     nc_cap = max(1, oracle.n_windows(int(lens.max())))
-    pooled = oracle.pool(kb, b.seq_start.cpu().numpy(), lens, nc_cap, bf16=pooled_bf16)
+    if kv_int8 is not None:
+        kc, ks, vc, vs = kv_int8
+        pooled = oracle.pool_int8(kc, ks, b.seq_start.cpu().numpy(), lens, nc_cap, bf16=pooled_bf16)
+    else:
+        pooled = oracle.pool(kb, b.seq_start.cpu().numpy(), lens, nc_cap, bf16=pooled_bf16)
     nb_cap = oracle.n_blocks(int(lens.max()))
     s = oracle.comp_scores(inputs.bf16_bits(b.q), pooled, lens, num_kv_heads=b.num_kv_heads,
                            scale=scale)
     S = oracle.block_scores(s, lens, nb_cap, num_kv_heads=b.num_kv_heads,
                             local_blocks=local_blocks)
     idx, cnt = oracle.topk(S, lens, topk, local_blocks=local_blocks)
-    out, lse = oracle.sparse_attention(inputs.bf16_bits(b.q), kb, inputs.bf16_bits(b.v_cache),
-                                       b.seq_start.cpu().numpy(), lens, idx, cnt, scale=scale,
-                                       local_blocks=local_blocks)
+    if kv_int8 is not None:
+        out, lse = oracle.sparse_attention_int8(inputs.bf16_bits(b.q), kc, ks, vc, vs, b.seq_start.cpu().numpy(),
+                                                lens, idx, cnt, scale=scale, local_blocks=local_blocks)
+    else:
+        out, lse = oracle.sparse_attention(inputs.bf16_bits(b.q), kb, inputs.bf16_bits(b.v_cache),
+                                           b.seq_start.cpu().numpy(), lens, idx, cnt, scale=scale,
+                                           local_blocks=local_blocks)
     return dict(pooled=pooled, comp_scores=s, block_scores=S, sel_idx=idx, sel_cnt=cnt, out=out,
                 lse=lse)
 
