@@ -294,6 +294,47 @@ NOSA_API int nosa_decode_step_device_paged(const nosa_params* p, const void* q, 
                                            int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* ws,
                                            size_t ws_bytes, void* stream);
 
+/* Sparse prefill (the pages' NOSAS mode, "NOSA 技术架构解析" §1.3: sparse
+ * attention in prefill as well as decode; the pages give no separate prefill
+ * rule, so each prefill token follows the decode rule on its own prefix).
+ * For every sequence s and query row r of q_start[s] <= e < q_start[s+1]
+ * (e = q_start[s] + r), the token at position t = q_pos[s] + r:
+ *   L_e     = t + 1 (the prefix the token sees, itself included)
+ *   sel[e]  = steps 2-3 above for q[e] against sequence s's pooled keys, L_e
+ *   out[e]  = step 4 above over sequence s's cache with L_e and sel[e]
+ * i.e. causal, each token selecting its own top-k blocks among the
+ * candidates of its prefix plus its local window.
+ *   q        bf16 [total_q, Hq, head_dim] (rows of all sequences, packed)
+ *   q_start  int32 [batch + 1] (device) non-decreasing row offsets into q,
+ *            q_start[0] = 0, q_start[batch] = total_q
+ *   q_pos    int32 [batch] (device) position of each sequence's first row
+ *   k/v_cache, seq_start: as for nosa_sparse_decode (one start per
+ *            sequence); the caches must already hold tokens [0, q_pos[s] +
+ *            rows) of each sequence
+ *   pooled   [batch, Hkv, nc_cap, head_dim] per sequence, holding every
+ *            window complete within each sequence's prefix (append the new
+ *            rows' windows first with nosa_pool_append, len_old = q_pos,
+ *            len_new = q_pos + rows, max_new_keys >= rows / 16 + 1)
+ *   sel_idx  int32 [total_q, Hkv, topk], sel_cnt int32 [total_q, Hkv]
+ *   out      bf16 [total_q, Hq, head_dim]; lse fp32 [total_q, Hq] nullable
+ * Each entry runs as one decode query of the step kernel (scoring, top-k and
+ * attention, no append): the selection is the one nosa_block_select gives
+ * for that token with L_e, and the output equals nosa_sparse_decode's up to
+ * rounding (the cluster size, and so the split of the tiles and the bf16
+ * rounding of the softmax weights, depends on how many entries one launch
+ * holds).  The
+ * workspace (nosa_prefill_workspace_size bytes, 256-byte aligned, zeroed once
+ * with nosa_workspace_init) holds the status word, spilled block scores and
+ * the entries' lengths.  A position past max_seq_len sets NOSA_DEV_MAX_LEN;
+ * a row outside its sequence's q_start range (q_start not non-decreasing)
+ * sets NOSA_DEV_BAD_LENGTH; those entries are skipped. */
+NOSA_API size_t nosa_prefill_workspace_size(const nosa_params* p, int total_q, int max_seq_len);
+NOSA_API int nosa_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                                 int64_t cache_rows, const int64_t* seq_start, const int32_t* q_start,
+                                 const int32_t* q_pos, int batch, int total_q, int max_seq_len, const void* pooled,
+                                 int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 /* One whole decode step from HOST buffers (the pages' per-token decode,
  * steps 1-4 above in order): copies q_host (bf16 [batch, Hq, D]) and the new
  * token's k_new_host / v_new_host (bf16 [batch, Hkv, D]) to the device,

@@ -86,6 +86,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // buffers of the host-buffer step (q, new K/V rows, out).
 struct Layout {
   size_t status, spill, stage_q, stage_k, stage_v, stage_out, total;
+  size_t entry_len, entry_seq;  // sparse prefill: per-entry lengths and sequence indices (int32)
   int nb_spill;  // candidates per pair in `spill` (0: block scores stay in shared memory)
 };
 
@@ -109,6 +110,27 @@ Layout layout_of(const nosa_params* p, int batch, int max_seq_len) {
   off = round_up(off + kvbytes, 256);
   l.stage_out = off;
   off = round_up(off + qbytes, 256);
+  l.total = off;
+  return l;
+}
+
+// Workspace of a sparse prefill over `total_q` query entries: the status
+// word, spilled block scores per entry, the entries' lengths and sequences
+// (no host-buffer staging).
+Layout prefill_layout_of(const nosa_params* p, int total_q, int max_seq_len) {
+  Layout l{};
+  const size_t pairs = static_cast<size_t>(total_q) * p->num_kv_heads;
+  const int64_t ncand_max = nosa::n_candidates(max_seq_len, p->local_blocks);
+  l.nb_spill = ncand_max > nosa::kSmemBlockScores ? static_cast<int>(ncand_max) : 0;
+  size_t off = 0;
+  l.status = off;
+  off += 256;
+  l.spill = off;
+  off = round_up(off + pairs * static_cast<size_t>(l.nb_spill) * 4, 256);
+  l.entry_len = off;
+  off = round_up(off + static_cast<size_t>(total_q) * 4, 256);
+  l.entry_seq = off;
+  off = round_up(off + static_cast<size_t>(total_q) * 4, 256);
   l.total = off;
   return l;
 }
@@ -466,6 +488,48 @@ int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new
   return ok();
 }
 
+// Sparse prefill (NOSAS): every query row of every sequence is one entry of
+// the step kernel (selection + attention, no append) with its own length
+// (position + 1), reading its sequence's cache and pooled keys.
+int do_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                      int64_t cache_rows, const int64_t* seq_start, const int32_t* q_start, const int32_t* q_pos,
+                      int batch, int total_q, int max_seq_len, const void* pooled, int nc_cap, int32_t* sel_idx,
+                      int32_t* sel_cnt, void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (int rc = check_common(p, total_q, max_seq_len)) return rc;
+  if (batch < 1) return fail(NOSA_ERR_INVALID_ARG, "batch must be >= 1");
+  if (total_q == 0) return ok();
+  const Layout l = prefill_layout_of(p, total_q, max_seq_len);
+  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
+  if (!q_start || !q_pos) return fail(NOSA_ERR_INVALID_ARG, "q_start and q_pos must not be NULL");
+  if (!aligned(q_start, 4) || !aligned(q_pos, 4)) return fail(NOSA_ERR_INVALID_ARG, "q_start / q_pos must be 4-byte aligned");
+  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, q_start, sel_idx,
+                                 sel_cnt, out))
+    return rc;
+  if (!pooled || nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "pooled must not be NULL and nc_cap >= 1");
+  if (!aligned(pooled, 16)) return fail(NOSA_ERR_INVALID_ARG, "pooled must be 16-byte aligned");
+  int32_t* entry_len = at<int32_t>(ws, l.entry_len);
+  int32_t* entry_seq = at<int32_t>(ws, l.entry_seq);
+  cudaError_t e = nosa::launch_prefill_entries(q_start, q_pos, batch, total_q, entry_len, entry_seq, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill entries launch");
+  nosa::StepArgs s = step_args(p, q, entry_len, total_q, max_seq_len, sel_idx, sel_cnt, ws, l);
+  s.seq_of = entry_seq;
+  s.seq_start = seq_start;
+  s.cache_rows = cache_rows;
+  s.pooled = const_cast<void*>(pooled);
+  s.nc_cap = nc_cap;
+  s.out = static_cast<__nv_bfloat16*>(out);
+  s.lse = lse;
+  s.mode = nosa::kStepScore | nosa::kStepDecode;
+  set_int8(s, p, const_cast<void*>(k_cache), v_cache, cache_rows);
+  nosa::StepMaps maps;
+  memset(&maps, 0, sizeof maps);
+  if (int rc = encode_cache_maps(&maps, p, k_cache, v_cache, cache_rows)) return rc;
+  if (int rc = encode_pooled_map(&maps.p, pooled, batch, p->num_kv_heads, nc_cap, p->pooled_bf16 != 0)) return rc;
+  e = nosa::launch_step(s, maps, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse_prefill launch");
+  return ok();
+}
+
 }  // namespace
 
 namespace nosa {
@@ -524,6 +588,20 @@ int nosa_quantize_kv_int8(const nosa_params* p, const void* src, void* cache, in
 size_t nosa_workspace_size(const nosa_params* p, int batch, int max_seq_len) {
   if (check_params(p) != NOSA_OK || batch < 0 || max_seq_len < 1) return 0;
   return layout_of(p, batch, max_seq_len).total;
+}
+
+size_t nosa_prefill_workspace_size(const nosa_params* p, int total_q, int max_seq_len) {
+  if (check_params(p) != NOSA_OK || total_q < 0 || max_seq_len < 1) return 0;
+  return prefill_layout_of(p, total_q, max_seq_len).total;
+}
+
+int nosa_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                        int64_t cache_rows, const int64_t* seq_start, const int32_t* q_start, const int32_t* q_pos,
+                        int batch, int total_q, int max_seq_len, const void* pooled, int nc_cap, int32_t* sel_idx,
+                        int32_t* sel_cnt, void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_params(p)) return rc;
+  return do_sparse_prefill(p, q, k_cache, v_cache, cache_rows, seq_start, q_start, q_pos, batch, total_q, max_seq_len,
+                           pooled, nc_cap, sel_idx, sel_cnt, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream) {

@@ -50,7 +50,9 @@ constexpr int kStepAppend = 4;  // write the new token's K/V rows and pool the w
 struct StepArgs {
   const __nv_bfloat16* q;        // [batch, hq, 128]
   const int32_t* seq_len;        // [batch]
-  const int64_t* seq_start;      // [batch] (decode / append, contiguous caches; nullptr when paged)
+  const int32_t* seq_of;         // nullable: [batch] sequence of each entry (multi-query prefill); else entry i
+                                 // is sequence i.  seq_start / page_table / pooled rows are per sequence.
+  const int64_t* seq_start;      // [sequences] (decode / append, contiguous caches; nullptr when paged)
   const int32_t* page_table;     // [batch, max_pages] (paged caches; nullptr: contiguous)
   int max_pages;
   int64_t cache_rows;
@@ -106,6 +108,11 @@ struct StepMaps {
   CUtensorMap k, v, p, ks, vs;
 };
 cudaError_t launch_step(const StepArgs& a, const StepMaps& maps, cudaStream_t stream);
+// Entries of a multi-query prefill: for sequence s with query rows
+// [q_start[s], q_start[s+1]) at positions q_pos[s] + r, entry e = q_start[s]
+// + r gets seq_len[e] = q_pos[s] + r + 1 and seq_of[e] = s.
+cudaError_t launch_prefill_entries(const int32_t* q_start, const int32_t* q_pos, int batch, int total_q,
+                                   int32_t* seq_len, int32_t* seq_of, cudaStream_t stream);
 cudaError_t launch_quantize_int8(const __nv_bfloat16* src, int8_t* codes, float* scales, int64_t scale_stride,
                                  int64_t row0, int64_t rows, int hkv, cudaStream_t stream);
 cudaError_t launch_select_only(const SelectArgs& a, cudaStream_t stream);

@@ -237,16 +237,20 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 
   // ---------------------------------------------------------------- geometry
   // (identical in every CTA of the cluster)
+  // Entry i is one query (its own length L, q, selection and output); si is
+  // the sequence whose cache and pooled keys it reads (si = i except for
+  // the multi-query prefill, where many entries share one sequence).
   const int i = pair / a.hkv, g = pair % a.hkv;
   const bool uses_cache = decoding || appending;
   const int L = a.seq_len[i];
+  const int si = a.seq_of ? a.seq_of[i] : i;
   const bool paged = a.page_table != nullptr;
-  const int64_t start_i = uses_cache && !paged ? a.seq_start[i] : 0;  // issued with the length load
+  const int64_t start_i = uses_cache && !paged ? a.seq_start[si] : 0;  // issued with the length load
   const bool bad_len = L < 1 || L > a.max_seq_len;
   const int64_t seq_base = bad_len ? 0 : start_i;
   KvRows kv;
   kv.base = seq_base;
-  kv.pages = paged ? a.page_table + static_cast<int64_t>(i) * a.max_pages : nullptr;
+  kv.pages = paged ? a.page_table + static_cast<int64_t>(si) * a.max_pages : nullptr;
   kv.num_pages = a.cache_rows / kPageTokens;
   const bool bad_rows = uses_cache && !bad_len &&
                         (paged ? static_cast<int64_t>(L) > static_cast<int64_t>(a.max_pages) * kPageTokens
@@ -328,7 +332,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       ok = __shfl_sync(0xffffffffu, good, 0) != 0;
       if (ok) ++r;
     };
-    const int row_base = pair * a.nc_cap;  // first pooled row of the pair (host: rows < 2^31)
+    const int row_base = (si * a.hkv + g) * a.nc_cap;  // first pooled row of the pair (host: rows < 2^31)
     for (int k = static_cast<int>(rank); k < nchunks && ok; k += static_cast<int>(C)) {
       issue([&](int s, uint8_t* st) {
         const int row0 = row_base + kChunkBlocks * kWindowsPerBlock * k - 1;
@@ -490,7 +494,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           const uint2* knew = a.k_new ? reinterpret_cast<const uint2*>(
                                             a.k_new + (static_cast<int64_t>(i) * a.hkv + g) * kHeadDim)
                                       : nullptr;
-          const int64_t at = (static_cast<int64_t>(pair) * a.nc_cap + j) * kHeadDim;
+          const int64_t at = ((static_cast<int64_t>(si) * a.hkv + g) * a.nc_cap + j) * kHeadDim;
           void* dst = a.pooled_bf16 ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.pooled) + at)
                                     : static_cast<void*>(static_cast<float*>(a.pooled) + at);
           if (kv.page_ok(j * kPoolStride) && kv.page_ok(j * kPoolStride + kPoolKernel - 1)) {

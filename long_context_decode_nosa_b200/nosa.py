@@ -70,6 +70,8 @@ _I64 = ctypes.c_int64
 _SIGNATURES = {
     "nosa_default_params": (None, [_P]),
     "nosa_kv_int8_bytes": (_SZ, [_I64, _I]),
+    "nosa_prefill_workspace_size": (_SZ, [_P, _I, _I]),
+    "nosa_sparse_prefill": (_I, [_P, _P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "nosa_quantize_kv_int8": (_I, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "nosa_workspace_size": (_SZ, [_P, _I, _I]),
     "nosa_workspace_init": (_I, [_P, _SZ, _P]),
@@ -325,6 +327,40 @@ def nosa_decode_step_device(p: nosa_params, q: torch.Tensor, k_cache: torch.Tens
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"),
         ws.numel(), _stream(stream))
     _check(rc, "nosa_decode_step_device")
+
+
+# ----------------------------------------------------------------------------- sparse prefill
+
+def prefill_workspace(p: nosa_params, total_q: int, max_seq_len: int, device="cuda", stream=None) -> torch.Tensor:
+    """A zero-initialised workspace for nosa_sparse_prefill over total_q query rows."""
+    n = lib().nosa_prefill_workspace_size(ctypes.byref(p), total_q, max_seq_len)
+    if n == 0:
+        raise NosaError(NOSA_ERR_INVALID_ARG, "nosa_prefill_workspace_size", "invalid parameters")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    nosa_workspace_init(ws, stream)
+    return ws
+
+
+def nosa_sparse_prefill(p: nosa_params, q: torch.Tensor, k_cache, v_cache, seq_start: torch.Tensor,
+                        q_start: torch.Tensor, q_pos: torch.Tensor, max_seq_len: int, pooled: torch.Tensor,
+                        sel_idx: torch.Tensor, sel_cnt: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, *,
+                        lse: Optional[torch.Tensor] = None, stream=None):
+    """Sparse prefill: every row of q (sequence s owns rows q_start[s] ..
+    q_start[s+1]-1 at positions q_pos[s] + r) is a decode query of its own
+    prefix (L = position + 1) against sequence s's cache and pooled keys."""
+    if sel_idx.shape[-1] != p.topk:
+        raise ValueError("sel_idx's last dimension must equal params.topk")
+    batch = q_pos.shape[0]
+    if q_start.shape[0] != batch + 1:
+        raise ValueError("q_start must have batch + 1 entries")
+    rc = lib().nosa_sparse_prefill(
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _cache(p, k_cache, "k_cache"), _cache(p, v_cache, "v_cache"),
+        k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"), _ptr(q_start, torch.int32, "q_start"),
+        _ptr(q_pos, torch.int32, "q_pos"), batch, q.shape[0], max_seq_len, _ptr(pooled, p.pooled_dtype, "pooled"),
+        pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
+        _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream))
+    _check(rc, "nosa_sparse_prefill")
 
 
 # ----------------------------------------------------------------------------- paged KV cache

@@ -255,3 +255,32 @@ def decode_step(q, k_cache, v_cache, seq_start, seq_len, pooled, topk_blocks, *,
                                 block_size=block_size, local_blocks=local_blocks)
     return {"comp_scores": s, "block_scores": S, "sel_idx": idx, "sel_cnt": cnt,
             "out": out, "lse": lse}
+
+
+def sparse_prefill(q, k_cache, v_cache, seq_start, q_start, q_pos, pooled, topk_blocks, *, scale=None,
+                   kernel=32, stride=16, block_size=64, local_blocks=16):
+    """Sparse prefill (the NOSAS mode): every query row e of sequence s (rows
+    q_start[s] .. q_start[s+1]-1, positions q_pos[s] + r) is one decode step
+    of its own prefix, L = position + 1, against sequence s's cache and
+    pooled keys -- ``decode_step`` applied token by token.  ``pooled``
+    [batch, Hkv, nc_cap, D] must hold every window of each prefix.  Returns
+    (sel_idx [total_q, Hkv, topk], sel_cnt [total_q, Hkv], out fp64
+    [total_q, Hq, D], lse fp64 [total_q, Hq])."""
+    q = _c(q, np.uint16)
+    total_q, hq, d = q.shape
+    hkv = k_cache.shape[1]
+    q_start = np.asarray(q_start, np.int64)
+    q_pos = np.asarray(q_pos, np.int64)
+    seq_start = np.asarray(seq_start, np.int64)
+    sel = np.full((total_q, hkv, topk_blocks), -1, np.int32)
+    cnt = np.zeros((total_q, hkv), np.int32)
+    out = np.zeros((total_q, hq, d), np.float64)
+    lse = np.zeros((total_q, hq), np.float64)
+    for s_ in range(len(q_pos)):
+        for e in range(int(q_start[s_]), int(q_start[s_ + 1])):
+            L = int(q_pos[s_]) + (e - int(q_start[s_])) + 1
+            r = decode_step(q[e:e + 1], k_cache, v_cache, seq_start[s_:s_ + 1], np.array([L], np.int32),
+                            pooled[s_:s_ + 1], topk_blocks, scale=scale, kernel=kernel, stride=stride,
+                            block_size=block_size, local_blocks=local_blocks)
+            sel[e], cnt[e], out[e], lse[e] = r["sel_idx"][0], r["sel_cnt"][0], r["out"][0], r["lse"][0]
+    return sel, cnt, out, lse

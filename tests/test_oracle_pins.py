@@ -506,3 +506,40 @@ def test_attention_int8_equals_attention_of_dequantized_cache(oracle_mod):
         l_ref = torch.logsumexp(logits.masked_fill(~m, -math.inf), dim=-1)[:, 0].numpy()
         np.testing.assert_allclose(out[0], o_ref, rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(lse[0], l_ref, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- sparse prefill
+
+def test_sparse_prefill_is_causal_attention_when_budget_covers_all(oracle_mod):
+    """With a top-k at least the number of candidates of every prefix, each
+    prefill token attends to exactly its whole prefix: the output is causal
+    attention (torch fp64 SDPA with a lower-triangular mask over the chunk's
+    rows), which pins the per-token length L = position + 1."""
+    lens = [2100, 1500]
+    b = inputs.make_batch(lens, num_q_heads=4, num_kv_heads=2, seed=31)
+    rows = [(1900, 200), (0, 1500)]                      # (first position, rows) per sequence
+    q_pos = np.array([r[0] for r in rows], np.int32)
+    q_start = np.concatenate([[0], np.cumsum([r[1] for r in rows])]).astype(np.int32)
+    total_q = int(q_start[-1])
+    gen = torch.Generator().manual_seed(32)
+    qf = torch.randn(total_q, 4, 128, generator=gen).to(torch.bfloat16)
+    nc_cap = oracle_mod.n_windows(max(lens))
+    pooled = oracle_mod.pool(_bits(b.k_cache), b.seq_start.numpy(), b.seq_len.numpy(), nc_cap)
+    topk = oracle_mod.n_candidates(max(lens))
+    sel, cnt, out, lse = oracle_mod.sparse_prefill(_bits(qf), _bits(b.k_cache), _bits(b.v_cache),
+                                                   b.seq_start.numpy(), q_start, q_pos, pooled, topk)
+    for s_, (p0, n) in enumerate(rows):
+        s0 = int(b.seq_start[s_])
+        Lmax = p0 + n
+        k = b.k_cache[s0:s0 + Lmax].double().permute(1, 0, 2).repeat_interleave(2, 0)   # [Hq, Lmax, D]
+        v = b.v_cache[s0:s0 + Lmax].double().permute(1, 0, 2).repeat_interleave(2, 0)
+        qq = qf[q_start[s_]:q_start[s_ + 1]].double().permute(1, 0, 2)                   # [Hq, n, D]
+        mask = torch.arange(Lmax)[None, :] <= (p0 + torch.arange(n))[:, None]           # [n, Lmax]
+        o_ref = F.scaled_dot_product_attention(qq, k, v, attn_mask=mask).permute(1, 0, 2).numpy()
+        np.testing.assert_allclose(out[q_start[s_]:q_start[s_ + 1]], o_ref, rtol=1e-10, atol=1e-12)
+        logits = (qq @ k.transpose(-1, -2)) / math.sqrt(128)
+        l_ref = torch.logsumexp(logits.masked_fill(~mask, -math.inf), dim=-1).t().numpy()
+        np.testing.assert_allclose(lse[q_start[s_]:q_start[s_ + 1]], l_ref, rtol=1e-12, atol=1e-12)
+        for e in range(q_start[s_], q_start[s_ + 1]):
+            L = p0 + (e - q_start[s_]) + 1
+            assert (cnt[e] == oracle_mod.n_candidates(L)).all()
