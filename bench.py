@@ -81,6 +81,9 @@ def parse():
                     help="pooled-key precision (bf16: the half-size variant)")
     ap.add_argument("--kv", choices=["bf16", "int8"], default="bf16",
                     help="K/V cache format (int8: codes + per-row scales, the 8-bit decode variant)")
+    ap.add_argument("--prefill", action="store_true",
+                    help="sparse prefill (NOSAS) of --batch sequences of --context tokens in --chunk-row chunks")
+    ap.add_argument("--chunk", type=int, default=4096, help="prefill chunk rows per sequence")
     ap.add_argument("--sweep", action="store_true",
                     help="NOSA-1B shape over context x batch x top-k (one JSON line per point)")
     return ap.parse_args()
@@ -620,6 +623,93 @@ def run_sweep(args):
     return 0
 
 
+def run_prefill(args):
+    """Sparse prefill (NOSAS): NOSA-1B attention shape, --batch sequences of
+    --context tokens, prefilled in chunks of --chunk rows; one prefill = per
+    chunk, the pool-append of the chunk's windows and one nosa_sparse_prefill
+    launch (every row a decode query of its own prefix).  K whole prefills
+    captured as one CUDA graph, CUDA events on the launching stream."""
+    from long_context_decode_nosa_b200 import nosa
+    nosa.lib()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    B = args.batch or 1
+    T = args.context or 16384
+    chunk = min(args.chunk, T)
+    topk = args.topk or 64
+    kv_int8 = args.kv == "int8"
+    p = nosa.params(16, 2, topk=topk, pooled_bf16=args.pooled == "bf16", kv_int8=kv_int8)
+    b = inputs.make_batch([T] * B, num_q_heads=16, num_kv_heads=2, seed=200, device=device)
+    kc, vc = b.k_cache, b.v_cache
+    if kv_int8:
+        kc, vc = nosa.Int8KvCache.from_bf16(p, kc), nosa.Int8KvCache.from_bf16(p, vc)
+    gen = torch.Generator(device=device).manual_seed(201)
+    q_all = torch.randn(B, T, 16, 128, generator=gen, device=device).to(torch.bfloat16)
+    nc_cap = max(1, nosa.n_windows(T))
+    pooled = torch.zeros(B, 2, nc_cap, 128, dtype=p.pooled_dtype, device=device)
+    ws_pool = nosa.workspace(p, B, T)
+    chunks = []
+    for c0 in range(0, T, chunk):
+        c1 = min(T, c0 + chunk)
+        n = c1 - c0
+        chunks.append(dict(
+            q=q_all[:, c0:c1].reshape(B * n, 16, 128).contiguous(),
+            q_start=torch.arange(0, B * n + 1, n, dtype=torch.int32, device=device),
+            q_pos=torch.full((B,), c0, dtype=torch.int32, device=device),
+            len_old=torch.full((B,), c0, dtype=torch.int32, device=device),
+            len_new=torch.full((B,), c1, dtype=torch.int32, device=device),
+            sel=torch.empty(B * n, 2, topk, dtype=torch.int32, device=device),
+            cnt=torch.empty(B * n, 2, dtype=torch.int32, device=device),
+            out=torch.empty(B * n, 16, 128, dtype=torch.bfloat16, device=device),
+            ws=nosa.prefill_workspace(p, B * n, T), n=n))
+
+    def prefill():
+        for c in chunks:
+            nosa.nosa_pool_append(p, kc, None, b.seq_start, c["len_new"], pooled, len_old=c["len_old"],
+                                  max_new_keys=c["n"] // 16 + 2, ws=ws_pool)
+            nosa.nosa_sparse_prefill(p, c["q"], kc, vc, b.seq_start, c["q_start"], c["q_pos"], T, pooled,
+                                     c["sel"], c["cnt"], c["out"], c["ws"])
+
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        prefill()
+    stream.synchronize()
+    for c in chunks:
+        rc, bits = nosa.nosa_read_device_status(c["ws"])
+        if rc:
+            raise SystemExit(f"sparse prefill reported device status 0x{bits:x}")
+    K = max(1, min(args.steps, 20))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(K):
+            prefill()
+    clocks = ClockSampler(0)
+    clocks.start()
+    with torch.cuda.stream(stream):
+        g.replay()
+        stream.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        stop = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        g.replay()
+        stop.record(stream)
+    stream.synchronize()
+    clk = clocks.stop()
+    ms = start.elapsed_time(stop) / K
+    tokens = B * T
+    line = {"metric": "sparse prefill tokens/s (NOSAS)", "value": tokens / (ms / 1e3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": K, "warmup": 1, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8+bf16" if kv_int8 else "bf16", "data": "synthetic",
+            "config": {"workload": f"NOSA-1B attention (16 q / 2 KV heads), {B} x {T}-token prefill in "
+                                   f"{chunk}-row chunks, top-k {topk} + 16 local blocks per token",
+                       "chunks": len(chunks), "pooled": args.pooled, "kv": args.kv},
+            "us_per_token": ms * 1e3 / tokens,
+            "gpu_launches": K * 2 * len(chunks), "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -628,6 +718,8 @@ def main():
         raise SystemExit("bench.py needs a CUDA device (B200); the CUDA path has no CPU fallback")
     if args.sweep:
         return run_sweep(args)
+    if args.prefill:
+        return run_prefill(args)
     return run_ours(args)
 
 
