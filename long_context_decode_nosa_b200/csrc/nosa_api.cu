@@ -519,7 +519,11 @@ int do_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache, 
   s.nc_cap = nc_cap;
   s.out = static_cast<__nv_bfloat16*>(out);
   s.lse = lse;
-  s.mode = nosa::kStepScore | nosa::kStepDecode;
+  // bf16 caches of sequences up to kPrefillMaxBlocks blocks: selection per
+  // entry in the step kernel, then the grouped attention kernel; otherwise
+  // the step kernel attends per entry as well.
+  const bool grouped = p->kv_int8 == 0 && nosa::n_blocks(max_seq_len) <= nosa::kPrefillMaxBlocks;
+  s.mode = grouped ? nosa::kStepScore : nosa::kStepScore | nosa::kStepDecode;
   set_int8(s, p, const_cast<void*>(k_cache), v_cache, cache_rows);
   nosa::StepMaps maps;
   memset(&maps, 0, sizeof maps);
@@ -527,6 +531,29 @@ int do_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache, 
   if (int rc = encode_pooled_map(&maps.p, pooled, batch, p->num_kv_heads, nc_cap, p->pooled_bf16 != 0)) return rc;
   e = nosa::launch_step(s, maps, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sparse_prefill launch");
+  if (grouped) {
+    nosa::PrefillAttnArgs pa{};
+    pa.q = static_cast<const __nv_bfloat16*>(q);
+    pa.entry_len = entry_len;
+    pa.entry_seq = entry_seq;
+    pa.seq_start = seq_start;
+    pa.cache_rows = cache_rows;
+    pa.sel_idx = sel_idx;
+    pa.sel_cnt = sel_cnt;
+    pa.out = static_cast<__nv_bfloat16*>(out);
+    pa.lse = lse;
+    pa.status = at<uint32_t>(ws, l.status);
+    pa.total_q = total_q;
+    pa.hq = p->num_q_heads;
+    pa.hkv = p->num_kv_heads;
+    pa.topk = p->topk;
+    pa.local_blocks = p->local_blocks;
+    pa.max_seq_len = max_seq_len;
+    pa.nb_words = static_cast<int>((nosa::n_blocks(max_seq_len) + 31) / 32);
+    pa.scale_log2 = s.scale_log2;
+    e = nosa::launch_prefill_attn(pa, maps.k, maps.v, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "sparse_prefill attention launch");
+  }
   return ok();
 }
 

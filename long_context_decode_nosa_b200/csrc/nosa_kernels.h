@@ -82,6 +82,27 @@ struct StepArgs {
   float scale_log2;  // softmax scale * log2(e)
 };
 
+// Attention of the sparse prefill over query groups (prefill_attn.cu).
+struct PrefillAttnArgs {
+  const __nv_bfloat16* q;     // [total_q, hq, 128]
+  const int32_t* entry_len;   // [total_q] L of each entry (position + 1)
+  const int32_t* entry_seq;   // [total_q] sequence of each entry
+  const int64_t* seq_start;   // [sequences] first cache row
+  int64_t cache_rows;
+  const int32_t* sel_idx;     // [total_q, hkv, topk]
+  const int32_t* sel_cnt;     // [total_q, hkv]
+  __nv_bfloat16* out;         // [total_q, hq, 128]
+  float* lse;                 // nullable: [total_q, hq]
+  uint32_t* status;
+  int total_q, hq, hkv, topk, local_blocks, max_seq_len;
+  int nb_words;               // 32-bit words of a block bitmap: ceil(nb(max_seq_len) / 32)
+  float scale_log2;
+};
+
+// Sequences up to this many blocks (256K tokens) use the grouped prefill
+// attention; longer ones run every entry through the step kernel.
+constexpr int kPrefillMaxBlocks = 4096;
+
 // Launches `kernel` with programmatic stream serialization, so that it can be
 // scheduled while the previous kernel on `stream` finishes (the kernels wait
 // on the dependency themselves before touching global memory).
@@ -113,6 +134,8 @@ cudaError_t launch_step(const StepArgs& a, const StepMaps& maps, cudaStream_t st
 // + r gets seq_len[e] = q_pos[s] + r + 1 and seq_of[e] = s.
 cudaError_t launch_prefill_entries(const int32_t* q_start, const int32_t* q_pos, int batch, int total_q,
                                    int32_t* seq_len, int32_t* seq_of, cudaStream_t stream);
+cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                cudaStream_t stream);
 cudaError_t launch_quantize_int8(const __nv_bfloat16* src, int8_t* codes, float* scales, int64_t scale_stride,
                                  int64_t row0, int64_t rows, int hkv, cudaStream_t stream);
 cudaError_t launch_select_only(const SelectArgs& a, cudaStream_t stream);
