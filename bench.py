@@ -35,6 +35,7 @@ import subprocess
 import sys
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -45,6 +46,7 @@ from long_context_decode_nosa_b200 import inputs, multirank  # noqa: E402
 
 METRIC = "sparse decode-attn queries/s and achieved HBM GB/s vs ~8 TB/s, 16K–64K ctx"
 UNIT = "queries/s"
+FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 
 WORKLOADS = {
@@ -240,6 +242,15 @@ def peak_hbm():
         return v, "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def peak_bf16():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def kernel_source_hash():
@@ -698,6 +709,34 @@ def run_prefill(args):
     clk = clocks.stop()
     ms = start.elapsed_time(stop) / K
     tokens = B * T
+    # Useful attention flops: every token's attended keys (its selected blocks
+    # and local window) x heads x (QK + PV) x 2.
+    keys = 0
+    for t in range(T):
+        L = t + 1
+        nb = -(-L // 64)
+        ncand = max(0, nb - 16)
+        keys += min(topk, ncand) * 64 + (L - 64 * ncand)
+    flops = 4.0 * 128 * 16 * keys * B
+    peak, peak_kind = peak_bf16()
+    achieved = flops / (ms / 1e3) / 1e12
+    # The oracle on a bounded sample: rows of the last chunk of sequence 0.
+    import oracle
+    nrows = 24
+    kb = inputs.bf16_bits(b.k_cache[:T].cpu())
+    vb = inputs.bf16_bits(b.v_cache[:T].cpu())
+    qs = inputs.bf16_bits(q_all[0, T - nrows:T].cpu())
+    pooled_h = oracle.pool(kb, np.array([0]), np.array([T], np.int32), nc_cap, bf16=args.pooled == "bf16")
+    threads = os.cpu_count() or 1
+    oracle.set_threads(threads)
+    t0 = time.perf_counter()
+    if kv_int8:
+        cpu_rows = None
+    else:
+        oracle.sparse_prefill(qs, kb, vb, np.array([0]), np.array([0, nrows]), np.array([T - nrows]), pooled_h,
+                              topk)
+        cpu_rows = nrows
+    cpu_s = time.perf_counter() - t0
     line = {"metric": "sparse prefill tokens/s (NOSAS)", "value": tokens / (ms / 1e3), "unit": "tokens/s",
             "n_gpus": 1, "steps": K, "warmup": 1, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8+bf16" if kv_int8 else "bf16", "data": "synthetic",
@@ -705,6 +744,13 @@ def run_prefill(args):
                                    f"{chunk}-row chunks, top-k {topk} + 16 local blocks per token",
                        "chunks": len(chunks), "pooled": args.pooled, "kv": args.kv},
             "us_per_token": ms * 1e3 / tokens,
+            "roofline": {"bound": "tensor", "kernel": "whole prefill (selection + grouped attention)",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_kind": f"{peak_kind} cuBLAS bf16", "traffic": None,
+                         "useful_flops_per_prefill": flops},
+            "cpu_baseline": None if cpu_rows is None else {
+                "value": cpu_rows / cpu_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                "sample": f"the last {cpu_rows} rows of a {T}-token prefill (decode rule per row, fp64 C oracle)"},
             "gpu_launches": K * 2 * len(chunks), "clocks": clk}
     print(json.dumps(line), flush=True)
     return 0
