@@ -76,10 +76,12 @@ def _run(nosa, g, p, q, q_start, q_pos, pooled, total_q, max_len):
     return sel, cnt, out, lse
 
 
-@pytest.mark.parametrize("hq,hkv,topk", [(16, 2, 16), (32, 8, 8), (8, 8, 4)])
+@pytest.mark.parametrize("hq,hkv,topk", [(16, 2, 16), (32, 8, 8), (8, 8, 4), (64, 4, 8), (4, 2, 12)])
 def test_sparse_prefill_matches_oracle(nosa, hq, hkv, topk):
     """Chunks at the start of a sequence, in its middle (crossing block and
-    local-window boundaries) and a single row; ragged lengths."""
+    local-window boundaries) and a single row; ragged lengths; every group
+    size (G = 8, 4, 1, 16, 2), so query groups of 8, 16, 64, 4 and 32 rows,
+    some holding rows of two sequences."""
     lens = [3000, 2600, 1200]
     rows = [(2900, 100), (0, 130), (1100, 1)]
     b, g, p, q, q_start, q_pos, pooled, total_q, lens_end = _setup(nosa, lens, rows, hq, hkv, topk, seed=41 + hq)
