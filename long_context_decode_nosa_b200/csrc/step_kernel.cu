@@ -175,10 +175,21 @@ struct MergeLayout {
   static constexpr int kPm = kMw + kConsumerWarps * G;               // [G] the CTA's row max
   static constexpr int kPl = kPm + G;                                // [G] the CTA's row sum
 };
-static_assert((MergeLayout<kMaxGroup>::kPl + kMaxGroup) * 4 <= kRingBytes, "merge scratch must fit in the ring");
+static_assert((MergeLayout<kMaxGroup>::kPl + kMaxGroup) * 4 <= 2 * kStageBytes,
+              "merge scratch must fit in the smallest ring (2 stages)");
+
+// Ring depths of a launch: the smaller one for two CTAs per SM, the larger
+// for one.  An INT8 stage carries two tiles plus their scale rows, so its
+// rings are 2 and 4 stages (4 and 8 tiles in flight): a 3-stage INT8 ring
+// with the scale slots no longer fits two CTAs per SM at long contexts.
+template <bool Q8>
+struct Rings {
+  static constexpr int kLo = Q8 ? 2 : kMinStages;
+  static constexpr int kHi = Q8 ? 4 : kMaxStages;
+};
 
 // S = ring stages: 3 (two CTAs per SM) or 6 (one CTA per SM, twice the
-// bytes in flight per CTA).
+// bytes in flight per CTA); with INT8 caches (Q8) 2 or 4 stages of two tiles.
 // Q8: the K/V caches are INT8 (codes + per-row scales).
 template <int G, int S, bool Q8>
 __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
@@ -904,7 +915,7 @@ cudaError_t capacity(size_t smem, const Capacity** out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   constexpr int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
-  Capacity& c = g_cap[gi][S == kMinStages ? 0 : 1][Q8 ? 1 : 0];
+  Capacity& c = g_cap[gi][S == Rings<Q8>::kLo ? 0 : 1][Q8 ? 1 : 0];
   if (c.dev != dev || c.smem != smem) {
     // The attribute is an upper bound: set to the largest size the device
     // allows next to the kernel's static shared memory, so that concurrent
@@ -1000,7 +1011,8 @@ cudaError_t launch_with(const StepArgs& a, const StepMaps& maps, size_t smem, in
 // next launch's clusters then become resident and run their prologue early;
 // when the grid fills the GPU, early-resident clusters of the next launch
 // only skew where the rest are placed.  NOSA_CLUSTER_SIZE (1..16) and
-// NOSA_RING_STAGES (3 or 6) override the choices.
+// NOSA_RING_STAGES (the smaller or the larger ring: 3 / 6, INT8 2 / 4)
+// override the choices.
 template <int G, bool Q8>
 cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t stream) {
   const int pairs = a.batch * a.hkv;
@@ -1017,24 +1029,25 @@ cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t 
   }();
   static const int forced_s = [] {
     const char* v = getenv("NOSA_RING_STAGES");
-    const int n = v ? atoi(v) : 0;
-    return n == kMinStages || n == kMaxStages ? n : 0;
+    return v ? atoi(v) : 0;
   }();
-  const size_t smem3 = step_smem_bytes<G, kMinStages, Q8>(a), smem6 = step_smem_bytes<G, kMaxStages, Q8>(a);
-  int csize, stages = kMinStages;
+  constexpr int kLo = Rings<Q8>::kLo, kHi = Rings<Q8>::kHi;
+  const size_t smem3 = step_smem_bytes<G, kLo, Q8>(a), smem6 = step_smem_bytes<G, kHi, Q8>(a);
+  int csize, stages = kLo;
   bool pdl;
   {
     std::lock_guard<std::mutex> lock(g_plan_mu);
     const Capacity* c3 = nullptr;
-    cudaError_t e = capacity<G, kMinStages, Q8>(smem3, &c3);
+    cudaError_t e = capacity<G, kLo, Q8>(smem3, &c3);
     if (e != cudaSuccess) return e;
     csize = choose_cluster(*c3, pairs, units);
     if (forced_c && c3->max_clusters[forced_c] > 0) csize = forced_c;
     pdl = static_cast<int64_t>(pairs) * csize * 2 <= c3->slots;
     const Capacity* c6 = nullptr;
-    const bool want6 = forced_s ? forced_s == kMaxStages : static_cast<int64_t>(pairs) * csize <= c3->sms;
-    if (want6 && capacity<G, kMaxStages, Q8>(smem6, &c6) == cudaSuccess && c6->max_clusters[csize] >= pairs) {
-      stages = kMaxStages;
+    const bool forced = forced_s == kLo || forced_s == kHi;
+    const bool want6 = forced ? forced_s == kHi : static_cast<int64_t>(pairs) * csize <= c3->sms;
+    if (want6 && capacity<G, kHi, Q8>(smem6, &c6) == cudaSuccess && c6->max_clusters[csize] >= pairs) {
+      stages = kHi;
       pdl = static_cast<int64_t>(pairs) * csize * 2 <= c6->slots;
     }
     cudaGetLastError();  // a 6-stage ring the device cannot host is simply not used
@@ -1043,8 +1056,8 @@ cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t 
             G, pairs, units, csize, stages, static_cast<int>(pdl), c3->slots, c6 ? c6->max_clusters[csize] : -1);
 #endif
   }
-  if (stages == kMaxStages) return launch_with<G, kMaxStages, Q8>(a, maps, smem6, csize, pdl, stream);
-  return launch_with<G, kMinStages, Q8>(a, maps, smem3, csize, pdl, stream);
+  if (stages == kHi) return launch_with<G, kHi, Q8>(a, maps, smem6, csize, pdl, stream);
+  return launch_with<G, kLo, Q8>(a, maps, smem3, csize, pdl, stream);
 }
 
 template <int G>
