@@ -529,9 +529,15 @@ def measure_e2e(nosa, wl: Workload, r: Replica, args, stream, info, device):
     if wl.layers > 1:
         return None
     b, st, p = r.b, r.st, r.p
-    q_h = b.q.cpu().pin_memory()
-    k_h = r.k_new.cpu().pin_memory()
-    v_h = r.v_new.cpu().pin_memory()
+    # q, k_new and v_new back to back in one pinned buffer (one copy per step)
+    nq, nk = b.q.numel(), r.k_new.numel()
+    packed = torch.empty(nq + 2 * nk, dtype=torch.bfloat16).pin_memory()
+    q_h = packed[:nq].view(b.q.shape)
+    k_h = packed[nq:nq + nk].view(r.k_new.shape)
+    v_h = packed[nq + nk:].view(r.v_new.shape)
+    q_h.copy_(b.q.cpu())
+    k_h.copy_(r.k_new.cpu())
+    v_h.copy_(r.v_new.cpu())
     o_h = torch.empty(wl.batch, wl.hq, 128, dtype=torch.bfloat16).pin_memory()
     n = max(10, min(args.steps, 500))
 

@@ -343,7 +343,9 @@ NOSA_API int nosa_sparse_prefill(const nosa_params* p, const void* q, const void
  * copies the bf16 output back to out_host.  seq_len (device) already counts
  * the new token.  All copies and kernels are enqueued on `stream`; the call
  * returns without waiting, so out_host is valid after the stream synchronises.
- * Host buffers should be pinned for the copies to be asynchronous.  The
+ * Host buffers should be pinned for the copies to be asynchronous; when
+ * q_host, k_new_host and v_new_host lie back to back in one host allocation
+ * (in that order) they travel in a single copy.  The
  * device staging area comes from `ws` (nosa_workspace_size covers it).  The
  * kernels run as in nosa_decode_step_device.
  * sel_idx / sel_cnt (device) receive the selection. */

@@ -157,10 +157,42 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// Recently encoded tensor maps of this host thread: a step re-encodes the
+// same K, V and pooled maps every call, and encoding costs microseconds of
+// host time per map.  Keyed by everything the encoding depends on.
+struct MapKey {
+  const void* base;
+  int64_t a, b;
+  int kind;
+  bool operator==(const MapKey& o) const { return base == o.base && a == o.a && b == o.b && kind == o.kind; }
+};
+struct MapCache {
+  static constexpr int kSlots = 16;
+  MapKey key[kSlots] = {};
+  CUtensorMap map[kSlots];
+  int next = 0;
+  const CUtensorMap* find(const MapKey& k) const {
+    for (int x = 0; x < kSlots; ++x)
+      if (key[x].base && key[x] == k) return &map[x];
+    return nullptr;
+  }
+  void put(const MapKey& k, const CUtensorMap& m) {
+    key[next] = k;
+    map[next] = m;
+    next = (next + 1) % kSlots;
+  }
+};
+thread_local MapCache g_maps;
+
 // 3-D map over a [rows, hkv, 128] cache: bf16 boxes of {64 dims, 1 head,
 // 64 tokens}, or INT8 boxes of {128 codes, 1 head, 64 tokens}; 128-byte rows
 // with the 128-byte swizzle, zero fill past `rows`.
 int encode_kv_map(CUtensorMap* map, const void* base, int hkv, int64_t rows, bool int8) {
+  const MapKey key{base, hkv, rows, int8 ? 1 : 0};
+  if (const CUtensorMap* hit = g_maps.find(key)) {
+    *map = *hit;
+    return NOSA_OK;
+  }
   auto enc = tensor_map_encoder();
   if (!enc) return fail(NOSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const cuuint64_t esize = int8 ? 1 : 2;
@@ -174,6 +206,7 @@ int encode_kv_map(CUtensorMap* map, const void* base, int hkv, int64_t rows, boo
                    const_cast<void*>(base), dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NOSA_ERR_INVALID_ARG, "tensor map encode failed (code %d)", static_cast<int>(r));
+  g_maps.put(key, *map);
   return NOSA_OK;
 }
 
@@ -182,6 +215,11 @@ int encode_kv_map(CUtensorMap* map, const void* base, int hkv, int64_t rows, boo
 // aligned token at or below its first row), no swizzle, zero fill past the
 // row.
 int encode_scale_map(CUtensorMap* map, const void* cache, int hkv, int64_t rows) {
+  const MapKey key{cache, hkv, rows, 2};
+  if (const CUtensorMap* hit = g_maps.find(key)) {
+    *map = *hit;
+    return NOSA_OK;
+  }
   auto enc = tensor_map_encoder();
   if (!enc) return fail(NOSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const int64_t stride = nosa::int8_scale_stride(rows);
@@ -193,6 +231,7 @@ int encode_scale_map(CUtensorMap* map, const void* cache, int hkv, int64_t rows)
                    elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NOSA_ERR_INVALID_ARG, "scale tensor map encode failed (code %d)", static_cast<int>(r));
+  g_maps.put(key, *map);
   return NOSA_OK;
 }
 
@@ -225,6 +264,11 @@ void set_int8(Args& a, const nosa_params* p, void* k_cache, const void* v_cache,
 // boxes of 128-byte rows ({32 fp32 or 64 bf16 columns, 61 rows}: one slice of
 // one scoring chunk), 128-byte swizzle, zero fill past the last row.
 int encode_pooled_map(CUtensorMap* map, const void* pooled, int batch, int hkv, int nc_cap, bool bf16) {
+  const MapKey key{pooled, static_cast<int64_t>(batch) * hkv, nc_cap, bf16 ? 4 : 3};
+  if (const CUtensorMap* hit = g_maps.find(key)) {
+    *map = *hit;
+    return NOSA_OK;
+  }
   auto enc = tensor_map_encoder();
   if (!enc) return fail(NOSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   const cuuint64_t rows = static_cast<cuuint64_t>(batch) * hkv * nc_cap;
@@ -241,6 +285,7 @@ int encode_pooled_map(CUtensorMap* map, const void* pooled, int batch, int hkv, 
                    elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NOSA_ERR_INVALID_ARG, "pooled tensor map encode failed (code %d)", static_cast<int>(r));
+  g_maps.put(key, *map);
   return NOSA_OK;
 }
 
@@ -748,9 +793,33 @@ int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new
   void* dv = at<void>(ws, l.stage_v);
   void* dout = at<void>(ws, l.stage_out);
   cudaError_t e;
-  if ((e = cudaMemcpyAsync(dq, q_host, qbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy q");
-  if ((e = cudaMemcpyAsync(dk, k_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy k_new");
-  if ((e = cudaMemcpyAsync(dv, v_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy v_new");
+  // The staging area holds q, k_new and v_new back to back (each a multiple
+  // of 256 bytes), so inputs that are back to back in host memory too go in
+  // one copy.
+  // Back-to-back addresses can still be separate pinned allocations, which
+  // one copy may not span: the runtime then refuses the copy up front
+  // (invalid value, nothing enqueued) and the three copies run instead.
+  const char* hq = static_cast<const char*>(q_host);
+  bool one_copy = static_cast<const char*>(k_new_host) == hq + qbytes &&
+                  static_cast<const char*>(v_new_host) == hq + qbytes + kvbytes &&
+                  static_cast<char*>(dk) == static_cast<char*>(dq) + qbytes &&
+                  static_cast<char*>(dv) == static_cast<char*>(dk) + kvbytes;
+  if (one_copy) {
+    e = cudaMemcpyAsync(dq, q_host, qbytes + 2 * kvbytes, cudaMemcpyHostToDevice, s);
+    if (e == cudaErrorInvalidValue) {
+      cudaGetLastError();
+      one_copy = false;
+    } else if (e != cudaSuccess) {
+      return cuda_fail(e, "copy q, k_new, v_new");
+    }
+  }
+  if (!one_copy) {
+    if ((e = cudaMemcpyAsync(dq, q_host, qbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy q");
+    if ((e = cudaMemcpyAsync(dk, k_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+      return cuda_fail(e, "copy k_new");
+    if ((e = cudaMemcpyAsync(dv, v_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+      return cuda_fail(e, "copy v_new");
+  }
   int rc = do_decode_step_device(p, dq, dk, dv, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, seq_len,
                                  batch, max_seq_len,
                                  pooled, nc_cap, sel_idx, sel_cnt, dout, nullptr, ws, ws_bytes, s);
