@@ -334,6 +334,15 @@ NOSA_API int nosa_sparse_prefill(const nosa_params* p, const void* q, const void
                                  const int32_t* q_pos, int batch, int total_q, int max_seq_len, const void* pooled,
                                  int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* ws,
                                  size_t ws_bytes, void* stream);
+/* The same over a paged cache (see the paged calls above): (num_pages,
+ * page_table, max_pages) in place of (cache_rows, seq_start); results are
+ * bit-identical to the contiguous call on the same tokens. */
+NOSA_API int nosa_sparse_prefill_paged(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                                       int64_t num_pages, const int32_t* page_table, int max_pages,
+                                       const int32_t* q_start, const int32_t* q_pos, int batch, int total_q,
+                                       int max_seq_len, const void* pooled, int nc_cap, int32_t* sel_idx,
+                                       int32_t* sel_cnt, void* out, float* lse, void* ws, size_t ws_bytes,
+                                       void* stream);
 
 /* One whole decode step from HOST buffers (the pages' per-token decode,
  * steps 1-4 above in order): copies q_host (bf16 [batch, Hq, D]) and the new

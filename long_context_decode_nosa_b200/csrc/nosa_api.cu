@@ -537,7 +537,7 @@ int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new
 // the step kernel (selection + attention, no append) with its own length
 // (position + 1), reading its sequence's cache and pooled keys.
 int do_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
-                      int64_t cache_rows, const int64_t* seq_start, const int32_t* q_start, const int32_t* q_pos,
+                      int64_t cache_rows, const KvLayout& kvl, const int32_t* q_start, const int32_t* q_pos,
                       int batch, int total_q, int max_seq_len, const void* pooled, int nc_cap, int32_t* sel_idx,
                       int32_t* sel_cnt, void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (int rc = check_common(p, total_q, max_seq_len)) return rc;
@@ -547,9 +547,7 @@ int do_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache, 
   if (int rc = check_ws(ws, ws_bytes, l)) return rc;
   if (!q_start || !q_pos) return fail(NOSA_ERR_INVALID_ARG, "q_start and q_pos must not be NULL");
   if (!aligned(q_start, 4) || !aligned(q_pos, 4)) return fail(NOSA_ERR_INVALID_ARG, "q_start / q_pos must be 4-byte aligned");
-  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, q_start, sel_idx,
-                                 sel_cnt, out))
-    return rc;
+  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, kvl, q_start, sel_idx, sel_cnt, out)) return rc;
   if (!pooled || nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "pooled must not be NULL and nc_cap >= 1");
   if (!aligned(pooled, 16)) return fail(NOSA_ERR_INVALID_ARG, "pooled must be 16-byte aligned");
   int32_t* entry_len = at<int32_t>(ws, l.entry_len);
@@ -558,7 +556,9 @@ int do_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache, 
   if (e != cudaSuccess) return cuda_fail(e, "prefill entries launch");
   nosa::StepArgs s = step_args(p, q, entry_len, total_q, max_seq_len, sel_idx, sel_cnt, ws, l);
   s.seq_of = entry_seq;
-  s.seq_start = seq_start;
+  s.seq_start = kvl.seq_start;
+  s.page_table = kvl.page_table;
+  s.max_pages = kvl.max_pages;
   s.cache_rows = cache_rows;
   s.pooled = const_cast<void*>(pooled);
   s.nc_cap = nc_cap;
@@ -581,7 +581,9 @@ int do_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache, 
     pa.q = static_cast<const __nv_bfloat16*>(q);
     pa.entry_len = entry_len;
     pa.entry_seq = entry_seq;
-    pa.seq_start = seq_start;
+    pa.seq_start = kvl.seq_start;
+    pa.page_table = kvl.page_table;
+    pa.max_pages = kvl.max_pages;
     pa.cache_rows = cache_rows;
     pa.sel_idx = sel_idx;
     pa.sel_cnt = sel_cnt;
@@ -672,8 +674,24 @@ int nosa_sparse_prefill(const nosa_params* p, const void* q, const void* k_cache
                         int batch, int total_q, int max_seq_len, const void* pooled, int nc_cap, int32_t* sel_idx,
                         int32_t* sel_cnt, void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
   if (int rc = check_params(p)) return rc;
-  return do_sparse_prefill(p, q, k_cache, v_cache, cache_rows, seq_start, q_start, q_pos, batch, total_q, max_seq_len,
-                           pooled, nc_cap, sel_idx, sel_cnt, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+  return do_sparse_prefill(p, q, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, q_start, q_pos, batch,
+                           total_q, max_seq_len, pooled, nc_cap, sel_idx, sel_cnt, out, lse, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int nosa_sparse_prefill_paged(const nosa_params* p, const void* q, const void* k_cache, const void* v_cache,
+                              int64_t num_pages, const int32_t* page_table, int max_pages, const int32_t* q_start,
+                              const int32_t* q_pos, int batch, int total_q, int max_seq_len, const void* pooled,
+                              int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* out, float* lse, void* ws,
+                              size_t ws_bytes, void* stream) {
+  if (int rc = check_params(p)) return rc;
+  if (!page_table) return fail(NOSA_ERR_INVALID_ARG, "page_table must not be NULL");
+  if (num_pages < 1 || num_pages >= (int64_t{1} << 31) / nosa::kPageTokens)
+    return fail(NOSA_ERR_UNSUPPORTED, "num_pages must be in [1, 2^31 / 64)");
+  return do_sparse_prefill(p, q, k_cache, v_cache, num_pages * nosa::kPageTokens,
+                           KvLayout{nullptr, page_table, max_pages}, q_start, q_pos, batch, total_q, max_seq_len,
+                           pooled, nc_cap, sel_idx, sel_cnt, out, lse, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int nosa_workspace_init(void* ws, size_t ws_bytes, void* stream) {

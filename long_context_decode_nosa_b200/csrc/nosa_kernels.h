@@ -87,7 +87,9 @@ struct PrefillAttnArgs {
   const __nv_bfloat16* q;     // [total_q, hq, 128]
   const int32_t* entry_len;   // [total_q] L of each entry (position + 1)
   const int32_t* entry_seq;   // [total_q] sequence of each entry
-  const int64_t* seq_start;   // [sequences] first cache row
+  const int64_t* seq_start;   // [sequences] first cache row (contiguous caches; nullptr when paged)
+  const int32_t* page_table;  // [sequences, max_pages] 64-token pages (paged caches; nullptr: contiguous)
+  int max_pages;
   int64_t cache_rows;
   const int32_t* sel_idx;     // [total_q, hkv, topk]
   const int32_t* sel_cnt;     // [total_q, hkv]

@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
   __shared__ int tok_seq[kTokens], tok_raw[kTokens], tok_raw_cnt[kTokens];  // loaded once per CTA
   __shared__ int tok_cnt[kTokens];  // selections used in the current segment
   __shared__ int seg_lo_blk, seg_hi_blk, seg_len;
+  __shared__ int sh_bad[kPfStages];  // the stage holds a tile whose page was invalid (masked)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.y;
@@ -182,7 +183,10 @@ __global__ void __launch_bounds__(kPfThreads, 2)
     const int sq = tok_seq[e_lo - e_begin];
     int e_hi = e_lo + 1;
     while (e_hi < e_end && tok_seq[e_hi - e_begin] == sq) ++e_hi;
-    const int64_t base = a.seq_start[sq];
+    // contiguous rows from seq_start, or 64-token pages through the table
+    const int64_t base = a.page_table ? 0 : a.seq_start[sq];
+    const int32_t* pages = a.page_table ? a.page_table + static_cast<int64_t>(sq) * a.max_pages : nullptr;
+    const int num_pages = static_cast<int>(a.cache_rows / kBlock);
     for (int x = tid; x < (kTokens + 1) * nbw; x += kPfThreads) sel_bm[x] = 0u;
     if (tid < kTokens) {
       const int e = e_begin + tid;
@@ -191,7 +195,8 @@ __global__ void __launch_bounds__(kPfThreads, 2)
         if (L < 1 || L > a.max_seq_len) {
           set_status(a.status, L < 1 ? NOSA_DEV_BAD_LENGTH : NOSA_DEV_MAX_LEN);
           L = 0;
-        } else if (base < 0 || base + L > a.cache_rows) {
+        } else if (pages ? static_cast<int64_t>(L) > static_cast<int64_t>(a.max_pages) * kBlock
+                         : base < 0 || base + L > a.cache_rows) {
           set_status(a.status, NOSA_DEV_CACHE_ROWS);
           L = 0;
         }
@@ -272,7 +277,19 @@ __global__ void __launch_bounds__(kPfThreads, 2)
               break;
             }
             uint8_t* st = smem + x * kStageBytes;
-            const int row = static_cast<int>(base + static_cast<int64_t>(b) * kBlock);
+            int row = static_cast<int>(base + static_cast<int64_t>(b) * kBlock);
+            if (pages) {
+              const int32_t pg = pages[b];
+              if (pg < 0 || pg >= num_pages) {
+                // an invalid page: stage the first page and mask the whole tile
+                set_status(a.status, NOSA_DEV_BAD_INDEX);
+                sh_bad[x] = 1;
+                row = 0;
+              } else {
+                sh_bad[x] = 0;
+                row = pg * kBlock;
+              }
+            }
             mbar_arrive_expect_tx(&full_bar[x], kTileTxBytes);
             tma_load_box(st, &tm_k, 0, g, row, &full_bar[x], policy);
             tma_load_box(st + kHalfBytes, &tm_k, 64, g, row, &full_bar[x], policy);
@@ -331,9 +348,10 @@ __global__ void __launch_bounds__(kPfThreads, 2)
               }
               pf_sync();
             }
-            const bool need0 = L0 > 0 && b < tok_nb[t0] &&
+            const bool bad = a.page_table != nullptr && sh_bad[x] != 0;
+            const bool need0 = !bad && L0 > 0 && b < tok_nb[t0] &&
                                (b >= tok_ncand[t0] || ((sel_bm[t0 * nbw + (b >> 5)] >> (b & 31)) & 1u));
-            const bool need1 = L1 > 0 && b < tok_nb[t1] &&
+            const bool need1 = !bad && L1 > 0 && b < tok_nb[t1] &&
                                (b >= tok_ncand[t1] || ((sel_bm[t1 * nbw + (b >> 5)] >> (b & 31)) & 1u));
             if (live && __any_sync(0xffffffffu, need0 || need1))
               attend_rows(att, qa, st, b, need0, need1, L0, L1, a.scale_log2, lane);

@@ -72,6 +72,8 @@ _SIGNATURES = {
     "nosa_kv_int8_bytes": (_SZ, [_I64, _I]),
     "nosa_prefill_workspace_size": (_SZ, [_P, _I, _I]),
     "nosa_sparse_prefill": (_I, [_P, _P, _P, _P, _I64, _P, _P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _SZ, _P]),
+    "nosa_sparse_prefill_paged": (_I, [_P, _P, _P, _P, _I64, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P,
+                                       _SZ, _P]),
     "nosa_quantize_kv_int8": (_I, [_P, _P, _P, _I64, _I64, _I64, _P]),
     "nosa_workspace_size": (_SZ, [_P, _I, _I]),
     "nosa_workspace_init": (_I, [_P, _SZ, _P]),
@@ -361,6 +363,26 @@ def nosa_sparse_prefill(p: nosa_params, q: torch.Tensor, k_cache, v_cache, seq_s
         _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
         _stream(stream))
     _check(rc, "nosa_sparse_prefill")
+
+
+def nosa_sparse_prefill_paged(p: nosa_params, q: torch.Tensor, k_cache, v_cache, page_table: torch.Tensor,
+                              q_start: torch.Tensor, q_pos: torch.Tensor, max_seq_len: int, pooled: torch.Tensor,
+                              sel_idx: torch.Tensor, sel_cnt: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, *,
+                              lse: Optional[torch.Tensor] = None, stream=None):
+    """nosa_sparse_prefill over a paged cache (page_table int32 [batch, max_pages])."""
+    if sel_idx.shape[-1] != p.topk:
+        raise ValueError("sel_idx's last dimension must equal params.topk")
+    batch = q_pos.shape[0]
+    if q_start.shape[0] != batch + 1 or page_table.shape[0] != batch:
+        raise ValueError("q_start must have batch + 1 entries and page_table batch rows")
+    rc = lib().nosa_sparse_prefill_paged(
+        ctypes.byref(p), _ptr(q, torch.bfloat16, "q"), _cache(p, k_cache, "k_cache"), _cache(p, v_cache, "v_cache"),
+        _pages(k_cache), _ptr(page_table, torch.int32, "page_table"), page_table.shape[1],
+        _ptr(q_start, torch.int32, "q_start"), _ptr(q_pos, torch.int32, "q_pos"), batch, q.shape[0], max_seq_len,
+        _ptr(pooled, p.pooled_dtype, "pooled"), pooled.shape[2], _ptr(sel_idx, torch.int32, "sel_idx"),
+        _ptr(sel_cnt, torch.int32, "sel_cnt"), _ptr(out, torch.bfloat16, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(rc, "nosa_sparse_prefill_paged")
 
 
 # ----------------------------------------------------------------------------- paged KV cache

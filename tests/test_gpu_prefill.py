@@ -179,3 +179,49 @@ def test_sparse_prefill_reports_rows_past_max_len(nosa):
     rc, bits = nosa.nosa_read_device_status(ws)
     assert rc == nosa.NOSA_ERR_DEVICE_CHECK and bits & nosa.NOSA_DEV_MAX_LEN
     assert (cnt[50:] == 0).all() and torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("kv_int8", [False, True])
+def test_sparse_prefill_paged_equals_contiguous(nosa, kv_int8):
+    """The same tokens in shuffled 64-token pages: selection, output and lse
+    bit-identical to the contiguous call (bf16 caches: grouped attention;
+    INT8: per-entry attention)."""
+    lens = [3000, 2600, 1200]
+    rows = [(2900, 100), (0, 130), (1100, 1)]
+    b, g, p, q, q_start, q_pos, pooled, total_q, _ = _setup(nosa, lens, rows, 16, 2, 16, seed=51, kv_int8=kv_int8)
+    sel, cnt, out, lse = _run(nosa, g, p, q, q_start, q_pos, pooled, total_q, max(lens))
+    # pages of the bf16 caches, quantized afresh for INT8 (same codes: per-row quantization)
+    cap = b.capacity.numpy()
+    need = [(int(c) + 63) // 64 for c in cap]
+    num_pages = sum(need) + 3
+    perm = np.random.default_rng(52).permutation(num_pages)
+    table = np.full((b.batch, max(need)), -1, np.int32)
+    src, dst, n = [], [], 0
+    for i in range(b.batch):
+        for pg in range(need[i]):
+            table[i, pg] = perm[n]
+            n += 1
+            t = np.arange(pg * 64, min(pg * 64 + 64, int(cap[i])))
+            src.append(int(b.seq_start[i]) + t)
+            dst.append(int(table[i, pg]) * 64 + t - pg * 64)
+    src = torch.from_numpy(np.concatenate(src)).to(DEV)
+    dst = torch.from_numpy(np.concatenate(dst)).to(DEV)
+    kb, vb = b.k_cache.to(DEV), b.v_cache.to(DEV)
+    kp = torch.zeros(num_pages * 64, 2, 128, dtype=torch.bfloat16, device=DEV)
+    vp = torch.zeros_like(kp)
+    kp[dst] = kb[src]
+    vp[dst] = vb[src]
+    if kv_int8:
+        kp, vp = nosa.Int8KvCache.from_bf16(p, kp), nosa.Int8KvCache.from_bf16(p, vp)
+    table_d = torch.from_numpy(table).to(DEV)
+    sel2 = torch.full_like(sel, -7)
+    cnt2 = torch.full_like(cnt, -7)
+    out2 = torch.empty_like(out)
+    lse2 = torch.empty_like(lse)
+    ws = nosa.prefill_workspace(p, total_q, max(lens))
+    nosa.nosa_sparse_prefill_paged(p, q.to(DEV), kp, vp, table_d, q_start.to(DEV), q_pos.to(DEV), max(lens), pooled,
+                                   sel2, cnt2, out2, ws, lse=lse2)
+    torch.cuda.synchronize()
+    _status_ok(nosa, ws)
+    assert torch.equal(sel, sel2) and torch.equal(cnt, cnt2)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
