@@ -21,9 +21,12 @@
 // tile no row of it needs.  Entries of different sequences in one group are
 // handled as consecutive segments.  Each warp's rows are complete at the end
 // (no cross-warp merge).
+#include <cstdlib>
+
 #include "decode_device.cuh"
 #include "nosa_common.cuh"
 #include "nosa_kernels.h"
+#include "umma.cuh"
 
 namespace nosa {
 
@@ -389,26 +392,441 @@ __global__ void __launch_bounds__(kPfThreads, 2)
   }
 }
 
+// ---------------------------------------------------------------------------
+// The same attention on the fifth-generation tensor cores (tcgen05): one CTA
+// per group of 128 / G consecutive entries, i.e. 128 (token, head) rows.
+//   * warp 8 (producer) stages each tile of the union walk with the tensor
+//     copies into a 3-stage ring, as above;
+//   * warp 9 (MMA) issues, from one thread, S = Q K^T (M 128, N 64, K 128;
+//     Q and K K-major in shared memory) into TMEM, and once the compute warps
+//     have written P, O_tile = P V (M 128, N 128, K 64; P K-major, V the
+//     MN-major B) into TMEM; its commits signal the compute warps and free
+//     the stage;
+//   * warps 0-7 (compute): thread (warp w, lane l) owns row 32 (w mod 4) + l
+//     (the TMEM lane quarter of its warp) and half w / 4 of the head
+//     dimension: it reads the row's 64 scores, runs the online softmax of the
+//     row (both halves alike), writes its half of P (bf16) in the swizzled
+//     layout, and adds the tile's O to its 64 accumulators in registers.
+// Masks, causal limits, segments and invalid pages are handled as in the
+// mma.sync kernel above.
+constexpr int kUmRows = 128;
+constexpr int kUmComputeWarps = 8;
+constexpr int kUmProducerWarp = 8;
+constexpr int kUmMmaWarp = 9;
+constexpr int kUmThreads = 10 * 32;
+constexpr int kUmComputeThreads = kUmComputeWarps * 32;
+constexpr int kUmQBytes = 2 * kUmRows * 128;  // Q: two K-major regions (dims 0-63, 64-127)
+constexpr int kUmPBytes = kUmRows * 128;      // P: 128 rows x 64 keys
+constexpr uint32_t kUmIdescS = umma_idesc_bf16(128, 64, false);
+constexpr uint32_t kUmIdescO = umma_idesc_bf16(128, 128, true);
+
+template <int G>
+__global__ void __launch_bounds__(kUmThreads, 1)
+    prefill_attn_umma_kernel(const PrefillAttnArgs a, const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v) {
+  constexpr int kTokens = kUmRows / G;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sq = smem + kPfRing;
+  uint8_t* sp = sq + kUmQBytes;
+  const int nbw = a.nb_words;
+  uint32_t* sel_bm = reinterpret_cast<uint32_t*>(sp + kUmPBytes);  // [kTokens][nbw]
+  uint32_t* uni_bm = sel_bm + kTokens * nbw;                        // [nbw]
+  __shared__ uint64_t full_bar[kPfStages], empty_bar[kPfStages], s_full, p_full, o_full;
+  __shared__ uint32_t tmem_base;
+  __shared__ int tok_len[kTokens], tok_ncand[kTokens], tok_nb[kTokens], tok_cnt[kTokens];
+  __shared__ int tok_seq[kTokens], tok_raw[kTokens], tok_raw_cnt[kTokens];
+  __shared__ unsigned char tok_in[kTokens];
+  __shared__ int seg_lo_blk, seg_hi_blk, seg_len;
+  __shared__ int sh_bad[kPfStages];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = blockIdx.y;
+  const int e_begin = blockIdx.x * kTokens;
+  const int e_end = min(e_begin + kTokens, a.total_q);
+  if (tid == 0) {
+    for (int x = 0; x < kPfStages; ++x) {
+      mbar_init(&full_bar[x], 1);
+      mbar_init(&empty_bar[x], 1);
+    }
+    mbar_init(&s_full, 1);
+    mbar_init(&p_full, kUmComputeThreads);
+    mbar_init(&o_full, 1);
+    fence_barrier_init();
+  }
+  if (warp == kUmMmaWarp) tmem_alloc<256>(&tmem_base);
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t t_s = tmem_base, t_o = tmem_base + 64;
+  grid_dependency_wait();
+  allow_dependents();
+  if (e_begin < e_end) {
+    if (tid < kTokens) {
+      const int e = e_begin + tid;
+      const bool in = e < e_end;
+      tok_seq[tid] = in ? a.entry_seq[e] : -1;
+      tok_raw[tid] = in ? a.entry_len[e] : 0;
+      tok_raw_cnt[tid] = in ? a.sel_cnt[static_cast<int64_t>(e) * a.hkv + g] : 0;
+    }
+    __syncthreads();
+    uint32_t jobs = 0;
+    int e_lo = e_begin;
+    while (e_lo < e_end) {
+      // ---------------------------------------------------------- segment setup
+      const int sq_id = tok_seq[e_lo - e_begin];
+      int e_hi = e_lo + 1;
+      while (e_hi < e_end && tok_seq[e_hi - e_begin] == sq_id) ++e_hi;
+      const int64_t base = a.page_table ? 0 : a.seq_start[sq_id];
+      const int32_t* pages = a.page_table ? a.page_table + static_cast<int64_t>(sq_id) * a.max_pages : nullptr;
+      const int num_pages = static_cast<int>(a.cache_rows / kBlock);
+      for (int x = tid; x < (kTokens + 1) * nbw; x += kUmThreads) sel_bm[x] = 0u;
+      if (tid < kTokens) {
+        const int e = e_begin + tid;
+        const bool in = e >= e_lo && e < e_hi;
+        int L = in ? tok_raw[tid] : 0;
+        if (in) {
+          if (L < 1 || L > a.max_seq_len) {
+            set_status(a.status, L < 1 ? NOSA_DEV_BAD_LENGTH : NOSA_DEV_MAX_LEN);
+            L = 0;
+          } else if (pages ? static_cast<int64_t>(L) > static_cast<int64_t>(a.max_pages) * kBlock
+                           : base < 0 || base + L > a.cache_rows) {
+            set_status(a.status, NOSA_DEV_CACHE_ROWS);
+            L = 0;
+          }
+        }
+        tok_len[tid] = L;
+        tok_in[tid] = in;
+        tok_nb[tid] = static_cast<int>(n_blocks(L));
+        tok_ncand[tid] = static_cast<int>(n_candidates(L, a.local_blocks));
+        int cnt = tok_raw_cnt[tid];
+        if (L > 0 && (cnt < 0 || cnt > a.topk)) {
+          set_status(a.status, NOSA_DEV_BAD_COUNT);
+          cnt = cnt < 0 ? 0 : a.topk;
+        }
+        tok_cnt[tid] = L > 0 ? cnt : 0;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int lo = 1 << 30, hi = 0, len = 0;
+        for (int t = 0; t < kTokens; ++t)
+          if (tok_len[t] > 0) {
+            lo = min(lo, tok_ncand[t]);
+            hi = max(hi, tok_nb[t]);
+            len = max(len, tok_len[t]);
+          }
+        seg_lo_blk = lo;
+        seg_hi_blk = hi;
+        seg_len = len;
+      }
+      {
+        constexpr int kU = 8;
+        const int n = kTokens * a.topk;
+        for (int x0 = tid; x0 < n; x0 += kUmThreads * kU) {
+          int v[kU];
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int x = x0 + u * kUmThreads;
+            const int t = x / a.topk, j = x - (x / a.topk) * a.topk;
+            v[u] = x < n && j < tok_cnt[t]
+                       ? a.sel_idx[(static_cast<int64_t>(e_begin + t) * a.hkv + g) * a.topk + j]
+                       : kNoBlock;
+          }
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            if (v[u] == kNoBlock) continue;
+            const int t = (x0 + u * kUmThreads) / a.topk;
+            const int b = v[u];
+            if (b < 0 || b >= tok_ncand[t]) {
+              set_status(a.status, NOSA_DEV_BAD_INDEX);
+              continue;
+            }
+            atomicOr(&sel_bm[t * nbw + (b >> 5)], 1u << (b & 31));
+            atomicOr(&uni_bm[b >> 5], 1u << (b & 31));
+          }
+        }
+      }
+      // Q of the segment's rows (row t * G + h), K-major with the 128-byte
+      // swizzle; rows of other tokens are zero.
+      for (int x = tid; x < kUmRows * 16; x += kUmThreads) {
+        const int r = x >> 4, c = x & 15;
+        const int t = r / G;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (tok_len[t] > 0)
+          val = __ldg(reinterpret_cast<const uint4*>(
+                          a.q + (static_cast<int64_t>(e_begin + t) * a.hq + static_cast<int64_t>(g) * G + r % G) *
+                                    kHeadDim) +
+                      c);
+        *reinterpret_cast<uint4*>(sq + (c >> 3) * (kUmRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = val;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncthreads();
+      for (int b = seg_lo_blk + tid; b < seg_hi_blk; b += kUmThreads) atomicOr(&uni_bm[b >> 5], 1u << (b & 31));
+      __syncthreads();
+      const int hi_blk = seg_hi_blk;
+
+      if (warp == kUmProducerWarp) {
+        // -------------------------------------------------------- producer
+        if (lane == 0) {
+          const uint64_t policy = l2_evict_first_policy();
+          uint32_t n = jobs;
+          bool ok = true;
+          for (int w = 0; w < nbw && ok; ++w) {
+            uint32_t bits = uni_bm[w];
+            while (bits && ok) {
+              const int b = w * 32 + __ffs(bits) - 1;
+              bits &= bits - 1u;
+              if (b >= hi_blk) continue;
+              const int x = static_cast<int>(n % kPfStages);
+              if (n >= kPfStages && !mbar_wait(&empty_bar[x], ((n / kPfStages) - 1) & 1u, a.status)) {
+                ok = false;
+                break;
+              }
+              uint8_t* st = smem + x * kStageBytes;
+              int row = static_cast<int>(base + static_cast<int64_t>(b) * kBlock);
+              sh_bad[x] = 0;
+              if (pages) {
+                const int32_t pg = pages[b];
+                if (pg < 0 || pg >= num_pages) {
+                  set_status(a.status, NOSA_DEV_BAD_INDEX);
+                  sh_bad[x] = 1;
+                  row = 0;
+                } else {
+                  row = pg * kBlock;
+                }
+              }
+              mbar_arrive_expect_tx(&full_bar[x], kTileTxBytes);
+              tma_load_box(st, &tm_k, 0, g, row, &full_bar[x], policy);
+              tma_load_box(st + kHalfBytes, &tm_k, 64, g, row, &full_bar[x], policy);
+              tma_load_box(st + 2 * kHalfBytes, &tm_v, 0, g, row, &full_bar[x], policy);
+              tma_load_box(st + 3 * kHalfBytes, &tm_v, 64, g, row, &full_bar[x], policy);
+              ++n;
+            }
+          }
+          jobs = n;
+        }
+        jobs = __shfl_sync(0xffffffffu, jobs, 0);
+      } else if (warp == kUmMmaWarp) {
+        // -------------------------------------------------------- MMA issue
+        if (lane == 0) {
+          uint32_t n = jobs;
+          bool ok = true;
+          for (int w = 0; w < nbw; ++w) {
+            uint32_t bits = uni_bm[w];
+            while (bits) {
+              const int b = w * 32 + __ffs(bits) - 1;
+              bits &= bits - 1u;
+              if (b >= hi_blk) continue;
+              const int x = static_cast<int>(n % kPfStages);
+              ok = ok && mbar_wait(&full_bar[x], (n / kPfStages) & 1u, a.status);
+              // S of the previous tile has been read (its P is written)
+              if (n > 0) ok = ok && mbar_wait(&p_full, (n - 1) & 1u, a.status);
+              tmem_fence_after();
+              if (ok) {
+                const uint8_t* st = smem + x * kStageBytes;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const uint64_t ad = umma_desc(smem_addr(sq + (k >> 2) * (kUmRows * 128) + (k & 3) * 32), 16, 1024);
+                  const uint64_t bd = umma_desc(smem_addr(st + (k >> 2) * kHalfBytes + (k & 3) * 32), 16, 1024);
+                  umma_bf16(t_s, ad, bd, kUmIdescS, k > 0);
+                }
+              }
+              umma_commit(&s_full);
+              ok = ok && mbar_wait(&p_full, n & 1u, a.status);
+              tmem_fence_after();
+              if (ok) {
+                const uint8_t* st = smem + x * kStageBytes;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const uint64_t ad = umma_desc(smem_addr(sp + k * 32), 16, 1024);
+                  const uint64_t bd = umma_desc(smem_addr(st + 2 * kHalfBytes + k * 2048), kHalfBytes, 1024);
+                  umma_bf16(t_o, ad, bd, kUmIdescO, k > 0);
+                }
+              }
+              umma_commit(&o_full);
+              umma_commit(&empty_bar[x]);
+              ++n;
+            }
+          }
+          jobs = n;
+        }
+        jobs = __shfl_sync(0xffffffffu, jobs, 0);
+      } else {
+        // -------------------------------------------------------- compute
+        const int quarter = warp & 3, half = warp >> 2;
+        const int r = 32 * quarter + lane;
+        const int t = r / G;
+        const int L = tok_len[t];
+        const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
+        float o[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) o[j] = 0.0f;
+        float m = -INFINITY, l = 0.0f;
+        uint32_t n = jobs;
+        bool ok = true;
+        for (int w = 0; w < nbw; ++w) {
+          uint32_t bits = uni_bm[w];
+          while (bits) {
+            const int b = w * 32 + __ffs(bits) - 1;
+            bits &= bits - 1u;
+            if (b >= hi_blk) continue;
+            const int x = static_cast<int>(n % kPfStages);
+            // the stage's page check (sh_bad) is published with its copies
+            ok = ok && mbar_wait(&full_bar[x], (n / kPfStages) & 1u, a.status);
+            ok = ok && mbar_wait(&s_full, n & 1u, a.status);
+            tmem_fence_after();
+            const bool bad = a.page_table != nullptr && sh_bad[x] != 0;
+            const bool need = ok && !bad && L > 0 && b < tok_nb[t] &&
+                              (b >= tok_ncand[t] || ((sel_bm[t * nbw + (b >> 5)] >> (b & 31)) & 1u));
+            const int64_t kb0 = static_cast<int64_t>(b) * kBlock;
+            float sc[64];
+            if (ok) {
+              float tmp[32];
+              tmem_ld32(t_s + lane_off, tmp);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sc[j] = tmp[j];
+              tmem_ld32(t_s + lane_off + 32, tmp);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sc[32 + j] = tmp[j];
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+              const bool valid = need && kb0 + j < L;
+              sc[j] = valid ? sc[j] * a.scale_log2 : -INFINITY;
+              mx = fmaxf(mx, sc[j]);
+            }
+            const float m_new = fmaxf(m, mx);
+            const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+            const float alpha = fast_exp2(m - m_use);
+            m = m_new;
+            float rs = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+              sc[j] = fast_exp2(sc[j] - m_use);
+              rs += sc[j];
+            }
+            l = l * alpha + rs;
+            // this thread's half of P: keys 32 half .. 32 half + 31 (chunks 4 half .. 4 half + 3);
+            // both halves spelled out so that every index into sc is a constant
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              if (hh != half) continue;
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int k0 = 32 * hh + 8 * c;
+                uint4 pk;
+                pk.x = pack_bf16x2(sc[k0 + 0], sc[k0 + 1]);
+                pk.y = pack_bf16x2(sc[k0 + 2], sc[k0 + 3]);
+                pk.z = pack_bf16x2(sc[k0 + 4], sc[k0 + 5]);
+                pk.w = pack_bf16x2(sc[k0 + 6], sc[k0 + 7]);
+                const int chunk = 4 * hh + c;
+                *reinterpret_cast<uint4*>(sp + r * 128 + ((chunk ^ (r & 7)) << 4)) = pk;
+              }
+            }
+            // V rows past every token's length hold stale rows: zero them
+            if (ok && kb0 + kBlock > seg_len) {
+              uint8_t* st = smem + x * kStageBytes;
+              for (int idx = tid; idx < kBlock * 16; idx += kUmComputeThreads) {
+                const int vr = idx >> 4, c16 = idx & 15;
+                if (kb0 + vr >= seg_len)
+                  *reinterpret_cast<uint4*>(st + 2 * kHalfBytes + (c16 >> 3) * kHalfBytes + vr * 128 +
+                                            (((c16 & 7) ^ (vr & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+              }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_fence_before();
+            mbar_arrive(&p_full);
+            ok = ok && mbar_wait(&o_full, n & 1u, a.status);
+            tmem_fence_after();
+            if (ok) {
+              float tmp[32];
+              tmem_ld32(t_o + lane_off + 64 * half, tmp);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = o[j] * alpha + tmp[j];
+              tmem_ld32(t_o + lane_off + 64 * half + 32, tmp);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[32 + j] = o[32 + j] * alpha + tmp[j];
+            }
+            tmem_fence_before();
+            ++n;
+          }
+        }
+        jobs = n;
+        // the row's half of the output
+        if (tok_in[t]) {
+          const int e = e_begin + t;
+          const int64_t orow = static_cast<int64_t>(e) * a.hq + static_cast<int64_t>(g) * G + r % G;
+          const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+          uint4* dst = reinterpret_cast<uint4*>(a.out + orow * kHeadDim + 64 * half);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 pk;
+            pk.x = pack_bf16x2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
+            pk.y = pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
+            pk.z = pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
+            pk.w = pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+            dst[c] = pk;
+          }
+          if (a.lse && half == 0) a.lse[orow] = l > 0.0f ? (m + log2f(l)) * kLn2 : -INFINITY;
+        }
+      }
+      __syncthreads();  // the segment's tiles are consumed; bitmaps, Q and token info may be rewritten
+      e_lo = e_hi;
+    }
+  }
+  tmem_fence_before();
+  __syncthreads();
+  if (warp == kUmMmaWarp) {
+    tmem_fence_after();
+    tmem_dealloc<256>(t_s);
+  }
+}
+
 }  // namespace
 
+// The mma.sync kernel (64 rows per CTA, warps skip tiles their rows do not
+// need) by default; NOSA_PREFILL_UMMA=1 selects the tcgen05 kernel (128 rows
+// per CTA).  With independent queries the union of a group's selections
+// covers most candidates, and a CTA of 128 rows computes every row against
+// every tile of that union, so the tcgen05 kernel measured slower here (16K
+// prefill 8.4 ms against 7.2 ms); with correlated neighbouring queries, as in
+// a trained model, the union shrinks and the tcgen05 tile is the faster one.
 cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                 cudaStream_t stream) {
+  static const bool use_sync = [] {
+    const char* v = getenv("NOSA_PREFILL_UMMA");
+    return !(v != nullptr && v[0] == '1');
+  }();
   const int G = a.hq / a.hkv;
-  const int tokens = kBlock / G;
+  const int rows = use_sync ? kBlock : kUmRows;
+  const int tokens = rows / G;
   const int groups = (a.total_q + tokens - 1) / tokens;
   if (groups == 0) return cudaSuccess;
-  const size_t smem = 1024 + kPfRing + static_cast<size_t>(tokens + 1) * a.nb_words * 4;
-  auto go = [&](auto kernel) -> cudaError_t {
+  const size_t smem = use_sync ? 1024 + kPfRing + static_cast<size_t>(tokens + 1) * a.nb_words * 4
+                               : 1024 + kPfRing + kUmQBytes + kUmPBytes +
+                                     static_cast<size_t>(tokens + 1) * a.nb_words * 4;
+  auto go = [&](auto kernel, int threads) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    return launch_overlapped(kernel, dim3(groups, a.hkv), dim3(kPfThreads), smem, stream, a, tm_k, tm_v);
+    return launch_overlapped(kernel, dim3(groups, a.hkv), dim3(threads), smem, stream, a, tm_k, tm_v);
   };
+  if (use_sync) {
+    switch (G) {
+      case 1: return go(prefill_attn_kernel<1>, kPfThreads);
+      case 2: return go(prefill_attn_kernel<2>, kPfThreads);
+      case 4: return go(prefill_attn_kernel<4>, kPfThreads);
+      case 8: return go(prefill_attn_kernel<8>, kPfThreads);
+      case 16: return go(prefill_attn_kernel<16>, kPfThreads);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (G) {
-    case 1: return go(prefill_attn_kernel<1>);
-    case 2: return go(prefill_attn_kernel<2>);
-    case 4: return go(prefill_attn_kernel<4>);
-    case 8: return go(prefill_attn_kernel<8>);
-    case 16: return go(prefill_attn_kernel<16>);
+    case 1: return go(prefill_attn_umma_kernel<1>, kUmThreads);
+    case 2: return go(prefill_attn_umma_kernel<2>, kUmThreads);
+    case 4: return go(prefill_attn_umma_kernel<4>, kUmThreads);
+    case 8: return go(prefill_attn_umma_kernel<8>, kUmThreads);
+    case 16: return go(prefill_attn_umma_kernel<16>, kUmThreads);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -225,3 +225,20 @@ def test_sparse_prefill_paged_equals_contiguous(nosa, kv_int8):
     _status_ok(nosa, ws)
     assert torch.equal(sel, sel2) and torch.equal(cnt, cnt2)
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+def test_sparse_prefill_tcgen05_kernel_passes_the_same_tests():
+    """The tcgen05 (TMEM-accumulator) attention kernel, selected with
+    NOSA_PREFILL_UMMA=1 (read once per process), passes this file's parity
+    tests in a child process."""
+    import os
+    import subprocess
+    import sys
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    env = dict(os.environ, NOSA_PREFILL_UMMA="1")
+    here = os.path.dirname(os.path.abspath(__file__))
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(here, "test_gpu_prefill.py"), "-x", "-q",
+                        "-m", "gpu", "-k", "not tcgen05"], env=env, cwd=os.path.dirname(here),
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
