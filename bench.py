@@ -81,6 +81,8 @@ def parse():
                     help="untimed repeated steps before timing, so clocks settle")
     ap.add_argument("--pooled", choices=["fp32", "bf16"], default="fp32",
                     help="pooled-key precision (bf16: the half-size variant)")
+    ap.add_argument("--paged", action="store_true",
+                    help="caches as shuffled 64-token pages through a page table (the paged entry points)")
     ap.add_argument("--kv", choices=["bf16", "int8"], default="bf16",
                     help="K/V cache format (int8: codes + per-row scales, the 8-bit decode variant)")
     ap.add_argument("--prefill", action="store_true",
@@ -115,8 +117,9 @@ class Workload:
         self.local_blocks = 16
         self.pooled_bf16 = getattr(args, "pooled", "fp32") == "bf16"
         self.kv_int8 = getattr(args, "kv", "bf16") == "int8"
+        self.paged = bool(getattr(args, "paged", False))
         self.desc = desc + (", bf16 pooled keys" if self.pooled_bf16 else "") + (
-            ", INT8 K/V cache" if self.kv_int8 else "")
+            ", INT8 K/V cache" if self.kv_int8 else "") + (", paged cache (shuffled 64-token pages)" if self.paged else "")
         if args.context or args.batch or args.topk:
             self.desc += f" [overridden: batch {self.batch}, context {max(self.lens)}, top-k {self.topk}]"
         self.max_len = max(self.lens)
@@ -151,13 +154,41 @@ class Replica:
                                    key_dist=wl.key_dist, device=device)
         self.p = nosa.params(wl.hq, wl.hkv, topk=wl.topk, local_blocks=wl.local_blocks, pooled_bf16=wl.pooled_bf16,
                              kv_int8=wl.kv_int8)
+        self.page_table = None
+        k_bf, v_bf = self.b.k_cache, self.b.v_cache
+        if wl.paged:     # the same tokens in randomly permuted 64-token pages (built untimed)
+            cap = self.b.capacity.cpu().tolist()
+            starts = self.b.seq_start.cpu().tolist()
+            need = [(c + 63) // 64 for c in cap]
+            perm = torch.randperm(sum(need), generator=torch.Generator().manual_seed(seed + 11))
+            table = torch.full((wl.batch, max(need)), -1, dtype=torch.int32)
+            src, dst, n = [], [], 0
+            for i in range(wl.batch):
+                for pg in range(need[i]):
+                    table[i, pg] = perm[n]
+                    n += 1
+                    t = torch.arange(pg * 64, min(pg * 64 + 64, cap[i]))
+                    src.append(starts[i] + t)
+                    dst.append(int(table[i, pg]) * 64 + t - pg * 64)
+            src = torch.cat(src).to(device)
+            dst = torch.cat(dst).to(device)
+            k_bf = torch.zeros(sum(need) * 64, wl.hkv, 128, dtype=torch.bfloat16, device=device)
+            v_bf = torch.zeros_like(k_bf)
+            k_bf[dst] = self.b.k_cache[src]
+            v_bf[dst] = self.b.v_cache[src]
+            self.page_table = table.to(device)
         if wl.kv_int8:   # the caches as the INT8 variant stores them (quantized on the GPU, untimed)
-            self.k_cache = nosa.Int8KvCache.from_bf16(self.p, self.b.k_cache)
-            self.v_cache = nosa.Int8KvCache.from_bf16(self.p, self.b.v_cache)
+            self.k_cache = nosa.Int8KvCache.from_bf16(self.p, k_bf)
+            self.v_cache = nosa.Int8KvCache.from_bf16(self.p, v_bf)
         else:
-            self.k_cache, self.v_cache = self.b.k_cache, self.b.v_cache
+            self.k_cache, self.v_cache = k_bf, v_bf
         self.st = nosa.DecodeState(self.p, wl.batch, wl.max_len, device=device)
-        self.st.rebuild_pooled(self.k_cache, self.b.seq_start, self.b.seq_len)
+        if wl.paged:
+            nosa.nosa_pool_append_paged(self.p, self.k_cache, None, self.page_table, self.b.seq_len, self.st.pooled,
+                                        len_old=torch.zeros_like(self.b.seq_len), max_new_keys=self.st.nc_cap,
+                                        ws=self.st.ws)
+        else:
+            self.st.rebuild_pooled(self.k_cache, self.b.seq_start, self.b.seq_len)
         self.k_new, self.v_new = inputs.random_kv_rows(wl.batch, wl.hkv, 128, seed=seed + 7,
                                                        device=device)
 
@@ -168,6 +199,26 @@ def step(nosa, r: Replica, events=None, fused=True):
     (nosa_decode_step_device); otherwise the three entry points in order, with
     ``events`` (4 CUDA events) recorded before each kernel and after the last."""
     b, st, p = r.b, r.st, r.p
+    if r.page_table is not None:
+        if fused:
+            nosa.nosa_decode_step_device_paged(p, b.q, r.k_cache, r.v_cache, r.page_table, b.seq_len,
+                                               st.max_seq_len, st.pooled, st.sel_idx, st.sel_cnt, st.out, st.ws,
+                                               k_new=r.k_new, v_new=r.v_new)
+            return
+        if events:
+            events[0].record()
+        nosa.nosa_pool_append_paged(p, r.k_cache, r.v_cache, r.page_table, b.seq_len, st.pooled, max_new_keys=1,
+                                    k_new=r.k_new, v_new=r.v_new, ws=st.ws)
+        if events:
+            events[1].record()
+        nosa.nosa_block_select(p, b.q, st.pooled, b.seq_len, st.max_seq_len, st.sel_idx, st.sel_cnt, st.ws)
+        if events:
+            events[2].record()
+        nosa.nosa_sparse_decode_paged(p, b.q, r.k_cache, r.v_cache, r.page_table, b.seq_len, st.max_seq_len,
+                                      st.sel_idx, st.sel_cnt, st.out, st.ws)
+        if events:
+            events[3].record()
+        return
     if fused:
         nosa.nosa_decode_step_device(p, b.q, r.k_cache, r.v_cache, b.seq_start, b.seq_len, st.max_seq_len,
                                      st.pooled, st.sel_idx, st.sel_cnt, st.out, st.ws, k_new=r.k_new,
@@ -468,12 +519,13 @@ def run_ours(args):
     fused_bytes_launch = step_bytes / wl.layers
     achieved = fused_bytes_launch / launch_s / 1e9
     traffic = None
-    if not (args.context or args.batch or args.topk):
+    # The committed counters cover the default variant of each named workload.
+    if not (args.context or args.batch or args.topk or wl.paged or wl.kv_int8 or wl.pooled_bf16):
         traffic = ncu_traffic(wl.name)
 
     # e2e through the host-buffer entry point, one layer (replica 0), pinned buffers.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not wl.paged:   # the host-buffer call takes contiguous caches
         e2e = measure_e2e(nosa, wl, rotation[0][0], args, stream, info, device)
 
     cpu = None
@@ -587,7 +639,7 @@ def run_sweep(args):
         for B in SWEEP_BATCHES:
             for K in SWEEP_TOPK:
                 a = argparse.Namespace(workload="nosa1b_b8_16k", context=L, batch=B, topk=K, pooled=args.pooled,
-                                       kv=args.kv)
+                                       kv=args.kv, paged=args.paged)
                 wl = Workload(a, 0)
                 layer_bytes = B * L * wl.hkv * 128 * 2 * 2
                 R = max(2, min(16, math.ceil(1.0e9 / layer_bytes)))
