@@ -245,6 +245,9 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   }
   grid_dependency_wait();
   allow_dependents();
+#ifdef NOSA_TRACE
+  if (tid == 0) NOSA_STAMP(6);
+#endif
 
   // ---------------------------------------------------------------- geometry
   // (identical in every CTA of the cluster)
@@ -298,9 +301,9 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   // CTA's shared memory.
   cluster_arrive();
 
-  // Who selects: one warp (the selector) for small candidate sets or block
-  // scores in global memory, else the selection group (uniform per pair).
-  const bool group_selects = scoring && !spill && ncand > kWarpSelectMax;
+  // Who selects: the selection group when the block scores are in shared
+  // memory, else (block scores in global memory) the selector alone.
+  const bool group_selects = scoring && !spill;
   // Top-k of the pair by the selection group, from the block scores in
   // shared memory; every member calls it (gtid = its index in the group).
   // The decision to give up after a timed-out wait is taken together.
@@ -311,12 +314,14 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     if (gtid == kConsumerThreads) NOSA_STAMP(3);
 #endif
     if (ok) {
-#ifdef NOSA_TRACE
-      group_topk<kSelectThreads>(bsm, false, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar,
-                                 &sh.tr[14]);
-#else
-      group_topk<kSelectThreads>(bsm, false, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
-#endif
+      // Sample select up to 7 candidates per thread (its pivot counting
+      // grows with the candidates), the radix select beyond.
+      if (ncand <= 2 * kSelectThreads)
+        sample_topk<kSelectThreads, 2>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
+      else if (ncand <= 7 * kSelectThreads)
+        sample_topk<kSelectThreads, 7>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
+      else
+        group_topk<kSelectThreads>(bsm, false, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
     } else {
       for (int x = gtid; x < a.topk; x += kSelectThreads) sel_list[x] = -1;
       if (gtid == 0) sh.sel_count = 0;
