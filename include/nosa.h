@@ -57,6 +57,11 @@
  *    bounded wait that gave up) never trap: the kernel skips that unit,
  *    writes zeros where it owns output, and sets a bit in the workspace's
  *    device status word, which nosa_read_device_status returns and clears.
+ *  * An empty batch (batch 0, or total_q 0 for the prefill calls) returns
+ *    NOSA_OK at once, before the other buffers are checked and without any
+ *    CUDA call; the paged calls still check the page pool's geometry (a
+ *    page table pointer and num_pages >= 1).  The no-workspace call resets
+ *    its built-in status word even then.
  *  * Calls that share one workspace must not overlap on the GPU (order them
  *    on one stream): the workspace holds the status word, block scores of
  *    very long sequences and the host-buffer step's staging.

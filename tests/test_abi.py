@@ -96,3 +96,35 @@ def test_null_and_workspace_checks(nosa):
                             ctypes.c_void_p(256), 1, ctypes.c_void_p(256), 1, 1,
                             ctypes.c_void_p(256), None, None, 0, None)
     assert rc == nosa.NOSA_ERR_INVALID_ARG
+
+
+# (entry point, index of batch (or total_q), index of max_seq_len or None, fixed args)
+_DUMMY = ctypes.c_void_p(256)  # a page table that an empty batch never reads
+_EMPTY_CALLS = [
+    ("nosa_block_select", 5, 6, {}),
+    ("nosa_sparse_decode", 7, 8, {}),
+    ("nosa_sparse_decode_paged", 8, 9, {4: 1, 5: _DUMMY}),
+    ("nosa_decode_step_device", 9, 10, {}),
+    ("nosa_decode_step_device_paged", 10, 11, {6: 1, 7: _DUMMY}),
+    ("nosa_decode_step", 10, 11, {}),
+    ("nosa_pool_append_paged", 8, None, {3: 1, 4: _DUMMY, 10: 1, 11: 1}),
+    ("nosa_sparse_prefill", 9, 10, {8: 1}),          # batch 1, total_q 0
+    ("nosa_sparse_prefill_paged", 10, 11, {4: 1, 5: _DUMMY, 9: 1}),
+]
+
+
+@pytest.mark.parametrize("name,i_batch,i_len,extra", _EMPTY_CALLS, ids=[c[0] for c in _EMPTY_CALLS])
+def test_empty_batch_is_a_no_op(nosa, name, i_batch, i_len, extra):
+    """An empty batch (or no prefill rows) returns NOSA_OK before any check
+    of the other buffers and before any CUDA call (none could run on this
+    host); the paged calls still check the page pool's geometry (a page
+    table pointer and at least one page)."""
+    p = nosa.params(16, 2)
+    fn = getattr(nosa.lib(), name)
+    args = [ctypes.byref(p)] + [None if t is nosa._P else 0 for t in fn.argtypes[1:]]
+    args[i_batch] = 0
+    if i_len is not None:
+        args[i_len] = 1024
+    for k, v in extra.items():
+        args[k] = v
+    assert fn(*args) == nosa.NOSA_OK, nosa.lib().nosa_last_error().decode()
