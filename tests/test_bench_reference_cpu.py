@@ -1,7 +1,9 @@
-"""The benchmark's reference arm (the oracle timed on the host cores) keeps
-the benchmark line contract: one JSON line on rank 0 with the metric, unit,
-direction and workload of the CUDA arm, a cpu_baseline describing the run and
-a zero-copy e2e; the other ranks of a torchrun launch exit 0 without work."""
+"""Host-side parts of the benchmark.  The reference arm (the oracle timed on
+the host cores) keeps the benchmark line contract: one JSON line on rank 0
+with the metric, unit, direction and workload of the CUDA arm, a
+cpu_baseline describing the run and a zero-copy e2e; the other ranks of a
+torchrun launch exit 0 without work.  The algorithmic byte count behind the
+roofline's `achieved` matches a count by hand."""
 import json
 import os
 import subprocess
@@ -45,3 +47,18 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert not [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+
+
+def test_algorithmic_bytes_of_the_default_step(monkeypatch):
+    """The roofline numerator of the default workload (NOSA-1B, B=8, L=16384,
+    16 q / 2 KV heads, top-k 64, 16 local blocks), counted by hand per
+    (sequence, KV head): 1023 windows, 256 blocks, 240 candidates."""
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    wl = bench.Workload(bench.parse(), 0)
+    G = 8
+    pool = 2 * 256 + 2 * 256 + 1 * (31 * 256 + 512)    # new K/V rows in and out; the window token 16383 completes
+    select = 960 * 512 + G * 256 + 64 * 4 + 4           # windows of the 240 candidate blocks (fp32), q, selection
+    decode = (64 * 64 + 16 * 64) * 2 * 256 + 2 * G * 256 + 64 * 4 + 4   # 80 tiles of K and V, q + out, selection
+    per_pair = pool + select + decode
+    m = wl.bytes_model()
+    assert sum(m.values()) == 16 * per_pair == 50_065_536
