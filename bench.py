@@ -30,6 +30,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -304,13 +305,26 @@ def peak_bf16():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+_COMMENT_OR_STRING = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', re.S)
+
+
+def _code_only(text: str) -> str:
+    """C/CUDA source without comments, whitespace runs collapsed (string
+    literals kept as they are)."""
+    text = _COMMENT_OR_STRING.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash():
+    """SHA-256 (16 hex digits) of the kernel sources with comments and
+    whitespace removed: a comment edit leaves the compiled kernels, and so
+    their ncu counters, unchanged."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_decode_nosa_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
