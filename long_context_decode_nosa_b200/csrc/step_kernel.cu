@@ -24,11 +24,12 @@
 //     into a ring of 32 KB stages (full / empty mbarriers); with INT8 caches
 //     a stage carries two tiles (half the bytes each) and their scale rows;
 //   * warp 5, selector: pools the window completed by the new token (rank
-//     0), waits until the block scores of the whole pair have arrived (one
-//     remote mbarrier arrival per CTA), runs the exact top-k (every CTA
-//     computes the same selection, so no second exchange is needed) and
-//     hands the selected blocks to the producer; rank 0 writes the
-//     selection out.
+//     0), waits until the block scores of the whole pair have arrived, runs
+//     the exact top-k with the consumers (the selection group: a sample
+//     select, or a radix select above 1120 candidates; alone when the block
+//     scores are kept in global memory) -- every CTA computes the same
+//     selection, so no second exchange is needed -- and hands the selected
+//     blocks to the producer; rank 0 writes the selection out.
 // Merge: each CTA merges its four warps into one partial (O, m, l) and
 // pushes it, slice by slice, into the receive buffers of the cluster's CTAs
 // (CTA r owns output slice r); after one cluster barrier, CTA r combines
