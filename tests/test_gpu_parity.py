@@ -203,12 +203,14 @@ def test_select_unplanted_ragged_valid(nosa):
     _status_ok(nosa, st.ws)
 
 
-@pytest.mark.parametrize("L", [16384, 65536, 132_000])
+@pytest.mark.parametrize("L", [5504, 7424, 16384, 65536, 132_000])
 def test_select_ties_resolved_to_lowest_index(nosa, L):
     """All keys zero except 10 planted blocks per KV head: every other block
-    scores exactly 0, so 54 of the 64 picks are ties that the lowest block
-    index must win -- through the whole scoring path (240, 1008 and 2047
-    candidates: every key count per thread of the selection group)."""
+    scores exactly 0, so most of the 64 picks are ties that the lowest block
+    index must win -- through the whole scoring path (70 and 100 candidates:
+    the sample select ranks tied survivors; 240 and 1008: too many ties for
+    its survivor list, so its radix fallback decides; 2047: the radix
+    select)."""
     b = inputs.make_batch(L, batch=1, num_q_heads=16, num_kv_heads=2, seed=41)
     b.k_cache.zero_()
     G = 8
