@@ -128,3 +128,40 @@ def test_empty_batch_is_a_no_op(nosa, name, i_batch, i_len, extra):
     for k, v in extra.items():
         args[k] = v
     assert fn(*args) == nosa.NOSA_OK, nosa.lib().nosa_last_error().decode()
+
+
+_C_CLIENT = r"""
+#include <stdio.h>
+#include "nosa.h"
+int main(void) {
+  nosa_params p;
+  nosa_default_params(&p);
+  p.num_q_heads = 16;
+  p.num_kv_heads = 2;
+  size_t ws = nosa_workspace_size(&p, 8, 16384);
+  printf("%zu|%s|%d\n", ws, nosa_status_string(NOSA_ERR_INVALID_ARG),
+         nosa_block_select(&p, NULL, NULL, 0, NULL, 0, 1024, NULL, 0, NULL, NULL, 0, NULL, NULL, NULL, 0, NULL));
+  return ws == 0;
+}
+"""
+
+
+def test_plain_c_client(nosa, tmp_path):
+    """The header compiles as strict C99 and a plain C program links against
+    the library and calls it (host-only calls: no GPU here), with no Python
+    or PyTorch involved."""
+    import shutil
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(_C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(nosa.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.dirname(HEADER), str(src),
+                    "-L", libdir, "-lnosa_b200", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.strip().split("|")
+    p = nosa.params(16, 2)
+    assert int(out[0]) == nosa.lib().nosa_workspace_size(ctypes.byref(p), 8, 16384) > 0
+    assert out[1] == nosa.lib().nosa_status_string(nosa.NOSA_ERR_INVALID_ARG).decode()
+    assert int(out[2]) == nosa.NOSA_OK  # batch 0
