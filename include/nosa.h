@@ -25,7 +25,9 @@
  *  * All tensor arguments are DEVICE pointers to caller-owned memory, except
  *    where an argument is documented as a host pointer.  The library keeps no
  *    global state besides a per-thread last-error string, and allocates no
- *    device memory: scratch space is the caller's workspace `ws`.
+ *    device memory: scratch space is the caller's workspace `ws`.  The one
+ *    exception is nosa_decode_step_device_noalloc, whose scratch is a fixed
+ *    array that the library defines in device memory (see there).
  *  * `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *    stream.  Every call only enqueues work on it (no host synchronisation),
  *    except nosa_read_device_status.
@@ -60,8 +62,7 @@
  *  * An empty batch (batch 0, or total_q 0 for the prefill calls) returns
  *    NOSA_OK at once, before the other buffers are checked and without any
  *    CUDA call; the paged calls still check the page pool's geometry (a
- *    page table pointer and num_pages >= 1).  The no-workspace call resets
- *    its built-in status word even then.
+ *    page table pointer and num_pages >= 1).
  *  * Calls that share one workspace must not overlap on the GPU (order them
  *    on one stream): the workspace holds the status word, block scores of
  *    very long sequences and the host-buffer step's staging.
@@ -248,17 +249,27 @@ NOSA_API int nosa_decode_step_device(const nosa_params* p, const void* q, const 
  * device pool and offers no workspace hook, or a serving loop that must not
  * call cudaMalloc once the KV cache has taken the free memory.  This entry
  * point takes the same arguments without `ws` and keeps its scratch in an
- * 8 MiB array that the library defines in device memory (every GPU that loads
- * the library holds it until the process exits).  It allocates nothing and
- * calls no allocating routine.
+ * 8 MiB array that the library defines in device memory.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *  * Host checks are those of nosa_decode_step_device and come first: a
+ *    rejected call returns its status code and enqueues nothing.  An empty
+ *    batch returns NOSA_OK with no CUDA call.
  *  * A batch whose nosa_workspace_size exceeds 8 MiB is rejected with
  *    NOSA_ERR_WORKSPACE (nothing is enqueued); use nosa_decode_step_device.
- *  * The first call on a device looks up the array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.
- *  * Every call on a device shares the one array: the call clears its
- *    status word first (asynchronously, on `stream`), but calls that
- *    overlap on the GPU race.  Order them on one stream.
+ *  * The array is part of the library's device code: CUDA creates it on a
+ *    device when it loads that code there, and it stays until the process
+ *    exits.  Under CUDA's default lazy loading that happens at the first
+ *    call on the device (with batch >= 1), so that first call -- like any
+ *    first kernel launch -- needs the 8 MiB of free device memory and may
+ *    synchronise: make it before the KV cache claims the free memory and
+ *    before any stream capture.  (CUDA_MODULE_LOADING=EAGER creates it when
+ *    the context is created instead.)  Every call looks the array's device
+ *    address up on the current device, so calls stay valid across devices
+ *    and after a device reset.
+ *  * Every call on a device shares the one array, which keeps what the last
+ *    call left: the call clears its status word first (asynchronously, on
+ *    `stream`), but calls that overlap on the GPU race.  Order them on one
+ *    stream.
  *  * Device-side data checks land in the array's status word, which no entry
  *    point reads back; callers that need those reports use the workspace
  *    variant and nosa_read_device_status. */
@@ -357,12 +368,12 @@ NOSA_API int nosa_sparse_prefill_paged(const nosa_params* p, const void* q, cons
  * copies the bf16 output back to out_host.  seq_len (device) already counts
  * the new token.  All copies and kernels are enqueued on `stream`; the call
  * returns without waiting, so out_host is valid after the stream synchronises.
- * Host buffers should be pinned for the copies to be asynchronous; when
- * q_host, k_new_host and v_new_host lie back to back in one host allocation
- * (in that order) they travel in a single copy.  The
- * device staging area comes from `ws` (nosa_workspace_size covers it).  The
- * kernels run as in nosa_decode_step_device.
- * sel_idx / sel_cnt (device) receive the selection. */
+ * Host buffers should be pinned for the copies to be asynchronous.  The
+ * three inputs travel in three copies (nosa_decode_step_packed below takes
+ * them as one buffer and one copy).  The device staging area comes from
+ * `ws` (nosa_workspace_size covers it).  The kernels run as in
+ * nosa_decode_step_device.  sel_idx / sel_cnt (device) receive the
+ * selection. */
 NOSA_API int nosa_decode_step(const nosa_params* p, const void* q_host,
                      const void* k_new_host, const void* v_new_host,
                      void* out_host, void* k_cache, void* v_cache,
@@ -370,6 +381,21 @@ NOSA_API int nosa_decode_step(const nosa_params* p, const void* q_host,
                      int batch, int max_seq_len, void* pooled, int nc_cap,
                      int32_t* sel_idx, int32_t* sel_cnt, void* ws,
                      size_t ws_bytes, void* stream);
+
+/* nosa_decode_step with the three inputs in ONE host buffer: qkv_host holds
+ * q (bf16 [batch, Hq, D]), then k_new (bf16 [batch, Hkv, D]), then v_new
+ * (bf16 [batch, Hkv, D]), back to back, batch * (Hq + 2 Hkv) * D * 2 bytes
+ * in all, within one host allocation (pinned, for the copy to be
+ * asynchronous).  It travels to the device in a single copy; everything else
+ * is as in nosa_decode_step, and the results are bit-identical to it.  The
+ * caller owns both host buffers; out_host is valid after `stream`
+ * synchronises.  Errors as in nosa_decode_step (NULL host buffer:
+ * NOSA_ERR_INVALID_ARG; a copy the runtime refuses: NOSA_ERR_CUDA). */
+NOSA_API int nosa_decode_step_packed(const nosa_params* p, const void* qkv_host, void* out_host,
+                                     void* k_cache, void* v_cache, int64_t cache_rows,
+                                     const int64_t* seq_start, const int32_t* seq_len, int batch,
+                                     int max_seq_len, void* pooled, int nc_cap, int32_t* sel_idx,
+                                     int32_t* sel_cnt, void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, reads and clears the workspace's device status word.
  * Returns NOSA_OK, NOSA_ERR_TIMEOUT (timeout bit set), NOSA_ERR_DEVICE_CHECK

@@ -481,6 +481,20 @@ int do_sparse_decode(const nosa_params* p, const void* q, const void* k_cache, c
   return ok();
 }
 
+// Buffer checks of the fused step (everything but the workspace).
+int check_step_buffers(const void* q, const void* k_new, const void* v_new, const void* k_cache, const void* v_cache,
+                       int64_t cache_rows, const KvLayout& kvl, const int32_t* seq_len, const void* pooled, int nc_cap,
+                       const int32_t* sel_idx, const int32_t* sel_cnt, const void* out) {
+  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, kvl, seq_len, sel_idx, sel_cnt, out)) return rc;
+  if (!pooled || nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "pooled must not be NULL and nc_cap >= 1");
+  if (!aligned(pooled, 16)) return fail(NOSA_ERR_INVALID_ARG, "pooled must be 16-byte aligned");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(NOSA_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+  if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16)))
+    return fail(NOSA_ERR_INVALID_ARG, "new-row pointers must be 16-byte aligned");
+  return NOSA_OK;
+}
+
 // The fused step on device buffers: one launch appends, pools, selects and
 // attends.  Needs at least two local blocks (then the window a new token
 // completes is never read by the same step's selection); otherwise the three
@@ -493,13 +507,9 @@ int do_decode_step_device(const nosa_params* p, const void* q, const void* k_new
   if (batch == 0) return ok();
   const Layout l = layout_of(p, batch, max_seq_len);
   if (int rc = check_ws(ws, ws_bytes, l)) return rc;
-  if (int rc = check_decode_ptrs(q, k_cache, v_cache, cache_rows, kvl, seq_len, sel_idx, sel_cnt, out)) return rc;
-  if (!pooled || nc_cap < 1) return fail(NOSA_ERR_INVALID_ARG, "pooled must not be NULL and nc_cap >= 1");
-  if (!aligned(pooled, 16)) return fail(NOSA_ERR_INVALID_ARG, "pooled must be 16-byte aligned");
-  if ((k_new == nullptr) != (v_new == nullptr))
-    return fail(NOSA_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
-  if (k_new && (!aligned(k_new, 16) || !aligned(v_new, 16)))
-    return fail(NOSA_ERR_INVALID_ARG, "new-row pointers must be 16-byte aligned");
+  if (int rc = check_step_buffers(q, k_new, v_new, k_cache, v_cache, cache_rows, kvl, seq_len, pooled, nc_cap,
+                                  sel_idx, sel_cnt, out))
+    return rc;
   if (p->local_blocks < 2) {
     int rc = do_pool_append(p, k_cache, v_cache, cache_rows, kvl, nullptr, seq_len, batch, pooled, nc_cap, 1,
                             k_new, v_new, at<uint32_t>(ws, l.status), stream);
@@ -614,6 +624,17 @@ size_t workspace_counter_bytes(const nosa_params* p, int batch, int max_seq_len)
 }
 
 int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
+int check_decode_step_device(const nosa_params* p, const void* q, const void* k_new, const void* v_new,
+                             const void* k_cache, const void* v_cache, int64_t cache_rows, const int64_t* seq_start,
+                             const int32_t* seq_len, int batch, int max_seq_len, const void* pooled, int nc_cap,
+                             const int32_t* sel_idx, const int32_t* sel_cnt, const void* out) {
+  if (int rc = check_params(p)) return rc;
+  if (int rc = check_common(p, batch, max_seq_len)) return rc;
+  if (batch == 0) return ok();
+  return check_step_buffers(q, k_new, v_new, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, seq_len,
+                            pooled, nc_cap, sel_idx, sel_cnt, out);
+}
 
 }  // namespace nosa
 
@@ -791,59 +812,78 @@ int nosa_decode_step_device_paged(const nosa_params* p, const void* q, const voi
                                sel_idx, sel_cnt, out, lse, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+namespace {
+
+// The host-buffer step after the input copies: the fused step on the
+// staging area, then the output copy back.
+int step_from_staging(const nosa_params* p, const Layout& l, void* out_host, void* k_cache, void* v_cache,
+                      int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch,
+                      int max_seq_len, void* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* ws,
+                      size_t ws_bytes, cudaStream_t s) {
+  const size_t qbytes = static_cast<size_t>(batch) * p->num_q_heads * nosa::kHeadDim * 2;
+  int rc = do_decode_step_device(p, at<void>(ws, l.stage_q), at<void>(ws, l.stage_k), at<void>(ws, l.stage_v), k_cache,
+                                 v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, seq_len, batch, max_seq_len,
+                                 pooled, nc_cap, sel_idx, sel_cnt, at<void>(ws, l.stage_out), nullptr, ws, ws_bytes, s);
+  if (rc) return rc;
+  cudaError_t e = cudaMemcpyAsync(out_host, at<void>(ws, l.stage_out), qbytes, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy out");
+  return ok();
+}
+
+int check_host_step(const nosa_params* p, int batch, int max_seq_len, void* ws, size_t ws_bytes, Layout* l) {
+  if (int rc = check_params(p)) return rc;
+  if (int rc = check_common(p, batch, max_seq_len)) return rc;
+  *l = layout_of(p, batch, max_seq_len);
+  return batch == 0 ? NOSA_OK : check_ws(ws, ws_bytes, *l);
+}
+
+}  // namespace
+
+extern "C" {
+
 int nosa_decode_step(const nosa_params* p, const void* q_host, const void* k_new_host,
                      const void* v_new_host, void* out_host, void* k_cache, void* v_cache,
                      int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch, int max_seq_len,
                      void* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* ws,
                      size_t ws_bytes, void* stream) {
-  if (int rc = check_params(p)) return rc;
-  if (int rc = check_common(p, batch, max_seq_len)) return rc;
+  Layout l;
+  if (int rc = check_host_step(p, batch, max_seq_len, ws, ws_bytes, &l)) return rc;
   if (batch == 0) return ok();
   if (!q_host || !k_new_host || !v_new_host || !out_host)
     return fail(NOSA_ERR_INVALID_ARG, "host buffers must not be NULL");
-  const Layout l = layout_of(p, batch, max_seq_len);
-  if (int rc = check_ws(ws, ws_bytes, l)) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t qbytes = static_cast<size_t>(batch) * p->num_q_heads * nosa::kHeadDim * 2;
   const size_t kvbytes = static_cast<size_t>(batch) * p->num_kv_heads * nosa::kHeadDim * 2;
-  void* dq = at<void>(ws, l.stage_q);
-  void* dk = at<void>(ws, l.stage_k);
-  void* dv = at<void>(ws, l.stage_v);
-  void* dout = at<void>(ws, l.stage_out);
   cudaError_t e;
-  // The staging area holds q, k_new and v_new back to back (each a multiple
-  // of 256 bytes), so inputs that are back to back in host memory too go in
-  // one copy.
-  // Back-to-back addresses can still be separate pinned allocations, which
-  // one copy may not span: the runtime then refuses the copy up front
-  // (invalid value, nothing enqueued) and the three copies run instead.
-  const char* hq = static_cast<const char*>(q_host);
-  bool one_copy = static_cast<const char*>(k_new_host) == hq + qbytes &&
-                  static_cast<const char*>(v_new_host) == hq + qbytes + kvbytes &&
-                  static_cast<char*>(dk) == static_cast<char*>(dq) + qbytes &&
-                  static_cast<char*>(dv) == static_cast<char*>(dk) + kvbytes;
-  if (one_copy) {
-    e = cudaMemcpyAsync(dq, q_host, qbytes + 2 * kvbytes, cudaMemcpyHostToDevice, s);
-    if (e == cudaErrorInvalidValue) {
-      cudaGetLastError();
-      one_copy = false;
-    } else if (e != cudaSuccess) {
-      return cuda_fail(e, "copy q, k_new, v_new");
-    }
-  }
-  if (!one_copy) {
-    if ((e = cudaMemcpyAsync(dq, q_host, qbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy q");
-    if ((e = cudaMemcpyAsync(dk, k_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
-      return cuda_fail(e, "copy k_new");
-    if ((e = cudaMemcpyAsync(dv, v_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
-      return cuda_fail(e, "copy v_new");
-  }
-  int rc = do_decode_step_device(p, dq, dk, dv, k_cache, v_cache, cache_rows, KvLayout{seq_start, nullptr, 0}, seq_len,
-                                 batch, max_seq_len,
-                                 pooled, nc_cap, sel_idx, sel_cnt, dout, nullptr, ws, ws_bytes, s);
-  if (rc) return rc;
-  if ((e = cudaMemcpyAsync(out_host, dout, qbytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess) return cuda_fail(e, "copy out");
-  return ok();
+  if ((e = cudaMemcpyAsync(at<void>(ws, l.stage_q), q_host, qbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+    return cuda_fail(e, "copy q");
+  if ((e = cudaMemcpyAsync(at<void>(ws, l.stage_k), k_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+    return cuda_fail(e, "copy k_new");
+  if ((e = cudaMemcpyAsync(at<void>(ws, l.stage_v), v_new_host, kvbytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+    return cuda_fail(e, "copy v_new");
+  return step_from_staging(p, l, out_host, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len,
+                           pooled, nc_cap, sel_idx, sel_cnt, ws, ws_bytes, s);
+}
+
+int nosa_decode_step_packed(const nosa_params* p, const void* qkv_host, void* out_host, void* k_cache, void* v_cache,
+                            int64_t cache_rows, const int64_t* seq_start, const int32_t* seq_len, int batch,
+                            int max_seq_len, void* pooled, int nc_cap, int32_t* sel_idx, int32_t* sel_cnt, void* ws,
+                            size_t ws_bytes, void* stream) {
+  Layout l;
+  if (int rc = check_host_step(p, batch, max_seq_len, ws, ws_bytes, &l)) return rc;
+  if (batch == 0) return ok();
+  if (!qkv_host || !out_host) return fail(NOSA_ERR_INVALID_ARG, "host buffers must not be NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t qbytes = static_cast<size_t>(batch) * p->num_q_heads * nosa::kHeadDim * 2;
+  const size_t kvbytes = static_cast<size_t>(batch) * p->num_kv_heads * nosa::kHeadDim * 2;
+  // q, k_new and v_new are whole 256-byte rows, so the staging area holds
+  // them back to back too: the packed buffer goes in one copy.
+  cudaError_t e = cudaMemcpyAsync(at<void>(ws, l.stage_q), qkv_host, qbytes + 2 * kvbytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy q, k_new, v_new");
+  return step_from_staging(p, l, out_host, k_cache, v_cache, cache_rows, seq_start, seq_len, batch, max_seq_len,
+                           pooled, nc_cap, sel_idx, sel_cnt, ws, ws_bytes, s);
 }
 
 int nosa_read_device_status(void* ws, size_t ws_bytes, void* stream) {

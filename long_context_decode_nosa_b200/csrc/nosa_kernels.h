@@ -155,4 +155,11 @@ size_t workspace_counter_bytes(const nosa_params* p, int batch, int max_seq_len)
 // Records `msg` as the calling thread's last error and returns `code`.
 int record_error(int code, const char* msg);
 
+// The host checks of nosa_decode_step_device except the workspace's (a
+// status code, recorded as the last error; nothing is enqueued).
+int check_decode_step_device(const nosa_params* p, const void* q, const void* k_new, const void* v_new,
+                             const void* k_cache, const void* v_cache, int64_t cache_rows, const int64_t* seq_start,
+                             const int32_t* seq_len, int batch, int max_seq_len, const void* pooled, int nc_cap,
+                             const int32_t* sel_idx, const int32_t* sel_cnt, const void* out);
+
 }  // namespace nosa

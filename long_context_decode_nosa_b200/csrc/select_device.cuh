@@ -713,6 +713,13 @@ __device__ inline void tma_load_keys(void* dst, const CUtensorMap* map, int col,
       : "memory");
 }
 
+// L2 prefetch of the same box (nothing lands in shared memory, nothing is
+// consumed: a later tma_load_keys of the box finds it in L2).
+__device__ inline void tma_prefetch_keys(const CUtensorMap* map, int col, int row) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(col), "r"(row)
+               : "memory");
+}
+
 template <int G>
 struct ScoreQ {
   static constexpr int kNTiles = G > 8 ? 2 : 1;  // n-tiles of 8 heads

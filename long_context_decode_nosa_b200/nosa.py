@@ -87,6 +87,7 @@ _SIGNATURES = {
     "nosa_decode_step_device_paged": (_I, [_P, _P, _P, _P, _P, _P, _I64, _P, _I, _P, _I, _I, _P, _I, _P, _P, _P,
                                            _P, _P, _SZ, _P]),
     "nosa_decode_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "nosa_decode_step_packed": (_I, [_P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "nosa_read_device_status": (_I, [_P, _SZ, _P]),
     "nosa_last_device_bits": (ctypes.c_uint32, []),
     "nosa_selftest_wait_timeout": (_I, [_P, _SZ, ctypes.c_uint32, _P]),
@@ -489,6 +490,27 @@ def nosa_decode_step(p: nosa_params, q_host: torch.Tensor, k_new_host: torch.Ten
         _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
     _check(rc, "nosa_decode_step")
+
+
+def nosa_decode_step_packed(p: nosa_params, qkv_host: torch.Tensor, out_host: torch.Tensor, k_cache: torch.Tensor,
+                            v_cache: torch.Tensor, seq_start: torch.Tensor, seq_len: torch.Tensor, max_seq_len: int,
+                            pooled: torch.Tensor, sel_idx: torch.Tensor, sel_cnt: torch.Tensor, ws: torch.Tensor,
+                            stream=None):
+    """nosa_decode_step with q, k_new and v_new back to back in one host
+    buffer (bf16, batch * (Hq + 2 Hkv) * 128 elements), copied in once."""
+    batch = seq_len.shape[0]
+    need = batch * (p.num_q_heads + 2 * p.num_kv_heads) * 128
+    if not qkv_host.is_contiguous() or qkv_host.numel() != need:
+        raise ValueError(f"qkv_host must be a contiguous buffer of {need} bf16 values")
+    rc = lib().nosa_decode_step_packed(
+        ctypes.byref(p), _ptr(qkv_host, torch.bfloat16, "qkv_host", cuda=False),
+        _ptr(out_host, torch.bfloat16, "out_host", cuda=False),
+        _cache(p, k_cache, "k_cache"), _cache(p, v_cache, "v_cache"),
+        k_cache.shape[0], _ptr(seq_start, torch.int64, "seq_start"), _ptr(seq_len, torch.int32, "seq_len"),
+        batch, max_seq_len, _ptr(pooled, p.pooled_dtype, "pooled"), pooled.shape[2],
+        _ptr(sel_idx, torch.int32, "sel_idx"), _ptr(sel_cnt, torch.int32, "sel_cnt"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream))
+    _check(rc, "nosa_decode_step_packed")
 
 
 def nosa_read_device_status(ws: torch.Tensor, stream=None):

@@ -107,6 +107,8 @@ _EMPTY_CALLS = [
     ("nosa_decode_step_device", 9, 10, {}),
     ("nosa_decode_step_device_paged", 10, 11, {6: 1, 7: _DUMMY}),
     ("nosa_decode_step", 10, 11, {}),
+    ("nosa_decode_step_packed", 8, 9, {}),
+    ("nosa_decode_step_device_noalloc", 9, 10, {}),
     ("nosa_pool_append_paged", 8, None, {3: 1, 4: _DUMMY, 10: 1, 11: 1}),
     ("nosa_sparse_prefill", 9, 10, {8: 1}),          # batch 1, total_q 0
     ("nosa_sparse_prefill_paged", 10, 11, {4: 1, 5: _DUMMY, 9: 1}),
@@ -128,6 +130,22 @@ def test_empty_batch_is_a_no_op(nosa, name, i_batch, i_len, extra):
     for k, v in extra.items():
         args[k] = v
     assert fn(*args) == nosa.NOSA_OK, nosa.lib().nosa_last_error().decode()
+
+
+def test_noalloc_host_checks_come_first(nosa):
+    """The scratch-free step runs the workspace entry point's host checks,
+    and its own size check, before any CUDA call (none could run on this
+    host): a NULL buffer and a batch beyond the built-in 8 MiB both return
+    their codes with nothing enqueued."""
+    p = nosa.params(16, 2, topk=64)
+    fn = nosa.lib().nosa_decode_step_device_noalloc
+    d = ctypes.c_void_p(256)
+    rc = fn(ctypes.byref(p), None, None, None, d, d, 100, d, d, 4, 1024, d, 1, d, d, d, None, None)
+    assert rc == nosa.NOSA_ERR_INVALID_ARG
+    assert nosa.workspace_size(p, 64, 1 << 20) > 8 << 20
+    rc = fn(ctypes.byref(p), d, None, None, d, d, 1 << 30, d, d, 64, 1 << 20, d, 1, d, d, d, None, None)
+    assert rc == nosa.NOSA_ERR_WORKSPACE
+    assert "8388608" in nosa.lib().nosa_last_error().decode()
 
 
 _C_CLIENT = r"""

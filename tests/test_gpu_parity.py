@@ -546,9 +546,11 @@ def test_decode_step_host_buffers_equals_device_path(nosa):
     _status_ok(nosa, st2.ws)
 
 
-def test_decode_step_host_buffers_packed_single_copy(nosa):
-    """q, k_new and v_new back to back in one pinned buffer (the single-copy
-    path) give the same step as separate buffers."""
+def test_decode_step_packed_equals_three_copies(nosa):
+    """nosa_decode_step_packed (q, k_new and v_new back to back in one pinned
+    buffer, one copy) gives the same step, bit for bit, as nosa_decode_step
+    (three buffers, three copies): output, appended caches, pooled keys and
+    selection."""
     lens = [3000, 1700, 5000]
     b = inputs.make_batch(lens, num_q_heads=16, num_kv_heads=2, seed=15, slack=16)
     kn, vn = inputs.random_kv_rows(3, 2, 128, seed=16)
@@ -558,20 +560,19 @@ def test_decode_step_host_buffers_packed_single_copy(nosa):
         g = b.to(DEV)
         p, st = _gpu_state(nosa, b, 64, max_seq_len=max(lens) + 1)
         st.rebuild_pooled(g.k_cache, g.seq_start, g.seq_len)
+        oh = torch.empty(3, 16, 128, dtype=torch.bfloat16).pin_memory()
         if packed:
-            buf = torch.empty(q.numel() + 2 * kn.numel(), dtype=torch.bfloat16).pin_memory()
-            qh = buf[:q.numel()].view(q.shape)
-            kh = buf[q.numel():q.numel() + kn.numel()].view(kn.shape)
-            vh = buf[q.numel() + kn.numel():].view(vn.shape)
-            qh.copy_(q), kh.copy_(kn), vh.copy_(vn)
+            buf = torch.cat([q.reshape(-1), kn.reshape(-1), vn.reshape(-1)]).pin_memory()
+            nosa.nosa_decode_step_packed(p, buf, oh, g.k_cache, g.v_cache, g.seq_start, g.seq_len + 1,
+                                         st.max_seq_len, st.pooled, st.sel_idx, st.sel_cnt, st.ws)
         else:
             qh, kh, vh = q.pin_memory(), kn.pin_memory(), vn.pin_memory()
-        oh = torch.empty(3, 16, 128, dtype=torch.bfloat16).pin_memory()
-        nosa.nosa_decode_step(p, qh, kh, vh, oh, g.k_cache, g.v_cache, g.seq_start, g.seq_len + 1,
-                              st.max_seq_len, st.pooled, st.sel_idx, st.sel_cnt, st.ws)
+            nosa.nosa_decode_step(p, qh, kh, vh, oh, g.k_cache, g.v_cache, g.seq_start, g.seq_len + 1,
+                                  st.max_seq_len, st.pooled, st.sel_idx, st.sel_cnt, st.ws)
         torch.cuda.synchronize()
         _status_ok(nosa, st.ws)
-        outs.append((oh.clone(), g.k_cache.cpu(), g.v_cache.cpu(), st.sel_idx.cpu()))
+        outs.append((oh.clone(), g.k_cache.cpu(), g.v_cache.cpu(), st.pooled.cpu(), st.sel_idx.cpu(),
+                     st.sel_cnt.cpu()))
     for x, y in zip(outs[0], outs[1]):
         assert torch.equal(x, y)
 
