@@ -147,6 +147,28 @@ class Workload:
                 "sparse_decode": decode * self.layers}
 
 
+def replica_plan(wl: Workload, args):
+    """(replicas R, bytes of one layer's K/V caches): R independent copies of
+    the caches are rotated so that no step finds its inputs in L2 (126 MB);
+    a multi-layer workload has its own caches per layer instead."""
+    layer_bytes = sum(wl.lens) * wl.hkv * (132 if wl.kv_int8 else 256) * 2
+    if wl.layers > 1:
+        return 1, layer_bytes
+    return args.replicas or max(2, min(16, math.ceil(1.0e9 / max(layer_bytes, 1)))), layer_bytes
+
+
+def run_config(wl: Workload, args, world: int):
+    """The `config` object of the JSON line (the same for both arms)."""
+    R, layer_bytes = replica_plan(wl, args)
+    return {"workload": wl.desc, "batch": wl.batch, "seq_len": wl.max_len,
+            "topk": wl.topk, "local_blocks": wl.local_blocks, "layers": wl.layers,
+            "parallelism": f"dp{world}" if world > 1 else "single GPU",
+            "l2": (f"inputs rotate over {R} cache replicas "
+                   f"({R * layer_bytes * wl.layers / 1e9:.2f} GB) > 126 MB L2"),
+            "clock_settle_ms": args.settle_ms,
+            "graph": "timed steps (one fused launch per layer-step) replayed as one CUDA graph"}
+
+
 class Replica:
     """One layer's device state: caches, pooled keys, selection, output."""
 
@@ -428,8 +450,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.desc, "batch": wl.batch, "seq_len": wl.max_len, "topk": wl.topk,
-                       "layers": wl.layers},
+            "config": run_config(wl, args, int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -450,13 +471,10 @@ def run_ours(args):
     seed0 = multirank.rank_seed(0, info)
 
     # Replicas so that no step finds its inputs in L2 (126 MB).
-    layer_bytes = sum(wl.lens) * wl.hkv * (132 if wl.kv_int8 else 256) * 2
+    R, layer_bytes = replica_plan(wl, args)
     if wl.layers > 1:
-        R = 1
-        layers = [Replica(nosa, wl, seed0 + 10 * l, device) for l in range(wl.layers)]
-        rotation = [layers]
+        rotation = [[Replica(nosa, wl, seed0 + 10 * l, device) for l in range(wl.layers)]]
     else:
-        R = args.replicas or max(2, min(16, math.ceil(1.0e9 / max(layer_bytes, 1))))
         rotation = [[Replica(nosa, wl, seed0 + 10 * r, device)] for r in range(R)]
     torch.cuda.synchronize()
 
@@ -537,10 +555,10 @@ def run_ours(args):
     if not (args.context or args.batch or args.topk or wl.paged or wl.kv_int8 or wl.pooled_bf16):
         traffic = ncu_traffic(wl.name)
 
-    # e2e through the host-buffer entry point, one layer (replica 0), pinned buffers.
+    # e2e through the host-buffer entry point, rotating over the same replicas, pinned buffers.
     e2e = None
     if not args.no_e2e and not wl.paged:   # the host-buffer call takes contiguous caches
-        e2e = measure_e2e(nosa, wl, rotation[0][0], args, stream, info, device)
+        e2e = measure_e2e(nosa, wl, rotation, args, stream, info, device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -564,13 +582,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8+bf16" if wl.kv_int8 else "bf16", "data": "synthetic",
-            "config": {"workload": wl.desc, "batch": wl.batch, "seq_len": wl.max_len,
-                       "topk": wl.topk, "local_blocks": wl.local_blocks, "layers": wl.layers,
-                       "parallelism": f"dp{world}" if world > 1 else "single GPU",
-                       "l2": (f"inputs rotate over {R} cache replicas "
-                              f"({R * layer_bytes * wl.layers / 1e9:.2f} GB) > 126 MB L2"),
-                       "clock_settle_ms": args.settle_ms,
-                       "graph": "timed steps (one fused launch per layer-step) replayed as one CUDA graph"},
+            "config": run_config(wl, args, world),
             "gpu_launches": args.steps * wl.layers,
             "hbm_gbs_step": step_bytes / (ms_step * 1e-3) / 1e9,
             "algorithmic_bytes_per_step": step_bytes,
@@ -589,44 +601,48 @@ def run_ours(args):
     return 0
 
 
-def measure_e2e(nosa, wl: Workload, r: Replica, args, stream, info, device):
-    """Same metric through nosa_decode_step with pinned host buffers: every
-    step copies q and the new K/V rows in and the output back."""
-    if wl.layers > 1:
-        return None
-    b, st, p = r.b, r.st, r.p
-    # q, k_new and v_new back to back in one pinned buffer (one copy per step)
-    nq, nk = b.q.numel(), r.k_new.numel()
-    packed = torch.empty(nq + 2 * nk, dtype=torch.bfloat16).pin_memory()
-    q_h = packed[:nq].view(b.q.shape)
-    k_h = packed[nq:nq + nk].view(r.k_new.shape)
-    v_h = packed[nq + nk:].view(r.v_new.shape)
-    q_h.copy_(b.q.cpu())
-    k_h.copy_(r.k_new.cpu())
-    v_h.copy_(r.v_new.cpu())
-    o_h = torch.empty(wl.batch, wl.hq, 128, dtype=torch.bfloat16).pin_memory()
-    n = max(10, min(args.steps, 500))
+def measure_e2e(nosa, wl: Workload, rotation, args, stream, info, device):
+    """Same metric through the host-buffer entry point (nosa_decode_step_packed)
+    with pinned host buffers: every layer-step copies q and the new K/V rows in
+    (one packed buffer, one copy) and the output back.  Steps rotate over the
+    same cache replicas as the device-timed region (each layer and replica with
+    its own pinned buffers), so the kernels inside run L2-cold as well."""
+    calls = []
+    for layers in rotation:
+        row = []
+        for r in layers:
+            b, st, p = r.b, r.st, r.p
+            packed = torch.cat([b.q.reshape(-1), r.k_new.reshape(-1), r.v_new.reshape(-1)]).cpu().pin_memory()
+            o_h = torch.empty(wl.batch, wl.hq, 128, dtype=torch.bfloat16).pin_memory()
+            row.append((r, packed, o_h))
+        calls.append(row)
+    n = max(len(calls), min(args.steps, 500))
 
-    def call():
-        nosa.nosa_decode_step(p, q_h, k_h, v_h, o_h, r.k_cache, r.v_cache, b.seq_start, b.seq_len,
-                              st.max_seq_len, st.pooled, st.sel_idx, st.sel_cnt, st.ws, stream=stream)
+    def step_e2e(s_):
+        for r, packed, o_h in calls[s_ % len(calls)]:
+            b, st, p = r.b, r.st, r.p
+            nosa.nosa_decode_step_packed(p, packed, o_h, r.k_cache, r.v_cache, b.seq_start, b.seq_len,
+                                         st.max_seq_len, st.pooled, st.sel_idx, st.sel_cnt, st.ws, stream=stream)
 
     with torch.cuda.stream(stream):
-        for _ in range(max(3, min(args.warmup, 50))):
-            call()
+        for s_ in range(max(3, min(args.warmup, 50))):
+            step_e2e(s_)
         stream.synchronize()
         multirank.barrier(info)
         start = torch.cuda.Event(enable_timing=True)
         stop = torch.cuda.Event(enable_timing=True)
         start.record(stream)
-        for _ in range(n):
-            call()
+        for s_ in range(n):
+            step_e2e(s_)
         stop.record(stream)
     stream.synchronize()
     ms = multirank.max_over_ranks(start.elapsed_time(stop), info, device)
-    return {"value": multirank.aggregate_rate(wl.batch * n, info, ms / 1e3), "unit": UNIT,
-            "h2d_bytes_per_step": q_h.numel() * 2 + k_h.numel() * 2 + v_h.numel() * 2,
-            "d2h_bytes_per_step": o_h.numel() * 2, "steps": n, "ms_per_step": ms / n}
+    packed0, out0 = calls[0][0][1], calls[0][0][2]
+    return {"value": multirank.aggregate_rate(wl.batch * wl.layers * n, info, ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": packed0.numel() * 2 * wl.layers,
+            "d2h_bytes_per_step": out0.numel() * 2 * wl.layers, "steps": n, "ms_per_step": ms / n,
+            "replicas": len(calls),
+            "api": "nosa_decode_step_packed (one host-to-device and one device-to-host copy per layer-step)"}
 
 
 # ----------------------------------------------------------------------------- sweep

@@ -281,8 +281,11 @@ NOSA_API int nosa_decode_step_device_noalloc(const nosa_params* p, const void* q
                                              int nc_cap, int32_t* sel_idx, int32_t* sel_cnt,
                                              void* out, float* lse, void* stream);
 
-/* Paged KV cache (a deployment layout; the pages have no counterpart).
- * The caches are a pool of 64-token pages, k_cache / v_cache bf16
+/* Paged KV cache.  "NOSA 技术架构解析" (devpress.csdn.net) §2.1
+ * (内核级优化技术, 内存池化管理) gives NOSI's memory pool a
+ * PagedAttention-style page layout, and §4.2 (典型问题排查, 问题3) lists the paged-cache switch
+ * `--use_paged_kv 1`; neither fixes a page size or table format, so the
+ * layout below is this library's.  The caches are a pool of 64-token pages, k_cache / v_cache bf16
  * [num_pages * 64, Hkv, head_dim]; token t of sequence i lives in row
  *     page_table[i * max_pages + t / 64] * 64 + t % 64,
  * page_table int32 [batch, max_pages].  The page size equals the block size,

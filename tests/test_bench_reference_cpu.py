@@ -38,6 +38,8 @@ def test_reference_arm_line(monkeypatch):
     cfg = d["config"]
     assert (cfg["batch"], cfg["seq_len"], cfg["topk"], cfg["layers"]) == (8, 16384, 64, 1)
     assert cfg["workload"] == default_desc
+    # the CUDA arm's config object, key for key
+    assert cfg == bench.run_config(bench.Workload(bench.parse(), 0), bench.parse(), 1)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
