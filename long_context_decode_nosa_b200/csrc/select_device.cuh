@@ -343,16 +343,14 @@ constexpr int kGroupKeys = 16;
 // Survivors the sample select ranks in shared memory (more fall back to the
 // radix select), and its taken-bit words (32 candidate slots each).
 constexpr int kSurvivorCap = 128;
-constexpr int kTakeWords = 64;
+constexpr int kTakeWords = 80;
 constexpr int kSampleWarps = 5;
 
 struct alignas(16) GroupTopkShared {
-  union {
-    uint32_t hist[256];           // radix select: digit histogram
-    uint64_t surv[kSurvivorCap];  // sample select: survivors, key << 32 | ~index
-  };
+  uint32_t hist[256];             // radix select: digit histogram; bucket select: bucket counts
+  uint64_t surv[kSurvivorCap];    // sample / bucket select: survivors, key << 32 | ~index
   uint32_t pcnt[kSampleWarps][32];  // sample select: per-range counts of the 32 pivots
-  uint32_t take[kTakeWords];      // sample select: taken bits
+  uint32_t take[kTakeWords];      // sample / bucket select: taken bits
   uint32_t red[2][8][2];  // per-warp partials, double-buffered
   uint32_t prefix, need, nsurv;
 };
@@ -671,6 +669,205 @@ __device__ void sample_topk(float* scores, int ncand, int topk, int32_t* sel_row
   }
   for (int x = k_eff + tid; x < topk; x += NT) sel_row[x] = -1;
   if (tid == 0) *sel_cnt = k_eff;
+}
+
+// The fp32 score an order-preserving key stands for (order_key's inverse;
+// -0.0 and NaN come back as +0.0 and -inf).
+__device__ inline float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Exact top-k of the selection group by bucket select: NT threads (a
+// multiple of 32, at most 8 warps; `tid` is the thread's index in the
+// group) and up to NT * M candidates, candidate b held by thread b mod NT in
+// register b / NT.  `scores` is the pair's block scores in shared memory;
+// they are overwritten by their order-preserving keys.
+//   1. Keys in registers and in place of the scores; the smallest and
+//      largest key over the group.
+//   2. Each key falls into one of 256 equal-width buckets of its score
+//      between the smallest and the largest, bucket(x) = floor((x - lo) *
+//      256 / (hi - lo)) clamped to 255: a non-decreasing function of the
+//      score (an fp32 subtraction and a multiplication by a positive
+//      constant never reverse an order), counted in a shared histogram.
+//   3. Every warp scans the histogram from the top for the bucket B that
+//      holds the k-th largest key; the keys of higher buckets are taken (one
+//      bit each in the taken-bit words, word q = candidates [32q, 32q + 32)),
+//      the keys of bucket B are listed as key << 32 | ~index.
+//   4. Each listed key is ranked among the list (key descending, then index
+//      ascending); the first k - (keys above B) set their taken bits.
+//   5. Placement in ascending index order: a candidate's position is the
+//      number of taken bits below its own.
+// One pass over the keys and four barriers; more than kSurvivorCap keys in
+// bucket B (many equal keys, or a range the buckets cannot split: an
+// infinite score, all scores equal) hand over to the radix select.
+template <int NT, int M>
+__device__ void bucket_topk(float* scores, int ncand, int topk, int32_t* sel_row, int32_t* sel_cnt, int tid,
+                            GroupTopkShared& sh, int bar_id, uint64_t* trace_stamps = nullptr) {
+#ifdef NOSA_TRACE
+#define BKT_STAMP(k) \
+  if (trace_stamps && tid == 0) trace_stamps[k] = global_timer_ns()
+#else
+#define BKT_STAMP(k)
+#endif
+  constexpr int kW = NT / 32;
+  constexpr int kQ = M * kW;  // taken-bit words of the NT * M candidate slots
+  static_assert(NT % 32 == 0 && kW <= 8, "the group is 1..8 whole warps");
+  static_assert(M >= 1 && kQ <= kTakeWords, "one taken-bit word per 32 candidate slots");
+  constexpr uint32_t kFull = 0xffffffffu;
+  const int lane = tid & 31, w = tid >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int k_eff = ncand < topk ? ncand : topk;
+  if (k_eff == ncand) {  // every candidate is taken
+    for (int b = tid; b < topk; b += NT) sel_row[b] = b < ncand ? b : -1;
+    if (tid == 0) *sel_cnt = k_eff;
+    return;
+  }
+  uint32_t* ords = reinterpret_cast<uint32_t*>(scores);
+  uint32_t key[M];
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    const int b = tid + m * NT;
+    const float f = scores[b < ncand ? b : 0];  // loads issued unconditionally
+    key[m] = b < ncand ? order_key(f) : 0u;     // valid keys are > 0
+    if (b < ncand) {
+      ords[b] = key[m];
+      kmin = min(kmin, key[m]);
+      kmax = max(kmax, key[m]);
+    }
+  }
+  for (int x = tid; x < 256; x += NT) sh.hist[x] = 0u;
+  if (tid == 0) sh.nsurv = 0u;
+  kmin = __reduce_min_sync(kFull, kmin);
+  kmax = __reduce_max_sync(kFull, kmax);
+  if (lane == 0) {
+    sh.red[0][w][0] = kmin;
+    sh.red[0][w][1] = kmax;
+  }
+  group_bar(bar_id, NT);
+  BKT_STAMP(0);
+#pragma unroll
+  for (int x = 0; x < kW; ++x) {
+    kmin = min(kmin, sh.red[0][x][0]);
+    kmax = max(kmax, sh.red[0][x][1]);
+  }
+  const float lo = key_float(kmin), range = key_float(kmax) - lo;
+  // range is +inf or NaN when a score is infinite: one bucket for all.
+  const float scale = range > 0.0f && range <= 3.0e38f ? 256.0f / range : 0.0f;
+  auto bucket = [&](uint32_t kk) -> int {
+    const float d = (key_float(kk) - lo) * scale;
+    return d >= 255.0f ? 255 : d > 0.0f ? static_cast<int>(d) : 0;
+  };
+  int bk[M];
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    bk[m] = tid + m * NT < ncand ? bucket(key[m]) : -1;
+    if (bk[m] >= 0) atomicAdd(&sh.hist[bk[m]], 1u);
+  }
+  group_bar(bar_id, NT);
+  BKT_STAMP(1);
+  // Lane l owns buckets [8l, 8l + 8); the bucket holding the k-th largest
+  // key is where the count from the top first reaches k.  Every warp finds
+  // it, so no barrier is needed to share it.
+  const uint32_t k = static_cast<uint32_t>(k_eff);
+  uint32_t c[8], sum = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    c[q] = sh.hist[8 * lane + q];
+    sum += c[q];
+  }
+  uint32_t suf = sum;  // sum over lanes >= this lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(kFull, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  int my_b = -1;
+  uint32_t my_above = 0;
+  if (suf - sum < k && k <= suf) {
+    uint32_t acc = suf - sum;
+#pragma unroll
+    for (int q = 7; q >= 0; --q) {
+      if (my_b < 0 && acc + c[q] >= k) {
+        my_b = 8 * lane + q;
+        my_above = acc;
+      }
+      acc += c[q];
+    }
+  }
+  const int src = __ffs(__ballot_sync(kFull, my_b >= 0)) - 1;  // exactly one lane
+  const int B = __shfl_sync(kFull, my_b, src);
+  const uint32_t c_above = __shfl_sync(kFull, my_above, src);
+  const uint32_t nsurv = sh.hist[B], need = k - c_above;
+  if (nsurv > static_cast<uint32_t>(kSurvivorCap)) {  // uniform over the group
+    group_topk<NT, true>(scores, false, ncand, topk, sel_row, sel_cnt, tid, sh, bar_id);
+    return;
+  }
+  const uint32_t nsurv4 = (nsurv + 3u) & ~3u;
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    const int b = tid + m * NT;
+    if (bk[m] == B) {
+      const uint32_t slot = atomicAdd(&sh.nsurv, 1u);
+      if (slot < nsurv) sh.surv[slot] = (static_cast<uint64_t>(key[m]) << 32) | ~static_cast<uint32_t>(b);
+    }
+    const uint32_t hb = __ballot_sync(kFull, bk[m] > B);
+    if (lane == 0) sh.take[m * kW + w] = hb;
+  }
+  if (tid < 4 && nsurv + tid < nsurv4) sh.surv[nsurv + tid] = 0u;  // below every entry
+  group_bar(bar_id, NT);
+  BKT_STAMP(2);
+  for (int t = tid; t < static_cast<int>(nsurv); t += NT) {
+    const uint64_t ct = sh.surv[t];
+    uint32_t r0 = 0, r1 = 0;
+#pragma unroll 4
+    for (uint32_t s2 = 0; s2 < nsurv4; s2 += 2) {
+      const ulonglong2 e = *reinterpret_cast<const ulonglong2*>(&sh.surv[s2]);
+      r0 += e.x > ct;
+      r1 += e.y > ct;
+    }
+    if (r0 + r1 < need) {
+      const uint32_t b = ~static_cast<uint32_t>(ct);
+      atomicOr(&sh.take[b >> 5], 1u << (b & 31u));
+    }
+  }
+  group_bar(bar_id, NT);
+  BKT_STAMP(3);
+  // Exclusive prefix of the words' bit counts, by every warp: lane j scans
+  // words [kPer j, kPer j + kPer).
+  constexpr int kPer = (kQ + 31) / 32;
+  uint32_t pe[kPer];
+  uint32_t tot = 0;
+#pragma unroll
+  for (int x = 0; x < kPer; ++x) {
+    const int qq = lane * kPer + x;
+    pe[x] = tot;
+    const uint32_t wd = sh.take[qq < kQ ? qq : 0];
+    tot += qq < kQ ? __popc(wd) : 0u;
+  }
+  uint32_t inc = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(kFull, inc, o);
+    if (lane >= o) inc += y;
+  }
+#pragma unroll
+  for (int x = 0; x < kPer; ++x) pe[x] += inc - tot;
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    const int q = m * kW + w;  // this thread's word (uniform over the warp)
+    uint32_t v = pe[0];
+#pragma unroll
+    for (int x = 1; x < kPer; ++x)
+      if (q % kPer == x) v = pe[x];
+    const uint32_t pre = __shfl_sync(kFull, v, q / kPer);
+    const uint32_t word = sh.take[q];
+    if ((word >> lane) & 1u) sel_row[pre + __popc(word & lt_mask)] = tid + m * NT;
+  }
+  for (int x = k_eff + tid; x < topk; x += NT) sel_row[x] = -1;
+  if (tid == 0) *sel_cnt = k_eff;
+  BKT_STAMP(4);
+#undef BKT_STAMP
 }
 
 // Top-k by one warp: register-resident keys up to kWarpTopkMax candidates,

@@ -315,12 +315,17 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     if (gtid == kConsumerThreads) NOSA_STAMP(3);
 #endif
     if (ok) {
-      // Sample select up to 7 candidates per thread (its pivot counting
-      // grows with the candidates), the radix select beyond.
+#ifdef NOSA_TRACE
+      uint64_t* stamps = &sh.tr[14];
+#else
+      uint64_t* stamps = nullptr;
+#endif
+      // Bucket select up to 7 candidates per thread (held in registers), the
+      // radix select beyond.
       if (ncand <= 2 * kSelectThreads)
-        sample_topk<kSelectThreads, 2>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
+        bucket_topk<kSelectThreads, 2>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
       else if (ncand <= 7 * kSelectThreads)
-        sample_topk<kSelectThreads, 7>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
+        bucket_topk<kSelectThreads, 7>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
       else
         group_topk<kSelectThreads>(bsm, false, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
     } else {
@@ -534,8 +539,10 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
         if (lane == 0) NOSA_STAMP(3);
 #endif
         if (ok) {
-          warp_select(spill ? a.bs_spill + static_cast<int64_t>(pair) * a.nb_spill : bsm, spill, ncand, a.topk,
-                      sel_list, &sh.sel_count, lane);
+          // Block scores in global memory: beyond the group's shared memory, so
+          // more than any register-resident selection holds.
+          warp_topk_mem(a.bs_spill + static_cast<int64_t>(pair) * a.nb_spill, true, ncand, a.topk, sel_list,
+                        &sh.sel_count, lane);
         } else {
           for (int t = lane; t < a.topk; t += 32) sel_list[t] = -1;
           if (lane == 0) sh.sel_count = 0;
