@@ -208,6 +208,14 @@ __device__ inline void st_async_f32(uint32_t addr, float v, uint32_t remote_bar)
                : "memory");
 }
 
+// As st_async_f32, four fp32 (16 bytes, 16-byte aligned address).
+__device__ inline void st_async_f32x4(uint32_t addr, float4 v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "r"(__float_as_uint(v.x)), "r"(__float_as_uint(v.y)), "r"(__float_as_uint(v.z)),
+               "r"(__float_as_uint(v.w)), "r"(remote_bar)
+               : "memory");
+}
+
 __device__ inline float ld_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");

@@ -32,8 +32,10 @@
 //     blocks to the producer; rank 0 writes the selection out.
 // Merge: each CTA merges its four warps into one partial (O, m, l) and
 // pushes it, slice by slice, into the receive buffers of the cluster's CTAs
-// (CTA r owns output slice r); after one cluster barrier, CTA r combines
-// the C partials of its slice from its own shared memory, in rank order.
+// (CTA r owns output slice r) with st.async, whose bytes complete on the
+// receiver's mbarrier; once its slice has arrived, CTA r combines the C
+// partials from its own shared memory, in rank order.  No cluster barrier
+// ends the kernel: a CTA only waits for what is pushed into it.
 //
 // No global-memory flags, tickets or work queues: the only cross-CTA
 // traffic is inside the cluster, and every wait is bounded (status bit
@@ -80,6 +82,7 @@ struct StepShared {
   uint64_t empty_bar[kMaxStages];
   uint64_t scores_bar;  // completes when every CTA of the cluster has sent its block scores
   uint64_t sel_bar;     // completes when the selection is in shared memory (selector -> producer)
+  uint64_t recv_bar;    // completes when every CTA of the cluster has pushed its share of this CTA's output slice
   int stage_blk[kMaxStages][2];   // the stage's tiles (second: kAbsentTile when one)
   int stage_soff[kMaxStages][2];  // INT8: position of the tile's first scale in its scale slot
   int sel_count;
@@ -116,6 +119,24 @@ __host__ __device__ constexpr int out_items() {
 template <int G>
 __host__ __device__ constexpr int recv_bytes() {
   return (out_items<G>() + kMaxCluster) * 16 + 2 * kMaxCluster * G * 4;
+}
+
+// Output float4s [f0, f1) of CTA `rank`'s slice of a pair's output.
+template <int G>
+__host__ __device__ inline void out_slice(int rank, int C, int* f0, int* f1) {
+  const int slice = (out_items<G>() + C - 1) / C;
+  *f0 = rank * slice < out_items<G>() ? rank * slice : out_items<G>();
+  *f1 = *f0 + slice < out_items<G>() ? *f0 + slice : out_items<G>();
+}
+// Bytes the cluster's CTAs push into CTA `rank` in the merge.
+template <int G>
+__device__ inline uint32_t recv_slice_bytes(int rank, int C) {
+  int f0, f1;
+  out_slice<G>(rank, C, &f0, &f1);
+  if (f1 <= f0) return 0u;
+  constexpr int kVec = kHeadDim / 4;
+  const int rows = (f1 - 1) / kVec - f0 / kVec + 1;
+  return static_cast<uint32_t>(C * (16 * (f1 - f0) + 8 * rows));
 }
 
 // Offset (from the aligned base) of the INT8 scale slots: after the receive
@@ -164,19 +185,15 @@ __device__ inline bool select_group_all(bool v) {
 }
 
 // Cross-warp merge scratch (in the drained ring): per warp O rows with a
-// padded stride (bank-conflict free float2 stores), row max / sum / weight,
-// then the CTA's row max / sum.
+// padded stride (bank-conflict free float2 stores), row max and row sum.
 constexpr int kMoStride = kHeadDim + 8;
 template <int G>
 struct MergeLayout {
   static constexpr int kMo = 0;                                      // [4][G][kMoStride]
   static constexpr int kMm = kMo + kConsumerWarps * G * kMoStride;   // [4][G]
   static constexpr int kMl = kMm + kConsumerWarps * G;               // [4][G]
-  static constexpr int kMw = kMl + kConsumerWarps * G;               // [4][G]
-  static constexpr int kPm = kMw + kConsumerWarps * G;               // [G] the CTA's row max
-  static constexpr int kPl = kPm + G;                                // [G] the CTA's row sum
 };
-static_assert((MergeLayout<kMaxGroup>::kPl + kMaxGroup) * 4 <= 2 * kStageBytes,
+static_assert((MergeLayout<kMaxGroup>::kMl + kConsumerWarps * kMaxGroup) * 4 <= 2 * kStageBytes,
               "merge scratch must fit in the smallest ring (2 stages)");
 
 // Ring depths of a launch: the smaller one for two CTAs per SM, the larger
@@ -226,6 +243,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     // every CTA of the cluster arrives once.
     mbar_init(&sh.scores_bar, spill ? C : 1);
     mbar_init(&sh.sel_bar, 1);
+    mbar_init(&sh.recv_bar, 1);
     fence_barrier_init();
 #ifdef NOSA_TRACE
     for (int k = 0; k < 24; ++k) sh.tr[k] = 0;
@@ -249,13 +267,38 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 #ifdef NOSA_TRACE
   if (tid == 0) NOSA_STAMP(6);
 #endif
+  const int i = pair / a.hkv, g = pair % a.hkv;
+  const __nv_bfloat16* q_group = a.q + (static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G) * kHeadDim;
+  // This CTA's first scoring chunk goes out before the sequence length is
+  // read: its rows depend only on the pair, so chunk `rank` is issued
+  // whenever a sequence of max_seq_len tokens has it; if the sequence turns
+  // out shorter the consumers release the stage unscored.  Meanwhile the
+  // selector warp pulls the group's queries into L1.
+  const int nchunks_max =
+      scoring && a.comp_out == nullptr && a.seq_of == nullptr ? (a.ncand_max + kChunkBlocks - 1) / kChunkBlocks : 0;
+  const bool early_chunk = static_cast<int>(rank) < nchunks_max;
+  if (early_chunk && warp == kProducerWarp && lane == 0) {
+    const int row0 = (i * a.hkv + g) * a.nc_cap + kChunkBlocks * kWindowsPerBlock * static_cast<int>(rank) - 1;
+    const uint64_t policy = l2_evict_first_policy();
+    if (a.pooled_bf16) {
+      mbar_arrive_expect_tx(&sh.full_bar[0], kScoreTxBytesBf16);
+      tma_load_keys(smem, tm_p, 0, row0, &sh.full_bar[0], policy);
+      tma_load_keys(smem + kScoreSlotBytes, tm_p, 64, row0, &sh.full_bar[0], policy);
+    } else {
+      mbar_arrive_expect_tx(&sh.full_bar[0], kScoreTxBytes);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tma_load_keys(smem + c * kScoreSlotBytes, tm_p, c * kBoxCols, row0, &sh.full_bar[0], policy);
+    }
+  }
+  if (warp == kSelectorWarp && lane < 2 * G)
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(q_group) + 128 * lane) : "memory");
 
   // ---------------------------------------------------------------- geometry
   // (identical in every CTA of the cluster)
   // Entry i is one query (its own length L, q, selection and output); si is
   // the sequence whose cache and pooled keys it reads (si = i except for
   // the multi-query prefill, where many entries share one sequence).
-  const int i = pair / a.hkv, g = pair % a.hkv;
   const bool uses_cache = decoding || appending;
   const int L = a.seq_len[i];
   const int si = a.seq_of ? a.seq_of[i] : i;
@@ -292,11 +335,14 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     if (bad_rows) set_status(a.status, NOSA_DEV_CACHE_ROWS);
     if (scoring && nc_all > a.nc_cap) set_status(a.status, NOSA_DEV_NC_CAP);
   }
-  const __nv_bfloat16* q_group = a.q + (static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G) * kHeadDim;
   // The selector expects the pair's block-score bytes before this CTA joins
   // cluster barrier phase 1, so no other CTA can send one before.
   if (scoring && !spill && warp == kSelectorWarp && lane == 0)
     mbar_arrive_expect_tx(&sh.scores_bar, 4u * static_cast<uint32_t>(ncand));
+  // The same for this CTA's output slice: C x (16 bytes per float4 of the
+  // slice + 8 bytes (row max, row sum) per row the slice touches).
+  if (decoding && warp == kSelectorWarp && lane == 0)
+    mbar_arrive_expect_tx(&sh.recv_bar, recv_slice_bytes<G>(static_cast<int>(rank), static_cast<int>(C)));
   // Cluster barrier phase 1: this CTA's barriers exist (and expect their
   // bytes).  Each thread waits on it before its first access to another
   // CTA's shared memory.
@@ -339,7 +385,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------------- producer
     const uint64_t policy = l2_evict_first_policy();
-    uint32_t r = 0;  // jobs issued
+    uint32_t r = early_chunk ? 1u : 0u;  // jobs issued
     bool ok = true;
     // Lane 0 waits for the stage, then issues the job's boxes.
     auto issue = [&](auto&& body) {
@@ -355,7 +401,8 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       if (ok) ++r;
     };
     const int row_base = (si * a.hkv + g) * a.nc_cap;  // first pooled row of the pair (host: rows < 2^31)
-    for (int k = static_cast<int>(rank); k < nchunks && ok; k += static_cast<int>(C)) {
+    for (int k = static_cast<int>(rank) + (early_chunk ? static_cast<int>(C) : 0); k < nchunks && ok;
+         k += static_cast<int>(C)) {
       issue([&](int s, uint8_t* st) {
         const int row0 = row_base + kChunkBlocks * kWindowsPerBlock * k - 1;
         if (a.pooled_bf16) {
@@ -569,7 +616,10 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     uint32_t r = 0;  // jobs consumed
     bool ok = true;
     if (scoring) {
-      if (static_cast<int>(rank) < nchunks) {
+      // Chunk jobs of this CTA: its chunks of the pair, or the early chunk
+      // alone when the sequence is too short to have it.
+      const int chunk_end = max(nchunks, early_chunk ? static_cast<int>(rank) + 1 : 0);
+      if (static_cast<int>(rank) < chunk_end) {
         const bool bf16 = a.pooled_bf16 != 0;
         ScoreQ<G> qf;
         ScoreQBf16<G> qfb;
@@ -577,16 +627,22 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           load_score_q_bf16<G>(qfb, q_group, lane);
         else
           load_score_q<G>(qf, q_group, lane);
-        for (int k = static_cast<int>(rank); k < nchunks; k += static_cast<int>(C)) {
+        for (int k = static_cast<int>(rank); k < chunk_end; k += static_cast<int>(C)) {
           const int s = static_cast<int>(r % S);
           const bool landed = consumer_all(mbar_wait(&sh.full_bar[s], (r / S) & 1u, a.status));
           if (!landed) {
             ok = false;
             break;
           }
+          if (k >= nchunks) {  // the early chunk of a short sequence
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
+            ++r;
+            continue;
+          }
 #ifdef NOSA_TRACE
-          const int cix = (k - static_cast<int>(rank)) / static_cast<int>(C);
-          if (tid == 0 && cix < 0) NOSA_STAMP(14 + 4 * cix);
+          if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(9);
+          if (tid == 0 && k == static_cast<int>(rank + C)) NOSA_STAMP(20);
 #endif
           if (bf16)
             score_stage_bf16<G>(qfb, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
@@ -597,7 +653,8 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           ++r;
           consumer_sync();  // the chunk's window scores are complete
 #ifdef NOSA_TRACE
-          if (tid == 0 && cix < 0) NOSA_STAMP(15 + 4 * cix);
+          if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(10);
+          if (tid == 0 && k == static_cast<int>(rank + C)) NOSA_STAMP(21);
 #endif
           const int b0 = kChunkBlocks * k;
           const int nblk = min(kChunkBlocks, ncand - b0);
@@ -623,9 +680,6 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
             }
           }
           consumer_sync();  // sh.blk is complete; ssm may be overwritten
-#ifdef NOSA_TRACE
-          if (tid == 0 && cix < 0) NOSA_STAMP(16 + 4 * cix);
-#endif
           if (!spill)
             for (int x = tid; x < nblk * static_cast<int>(C); x += kConsumerThreads) {
               const int b = x / static_cast<int>(C);
@@ -634,7 +688,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
                            map_shared_rank(smem_addr(&sh.scores_bar), dst));
             }
 #ifdef NOSA_TRACE
-          if (tid == 0 && cix < 0) NOSA_STAMP(17 + 4 * cix);
+          if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(19);
 #endif
         }
       }
@@ -759,73 +813,59 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       }
     }
     __syncthreads();
-    for (int row = tid; row < G; row += kStepThreads) {
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mf[ML::kMm + w * G + row]);
-      float lsum = 0.0f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float m_w = mf[ML::kMm + w * G + row];
-        const float f = m_w == -INFINITY ? 0.0f : exp2f(m_w - M);
-        mf[ML::kMw + w * G + row] = f;
-        lsum += mf[ML::kMl + w * G + row] * f;
-      }
-      mf[ML::kPm + row] = M;
-      mf[ML::kPl + row] = lsum;
-    }
-    __syncthreads();
-    // Push: output float4 f of this CTA's partial goes to CTA f / slice of
-    // the cluster (slot [rank][f % slice] of its receive buffer), and this
-    // CTA's row maxima and sums go to every CTA.
+    // Push: output float4 f of this CTA's partial (its four warps combined,
+    // weights 2^(m_w - M)) goes to CTA f / slice of the cluster (slot
+    // [rank][f % slice] of its receive buffer), and the first float4 of each
+    // row in a slice also carries the row's max and sum.  st.async completes
+    // the bytes on the receiver's recv_bar: no cluster barrier.
     constexpr int kVec = kHeadDim / 4;
     const int slice = (out_items<G>() + static_cast<int>(C) - 1) / static_cast<int>(C);
     float* recv_m = recv + 4 * static_cast<int>(C) * slice;  // [C][G]
     float* recv_l = recv_m + static_cast<int>(C) * G;         // [C][G]
     for (int f = tid; f < out_items<G>(); f += kStepThreads) {
       const int row = f / kVec, d4 = f % kVec;
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      float mw[kConsumerWarps];
+      float M = -INFINITY;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) {
-        const float fw = mf[ML::kMw + w * G + row];
+        mw[w] = mf[ML::kMm + w * G + row];
+        M = fmaxf(M, mw[w]);
+      }
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      float lsum = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float fw = mw[w] == -INFINITY ? 0.0f : fast_exp2(mw[w] - M);
         const float4 x = *reinterpret_cast<const float4*>(mf + ML::kMo + (w * G + row) * kMoStride + 4 * d4);
         o.x = fmaf(fw, x.x, o.x);
         o.y = fmaf(fw, x.y, o.y);
         o.z = fmaf(fw, x.z, o.z);
         o.w = fmaf(fw, x.w, o.w);
+        lsum = fmaf(fw, mf[ML::kMl + w * G + row], lsum);
       }
       const int dst = f / slice;
-      st_cluster_f32x4(map_shared_rank(smem_addr(recv + 4 * (static_cast<int>(rank) * slice + (f - dst * slice))),
-                                       static_cast<uint32_t>(dst)),
-                       o);
+      const uint32_t bar = map_shared_rank(smem_addr(&sh.recv_bar), static_cast<uint32_t>(dst));
+      st_async_f32x4(map_shared_rank(smem_addr(recv + 4 * (static_cast<int>(rank) * slice + (f - dst * slice))),
+                                     static_cast<uint32_t>(dst)),
+                     o, bar);
+      if (f == max(row * kVec, dst * slice)) {
+        st_async_f32(map_shared_rank(smem_addr(recv_m + static_cast<int>(rank) * G + row), static_cast<uint32_t>(dst)),
+                     M, bar);
+        st_async_f32(map_shared_rank(smem_addr(recv_l + static_cast<int>(rank) * G + row), static_cast<uint32_t>(dst)),
+                     lsum, bar);
+      }
     }
-    for (int t = tid; t < G * static_cast<int>(C); t += kStepThreads) {
-      const int row = t % G;
-      const uint32_t dst = static_cast<uint32_t>(t / G);
-      st_cluster_f32(map_shared_rank(smem_addr(recv_m + static_cast<int>(rank) * G + row), dst), mf[ML::kPm + row]);
-      st_cluster_f32(map_shared_rank(smem_addr(recv_l + static_cast<int>(rank) * G + row), dst), mf[ML::kPl + row]);
-    }
-  }
-  // Cluster barrier phase 2: every CTA's pushes have landed.  Nothing
-  // touches another CTA's shared memory after it, so no CTA needs to wait
-  // for the others before leaving.
 #ifdef NOSA_TRACE
-  if (tid == 0) NOSA_STAMP(11);
+    if (tid == 0) NOSA_STAMP(11);
 #endif
-  cluster_arrive();
-  cluster_wait();
+    // This CTA's slice of the output, once all C partials have arrived:
+    // combined in rank order.
+    int f0, f1;
+    out_slice<G>(static_cast<int>(rank), static_cast<int>(C), &f0, &f1);
+    const bool arrived = tid < f1 - f0 && mbar_wait(&sh.recv_bar, 0, a.status);
 #ifdef NOSA_TRACE
-  if (tid == 0) NOSA_STAMP(12);
+    if (tid == 0) NOSA_STAMP(12);
 #endif
-  if (decoding) {
-    // This CTA's slice of the output: all C partials from the receive
-    // buffer, combined in rank order.
-    constexpr int kVec = kHeadDim / 4;
-    const int slice = (out_items<G>() + static_cast<int>(C) - 1) / static_cast<int>(C);
-    const float* recv_m = recv + 4 * static_cast<int>(C) * slice;
-    const float* recv_l = recv_m + static_cast<int>(C) * G;
-    const int f0 = static_cast<int>(rank) * slice;
-    const int f1 = min(f0 + slice, out_items<G>());
     for (int f = f0 + tid; f < f1; f += kStepThreads) {
       const int row = f / kVec, d4 = f % kVec;
       float M = -INFINITY;
@@ -834,13 +874,18 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int k = 0; k < static_cast<int>(C); ++k) {
         const float mk = recv_m[k * G + row];
-        const float w = mk == -INFINITY ? 0.0f : exp2f(mk - M);
-        lsum += recv_l[k * G + row] * w;
+        const float w = mk == -INFINITY ? 0.0f : fast_exp2(mk - M);
+        lsum = fmaf(recv_l[k * G + row], w, lsum);
         const float4 x = *reinterpret_cast<const float4*>(recv + 4 * (k * slice + (f - f0)));
         o.x = fmaf(w, x.x, o.x);
         o.y = fmaf(w, x.y, o.y);
         o.z = fmaf(w, x.z, o.z);
         o.w = fmaf(w, x.w, o.w);
+      }
+      if (!arrived) {  // a push never came (status bit set): write zeros
+        o = make_float4(0.f, 0.f, 0.f, 0.f);
+        lsum = 0.0f;
+        M = -INFINITY;
       }
       const int64_t orow = static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G + row;
       const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
