@@ -1078,8 +1078,9 @@ __device__ inline void score_stage_bf16(const ScoreQBf16<G>& qf, uint32_t stage,
 // 4b-1 .. 4b+3 that exist (0 <= j < nc), i.e. rows 4t .. 4t+4 for block
 // b = 15k + t.  Spread over the consumer threads: min(G, 8) lanes per block,
 // each taking the window max of G / min(G, 8) heads, then a fixed shuffle
-// tree sums the heads.  Every thread of the (full) warps calls it; lane
-// `hl == 0` of block t's lanes returns S[b] in *out and true.
+// tree sums the heads.  Every thread of the (full) warps calls it; every
+// lane of block t's lanes gets S[b] in *out (the butterfly adds the same
+// operands in every lane, so they agree bit for bit) and true.
 template <int G>
 __device__ inline bool block_rule(const float* __restrict__ ssm, int k, int nblk, int64_t nc, int tid, float* out) {
   constexpr int kLanes = G < 8 ? G : 8;   // lanes per block
@@ -1103,7 +1104,7 @@ __device__ inline bool block_rule(const float* __restrict__ ssm, int k, int nblk
 #pragma unroll
   for (int o = kLanes / 2; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
   *out = part;
-  return t < nblk && hl == 0;
+  return t < nblk;
 }
 
 }  // namespace nosa

@@ -86,7 +86,6 @@ struct StepShared {
   int stage_blk[kMaxStages][2];   // the stage's tiles (second: kAbsentTile when one)
   int stage_soff[kMaxStages][2];  // INT8: position of the tile's first scale in its scale slot
   int sel_count;
-  float blk[kChunkBlocks];  // block scores of the chunk being sent
   GroupTopkShared gtk;      // the selection group's exchange (consumers + selector)
 #ifdef NOSA_TRACE
   uint64_t tr[24];
@@ -98,15 +97,19 @@ constexpr int kAbsentTile = -2;
 
 // Shared memory of the step kernel (dynamic, from a 1024-byte aligned base):
 //   ring  kRingBytes                      kStages stages of 32 KB
-//   ssm   G x kScoreStride floats         window scores of the chunk being scored
 //   sel   round16(4 * topk) bytes         the pair's selection (ascending block indices)
 //   bsm   4 * ncand_max bytes             the pair's block scores (unless kept in global memory)
 //   recv  recv_bytes<G>()                 the partials the cluster's CTAs push for this CTA's
-//                                         share of the output (see the merge)
+//                                         share of the output (see the merge); before that,
+//                                         two G x kScoreStride float buffers of window scores
+//                                         (chunks alternate between them)
 //   scl   S x kScaleStageBytes            INT8 caches: the scale rows of each stage's tiles
+// The window-score buffers can share the receive buffer: another CTA pushes
+// into it only after its selection, i.e. after every CTA of the cluster --
+// this one too -- has sent its last block score, the last use of them.
 template <int G>
-__host__ __device__ constexpr int ssm_bytes() {
-  return G * kScoreStride * 4;
+__host__ __device__ constexpr int ssm_floats() {
+  return G * kScoreStride;
 }
 __host__ __device__ constexpr int round16(int x) { return (x + 15) & ~15; }
 // Output float4s of a pair and the receive buffer that holds, for any
@@ -120,6 +123,8 @@ template <int G>
 __host__ __device__ constexpr int recv_bytes() {
   return (out_items<G>() + kMaxCluster) * 16 + 2 * kMaxCluster * G * 4;
 }
+static_assert(recv_bytes<1>() >= 8 * ssm_floats<1>() && recv_bytes<16>() >= 8 * ssm_floats<16>(),
+              "two window-score buffers fit in the receive buffer");
 
 // Output float4s [f0, f1) of CTA `rank`'s slice of a pair's output.
 template <int G>
@@ -143,8 +148,8 @@ __device__ inline uint32_t recv_slice_bytes(int rank, int C) {
 // buffer, 128-byte aligned.
 template <int G, int S>
 __host__ __device__ inline int step_scale_offset(const StepArgs& a) {
-  const int end = S * kStageBytes + ssm_bytes<G>() + round16(4 * a.topk) +
-                  (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))) + recv_bytes<G>();
+  const int end = S * kStageBytes + round16(4 * a.topk) + (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))) +
+                  recv_bytes<G>();
   return (end + 127) & ~127;
 }
 
@@ -219,9 +224,10 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzled TMA boxes want 1024-byte aligned destinations.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* ssm = reinterpret_cast<float*>(smem + kRing);
-  int32_t* sel_list = reinterpret_cast<int32_t*>(smem + kRing + ssm_bytes<G>());
-  float* bsm = reinterpret_cast<float*>(smem + kRing + ssm_bytes<G>() + round16(4 * a.topk));
+  int32_t* sel_list = reinterpret_cast<int32_t*>(smem + kRing);
+  float* bsm = reinterpret_cast<float*>(smem + kRing + round16(4 * a.topk));
+  float* recv = reinterpret_cast<float*>(smem + kRing + round16(4 * a.topk) +
+                                         (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))));
   __shared__ StepShared sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -290,6 +296,9 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
       for (int c = 0; c < 4; ++c)
         tma_load_keys(smem + c * kScoreSlotBytes, tm_p, c * kBoxCols, row0, &sh.full_bar[0], policy);
     }
+#ifdef NOSA_TRACE
+    NOSA_STAMP(13);
+#endif
   }
   if (warp == kSelectorWarp && lane < 2 * G)
     asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<const uint8_t*>(q_group) + 128 * lane) : "memory");
@@ -305,6 +314,9 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   const bool paged = a.page_table != nullptr;
   const int64_t start_i = uses_cache && !paged ? a.seq_start[si] : 0;  // issued with the length load
   const bool bad_len = L < 1 || L > a.max_seq_len;
+#ifdef NOSA_TRACE
+  if (warp == kProducerWarp && lane == 0 && !bad_len) NOSA_STAMP(8);
+#endif
   const int64_t seq_base = bad_len ? 0 : start_i;
   KvRows kv;
   kv.base = seq_base;
@@ -347,6 +359,9 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   // bytes).  Each thread waits on it before its first access to another
   // CTA's shared memory.
   cluster_arrive();
+#ifdef NOSA_TRACE
+  if (warp == kProducerWarp && lane == 0) NOSA_STAMP(23);
+#endif
 
   // Who selects: the selection group when the block scores are in shared
   // memory, else (block scores in global memory) the selector alone.
@@ -612,7 +627,14 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
     if (lane == 0) mbar_arrive(&sh.sel_bar);
   } else {
     // ---------------------------------------------------------------- consumers
-    cluster_wait();
+    // Cluster barrier phase 1 is awaited just before the first access to
+    // another CTA's shared memory (the first block-score send), so that the
+    // first chunk is scored meanwhile.
+    bool joined = false;
+    auto join_cluster = [&] {
+      if (!joined) cluster_wait();
+      joined = true;
+    };
     uint32_t r = 0;  // jobs consumed
     bool ok = true;
     if (scoring) {
@@ -644,6 +666,10 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(9);
           if (tid == 0 && k == static_cast<int>(rank + C)) NOSA_STAMP(20);
 #endif
+          // Chunks alternate between two window-score buffers: a buffer is
+          // rewritten two chunks later, after every warp has passed the
+          // next chunk's barrier and so has finished reading it.
+          float* ssm = recv + ((k - static_cast<int>(rank)) / static_cast<int>(C) & 1) * ssm_floats<G>();
           if (bf16)
             score_stage_bf16<G>(qfb, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
           else
@@ -658,16 +684,6 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 #endif
           const int b0 = kChunkBlocks * k;
           const int nblk = min(kChunkBlocks, ncand - b0);
-          {
-            float bscore;
-            if (block_rule<G>(ssm, k, nblk, nc, tid, &bscore)) {
-              constexpr int kLanes = G < 8 ? G : 8;
-              const int t = tid / kLanes;
-              sh.blk[t] = bscore;
-              if (a.bs_out) a.bs_out[static_cast<int64_t>(pair) * a.nb_out + b0 + t] = bscore;
-              if (spill) a.bs_spill[static_cast<int64_t>(pair) * a.nb_spill + b0 + t] = bscore;
-            }
-          }
           if (a.comp_out) {
             // windows [60k, min(60k + 60, nc)); the row of window j is j - 60k + 1
             const int64_t j0 = static_cast<int64_t>(kChunkBlocks) * kWindowsPerBlock * k;
@@ -679,19 +695,28 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
                     ssm[h * kScoreStride + x + 1];
             }
           }
-          consumer_sync();  // sh.blk is complete; ssm may be overwritten
-          if (!spill)
-            for (int x = tid; x < nblk * static_cast<int>(C); x += kConsumerThreads) {
-              const int b = x / static_cast<int>(C);
-              const uint32_t dst = static_cast<uint32_t>(x % static_cast<int>(C));
-              st_async_f32(map_shared_rank(smem_addr(bsm + b0 + b), dst), sh.blk[b],
-                           map_shared_rank(smem_addr(&sh.scores_bar), dst));
+          join_cluster();
+          {
+            // Every lane of block t's group holds its score: lane hl sends it
+            // to CTAs hl, hl + kLanes, ... of the cluster.
+            constexpr int kLanes = G < 8 ? G : 8;
+            const int t = tid / kLanes, hl = tid % kLanes;
+            float bscore;
+            if (block_rule<G>(ssm, k, nblk, nc, tid, &bscore)) {
+              if (!spill)
+                for (int d = hl; d < static_cast<int>(C); d += kLanes)
+                  st_async_f32(map_shared_rank(smem_addr(bsm + b0 + t), static_cast<uint32_t>(d)), bscore,
+                               map_shared_rank(smem_addr(&sh.scores_bar), static_cast<uint32_t>(d)));
+              if (hl == 0 && a.bs_out) a.bs_out[static_cast<int64_t>(pair) * a.nb_out + b0 + t] = bscore;
+              if (hl == 0 && spill) a.bs_spill[static_cast<int64_t>(pair) * a.nb_spill + b0 + t] = bscore;
             }
+          }
 #ifdef NOSA_TRACE
           if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(19);
 #endif
         }
       }
+      join_cluster();
       if (spill) {
         // Block scores in global memory: tell every CTA of the cluster (this
         // one included) that this CTA's are in place.
@@ -705,6 +730,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 #endif
       if (group_selects) group_select(tid);
     }
+    join_cluster();
     attn_init(att);
     if (decoding && ok) {
       // This CTA's tiles: local t = rank, rank + C, ... < min(nloc, ntiles),
@@ -733,7 +759,6 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
           if (!mbar_wait(&sh.full_bar[s], (r / S) & 1u, a.status)) break;
 #ifdef NOSA_TRACE
           if (tid == 0 && n == 0) NOSA_STAMP(22);
-          if (tid == 0 && n == 2) NOSA_STAMP(23);
 #endif
           if constexpr (Q8) {
             const uint8_t* st = smem + s * kStageBytes;
@@ -744,7 +769,6 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
                                          scl + 3 * (kScaleSlot / 4) + sh.stage_soff[s][1]};
 #ifdef NOSA_TRACE
             uint64_t* stamps = tid == 0 && n == 1 ? &sh.tr[14] : nullptr;
-            if (stamps) NOSA_STAMP(8);
 #else
             uint64_t* stamps = nullptr;
 #endif
@@ -753,17 +777,8 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
             else
               attend_stage_int8<2>(att, qa, qpow, st, ksc, vsc, blk, L, a.scale_log2, warp, lane, stamps);
           } else {
-#ifdef NOSA_TRACE
-            if (tid == 0 && n == 1) NOSA_STAMP(8);
-#endif
             attend_tile(att, qa, smem + s * kStageBytes, sh.stage_blk[s][0], L, a.scale_log2, warp, lane);
           }
-#ifdef NOSA_TRACE
-          if (tid == 0 && n == 1) {
-            asm volatile("" ::"f"(att.acc[0][0]), "f"(att.acc[15][3]));
-            NOSA_STAMP(13);
-          }
-#endif
           if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
           ++r;
         }
@@ -779,8 +794,7 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
   // ---------------------------------------------------------------- merge
   using ML = MergeLayout<G>;
   float* mf = reinterpret_cast<float*>(smem);
-  float* recv = reinterpret_cast<float*>(smem + kRing + ssm_bytes<G>() + round16(4 * a.topk) +
-                                         (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))));
+
   if (decoding) {
     // The four warps' states, in warp order, into this CTA's partial.
     if (warp < kConsumerWarps) {
