@@ -758,12 +758,9 @@ __device__ void bucket_topk(float* scores, int ncand, int topk, int32_t* sel_row
     const float d = (key_float(kk) - lo) * scale;
     return d >= 255.0f ? 255 : d > 0.0f ? static_cast<int>(d) : 0;
   };
-  int bk[M];
 #pragma unroll
-  for (int m = 0; m < M; ++m) {
-    bk[m] = tid + m * NT < ncand ? bucket(key[m]) : -1;
-    if (bk[m] >= 0) atomicAdd(&sh.hist[bk[m]], 1u);
-  }
+  for (int m = 0; m < M; ++m)
+    if (tid + m * NT < ncand) atomicAdd(&sh.hist[bucket(key[m])], 1u);
   group_bar(bar_id, NT);
   BKT_STAMP(1);
   // Lane l owns buckets [8l, 8l + 8); the bucket holding the k-th largest
@@ -807,11 +804,12 @@ __device__ void bucket_topk(float* scores, int ncand, int topk, int32_t* sel_row
 #pragma unroll
   for (int m = 0; m < M; ++m) {
     const int b = tid + m * NT;
-    if (bk[m] == B) {
+    const int bkm = b < ncand ? bucket(key[m]) : -1;
+    if (bkm == B) {
       const uint32_t slot = atomicAdd(&sh.nsurv, 1u);
       if (slot < nsurv) sh.surv[slot] = (static_cast<uint64_t>(key[m]) << 32) | ~static_cast<uint32_t>(b);
     }
-    const uint32_t hb = __ballot_sync(kFull, bk[m] > B);
+    const uint32_t hb = __ballot_sync(kFull, bkm > B);
     if (lane == 0) sh.take[m * kW + w] = hb;
   }
   if (tid < 4 && nsurv + tid < nsurv4) sh.surv[nsurv + tid] = 0u;  // below every entry
@@ -923,19 +921,27 @@ struct ScoreQ {
   uint32_t b[kNTiles][16][2];
 };
 
-// The group's queries as TF32 B fragments of mma m16n8k8 (k = dimension,
-// n = head; heads >= G are zero).  bf16 widens to TF32 exactly.
+// The group's queries as TF32 B fragments of mma m16n8k8 (n = head; heads
+// >= G are zero), bf16 widened exactly.  The k slots of each k-step are
+// permuted so that a lane's A values are four consecutive dimensions of a
+// row (one 16-byte load; see score_stage): with d(u, t) = 32 (u / 2) +
+// 4 (2t + u % 2), k-step 2u covers dimensions d + {0, 1} in slots t and
+// t + 4, k-step 2u + 1 dimensions d + {2, 3} (t = the lane's quad
+// position).  A dot product does not depend on the order of its terms.
 template <int G>
 __device__ inline void load_score_q(ScoreQ<G>& f, const __nv_bfloat16* __restrict__ q_group, int lane) {
   const int grp = lane >> 2, tig = lane & 3;
-  const uint16_t* bits = reinterpret_cast<const uint16_t*>(q_group);
 #pragma unroll
   for (int nt = 0; nt < ScoreQ<G>::kNTiles; ++nt) {
     const int head = nt * 8 + grp;
 #pragma unroll
-    for (int ks = 0; ks < 16; ++ks) {
-      f.b[nt][ks][0] = head < G ? static_cast<uint32_t>(__ldg(bits + head * kHeadDim + 8 * ks + tig)) << 16 : 0u;
-      f.b[nt][ks][1] = head < G ? static_cast<uint32_t>(__ldg(bits + head * kHeadDim + 8 * ks + tig + 4)) << 16 : 0u;
+    for (int u = 0; u < 8; ++u) {
+      const int d = 32 * (u >> 1) + 4 * (2 * tig + (u & 1));
+      const uint2 w = head < G ? __ldg(reinterpret_cast<const uint2*>(q_group + head * kHeadDim + d)) : make_uint2(0u, 0u);
+      f.b[nt][2 * u][0] = w.x << 16;
+      f.b[nt][2 * u][1] = w.x & 0xFFFF0000u;
+      f.b[nt][2 * u + 1][0] = w.y << 16;
+      f.b[nt][2 * u + 1][1] = w.y & 0xFFFF0000u;
     }
   }
 }
@@ -944,11 +950,15 @@ __device__ inline void load_score_q(ScoreQ<G>& f, const __nv_bfloat16* __restric
 // computes rows [16w, 16w+16) of S^T = K * Q^T (mma.sync m16n8k8, TF32
 // inputs, fp32 accumulation) and stores scale * s into ssm[head][row] for
 // rows < 61.  Each fp32 pooled value x is split into hi (x with its low 13
-// mantissa bits cleared, exact in TF32) and lo (x - hi, exact in fp32, with
-// its low 13 mantissa bits cleared too); the hi and lo products go to
-// separate fp32 accumulators (even and odd k-steps apart) that are added at
-// the end, so the only input rounding is that of lo, below 2^-20 of |x| ("NOSA-1B
-// 性能基准全解析" §三.3: scores of the pooled keys).
+// mantissa bits cleared, exact in TF32) and lo = x - hi (exact in fp32, of
+// which the tensor core reads the TF32 part); the hi and lo products go to
+// separate fp32 accumulators that are added at the end, so the only input
+// rounding is that of lo, below 2^-20 of |x| ("NOSA-1B 性能基准全解析" §三.3:
+// scores of the pooled keys).  A lane reads its four dimensions of a row
+// (see load_score_q) with one 16-byte load per row and k-step pair: 16-byte
+// unit 2t + u % 2 of the row's 128-byte box row, so that the two rows a
+// quarter warp reads (their row indices differ in the lowest bit, which the
+// 128-byte swizzle XORs into the unit) fall on disjoint banks.
 template <int G>
 __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* __restrict__ ssm, float scale,
                                    int warp, int lane) {
@@ -966,29 +976,30 @@ __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* _
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc_hi[c][nt][e] = acc_lo[c][nt][e] = 0.0f;
 #pragma unroll
-  for (int ks = 0; ks < 16; ++ks) {
-    const uint32_t box = stage + (ks >> 2) * kScoreSlotBytes;
-    const int unit = 2 * (ks & 3);  // 16-byte unit of dimension 8*(ks%4) within the 128-byte row
-    float x[4];
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(x[0]) : "r"(box + ra * 128 + ((unit ^ (ra & 7)) << 4) + tig * 4));
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(x[1]) : "r"(box + rb * 128 + ((unit ^ (rb & 7)) << 4) + tig * 4));
-    asm volatile("ld.shared.f32 %0, [%1];"
-                 : "=f"(x[2])
-                 : "r"(box + ra * 128 + (((unit + 1) ^ (ra & 7)) << 4) + tig * 4));
-    asm volatile("ld.shared.f32 %0, [%1];"
-                 : "=f"(x[3])
-                 : "r"(box + rb * 128 + (((unit + 1) ^ (rb & 7)) << 4) + tig * 4));
-    uint32_t hi[4], lo[4];
+  for (int u = 0; u < 8; ++u) {  // k-steps 2u, 2u + 1
+    const uint32_t box = stage + (u >> 1) * kScoreSlotBytes;
+    const int unit = 2 * tig + (u & 1);  // dimensions d(u, tig) .. + 3 of the box row
+    uint32_t va[4], vb[4];
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(va[0]), "=r"(va[1]), "=r"(va[2]), "=r"(va[3])
+                 : "r"(box + ra * 128 + ((unit ^ (ra & 7)) << 4)));
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(vb[0]), "=r"(vb[1]), "=r"(vb[2]), "=r"(vb[3])
+                 : "r"(box + rb * 128 + ((unit ^ (rb & 7)) << 4)));
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      hi[e] = __float_as_uint(x[e]) & 0xffffe000u;
-      const float r = x[e] - __uint_as_float(hi[e]);  // exact; NaN only for infinite x
-      lo[e] = __float_as_uint(r == r ? r : 0.0f) & 0xffffe000u;
-    }
+    for (int h = 0; h < 2; ++h) {  // k-step 2u + h: dimensions d(u, tig) + 2h + {0, 1}
+      const uint32_t x[4] = {va[2 * h], vb[2 * h], va[2 * h + 1], vb[2 * h + 1]};
+      uint32_t hi[4], lo[4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      mma_tf32_1688(acc_hi[ks & 1][nt], hi, qf.b[nt][ks][0], qf.b[nt][ks][1]);
-      mma_tf32_1688(acc_lo[ks & 1][nt], lo, qf.b[nt][ks][0], qf.b[nt][ks][1]);
+      for (int e = 0; e < 4; ++e) {
+        hi[e] = x[e] & 0xffffe000u;
+        lo[e] = __float_as_uint(__uint_as_float(x[e]) - __uint_as_float(hi[e]));
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_tf32_1688(acc_hi[h][nt], hi, qf.b[nt][2 * u + h][0], qf.b[nt][2 * u + h][1]);
+        mma_tf32_1688(acc_lo[h][nt], lo, qf.b[nt][2 * u + h][0], qf.b[nt][2 * u + h][1]);
+      }
     }
   }
   // acc[nt][0..1]: row ra, heads nt*8 + 2*tig + {0,1}; [2..3]: row rb.

@@ -381,14 +381,14 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 #else
       uint64_t* stamps = nullptr;
 #endif
-      // Bucket select up to 7 candidates per thread (held in registers), the
-      // radix select beyond.
+      // Bucket select, the candidates held in registers (up to 13 per thread:
+      // every count shared memory holds).
       if (ncand <= 2 * kSelectThreads)
         bucket_topk<kSelectThreads, 2>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
       else if (ncand <= 7 * kSelectThreads)
         bucket_topk<kSelectThreads, 7>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
       else
-        group_topk<kSelectThreads>(bsm, false, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
+        bucket_topk<kSelectThreads, 13>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
     } else {
       for (int x = gtid; x < a.topk; x += kSelectThreads) sel_list[x] = -1;
       if (gtid == 0) sh.sel_count = 0;
