@@ -1082,9 +1082,9 @@ cudaError_t launch_with(const StepArgs& a, const StepMaps& maps, size_t smem, in
 // only when the grid leaves at least half of the resident slots free: the
 // next launch's clusters then become resident and run their prologue early;
 // when the grid fills the GPU, early-resident clusters of the next launch
-// only skew where the rest are placed.  NOSA_CLUSTER_SIZE (1..16) and
-// NOSA_RING_STAGES (the smaller or the larger ring: 3 / 6, INT8 2 / 4)
-// override the choices.
+// only skew where the rest are placed.  NOSA_CLUSTER_SIZE (1..16),
+// NOSA_RING_STAGES (the smaller or the larger ring: 3 / 6, INT8 2 / 4) and
+// NOSA_PDL (0 / 1) override the choices.
 template <int G, bool Q8>
 cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t stream) {
   const int pairs = a.batch * a.hkv;
@@ -1103,6 +1103,10 @@ cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t 
     const char* v = getenv("NOSA_RING_STAGES");
     return v ? atoi(v) : 0;
   }();
+  static const int forced_pdl = [] {
+    const char* v = getenv("NOSA_PDL");
+    return v && (atoi(v) == 0 || atoi(v) == 1) ? atoi(v) : -1;
+  }();
   constexpr int kLo = Rings<Q8>::kLo, kHi = Rings<Q8>::kHi;
   const size_t smem3 = step_smem_bytes<G, kLo, Q8>(a), smem6 = step_smem_bytes<G, kHi, Q8>(a);
   int csize, stages = kLo;
@@ -1114,13 +1118,13 @@ cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t 
     if (e != cudaSuccess) return e;
     csize = choose_cluster(*c3, pairs, units);
     if (forced_c && c3->max_clusters[forced_c] > 0) csize = forced_c;
-    pdl = static_cast<int64_t>(pairs) * csize * 2 <= c3->slots;
+    pdl = forced_pdl >= 0 ? forced_pdl != 0 : static_cast<int64_t>(pairs) * csize * 2 <= c3->slots;
     const Capacity* c6 = nullptr;
     const bool forced = forced_s == kLo || forced_s == kHi;
     const bool want6 = forced ? forced_s == kHi : static_cast<int64_t>(pairs) * csize <= c3->sms;
     if (want6 && capacity<G, kHi, Q8>(smem6, &c6) == cudaSuccess && c6->max_clusters[csize] >= pairs) {
       stages = kHi;
-      pdl = static_cast<int64_t>(pairs) * csize * 2 <= c6->slots;
+      pdl = forced_pdl >= 0 ? forced_pdl != 0 : static_cast<int64_t>(pairs) * csize * 2 <= c6->slots;
     }
     cudaGetLastError();  // a 6-stage ring the device cannot host is simply not used
 #ifdef NOSA_TRACE
