@@ -74,6 +74,7 @@ def parse():
     ap.add_argument("--context", type=int, default=0, help="override the context length")
     ap.add_argument("--batch", type=int, default=0, help="override the batch size")
     ap.add_argument("--topk", type=int, default=0, help="override top-k blocks")
+    ap.add_argument("--layers", type=int, default=0, help="override the number of layers of a step")
     ap.add_argument("--replicas", type=int, default=0, help="cache replicas rotated (0: auto)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline time budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -113,7 +114,7 @@ class Workload:
             self.lens = [int(lens)] * self.batch
         self.hq, self.hkv = hq, hkv
         self.topk = args.topk or topk
-        self.layers = layers
+        self.layers = getattr(args, "layers", 0) or layers
         self.key_dist = kdist
         self.local_blocks = 16
         self.pooled_bf16 = getattr(args, "pooled", "fp32") == "bf16"
@@ -121,8 +122,9 @@ class Workload:
         self.paged = bool(getattr(args, "paged", False))
         self.desc = desc + (", bf16 pooled keys" if self.pooled_bf16 else "") + (
             ", INT8 K/V cache" if self.kv_int8 else "") + (", paged cache (shuffled 64-token pages)" if self.paged else "")
-        if args.context or args.batch or args.topk:
-            self.desc += f" [overridden: batch {self.batch}, context {max(self.lens)}, top-k {self.topk}]"
+        if args.context or args.batch or args.topk or getattr(args, "layers", 0):
+            self.desc += (f" [overridden: batch {self.batch}, context {max(self.lens)}, top-k {self.topk}, "
+                          f"layers {self.layers}]")
         self.max_len = max(self.lens)
 
     # Algorithmic bytes per kernel for one layer-step (see the byte model in the design notes).
@@ -552,7 +554,7 @@ def run_ours(args):
     achieved = fused_bytes_launch / launch_s / 1e9
     traffic = None
     # The committed counters cover the default variant of each named workload.
-    if not (args.context or args.batch or args.topk or wl.paged or wl.kv_int8 or wl.pooled_bf16):
+    if not (args.context or args.batch or args.topk or args.layers or wl.paged or wl.kv_int8 or wl.pooled_bf16):
         traffic = ncu_traffic(wl.name)
 
     # e2e through the host-buffer entry point, rotating over the same replicas, pinned buffers.
