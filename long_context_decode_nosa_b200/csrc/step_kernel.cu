@@ -215,7 +215,7 @@ struct Rings {
 // bytes in flight per CTA); with INT8 caches (Q8) 2 or 4 stages of two tiles.
 // Q8: the K/V caches are INT8 (codes + per-row scales).
 template <int G, int S, bool Q8>
-__global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasPerSm)
     step_kernel(const StepArgs a, const __grid_constant__ StepMaps maps) {
   constexpr int kRing = S * kStageBytes;
   const CUtensorMap* tm_k = &maps.k;
@@ -381,14 +381,17 @@ __global__ void __launch_bounds__(kStepThreads, kCtasPerSm)
 #else
       uint64_t* stamps = nullptr;
 #endif
-      // Bucket select, the candidates held in registers (up to 13 per thread:
-      // every count shared memory holds).
+      // Bucket select, the candidates held in registers: up to 7 per thread,
+      // and with one CTA per SM (registers to spare) up to 13, every count
+      // shared memory holds; the radix select beyond.
       if (ncand <= 2 * kSelectThreads)
         bucket_topk<kSelectThreads, 2>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
       else if (ncand <= 7 * kSelectThreads)
         bucket_topk<kSelectThreads, 7>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
-      else
+      else if constexpr (S == Rings<Q8>::kHi)
         bucket_topk<kSelectThreads, 13>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
+      else
+        group_topk<kSelectThreads>(bsm, false, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
     } else {
       for (int x = gtid; x < a.topk; x += kSelectThreads) sel_list[x] = -1;
       if (gtid == 0) sh.sel_count = 0;
