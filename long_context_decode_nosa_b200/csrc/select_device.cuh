@@ -1016,6 +1016,70 @@ __device__ inline void score_stage(const ScoreQ<G>& qf, uint32_t stage, float* _
   }
 }
 
+// Two chunks in one pass (stage[c] -> ssm[c]), each scored exactly as
+// score_stage scores it: the chunks' products are independent accumulation
+// chains, so the pass keeps twice as many tensor-core operations in flight.
+template <int G>
+__device__ inline void score_stage_pair(const ScoreQ<G>& qf, const uint32_t (&stage)[2], float* const (&ssm)[2],
+                                        float scale, int warp, int lane) {
+  constexpr int NT = ScoreQ<G>::kNTiles;
+  const int grp = lane >> 2, tig = lane & 3;
+  const int r0 = warp * 16;
+  const int ra = r0 + grp, rb = ra + 8;
+  float acc_hi[2][2][NT][4], acc_lo[2][2][NT][4];  // [chunk][k-step parity][n-tile][fragment]
+#pragma unroll
+  for (int x = 0; x < 2; ++x)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc_hi[x][c][nt][e] = acc_lo[x][c][nt][e] = 0.0f;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {  // k-steps 2u, 2u + 1
+    const int unit = 2 * tig + (u & 1);
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const uint32_t box = stage[x] + (u >> 1) * kScoreSlotBytes;
+      uint32_t va[4], vb[4];
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(va[0]), "=r"(va[1]), "=r"(va[2]), "=r"(va[3])
+                   : "r"(box + ra * 128 + ((unit ^ (ra & 7)) << 4)));
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(vb[0]), "=r"(vb[1]), "=r"(vb[2]), "=r"(vb[3])
+                   : "r"(box + rb * 128 + ((unit ^ (rb & 7)) << 4)));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t xv[4] = {va[2 * h], vb[2 * h], va[2 * h + 1], vb[2 * h + 1]};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[e] = xv[e] & 0xffffe000u;
+          lo[e] = __float_as_uint(__uint_as_float(xv[e]) - __uint_as_float(hi[e]));
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_tf32_1688(acc_hi[x][h][nt], hi, qf.b[nt][2 * u + h][0], qf.b[nt][2 * u + h][1]);
+          mma_tf32_1688(acc_lo[x][h][nt], lo, qf.b[nt][2 * u + h][0], qf.b[nt][2 * u + h][1]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < 2; ++x)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int head = nt * 8 + 2 * tig + (e & 1);
+        const int row = (e >> 1) ? rb : ra;
+        if (head < G && row < kChunkWindows)
+          ssm[x][head * kScoreStride + row] =
+              ((acc_hi[x][0][nt][e] + acc_hi[x][1][nt][e]) + (acc_lo[x][0][nt][e] + acc_lo[x][1][nt][e])) * scale;
+      }
+    }
+}
+
 // bf16 pooled keys: a chunk's rows arrive as two 2-D TMA boxes of {64 bf16
 // columns, 61 rows} (128-byte swizzle), box c holding dimensions
 // [64c, 64c+64), in the first two 8 KB slots of the stage.

@@ -214,7 +214,9 @@ struct Rings {
 // S = ring stages: 3 (two CTAs per SM) or 6 (one CTA per SM, twice the
 // bytes in flight per CTA); with INT8 caches (Q8) 2 or 4 stages of two tiles.
 // Q8: the K/V caches are INT8 (codes + per-row scales).
-template <int G, int S, bool Q8>
+// P: fp32 pooled keys scored two chunks per pass after the first (the deep
+// ring, for CTAs with many scoring chunks).
+template <int G, int S, bool Q8, bool P = false>
 __global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasPerSm)
     step_kernel(const StepArgs a, const __grid_constant__ StepMaps maps) {
   constexpr int kRing = S * kStageBytes;
@@ -652,56 +654,90 @@ __global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasP
           load_score_q_bf16<G>(qfb, q_group, lane);
         else
           load_score_q<G>(qf, q_group, lane);
-        for (int k = static_cast<int>(rank); k < chunk_end; k += static_cast<int>(C)) {
-          const int s = static_cast<int>(r % S);
-          const bool landed = consumer_all(mbar_wait(&sh.full_bar[s], (r / S) & 1u, a.status));
-          if (!landed) {
-            ok = false;
-            break;
-          }
-          if (k >= nchunks) {  // the early chunk of a short sequence
+        if constexpr (!P) {
+          for (int k = static_cast<int>(rank); k < chunk_end; k += static_cast<int>(C)) {
+            const int s = static_cast<int>(r % S);
+            const bool landed = consumer_all(mbar_wait(&sh.full_bar[s], (r / S) & 1u, a.status));
+            if (!landed) {
+              ok = false;
+              break;
+            }
+            if (k >= nchunks) {  // the early chunk of a short sequence
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
+              ++r;
+              continue;
+            }
+#ifdef NOSA_TRACE
+            if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(9);
+            if (tid == 0 && k == static_cast<int>(rank + C)) NOSA_STAMP(20);
+#endif
+            // Chunks alternate between two window-score buffers: a buffer is
+            // rewritten two chunks later, after every warp has passed the
+            // next chunk's barrier and so has finished reading it.
+            float* ssm = recv + ((k - static_cast<int>(rank)) / static_cast<int>(C) & 1) * ssm_floats<G>();
+            if (bf16)
+              score_stage_bf16<G>(qfb, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
+            else
+              score_stage<G>(qf, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
             ++r;
-            continue;
-          }
+            consumer_sync();  // the chunk's window scores are complete
 #ifdef NOSA_TRACE
-          if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(9);
-          if (tid == 0 && k == static_cast<int>(rank + C)) NOSA_STAMP(20);
+            if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(10);
+            if (tid == 0 && k == static_cast<int>(rank + C)) NOSA_STAMP(21);
 #endif
-          // Chunks alternate between two window-score buffers: a buffer is
-          // rewritten two chunks later, after every warp has passed the
-          // next chunk's barrier and so has finished reading it.
-          float* ssm = recv + ((k - static_cast<int>(rank)) / static_cast<int>(C) & 1) * ssm_floats<G>();
-          if (bf16)
-            score_stage_bf16<G>(qfb, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
-          else
-            score_stage<G>(qf, smem_addr(smem + s * kStageBytes), ssm, a.scale, warp, lane);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
-          ++r;
-          consumer_sync();  // the chunk's window scores are complete
-#ifdef NOSA_TRACE
-          if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(10);
-          if (tid == 0 && k == static_cast<int>(rank + C)) NOSA_STAMP(21);
-#endif
-          const int b0 = kChunkBlocks * k;
-          const int nblk = min(kChunkBlocks, ncand - b0);
-          if (a.comp_out) {
-            // windows [60k, min(60k + 60, nc)); the row of window j is j - 60k + 1
-            const int64_t j0 = static_cast<int64_t>(kChunkBlocks) * kWindowsPerBlock * k;
-            constexpr int kWin = kChunkBlocks * kWindowsPerBlock;
-            for (int t = tid; t < G * kWin; t += kConsumerThreads) {
-              const int h = t / kWin, x = t % kWin;
-              if (j0 + x < nc)
-                a.comp_out[(static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G + h) * a.nc_cap + j0 + x] =
-                    ssm[h * kScoreStride + x + 1];
+            const int b0 = kChunkBlocks * k;
+            const int nblk = min(kChunkBlocks, ncand - b0);
+            if (a.comp_out) {
+              // windows [60k, min(60k + 60, nc)); the row of window j is j - 60k + 1
+              const int64_t j0 = static_cast<int64_t>(kChunkBlocks) * kWindowsPerBlock * k;
+              constexpr int kWin = kChunkBlocks * kWindowsPerBlock;
+              for (int t = tid; t < G * kWin; t += kConsumerThreads) {
+                const int h = t / kWin, x = t % kWin;
+                if (j0 + x < nc)
+                  a.comp_out[(static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G + h) * a.nc_cap + j0 + x] =
+                      ssm[h * kScoreStride + x + 1];
+              }
             }
+            join_cluster();
+            {
+              // Every lane of block t's group holds its score: lane hl sends it
+              // to CTAs hl, hl + kLanes, ... of the cluster.
+              constexpr int kLanes = G < 8 ? G : 8;
+              const int t = tid / kLanes, hl = tid % kLanes;
+              float bscore;
+              if (block_rule<G>(ssm, k, nblk, nc, tid, &bscore)) {
+                if (!spill)
+                  for (int d = hl; d < static_cast<int>(C); d += kLanes)
+                    st_async_f32(map_shared_rank(smem_addr(bsm + b0 + t), static_cast<uint32_t>(d)), bscore,
+                                 map_shared_rank(smem_addr(&sh.scores_bar), static_cast<uint32_t>(d)));
+                if (hl == 0 && a.bs_out) a.bs_out[static_cast<int64_t>(pair) * a.nb_out + b0 + t] = bscore;
+                if (hl == 0 && spill) a.bs_spill[static_cast<int64_t>(pair) * a.nb_spill + b0 + t] = bscore;
+              }
+            }
+#ifdef NOSA_TRACE
+            if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(19);
+#endif
           }
-          join_cluster();
-          {
-            // Every lane of block t's group holds its score: lane hl sends it
-            // to CTAs hl, hl + kLanes, ... of the cluster.
+        } else {
+          // The block rule and the sends of chunk k from its window scores
+          // (as in the single-chunk loop above).
+          auto send_chunk = [&](int k, const float* ssm) {
+            const int b0 = kChunkBlocks * k;
+            const int nblk = min(kChunkBlocks, ncand - b0);
+            if (a.comp_out) {
+              const int64_t j0 = static_cast<int64_t>(kChunkBlocks) * kWindowsPerBlock * k;
+              constexpr int kWin = kChunkBlocks * kWindowsPerBlock;
+              for (int t = tid; t < G * kWin; t += kConsumerThreads) {
+                const int h = t / kWin, x = t % kWin;
+                if (j0 + x < nc)
+                  a.comp_out[(static_cast<int64_t>(i) * a.hq + static_cast<int64_t>(g) * G + h) * a.nc_cap + j0 +
+                             x] = ssm[h * kScoreStride + x + 1];
+              }
+            }
+            join_cluster();
             constexpr int kLanes = G < 8 ? G : 8;
             const int t = tid / kLanes, hl = tid % kLanes;
             float bscore;
@@ -713,10 +749,45 @@ __global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasP
               if (hl == 0 && a.bs_out) a.bs_out[static_cast<int64_t>(pair) * a.nb_out + b0 + t] = bscore;
               if (hl == 0 && spill) a.bs_spill[static_cast<int64_t>(pair) * a.nb_spill + b0 + t] = bscore;
             }
+          };
+          // The first chunk alone (scored as soon as it lands), then pairs of
+          // chunks k, k + C into the two window-score buffers.  Every pass
+          // starts with the consumers' barrier, after every warp has finished
+          // reading the buffers of the pass before.
+          float* const ssm2[2] = {recv, recv + ssm_floats<G>()};
+          for (int k = static_cast<int>(rank); k < chunk_end;) {
+            const bool two = k != static_cast<int>(rank) && k + static_cast<int>(C) < nchunks;
+            const int s = static_cast<int>(r % S), s1 = static_cast<int>((r + 1) % S);
+            bool landed = mbar_wait(&sh.full_bar[s], (r / S) & 1u, a.status);
+            if (two) landed = mbar_wait(&sh.full_bar[s1], ((r + 1) / S) & 1u, a.status) && landed;
+            if (!consumer_all(landed)) {
+              ok = false;
+              break;
+            }
+            if (k >= nchunks) {  // the early chunk of a short sequence
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sh.empty_bar[s]);
+              ++r;
+              k += static_cast<int>(C);
+              continue;
+            }
+            if (two) {
+              const uint32_t st[2] = {smem_addr(smem + s * kStageBytes), smem_addr(smem + s1 * kStageBytes)};
+              score_stage_pair<G>(qf, st, ssm2, a.scale, warp, lane);
+            } else {
+              score_stage<G>(qf, smem_addr(smem + s * kStageBytes), ssm2[0], a.scale, warp, lane);
+            }
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(&sh.empty_bar[s]);
+              if (two) mbar_arrive(&sh.empty_bar[s1]);
+            }
+            r += two ? 2u : 1u;
+            consumer_sync();  // the chunks' window scores are complete
+            send_chunk(k, ssm2[0]);
+            if (two) send_chunk(k + static_cast<int>(C), ssm2[1]);
+            k += (two ? 2 : 1) * static_cast<int>(C);
           }
-#ifdef NOSA_TRACE
-          if (tid == 0 && k == static_cast<int>(rank)) NOSA_STAMP(19);
-#endif
         }
       }
       join_cluster();
@@ -1058,7 +1129,7 @@ int choose_cluster(const Capacity& c, int pairs, int units) {
   return best;
 }
 
-template <int G, int S, bool Q8>
+template <int G, int S, bool Q8, bool P = false>
 cudaError_t launch_with(const StepArgs& a, const StepMaps& maps, size_t smem, int csize, bool pdl,
                         cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
@@ -1075,7 +1146,31 @@ cudaError_t launch_with(const StepArgs& a, const StepMaps& maps, size_t smem, in
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, step_kernel<G, S, Q8>, a, maps);
+  return cudaLaunchKernelEx(&cfg, step_kernel<G, S, Q8, P>, a, maps);
+}
+
+// The pair-scoring instance of the deep ring: the same shared-memory
+// attributes as its base instance (set once per device), and the same
+// residency (one CTA per SM, equal shared memory).
+template <int G, bool Q8>
+cudaError_t prepare_pairs() {
+  static int prepared_dev = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || prepared_dev == dev) return e;
+  constexpr int kHi = Rings<Q8>::kHi;
+  int optin = 0;
+  cudaFuncAttributes fa;
+  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+  if ((e = cudaFuncGetAttributes(&fa, step_kernel<G, kHi, Q8, true>)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(step_kernel<G, kHi, Q8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                optin - static_cast<int>(fa.sharedSizeBytes))) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(step_kernel<G, kHi, Q8, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
+      cudaSuccess)
+    return e;
+  prepared_dev = dev;
+  return cudaSuccess;
 }
 
 // Launch plan: the cluster size (choose_cluster) on the 3-stage ring, two
@@ -1087,7 +1182,13 @@ cudaError_t launch_with(const StepArgs& a, const StepMaps& maps, size_t smem, in
 // when the grid fills the GPU, early-resident clusters of the next launch
 // only skew where the rest are placed.  NOSA_CLUSTER_SIZE (1..16),
 // NOSA_RING_STAGES (the smaller or the larger ring: 3 / 6, INT8 2 / 4) and
-// NOSA_PDL (0 / 1) override the choices.
+// NOSA_PDL (0 / 1) override the choices.  With the deep ring, fp32 pooled
+// keys and at least kPairChunks scoring chunks per CTA, chunks after the
+// first are scored two per pass (NOSA_PAIRS 0 / 1 overrides): the scoring of
+// long contexts is bound by the consumers' tensor-core chains, while with
+// few chunks per CTA a pair would hold the second chunk's scores back.
+constexpr int kPairChunks = 8;
+
 template <int G, bool Q8>
 cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t stream) {
   const int pairs = a.batch * a.hkv;
@@ -1108,6 +1209,10 @@ cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t 
   }();
   static const int forced_pdl = [] {
     const char* v = getenv("NOSA_PDL");
+    return v && (atoi(v) == 0 || atoi(v) == 1) ? atoi(v) : -1;
+  }();
+  static const int forced_pairs = [] {
+    const char* v = getenv("NOSA_PAIRS");
     return v && (atoi(v) == 0 || atoi(v) == 1) ? atoi(v) : -1;
   }();
   constexpr int kLo = Rings<Q8>::kLo, kHi = Rings<Q8>::kHi;
@@ -1135,7 +1240,22 @@ cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t 
             G, pairs, units, csize, stages, static_cast<int>(pdl), c3->slots, c6 ? c6->max_clusters[csize] : -1);
 #endif
   }
-  if (stages == kHi) return launch_with<G, kHi, Q8>(a, maps, smem6, csize, pdl, stream);
+  if (stages == kHi) {
+    if constexpr (!Q8 && G <= 8) {
+      const bool pairs_mode =
+          !a.pooled_bf16 && (forced_pairs >= 0 ? forced_pairs == 1 : (units + csize - 1) / csize >= kPairChunks);
+      if (pairs_mode) {
+        cudaError_t e;
+        {
+          std::lock_guard<std::mutex> lock(g_plan_mu);
+          e = prepare_pairs<G, Q8>();
+        }
+        if (e != cudaSuccess) return e;
+        return launch_with<G, kHi, Q8, true>(a, maps, smem6, csize, pdl, stream);
+      }
+    }
+    return launch_with<G, kHi, Q8>(a, maps, smem6, csize, pdl, stream);
+  }
   return launch_with<G, kLo, Q8>(a, maps, smem3, csize, pdl, stream);
 }
 

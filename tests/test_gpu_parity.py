@@ -371,6 +371,47 @@ def test_attention_invariant_to_cluster_partition(nosa, tmp_path):
     np.testing.assert_allclose(res[1]["out"], res[8]["out"], atol=2e-3, rtol=8e-3)
 
 
+_PAIRS_SCRIPT = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+from long_context_decode_nosa_b200 import inputs, nosa
+b = inputs.make_batch([65536, 40000, 9000, 130], num_q_heads=16, num_kv_heads=2, seed=53, device="cuda")
+p = nosa.params(16, 2, topk=64)
+st = nosa.DecodeState(p, b.batch, b.max_seq_len)
+st.rebuild_pooled(b.k_cache, b.seq_start, b.seq_len)
+bsc = torch.full((b.batch, 2, nosa.n_blocks(b.max_seq_len)), float("nan"), device="cuda")
+nosa.nosa_block_select(p, b.q, st.pooled, b.seq_len, b.max_seq_len, st.sel_idx, st.sel_cnt, st.ws,
+                       block_scores_out=bsc)
+sel0 = st.sel_idx.cpu().numpy()
+st.step(b.q, b.k_cache, b.v_cache, b.seq_start, b.seq_len, append=False, with_lse=True)
+torch.cuda.synchronize()
+rc, bits = nosa.nosa_read_device_status(st.ws)
+assert rc == 0, (rc, bits)
+np.savez(sys.argv[2], out=st.out.float().cpu().numpy(), lse=st.lse.cpu().numpy(),
+         sel=st.sel_idx.cpu().numpy(), sel0=sel0, bsc=bsc.cpu().numpy())
+"""
+
+
+def test_pair_scoring_is_bit_identical(nosa, tmp_path):
+    """Scoring two chunks per pass (the deep ring's mode for CTAs with many
+    chunks; NOSA_PAIRS forces it on or off, read once per process) performs
+    every chunk's arithmetic exactly as the one-chunk pass: block scores,
+    selections, outputs and lse are bit-identical, for the fused step and the
+    selection launch, over sequences of 64K down to a single candidate."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = {}
+    for v in ("0", "1"):
+        env = dict(os.environ, NOSA_PAIRS=v)
+        path = str(tmp_path / f"p{v}.npz")
+        subprocess.run([sys.executable, "-c", _PAIRS_SCRIPT, root, path], env=env, check=True, timeout=300)
+        res[v] = np.load(path)
+    for key in ("bsc", "sel0", "sel", "lse", "out"):
+        np.testing.assert_array_equal(res["0"][key], res["1"][key], err_msg=key)
+
+
 def test_full_step_edge_lengths(nosa):
     """Lengths at every geometric edge in one ragged batch, whole step."""
     lens = [1, 2, 31, 32, 33, 63, 64, 65, 1023, 1024, 1025, 1088, 1089, 64 * 17 + 63, 2049, 4096]
