@@ -99,7 +99,7 @@ constexpr int kAbsentTile = -2;
 //   ring  kRingBytes                      kStages stages of 32 KB
 //   sel   round16(4 * topk) bytes         the pair's selection (ascending block indices)
 //   bsm   4 * ncand_max bytes             the pair's block scores (unless kept in global memory)
-//   recv  recv_bytes<G>()                 the partials the cluster's CTAs push for this CTA's
+//   recv  recv_bytes<G>(C)                the partials the cluster's CTAs push for this CTA's
 //                                         share of the output (see the merge); before that,
 //                                         two G x kScoreStride float buffers of window scores
 //                                         (chunks alternate between them)
@@ -112,19 +112,20 @@ __host__ __device__ constexpr int ssm_floats() {
   return G * kScoreStride;
 }
 __host__ __device__ constexpr int round16(int x) { return (x + 15) & ~15; }
-// Output float4s of a pair and the receive buffer that holds, for any
-// cluster size C <= 16, C x ceil(items / C) pushed float4s plus C x G row
-// maxima and C x G row sums.
+// Output float4s of a pair and the receive buffer of a cluster of C CTAs:
+// C x ceil(items / C) pushed float4s plus C x G row maxima and C x G row
+// sums, and at least the two window-score buffers.  Sized for the launch's
+// own cluster size (the host sizes shared memory for an upper bound of it).
 template <int G>
 __host__ __device__ constexpr int out_items() {
   return G * kHeadDim / 4;
 }
 template <int G>
-__host__ __device__ constexpr int recv_bytes() {
-  return (out_items<G>() + kMaxCluster) * 16 + 2 * kMaxCluster * G * 4;
+__host__ __device__ constexpr int recv_bytes(int C) {
+  return (out_items<G>() + C) * 16 + 2 * C * G * 4 > 8 * ssm_floats<G>()
+             ? (out_items<G>() + C) * 16 + 2 * C * G * 4
+             : 8 * ssm_floats<G>();
 }
-static_assert(recv_bytes<1>() >= 8 * ssm_floats<1>() && recv_bytes<16>() >= 8 * ssm_floats<16>(),
-              "two window-score buffers fit in the receive buffer");
 
 // Output float4s [f0, f1) of CTA `rank`'s slice of a pair's output.
 template <int G>
@@ -145,11 +146,11 @@ __device__ inline uint32_t recv_slice_bytes(int rank, int C) {
 }
 
 // Offset (from the aligned base) of the INT8 scale slots: after the receive
-// buffer, 128-byte aligned.
+// buffer of a cluster of C CTAs, 128-byte aligned.
 template <int G, int S>
-__host__ __device__ inline int step_scale_offset(const StepArgs& a) {
+__host__ __device__ inline int step_scale_offset(const StepArgs& a, int C) {
   const int end = S * kStageBytes + round16(4 * a.topk) + (a.bs_spill ? 0 : round16(4 * max(a.ncand_max, 1))) +
-                  recv_bytes<G>();
+                  recv_bytes<G>(C);
   return (end + 127) & ~127;
 }
 
@@ -463,7 +464,7 @@ __global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasP
         sh.stage_blk[s][0] = blk0;
         sh.stage_blk[s][1] = blk1;
         if constexpr (Q8) {
-          uint8_t* scl = smem + step_scale_offset<G, S>(a) + s * kScaleStageBytes;
+          uint8_t* scl = smem + step_scale_offset<G, S>(a, static_cast<int>(C)) + s * kScaleStageBytes;
           const int n = blk1 == kAbsentTile ? 1 : 2;
           mbar_arrive_expect_tx(&sh.full_bar[s], n * kTileTxBytesInt8);
           for (int x = 0; x < n; ++x) {
@@ -836,7 +837,7 @@ __global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasP
 #endif
           if constexpr (Q8) {
             const uint8_t* st = smem + s * kStageBytes;
-            const float* scl = reinterpret_cast<const float*>(smem + step_scale_offset<G, S>(a) + s * kScaleStageBytes);
+            const float* scl = reinterpret_cast<const float*>(smem + step_scale_offset<G, S>(a, static_cast<int>(C)) + s * kScaleStageBytes);
             const int blk[2] = {sh.stage_blk[s][0], sh.stage_blk[s][1]};
             const float* const ksc[2] = {scl + sh.stage_soff[s][0], scl + 2 * (kScaleSlot / 4) + sh.stage_soff[s][1]};
             const float* const vsc[2] = {scl + (kScaleSlot / 4) + sh.stage_soff[s][0],
@@ -1039,9 +1040,10 @@ __global__ void wait_selftest_kernel(uint32_t* status, uint32_t max_iters) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, status, max_iters, 1000u);
 }
 
+// Shared memory of a launch whose clusters have at most C CTAs.
 template <int G, int S, bool Q8>
-size_t step_smem_bytes(const StepArgs& a) {
-  return 1024 + step_scale_offset<G, S>(a) + (Q8 ? static_cast<size_t>(S) * kScaleStageBytes : 0);
+size_t step_smem_bytes(const StepArgs& a, int C) {
+  return 1024 + step_scale_offset<G, S>(a, C) + (Q8 ? static_cast<size_t>(S) * kScaleStageBytes : 0);
 }
 
 // Residency of the step kernel at a given shared-memory size: resident
@@ -1053,15 +1055,18 @@ struct Capacity {
   int max_clusters[kMaxCluster + 1] = {};  // C = 1..16
 };
 std::mutex g_plan_mu;
-Capacity g_cap[5][2][2];  // [group size][ring: 3 or 6 stages][bf16 / INT8 caches]
+// [group size][ring: 3 or 6 stages][bf16 / INT8 caches][receive buffer for
+// clusters of up to 16 / up to kSmallCluster CTAs]
+Capacity g_cap[5][2][2][2];
+constexpr int kSmallCluster = 4;
 
 template <int G, int S, bool Q8>
-cudaError_t capacity(size_t smem, const Capacity** out) {
+cudaError_t capacity(size_t smem, bool small_recv, const Capacity** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   constexpr int gi = G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : G == 8 ? 3 : 4;
-  Capacity& c = g_cap[gi][S == Rings<Q8>::kLo ? 0 : 1][Q8 ? 1 : 0];
+  Capacity& c = g_cap[gi][S == Rings<Q8>::kLo ? 0 : 1][Q8 ? 1 : 0][small_recv ? 1 : 0];
   if (c.dev != dev || c.smem != smem) {
     // The attribute is an upper bound: set to the largest size the device
     // allows next to the kernel's static shared memory, so that concurrent
@@ -1111,14 +1116,14 @@ cudaError_t capacity(size_t smem, const Capacity** out) {
   return cudaSuccess;
 }
 
-// Among the cluster sizes whose pairs x C CTAs are all resident at once,
-// the smallest C with the fewest scoring chunks per CTA (`units` of the
-// longest pair): a larger cluster would not shorten the longest CTA's
+// Among the cluster sizes up to max_c whose pairs x C CTAs are all resident
+// at once, the smallest C with the fewest scoring chunks per CTA (`units` of
+// the longest pair): a larger cluster would not shorten the longest CTA's
 // scoring and only costs wider exchanges.  1 when no larger cluster fits
 // (then clusters run in waves).
-int choose_cluster(const Capacity& c, int pairs, int units) {
+int choose_cluster(const Capacity& c, int pairs, int units, int max_c) {
   int best = 1, best_units = units;
-  for (int cs = 2; cs <= kMaxCluster; ++cs) {
+  for (int cs = 2; cs <= max_c; ++cs) {
     if (static_cast<int64_t>(pairs) * cs > c.slots || c.max_clusters[cs] < pairs) continue;
     const int per_cta = (units + cs - 1) / cs;
     if (per_cta < best_units) {
@@ -1216,21 +1221,40 @@ cudaError_t launch_step_g(const StepArgs& a, const StepMaps& maps, cudaStream_t 
     return v && (atoi(v) == 0 || atoi(v) == 1) ? atoi(v) : -1;
   }();
   constexpr int kLo = Rings<Q8>::kLo, kHi = Rings<Q8>::kHi;
-  const size_t smem3 = step_smem_bytes<G, kLo, Q8>(a), smem6 = step_smem_bytes<G, kHi, Q8>(a);
+  const size_t smem6 = step_smem_bytes<G, kHi, Q8>(a, kMaxCluster);
+  size_t smem3 = step_smem_bytes<G, kLo, Q8>(a, kMaxCluster);
+  const size_t smem3_small = step_smem_bytes<G, kLo, Q8>(a, kSmallCluster);
   int csize, stages = kLo;
   bool pdl;
   {
     std::lock_guard<std::mutex> lock(g_plan_mu);
     const Capacity* c3 = nullptr;
-    cudaError_t e = capacity<G, kLo, Q8>(smem3, &c3);
+    cudaError_t e = capacity<G, kLo, Q8>(smem3, false, &c3);
     if (e != cudaSuccess) return e;
-    csize = choose_cluster(*c3, pairs, units);
-    if (forced_c && c3->max_clusters[forced_c] > 0) csize = forced_c;
+    csize = choose_cluster(*c3, pairs, units, kMaxCluster);
+    if (forced_c && c3->max_clusters[forced_c] > 0) {
+      csize = forced_c;
+    } else if (smem3_small < smem3 && c3->slots <= c3->sms) {
+      // The receive buffer of 16-CTA clusters keeps the 3-stage ring at one
+      // CTA per SM (long contexts: the block scores take the room); sized for
+      // clusters of at most kSmallCluster CTAs it may fit two.  That plan is
+      // taken when it gives fewer scoring chunks per CTA.
+      const Capacity* c3s = nullptr;
+      if (capacity<G, kLo, Q8>(smem3_small, true, &c3s) == cudaSuccess && c3s->slots > c3->slots) {
+        const int cs = choose_cluster(*c3s, pairs, units, kSmallCluster);
+        if ((units + cs - 1) / cs < (units + csize - 1) / csize) {
+          csize = cs;
+          c3 = c3s;
+          smem3 = smem3_small;
+        }
+      }
+      cudaGetLastError();
+    }
     pdl = forced_pdl >= 0 ? forced_pdl != 0 : static_cast<int64_t>(pairs) * csize * 2 <= c3->slots;
     const Capacity* c6 = nullptr;
     const bool forced = forced_s == kLo || forced_s == kHi;
     const bool want6 = forced ? forced_s == kHi : static_cast<int64_t>(pairs) * csize <= c3->sms;
-    if (want6 && capacity<G, kHi, Q8>(smem6, &c6) == cudaSuccess && c6->max_clusters[csize] >= pairs) {
+    if (want6 && capacity<G, kHi, Q8>(smem6, false, &c6) == cudaSuccess && c6->max_clusters[csize] >= pairs) {
       stages = kHi;
       pdl = forced_pdl >= 0 ? forced_pdl != 0 : static_cast<int64_t>(pairs) * csize * 2 <= c6->slots;
     }
