@@ -671,6 +671,16 @@ __device__ void sample_topk(float* scores, int ncand, int topk, int32_t* sel_row
   if (tid == 0) *sel_cnt = k_eff;
 }
 
+// The bucket select's hand-over to the radix select (more survivors in the
+// k-th bucket than its list holds: ties, or a range the buckets cannot
+// split).  Out of line: it almost never runs, and inlined it would sit in
+// the middle of the bucket select's code.
+template <int NT>
+__device__ __noinline__ void group_topk_from_keys(float* scores, int ncand, int topk, int32_t* sel_row,
+                                                  int32_t* sel_cnt, int tid, GroupTopkShared& sh, int bar_id) {
+  group_topk<NT, true>(scores, false, ncand, topk, sel_row, sel_cnt, tid, sh, bar_id);
+}
+
 // The fp32 score an order-preserving key stands for (order_key's inverse;
 // -0.0 and NaN come back as +0.0 and -inf).
 __device__ inline float key_float(uint32_t k) {
@@ -797,7 +807,7 @@ __device__ void bucket_topk(float* scores, int ncand, int topk, int32_t* sel_row
   const uint32_t c_above = __shfl_sync(kFull, my_above, src);
   const uint32_t nsurv = sh.hist[B], need = k - c_above;
   if (nsurv > static_cast<uint32_t>(kSurvivorCap)) {  // uniform over the group
-    group_topk<NT, true>(scores, false, ncand, topk, sel_row, sel_cnt, tid, sh, bar_id);
+    group_topk_from_keys<NT>(scores, ncand, topk, sel_row, sel_cnt, tid, sh, bar_id);
     return;
   }
   const uint32_t nsurv4 = (nsurv + 3u) & ~3u;

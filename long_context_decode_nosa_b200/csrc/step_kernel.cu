@@ -77,6 +77,21 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;    // 128
 constexpr int kCtasPerSm = 2;
 constexpr int kSelOnlyThreads = 256;
 
+// Cold paths of the step kernel, out of line so that they do not sit in the
+// middle of the code every launch runs: the selector's top-k over block
+// scores in global memory (very long sequences only), and the pooling of
+// the window the new token completes (one warp of one CTA per pair, once per
+// launch, off the scoring chain).
+__device__ __noinline__ void select_spilled(const float* scores, int ncand, int topk, int32_t* sel_row,
+                                            int32_t* sel_cnt, int lane) {
+  warp_topk_mem(scores, true, ncand, topk, sel_row, sel_cnt, lane);
+}
+__device__ __noinline__ void pool_new_window(const __nv_bfloat16* k_cache, int hkv, const KvRows& kv, int g,
+                                             int64_t j, int64_t new_row, const uint2* knew, void* dst, bool bf16,
+                                             int lane) {
+  pool_window_warp(k_cache, hkv, kv, g, j, new_row, knew, dst, bf16, lane);
+}
+
 struct StepShared {
   uint64_t full_bar[kMaxStages];
   uint64_t empty_bar[kMaxStages];
@@ -592,7 +607,7 @@ __global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasP
               pool_window_warp_int8(Int8Cache{reinterpret_cast<int8_t*>(a.k_cache), a.k_scale, a.scale_stride}, a.hkv,
                                     kv, g, j, knew ? L - 1 : -1, knew, dst, a.pooled_bf16 != 0, lane);
             else
-              pool_window_warp(a.k_cache, a.hkv, kv, g, j, knew ? L - 1 : -1, knew, dst, a.pooled_bf16 != 0, lane);
+              pool_new_window(a.k_cache, a.hkv, kv, g, j, knew ? L - 1 : -1, knew, dst, a.pooled_bf16 != 0, lane);
           } else if (lane == 0)
             set_status(a.status, NOSA_DEV_BAD_INDEX);
         }
@@ -609,8 +624,8 @@ __global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasP
         if (ok) {
           // Block scores in global memory: beyond the group's shared memory, so
           // more than any register-resident selection holds.
-          warp_topk_mem(a.bs_spill + static_cast<int64_t>(pair) * a.nb_spill, true, ncand, a.topk, sel_list,
-                        &sh.sel_count, lane);
+          select_spilled(a.bs_spill + static_cast<int64_t>(pair) * a.nb_spill, ncand, a.topk, sel_list,
+                         &sh.sel_count, lane);
         } else {
           for (int t = lane; t < a.topk; t += 32) sel_list[t] = -1;
           if (lane == 0) sh.sel_count = 0;
