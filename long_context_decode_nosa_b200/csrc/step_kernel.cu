@@ -79,12 +79,17 @@ constexpr int kSelOnlyThreads = 256;
 
 // Cold paths of the step kernel, out of line so that they do not sit in the
 // middle of the code every launch runs: the selector's top-k over block
-// scores in global memory (very long sequences only), and the pooling of
-// the window the new token completes (one warp of one CTA per pair, once per
-// launch, off the scoring chain).
+// scores in global memory (very long sequences only), the selection group's
+// radix select (above the register-resident bucket select's candidates), and
+// the pooling of the window the new token completes (one warp of one CTA per
+// pair, once per launch, off the scoring chain).
 __device__ __noinline__ void select_spilled(const float* scores, int ncand, int topk, int32_t* sel_row,
                                             int32_t* sel_cnt, int lane) {
   warp_topk_mem(scores, true, ncand, topk, sel_row, sel_cnt, lane);
+}
+__device__ __noinline__ void select_radix(const float* scores, int ncand, int topk, int32_t* sel_row,
+                                          int32_t* sel_cnt, int gtid, GroupTopkShared& gtk, int bar_id) {
+  group_topk<kConsumerThreads + 32>(scores, false, ncand, topk, sel_row, sel_cnt, gtid, gtk, bar_id);
 }
 __device__ __noinline__ void pool_new_window(const __nv_bfloat16* k_cache, int hkv, const KvRows& kv, int g,
                                              int64_t j, int64_t new_row, const uint2* knew, void* dst, bool bf16,
@@ -409,7 +414,7 @@ __global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasP
       else if constexpr (S == Rings<Q8>::kHi)
         bucket_topk<kSelectThreads, 13>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
       else
-        group_topk<kSelectThreads>(bsm, false, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
+        select_radix(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
     } else {
       for (int x = gtid; x < a.topk; x += kSelectThreads) sel_list[x] = -1;
       if (gtid == 0) sh.sel_count = 0;
