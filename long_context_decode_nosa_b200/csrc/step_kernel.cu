@@ -77,12 +77,13 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;    // 128
 constexpr int kCtasPerSm = 2;
 constexpr int kSelOnlyThreads = 256;
 
-// Cold paths of the step kernel, out of line so that they do not sit in the
+// Paths of the step kernel kept out of line, so that they do not sit in the
 // middle of the code every launch runs: the selector's top-k over block
 // scores in global memory (very long sequences only), the selection group's
-// radix select (above the register-resident bucket select's candidates), and
-// the pooling of the window the new token completes (one warp of one CTA per
-// pair, once per launch, off the scoring chain).
+// radix select and the bucket selects of more than two keys per thread (the
+// two-key one, the small-batch case, stays inline), and the pooling of the
+// window the new token completes (one warp of one CTA per pair, once per
+// launch, off the scoring chain).  Each runs at most once per launch.
 __device__ __noinline__ void select_spilled(const float* scores, int ncand, int topk, int32_t* sel_row,
                                             int32_t* sel_cnt, int lane) {
   warp_topk_mem(scores, true, ncand, topk, sel_row, sel_cnt, lane);
@@ -90,6 +91,11 @@ __device__ __noinline__ void select_spilled(const float* scores, int ncand, int 
 __device__ __noinline__ void select_radix(const float* scores, int ncand, int topk, int32_t* sel_row,
                                           int32_t* sel_cnt, int gtid, GroupTopkShared& gtk, int bar_id) {
   group_topk<kConsumerThreads + 32>(scores, false, ncand, topk, sel_row, sel_cnt, gtid, gtk, bar_id);
+}
+template <int M>
+__device__ __noinline__ void select_bucket(float* scores, int ncand, int topk, int32_t* sel_row, int32_t* sel_cnt,
+                                           int gtid, GroupTopkShared& gtk, int bar_id, uint64_t* stamps) {
+  bucket_topk<kConsumerThreads + 32, M>(scores, ncand, topk, sel_row, sel_cnt, gtid, gtk, bar_id, stamps);
 }
 __device__ __noinline__ void pool_new_window(const __nv_bfloat16* k_cache, int hkv, const KvRows& kv, int g,
                                              int64_t j, int64_t new_row, const uint2* knew, void* dst, bool bf16,
@@ -410,9 +416,9 @@ __global__ void __launch_bounds__(kStepThreads, S == Rings<Q8>::kHi ? 1 : kCtasP
       if (ncand <= 2 * kSelectThreads)
         bucket_topk<kSelectThreads, 2>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
       else if (ncand <= 7 * kSelectThreads)
-        bucket_topk<kSelectThreads, 7>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
+        select_bucket<7>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
       else if constexpr (S == Rings<Q8>::kHi)
-        bucket_topk<kSelectThreads, 13>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
+        select_bucket<13>(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar, stamps);
       else
         select_radix(bsm, ncand, a.topk, sel_list, &sh.sel_count, gtid, sh.gtk, kSelectBar);
     } else {
