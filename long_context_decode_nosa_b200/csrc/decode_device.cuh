@@ -87,14 +87,6 @@ __device__ inline void tma_load_box(void* dst, const CUtensorMap* map, int dim0,
       : "memory");
 }
 
-// L2 prefetch of the same box (nothing lands in shared memory, nothing is
-// consumed: a later tma_load_box of the box finds it in L2).
-__device__ inline void tma_prefetch_box(const CUtensorMap* map, int dim0, int head, int row) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(dim0),
-               "r"(head), "r"(row)
-               : "memory");
-}
-
 // Address of 16-byte chunk `chunk` (0..7) of row `row` in a box written with
 // the 128-byte swizzle: chunks are permuted by XOR with (row mod 8).
 __device__ inline uint32_t swz(uint32_t box_base, int row, int chunk) {

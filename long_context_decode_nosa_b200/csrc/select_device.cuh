@@ -340,17 +340,15 @@ __device__ inline void warp_topk_mem(const float* scores, bool coherent, int nca
 // arguments; `tid` is the thread's index in the group.
 constexpr int kGroupKeys = 16;
 
-// Survivors the sample select ranks in shared memory (more fall back to the
+// Survivors the bucket select ranks in shared memory (more fall back to the
 // radix select), and its taken-bit words (32 candidate slots each).
 constexpr int kSurvivorCap = 128;
 constexpr int kTakeWords = 80;
-constexpr int kSampleWarps = 5;
 
 struct alignas(16) GroupTopkShared {
   uint32_t hist[256];             // radix select: digit histogram; bucket select: bucket counts
-  uint64_t surv[kSurvivorCap];    // sample / bucket select: survivors, key << 32 | ~index
-  uint32_t pcnt[kSampleWarps][32];  // sample select: per-range counts of the 32 pivots
-  uint32_t take[kTakeWords];      // sample / bucket select: taken bits
+  uint64_t surv[kSurvivorCap];    // bucket select: survivors, key << 32 | ~index
+  uint32_t take[kTakeWords];      // bucket select: taken bits
   uint32_t red[2][8][2];  // per-warp partials, double-buffered
   uint32_t prefix, need, nsurv;
 };
@@ -514,161 +512,6 @@ __device__ void group_topk(const float* scores, bool coherent, int ncand, int to
   if (tid == 0) *sel_cnt = k_eff;
   GTK_STAMP(5);
 #undef GTK_STAMP
-}
-
-// Exact top-k of the selection group by sample select: NT threads (a
-// multiple of 32, at most 5 warps; `tid` is the thread's index in the group)
-// and up to NT * M candidates, candidate b held by thread b mod NT in
-// register b / NT.  `scores` is the pair's block scores in shared memory
-// (16-byte aligned, room for round4(ncand) entries); they are overwritten by
-// their order-preserving keys (larger score, larger key; every valid key is
-// above 0).
-//   1. Keys: in registers and in place of the scores (zero-padded to 4).
-//   2. 32 pivots, the keys of candidates floor(p * ncand / 32): lane p of
-//      warp w counts the keys >= pivot p in the w-th of NT / 32 ranges.
-//   3. Every warp sums the counts and brackets the k-th largest key T:
-//      lo = the largest pivot with count >= k (T >= lo, else lo = 0) and
-//      hi = the smallest pivot with count < k (T < hi, else no bound).  The
-//      c_hi keys >= hi are all taken (one bit each in the taken-bit words,
-//      word q = candidates [32q, 32q + 32)); the keys in [lo, hi) survive
-//      and are listed in shared memory as key << 32 | ~index.
-//   4. Each survivor is ranked among the survivors (the list entries are
-//      unique: key descending, then index ascending); the first k - c_hi
-//      set their taken bits.  More than kSurvivorCap survivors (many equal
-//      keys): the radix select decides instead.
-//   5. Placement in ascending index order: a candidate's position is the
-//      number of taken bits below its own.
-// Four barriers, each phase a few independent loads deep: no chain of
-// dependent steps over the key bits.
-template <int NT, int M>
-__device__ void sample_topk(float* scores, int ncand, int topk, int32_t* sel_row, int32_t* sel_cnt, int tid,
-                            GroupTopkShared& sh, int bar_id) {
-  constexpr int kW = NT / 32;
-  constexpr int kQ = M * kW;  // taken-bit words of the NT * M candidate slots
-  static_assert(NT % 32 == 0 && NT <= 32 * kSampleWarps, "the group is 1..5 whole warps");
-  static_assert(M >= 1 && kQ <= kTakeWords, "keys held in registers; one taken-bit word per 32 slots");
-  constexpr uint32_t kFull = 0xffffffffu;
-  const int lane = tid & 31, w = tid >> 5;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  const int k_eff = ncand < topk ? ncand : topk;
-  if (k_eff == ncand) {  // every candidate is taken
-    for (int b = tid; b < topk; b += NT) sel_row[b] = b < ncand ? b : -1;
-    if (tid == 0) *sel_cnt = k_eff;
-    return;
-  }
-  uint32_t* ords = reinterpret_cast<uint32_t*>(scores);
-  const int n4 = (ncand + 3) & ~3;
-  uint32_t key[M];
-#pragma unroll
-  for (int m = 0; m < M; ++m) {
-    const int b = tid + m * NT;
-    const float f = scores[b < ncand ? b : 0];  // loads issued unconditionally
-    key[m] = b < ncand ? order_key(f) : 0u;
-    if (b < n4) ords[b] = key[m];
-  }
-  if (tid == 0) sh.nsurv = 0u;
-  group_bar(bar_id, NT);
-
-  const uint32_t piv = ords[(lane * ncand) >> 5];
-  {
-    // Range w: [r0, r1), 4-aligned, at most NT * M / kW + 4 keys.
-    const int r0 = ((w * n4) / kW) & ~3;
-    const int r1 = w == kW - 1 ? n4 : (((w + 1) * n4) / kW) & ~3;
-    // Every chunk load is issued unconditionally (clamped into the keys) so
-    // that they are all in flight at once; chunks past r1 count nothing.
-    constexpr int kMaxChunks = (NT * M) / (4 * kW) + 1;
-    uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0;
-#pragma unroll
-    for (int j = 0; j < kMaxChunks; ++j) {
-      const int c = r0 + 4 * j;
-      const uint4 v = *reinterpret_cast<const uint4*>(ords + (c < n4 ? c : n4 - 4));
-      const uint32_t p = c < r1 ? piv : 0xFFFFFFFFu;  // no valid key reaches 0xFFFFFFFF
-      c0 += v.x >= p;
-      c1 += v.y >= p;
-      c2 += v.z >= p;
-      c3 += v.w >= p;
-    }
-    sh.pcnt[w][lane] = (c0 + c1) + (c2 + c3);
-  }
-  group_bar(bar_id, NT);
-
-  uint32_t cp = 0;
-#pragma unroll
-  for (int x = 0; x < kW; ++x) cp += sh.pcnt[x][lane];
-  const uint32_t k = static_cast<uint32_t>(k_eff);
-  const bool at_least_k = cp >= k;
-  const uint32_t lo = __reduce_max_sync(kFull, at_least_k ? piv : 0u);
-  const uint32_t c_lo = __reduce_min_sync(kFull, at_least_k ? cp : static_cast<uint32_t>(ncand));
-  const uint32_t hi = __reduce_min_sync(kFull, at_least_k ? 0xFFFFFFFFu : piv);
-  const uint32_t c_hi = __reduce_max_sync(kFull, at_least_k ? 0u : cp);
-  const uint32_t nsurv = c_lo - c_hi, need = k - c_hi;
-  if (nsurv > static_cast<uint32_t>(kSurvivorCap)) {  // uniform over the group
-    group_topk<NT, true>(scores, false, ncand, topk, sel_row, sel_cnt, tid, sh, bar_id);
-    return;
-  }
-  const uint32_t nsurv4 = (nsurv + 3u) & ~3u;
-#pragma unroll
-  for (int m = 0; m < M; ++m) {
-    const int b = tid + m * NT;
-    if (key[m] != 0u && key[m] >= lo && key[m] < hi) {
-      const uint32_t slot = atomicAdd(&sh.nsurv, 1u);
-      if (slot < nsurv) sh.surv[slot] = (static_cast<uint64_t>(key[m]) << 32) | ~static_cast<uint32_t>(b);
-    }
-    const uint32_t hb = __ballot_sync(kFull, key[m] >= hi);  // hi >= 1: no padding slot
-    if (lane == 0) sh.take[m * kW + w] = hb;
-  }
-  if (tid < 4 && nsurv + tid < nsurv4) sh.surv[nsurv + tid] = 0u;  // below every entry
-  group_bar(bar_id, NT);
-
-  for (int t = tid; t < static_cast<int>(nsurv); t += NT) {
-    const uint64_t ct = sh.surv[t];
-    uint32_t r0 = 0, r1 = 0;
-#pragma unroll 4
-    for (uint32_t s2 = 0; s2 < nsurv4; s2 += 2) {
-      const ulonglong2 e = *reinterpret_cast<const ulonglong2*>(&sh.surv[s2]);
-      r0 += e.x > ct;
-      r1 += e.y > ct;
-    }
-    if (r0 + r1 < need) {
-      const uint32_t b = ~static_cast<uint32_t>(ct);
-      atomicOr(&sh.take[b >> 5], 1u << (b & 31u));
-    }
-  }
-  group_bar(bar_id, NT);
-
-  // Exclusive prefix of the words' bit counts, by every warp: lane j scans
-  // words [kPer j, kPer j + kPer).
-  constexpr int kPer = (kQ + 31) / 32;
-  uint32_t pe[kPer];
-  uint32_t tot = 0;
-#pragma unroll
-  for (int x = 0; x < kPer; ++x) {
-    const int qq = lane * kPer + x;
-    pe[x] = tot;
-    const uint32_t wd = sh.take[qq < kQ ? qq : 0];
-    tot += qq < kQ ? __popc(wd) : 0u;
-  }
-  uint32_t inc = tot;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(kFull, inc, o);
-    if (lane >= o) inc += y;
-  }
-#pragma unroll
-  for (int x = 0; x < kPer; ++x) pe[x] += inc - tot;
-#pragma unroll
-  for (int m = 0; m < M; ++m) {
-    const int q = m * kW + w;  // this thread's word (uniform over the warp)
-    uint32_t v = pe[0];
-#pragma unroll
-    for (int x = 1; x < kPer; ++x)
-      if (q % kPer == x) v = pe[x];
-    const uint32_t pre = __shfl_sync(kFull, v, q / kPer);
-    const uint32_t word = sh.take[q];
-    if ((word >> lane) & 1u) sel_row[pre + __popc(word & lt_mask)] = tid + m * NT;
-  }
-  for (int x = k_eff + tid; x < topk; x += NT) sel_row[x] = -1;
-  if (tid == 0) *sel_cnt = k_eff;
 }
 
 // The bucket select's hand-over to the radix select (more survivors in the
@@ -878,18 +721,6 @@ __device__ void bucket_topk(float* scores, int ncand, int topk, int32_t* sel_row
 #undef BKT_STAMP
 }
 
-// Top-k by one warp: register-resident keys up to kWarpTopkMax candidates,
-// memory-resident beyond.
-__device__ inline void warp_select(const float* scores, bool coherent, int ncand, int topk, int32_t* sel_row,
-                                   int32_t* sel_cnt, int lane, uint64_t* trace_stamps = nullptr) {
-  if (ncand <= 256)
-    warp_topk<8>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane, trace_stamps);
-  else if (ncand <= kWarpTopkMax)
-    warp_topk<32>(scores, coherent, ncand, topk, sel_row, sel_cnt, lane, trace_stamps);
-  else
-    warp_topk_mem(scores, coherent, ncand, topk, sel_row, sel_cnt, lane);
-}
-
 // ---------------------------------------------------------------- scoring
 // A scoring chunk k of a (sequence, KV head) covers blocks [15k, 15k+15)
 // and pooled windows [60k-1, 60k+60) (61 rows; row r is window 60k-1+r).
@@ -916,13 +747,6 @@ __device__ inline void tma_load_keys(void* dst, const CUtensorMap* map, int col,
       "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
       "l"(map), "r"(col), "r"(row), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
-}
-
-// L2 prefetch of the same box (nothing lands in shared memory, nothing is
-// consumed: a later tma_load_keys of the box finds it in L2).
-__device__ inline void tma_prefetch_keys(const CUtensorMap* map, int col, int row) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(col), "r"(row)
-               : "memory");
 }
 
 template <int G>

@@ -25,8 +25,9 @@
 //     a stage carries two tiles (half the bytes each) and their scale rows;
 //   * warp 5, selector: pools the window completed by the new token (rank
 //     0), waits until the block scores of the whole pair have arrived, runs
-//     the exact top-k with the consumers (the selection group: a sample
-//     select, or a radix select above 1120 candidates; alone when the block
+//     the exact top-k with the consumers (the selection group: a bucket
+//     select with the keys in registers -- up to 7 per thread, 13 with one
+//     CTA per SM -- or a radix select above that; alone when the block
 //     scores are kept in global memory) -- every CTA computes the same
 //     selection, so no second exchange is needed -- and hands the selected
 //     blocks to the producer; rank 0 writes the selection out.
